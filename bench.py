@@ -1,0 +1,414 @@
+"""Benchmark of the block-quantized product path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step runs the hot path once over one batch of synthetic input: for the
+headline workload (Q4_K decode GEMV, W 4096x4096, x bf16 batch 1) the batch is
+a pool of independent weight matrices whose total size is at least four times
+the L2 cache, each multiplied by its own activation vector -- so every call
+streams its weights from HBM (no L2 flush needed).  Steps are replayed from a
+CUDA graph; the timed region is bracketed by a barrier and a synchronize and
+timed with CUDA events on the launching stream (max over ranks).
+
+Under torchrun (N > 1) every rank runs an independent replica (no collective:
+the path has no exchange step) and the value is the sum over ranks of the
+bytes moved divided by the slowest rank's time.
+
+`--impl reference` times the CPU oracle (fp64, plain C) on the host cores on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+HEADLINE = "q4_k_gemv_4096x4096"
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def kernel_source_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "block_quantized_matmul_quant_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel_key, sources):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        e = t[kernel_key]
+        if e["source_hash"] == kernel_source_hash(sources):
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workloads on the GPU
+
+def _torch_setup():
+    import torch
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    return torch, rank, world, local, pg
+
+
+def _x_tensor(torch, x, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16) if dtype == "bf16" else t
+
+
+class GemvStep:
+    """One step = every weight matrix of the pool multiplied by its activations."""
+
+    def __init__(self, torch, kq, wl, l2_bytes):
+        w, x, _ = synth.make_inputs(wl)
+        self.wl = wl
+        self.wbytes = w.nbytes
+        self.pool = max(8, -(-4 * l2_bytes // w.nbytes))
+        base = torch.from_numpy(w).cuda()
+        # replicas of the seeded matrix: distinct HBM addresses, same values
+        self.ws = [base.clone() for _ in range(self.pool)]
+        xt = _x_tensor(torch, x, wl.x_dtype).cuda()
+        self.xs = [xt.clone() for _ in range(self.pool)]
+        ydt = torch.float32 if wl.y_dtype == "f32" else torch.bfloat16
+        self.ys = [torch.empty((wl.m, wl.n), dtype=ydt, device="cuda") for _ in range(self.pool)]
+        self.kq = kq
+        self.launches = self.pool
+        self.x_bytes = x.size * (2 if wl.x_dtype == "bf16" else 4)
+        self.y_bytes = wl.m * wl.n * (4 if wl.y_dtype == "f32" else 2)
+        self.algo_bytes_per_launch = self.wbytes + self.x_bytes + self.y_bytes
+        self.host_w = torch.from_numpy(w).pin_memory()
+        self.host_x = _x_tensor(torch, x, wl.x_dtype).pin_memory()
+        self.host_y = torch.empty((wl.m, wl.n), dtype=ydt).pin_memory()
+
+    def run(self):
+        for i in range(self.pool):
+            self.kq.matmul(self.ws[i], self.wl.codec, self.xs[i], out=self.ys[i],
+                           const_weights=True)
+
+    def run_e2e(self):
+        """Through the public API from pinned host buffers: copy the step's
+        weights and activations in, multiply, copy the result out."""
+        for i in range(self.pool):
+            self.ws[i].copy_(self.host_w, non_blocking=True)
+            self.xs[i].copy_(self.host_x, non_blocking=True)
+            self.kq.matmul(self.ws[i], self.wl.codec, self.xs[i], out=self.ys[i])
+            self.host_y.copy_(self.ys[i], non_blocking=True)
+
+    def step_units(self):
+        return self.wbytes * self.pool  # weight bytes per step
+
+
+def time_graph(torch, fn, steps, warmup, pg):
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            fn()
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        for _ in range(steps):
+            g.replay()
+        b.record(s)
+        b.synchronize()
+        torch.cuda.synchronize()
+        if pg is not None:
+            pg.barrier()
+    ms = a.elapsed_time(b)
+    del g
+    return ms
+
+
+def time_eager(torch, fn, steps, warmup, pg):
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        if pg is not None:
+            pg.barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        for _ in range(steps):
+            fn()
+        b.record(s)
+        b.synchronize()
+        if pg is not None:
+            pg.barrier()
+    return a.elapsed_time(b)
+
+
+def max_over_ranks(torch, pg, v):
+    if pg is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline_gemv(wl, budget_s=10.0):
+    """The oracle as it stands, on the host's cores, over whole GEMVs of the
+    workload repeated until ~budget_s of CPU work; GB/s of weight bytes."""
+    import oracle
+
+    w, x, _ = synth.make_inputs(wl)
+    cores = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle.matmul(wl.codec, w, wl.k, x, threads=cores)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 10000:
+            break
+    return {"value": w.nbytes * n / el / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} whole {wl.n}x{wl.k} {synth.CODEC_NAMES[wl.codec]} GEMVs (fp64 accumulate) "
+                      f"in {el:.1f} s on {cores} threads"}
+
+
+def run_gpu(args):
+    torch, rank, world, local, pg = _torch_setup()
+    import block_quantized_matmul_quant_b200 as kq
+
+    kq.lib()
+    wl = synth.WORKLOADS[args.workload]
+    if wl.kind != "gemv":
+        raise SystemExit("the bench's headline step is the decode GEMV workload")
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    step = GemvStep(torch, kq, wl, l2)
+    peaks = load_peaks()
+    with ClockSampler(local) as clk:
+        ms = time_graph(torch, step.run, args.steps, args.warmup, pg)
+    ms = max_over_ranks(torch, pg, ms)
+    e2e_ms = time_eager(torch, step.run_e2e, max(1, args.steps // 4), 1, pg)
+    e2e_ms = max_over_ranks(torch, pg, e2e_ms) / max(1, args.steps // 4)
+    per_step_ms = ms / args.steps
+    total_bytes = step.step_units() * args.steps * world
+    value = total_bytes / (ms / 1e3) / 1e9
+    launch_us = ms * 1e3 / (args.steps * step.launches)
+    achieved = step.algo_bytes_per_launch / (launch_us * 1e-6) / 1e9
+    traffic = measured_traffic("gemv_q4k_4096x4096", ["kq_gemv.cu", "kq_ptx.cuh", "kq_common.cuh"])
+    out = {
+        "metric": "Q4_K GEMV weight GB/s",
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(per_step_ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u8 Q4_K weights x bf16 activations, fp32 accumulate",
+        "data": "synthetic (seeded Q4_K wire bytes and N(0,1) bf16 activations)",
+        "config": {
+            "workload": wl.name,
+            "weights": f"{wl.n}x{wl.k} Q4_K ({step.wbytes} B)",
+            "x": f"bf16 [{wl.m},{wl.k}]",
+            "y": f"{wl.y_dtype} [{wl.m},{wl.n}]",
+            "pool_matrices_per_step": step.pool,
+            "l2_policy": f"inputs larger than L2: each step streams {step.pool} distinct weight "
+                         f"matrices ({step.pool * step.wbytes / 1e6:.0f} MB > 4x L2 {l2 / 1e6:.0f} MB)",
+            "parallelism": f"replicas x{world}",
+        },
+        "gpu_launches": args.steps * step.launches,
+        "e2e": {
+            "value": round(step.step_units() / (e2e_ms / 1e3) / 1e9 * world, 3),
+            "unit": "GB/s",
+            "h2d_bytes_per_step": (step.wbytes + step.x_bytes) * step.pool,
+            "d2h_bytes_per_step": step.y_bytes * step.pool,
+        },
+        "roofline": {
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"],
+            "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic,
+            "peak_source": peaks["source"],
+            "kernel": "gemv_q4k_kernel",
+            "launch_us": round(launch_us, 4),
+        },
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1:
+        out["cpu_baseline"] = cpu_baseline_gemv(wl, budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle (CPU) as the reference arm: each step is one whole GEMV of
+    the workload on all host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+
+    wl = synth.WORKLOADS[args.workload]
+    w, x, _ = synth.make_inputs(wl)
+    cores = len(os.sched_getaffinity(0))
+    for _ in range(args.warmup):
+        oracle.matmul(wl.codec, w, wl.k, x, threads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.matmul(wl.codec, w, wl.k, x, threads=cores)
+    el = time.perf_counter() - t0
+    value = w.nbytes * args.steps / el / 1e9
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "Q4_K GEMV weight GB/s",
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(el * 1e3 / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u8 Q4_K weights, fp64 accumulate",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "weights": f"{wl.n}x{wl.k} Q4_K", "x": f"bf16 [{wl.m},{wl.k}]"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"one whole {wl.n}x{wl.k} GEMV per step on {cores} threads"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="kq", choices=["kq", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,200 @@
+"""Python binding of libkq (block-quantized matrix products on B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libkq.so`` (built in-tree from ``csrc/`` by ``_build.py``).  torch
+supplies device memory and the current stream.  There is no CPU fallback:
+when the library is missing or the device is not an sm_100 GPU the calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import _build
+
+Q8_0, Q2_K, Q4_K, TQ1_G128 = 8, 10, 12, 1001
+CODECS = {"q8_0": Q8_0, "q2_k": Q2_K, "q4_k": Q4_K, "tq1_g128": TQ1_G128}
+F32, BF16, F16 = 0, 1, 2
+PATH_AUTO, PATH_SIMPLE, PATH_GEMV, PATH_GEMM = 0, 1, 2, 3
+FLAG_CONST_WEIGHTS = 0x100
+
+_DT = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}
+
+LIB_PATH = _build.LIB
+
+
+class KQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+def ensure_built() -> str:
+    """Build libkq.so if it is missing or older than its sources."""
+    return _build.build()
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
+                "or python -m block_quantized_matmul_quant_b200._build")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, vp, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+        sz = ctypes.c_size_t
+        L.kq_block_weights.argtypes = [i32]
+        L.kq_block_bytes.argtypes = [i32]
+        L.kq_row_bytes.argtypes = [i32, i64]
+        L.kq_row_bytes.restype = i64
+        L.kq_dequantize.argtypes = [i32, vp, i64, i64, vp, i32, vp]
+        L.kq_matmul.argtypes = [i32, vp, i64, i64, vp, i32, i64, vp, i32, vp]
+        L.kq_matmul_ex.argtypes = [i32, vp, i64, i64, vp, i32, i64, vp, i32, i32, vp]
+        L.kq_matmul_id_workspace_bytes.argtypes = [i64, i64, i64]
+        L.kq_matmul_id_workspace_bytes.restype = sz
+        L.kq_matmul_id.argtypes = [i32, vp, i64, i64, i64, i64, vp, i32, i64, vp, i64, vp, i32,
+                                   vp, sz, vp]
+        L.kq_matmul_id_ex.argtypes = [i32, vp, i64, i64, i64, i64, vp, i32, i64, vp, i64, vp, i32,
+                                      vp, sz, i32, vp]
+        L.kq_moe_group.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+        L.kq_validate.argtypes = [i32, vp, i64, i64, ctypes.POINTER(i64), vp]
+        L.kq_device_status.argtypes = [vp]
+        L.kq_status_string.argtypes = [i32]
+        L.kq_status_string.restype = ctypes.c_char_p
+        for f in ("kq_block_weights", "kq_block_bytes", "kq_dequantize", "kq_matmul",
+                  "kq_matmul_ex", "kq_matmul_id", "kq_matmul_id_ex", "kq_moe_group", "kq_validate",
+                  "kq_device_status"):
+            getattr(L, f).restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().kq_status_string(int(status)).decode()
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise KQError(st, what)
+
+
+def _codec(c) -> int:
+    return CODECS[c] if isinstance(c, str) else int(c)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t: torch.Tensor):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def block_weights(codec) -> int:
+    return lib().kq_block_weights(_codec(codec))
+
+
+def block_bytes(codec) -> int:
+    return lib().kq_block_bytes(_codec(codec))
+
+
+def row_bytes(codec, k: int) -> int:
+    return int(lib().kq_row_bytes(_codec(codec), int(k)))
+
+
+def _weights(w: torch.Tensor, codec: int, k: int):
+    if w.dtype != torch.uint8 or not w.is_contiguous() or not w.is_cuda:
+        raise ValueError("w must be a contiguous uint8 CUDA tensor of wire blocks")
+    rb = row_bytes(codec, k)
+    if rb <= 0 or w.numel() % rb:
+        raise ValueError(f"w holds {w.numel()} bytes, not a whole number of {rb}-byte rows")
+    return w.numel() // rb
+
+
+def dequantize(w: torch.Tensor, codec, k: int, dtype=torch.float32, out=None) -> torch.Tensor:
+    """Decode wire blocks [rows, row_bytes] into a [rows, k] float tensor."""
+    c = _codec(codec)
+    rows = _weights(w, c, k)
+    if out is None:
+        out = torch.empty((rows, k), dtype=dtype, device=w.device)
+    _check(lib().kq_dequantize(c, _ptr(w), rows, k, _ptr(out), _DT[out.dtype], _stream()),
+           "kq_dequantize")
+    return out
+
+
+def matmul(w: torch.Tensor, codec, x: torch.Tensor, out=None, out_dtype=torch.float32,
+           path: int = PATH_AUTO, const_weights: bool = False) -> torch.Tensor:
+    """y[m, n] = sum_k dequant(w)[n, k] * x[m, k]; x [m, k] fp32/bf16."""
+    c = _codec(codec)
+    if x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous [m, k] tensor")
+    m, k = x.shape
+    n = _weights(w, c, k)
+    if out is None:
+        out = torch.empty((m, n), dtype=out_dtype, device=x.device)
+    flags = path | (FLAG_CONST_WEIGHTS if const_weights else 0)
+    _check(lib().kq_matmul_ex(c, _ptr(w), n, k, _ptr(x), _DT[x.dtype], m, _ptr(out),
+                              _DT[out.dtype], flags, _stream()), "kq_matmul")
+    return out
+
+
+def matmul_id_workspace_bytes(n_tokens: int, top_k: int, n_experts: int) -> int:
+    return int(lib().kq_matmul_id_workspace_bytes(n_tokens, top_k, n_experts))
+
+
+def matmul_id(w: torch.Tensor, codec, x: torch.Tensor, ids: torch.Tensor, out=None,
+              out_dtype=torch.float32, workspace=None, path: int = PATH_AUTO) -> torch.Tensor:
+    """y[t, s, n] = sum_k dequant(w[ids[t, s]])[n, k] * x[t, k].
+    w: [E, n, row_bytes] uint8; x: [T, k]; ids: [T, top_k] int32."""
+    c = _codec(codec)
+    if w.dim() != 3:
+        raise ValueError("w must be [n_experts, n, row_bytes]")
+    e, n, rb = w.shape
+    t, k = x.shape
+    if rb != row_bytes(c, k):
+        raise ValueError("w's last dimension does not match k")
+    if ids.dtype != torch.int32 or ids.dim() != 2 or ids.shape[0] != t:
+        raise ValueError("ids must be int32 [n_tokens, top_k]")
+    top_k = ids.shape[1]
+    if out is None:
+        out = torch.empty((t, top_k, n), dtype=out_dtype, device=x.device)
+    need = matmul_id_workspace_bytes(t, top_k, e)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    _check(lib().kq_matmul_id_ex(c, _ptr(w), e, n, k, w.stride(0), _ptr(x), _DT[x.dtype], t,
+                                 _ptr(ids), top_k, _ptr(out), _DT[out.dtype], _ptr(workspace),
+                                 workspace.numel(), path, _stream()), "kq_matmul_id")
+    return out
+
+
+def moe_group(ids: torch.Tensor, n_experts: int):
+    """(counts [E], offsets [E+1], perm [P]) of the device-side expert grouping."""
+    ids = ids.contiguous().view(-1)
+    p = ids.numel()
+    counts = torch.empty(n_experts, dtype=torch.int32, device=ids.device)
+    offsets = torch.empty(n_experts + 1, dtype=torch.int32, device=ids.device)
+    perm = torch.empty(p, dtype=torch.int32, device=ids.device)
+    _check(lib().kq_moe_group(_ptr(ids), p, n_experts, _ptr(counts), _ptr(offsets), _ptr(perm),
+                              _stream()), "kq_moe_group")
+    return counts, offsets, perm
+
+
+def validate(w: torch.Tensor, codec, k: int) -> int:
+    """Index of the first block with an illegal TQ1 byte, or -1 (synchronizes)."""
+    c = _codec(codec)
+    rows = _weights(w, c, k)
+    out = ctypes.c_int64(-1)
+    _check(lib().kq_validate(c, _ptr(w), rows, k, ctypes.byref(out), _stream()), "kq_validate")
+    return out.value
+
+
+def device_status() -> int:
+    """Synchronize and return (and clear) the device error word as a status code."""
+    return int(lib().kq_device_status(_stream()))

@@ -1,0 +1,313 @@
+// kq_api.cu -- the C ABI (include/kq.h): argument validation, dispatch and
+// the device status word.  All validation happens before any launch.
+#include <mutex>
+#include <string.h>
+
+#include "kq_common.cuh"
+#include "kq_launch.h"
+
+namespace kq {
+
+__device__ unsigned long long g_scan_first_bad;
+__device__ unsigned int g_error_word = 0;
+
+// Device address of this device's error word (cached per device ordinal).
+unsigned int *error_word() {
+    static unsigned int *cache[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (cache[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_error_word) == cudaSuccess) cache[dev] = static_cast<unsigned int *>(p);
+    }
+    return cache[dev];
+}
+
+static int block_weights(int type) {
+    switch (type) {
+    case KQ_Q8_0: return Geom<KQ_Q8_0>::QK;
+    case KQ_Q2_K: return Geom<KQ_Q2_K>::QK;
+    case KQ_Q4_K: return Geom<KQ_Q4_K>::QK;
+    case KQ_TQ1_G128: return Geom<KQ_TQ1_G128>::QK;
+    default: return 0;
+    }
+}
+static int block_bytes(int type) {
+    switch (type) {
+    case KQ_Q8_0: return Geom<KQ_Q8_0>::BB;
+    case KQ_Q2_K: return Geom<KQ_Q2_K>::BB;
+    case KQ_Q4_K: return Geom<KQ_Q4_K>::BB;
+    case KQ_TQ1_G128: return Geom<KQ_TQ1_G128>::BB;
+    default: return 0;
+    }
+}
+
+static bool mul_ok(int64_t a, int64_t b, int64_t *r) { return !__builtin_mul_overflow(a, b, r); }
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Current device must be sm_100 (B200); cached per device ordinal.
+static int check_device() {
+    static int cache[64];  // 0 unknown, 1 ok, -1 not sm_100
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KQ_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return KQ_ERR_UNSUPPORTED;
+    if (cache[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return KQ_ERR_CUDA;
+        cache[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    return cache[dev] == 1 ? KQ_OK : KQ_ERR_UNSUPPORTED;
+}
+
+static int to_status(cudaError_t e) { return e == cudaSuccess ? KQ_OK : KQ_ERR_CUDA; }
+
+// Shared checks of a weight matrix [n, k] of `type`.
+static int check_weights(int type, const void *w, int64_t n, int64_t k, int64_t *row_bytes) {
+    const int qk = block_weights(type);
+    if (qk == 0) return KQ_ERR_TYPE;
+    if (w == nullptr) return KQ_ERR_ARG;
+    if (n <= 0 || k <= 0) return KQ_ERR_ARG;
+    if (k % qk) return KQ_ERR_SHAPE;
+    if (!aligned16(w)) return KQ_ERR_ALIGN;
+    int64_t rb = (k / qk) * block_bytes(type), total;
+    if (!mul_ok(rb, n, &total)) return KQ_ERR_OVERFLOW;
+    *row_bytes = rb;
+    return KQ_OK;
+}
+
+static int check_act(const void *p, int dtype, int64_t rows, int64_t cols, bool allow_f16) {
+    if (p == nullptr) return KQ_ERR_ARG;
+    if (dtype != KQ_F32 && dtype != KQ_BF16 && !(allow_f16 && dtype == KQ_F16)) return KQ_ERR_DTYPE;
+    if (!aligned16(p)) return KQ_ERR_ALIGN;
+    int64_t e, b;
+    if (!mul_ok(rows, cols, &e) || !mul_ok(e, 4, &b)) return KQ_ERR_OVERFLOW;
+    return KQ_OK;
+}
+
+// Workspace layout of kq_matmul_id (256-byte aligned sections).
+struct IdWorkspace {
+    size_t counts, offsets, perm, tiles, n_tiles, total;
+};
+static size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
+static bool id_workspace_layout(int64_t n_tokens, int64_t top_k, int64_t n_experts, IdWorkspace *l) {
+    int64_t pairs;
+    if (n_tokens <= 0 || top_k <= 0 || n_experts <= 0) return false;
+    if (!mul_ok(n_tokens, top_k, &pairs) || pairs > INT32_MAX) return false;
+    size_t off = 0;
+    l->counts = off;  off += up256(4 * (size_t)n_experts);
+    l->offsets = off; off += up256(4 * (size_t)(n_experts + 1));
+    l->perm = off;    off += up256(4 * (size_t)pairs);
+    l->tiles = off;   off += up256(8 * (size_t)(pairs / 16 + n_experts + 1));
+    l->n_tiles = off; off += 256;
+    l->total = off;
+    return true;
+}
+
+// Threshold of activation rows above which the tensor-core kernel serves
+// bf16 inputs (measured on B200; see the dispatch table in DESIGN).
+constexpr int64_t GEMM_MIN_M = 16;
+
+}  // namespace kq
+
+using namespace kq;
+
+extern "C" {
+
+int kq_block_weights(int type) { return block_weights(type); }
+int kq_block_bytes(int type) { return block_bytes(type); }
+int64_t kq_row_bytes(int type, int64_t k) {
+    const int qk = block_weights(type);
+    if (qk == 0 || k < 0 || k % qk) return -1;
+    return (k / qk) * block_bytes(type);
+}
+
+int kq_dequantize(int type, const void *w, int64_t rows, int64_t k, void *out, int out_dtype,
+                  void *stream) {
+    int64_t rb;
+    int st = check_weights(type, w, rows, k, &rb);
+    if (st) return st;
+    if ((st = check_act(out, out_dtype, rows, k, true))) return st;
+    if ((st = check_device())) return st;
+    return to_status(launch_dequant(type, w, rows, k, out, out_dtype, (cudaStream_t)stream));
+}
+
+int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, int x_dtype,
+                 int64_t m, void *y, int y_dtype, int path, void *stream) {
+    int64_t rb;
+    int st = check_weights(type, w, n, k, &rb);
+    if (st) return st;
+    if (m <= 0) return KQ_ERR_ARG;
+    if ((st = check_act(x, x_dtype, m, k, false))) return st;
+    if ((st = check_act(y, y_dtype, m, n, false))) return st;
+    const bool const_w = (path & KQ_FLAG_CONST_WEIGHTS) != 0;
+    path &= ~KQ_FLAG_CONST_WEIGHTS;
+    if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMM) return KQ_ERR_ARG;
+    if ((st = check_device())) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool can_gemm = gemm_supported(type, n, k, x_dtype, y_dtype);
+    const bool can_gemv = gemv_supported(type, n, k, x_dtype, m);
+    if (path == KQ_PATH_AUTO) {
+        if (can_gemm && m >= GEMM_MIN_M) path = KQ_PATH_GEMM;
+        else if (can_gemv) path = KQ_PATH_GEMV;
+        else path = KQ_PATH_SIMPLE;
+    }
+    switch (path) {
+    case KQ_PATH_GEMM:
+        if (!can_gemm) return KQ_ERR_UNSUPPORTED;
+        return to_status(launch_gemm(type, w, n, k, x, m, y, y_dtype, s));
+    case KQ_PATH_GEMV:
+        if (!can_gemv) return KQ_ERR_UNSUPPORTED;
+        return to_status(launch_gemv(type, w, n, k, x, x_dtype, m, y, y_dtype, const_w, s));
+    default:
+        return to_status(launch_simple_matmul(type, w, n, k, x, x_dtype, m, y, y_dtype, s));
+    }
+}
+
+int kq_matmul(int type, const void *w, int64_t n, int64_t k, const void *x, int x_dtype, int64_t m,
+              void *y, int y_dtype, void *stream) {
+    return kq_matmul_ex(type, w, n, k, x, x_dtype, m, y, y_dtype, KQ_PATH_AUTO, stream);
+}
+
+size_t kq_matmul_id_workspace_bytes(int64_t n_tokens, int64_t top_k, int64_t n_experts) {
+    IdWorkspace l;
+    if (!id_workspace_layout(n_tokens, top_k, n_experts, &l)) return 0;
+    return l.total;
+}
+
+int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
+                    int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
+                    const int32_t *ids, int64_t top_k, void *y, int y_dtype, void *workspace,
+                    size_t workspace_bytes, int path, void *stream) {
+    int64_t rb;
+    int st = check_weights(type, w, n, k, &rb);
+    if (st) return st;
+    if (n_experts <= 0 || n_experts > 65535 || n_tokens <= 0) return KQ_ERR_ARG;
+    if (top_k <= 0 || top_k > n_experts) return KQ_ERR_ARG;
+    int64_t per_expert, last, pairs, ypairs;
+    if (!mul_ok(n, rb, &per_expert)) return KQ_ERR_OVERFLOW;
+    if (expert_stride < per_expert || (expert_stride & 15)) return KQ_ERR_SHAPE;
+    if (!mul_ok(n_experts - 1, expert_stride, &last) ||
+        __builtin_add_overflow(last, per_expert, &last))
+        return KQ_ERR_OVERFLOW;
+    if (!mul_ok(n_tokens, top_k, &pairs) || pairs > INT32_MAX) return KQ_ERR_OVERFLOW;
+    if (!mul_ok(pairs, n, &ypairs)) return KQ_ERR_OVERFLOW;
+    if ((st = check_act(x, x_dtype, n_tokens, k, false))) return st;
+    if ((st = check_act(y, y_dtype, pairs, n, false))) return st;
+    if (ids == nullptr) return KQ_ERR_ARG;
+    if (!aligned16(ids)) return KQ_ERR_ALIGN;
+    IdWorkspace l;
+    if (!id_workspace_layout(n_tokens, top_k, n_experts, &l)) return KQ_ERR_OVERFLOW;
+    if (workspace == nullptr || workspace_bytes < l.total) return KQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KQ_ERR_ALIGN;
+    if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMM) return KQ_ERR_ARG;
+    if ((st = check_device())) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    char *ws = static_cast<char *>(workspace);
+    IdArgs a;
+    a.type = type; a.w = w; a.n_experts = n_experts; a.n = n; a.k = k;
+    a.expert_stride = expert_stride; a.x = x; a.x_dtype = x_dtype; a.n_tokens = n_tokens;
+    a.top_k = top_k; a.y = y; a.y_dtype = y_dtype;
+    a.counts = reinterpret_cast<int32_t *>(ws + l.counts);
+    a.offsets = reinterpret_cast<int32_t *>(ws + l.offsets);
+    a.perm = reinterpret_cast<int32_t *>(ws + l.perm);
+    a.tiles = reinterpret_cast<int32_t *>(ws + l.tiles);
+    a.n_tiles = reinterpret_cast<int32_t *>(ws + l.n_tiles);
+    const bool can_gemv = gemv_id_supported(type, k, x_dtype);
+    if (path == KQ_PATH_AUTO) path = can_gemv ? KQ_PATH_GEMV : KQ_PATH_SIMPLE;
+    if (path == KQ_PATH_GEMM) return KQ_ERR_UNSUPPORTED;
+    if (path == KQ_PATH_GEMV && !can_gemv) return KQ_ERR_UNSUPPORTED;
+    cudaError_t e = launch_moe_group(ids, pairs, n_experts, const_cast<int32_t *>(a.counts),
+                                     const_cast<int32_t *>(a.offsets),
+                                     const_cast<int32_t *>(a.perm), y, y_dtype, n, s);
+    if (e != cudaSuccess) return KQ_ERR_CUDA;
+    if (path == KQ_PATH_GEMV) return to_status(launch_gemv_id(a, s));
+    return to_status(launch_simple_id(a, s));
+}
+
+int kq_matmul_id(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
+                 int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
+                 const int32_t *ids, int64_t top_k, void *y, int y_dtype, void *workspace,
+                 size_t workspace_bytes, void *stream) {
+    return kq_matmul_id_ex(type, w, n_experts, n, k, expert_stride, x, x_dtype, n_tokens, ids,
+                           top_k, y, y_dtype, workspace, workspace_bytes, KQ_PATH_AUTO, stream);
+}
+
+int kq_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_experts, int32_t *counts,
+                 int32_t *offsets, int32_t *perm, void *stream) {
+    if (!ids || !counts || !offsets || !perm) return KQ_ERR_ARG;
+    if (n_pairs <= 0 || n_pairs > INT32_MAX || n_experts <= 0 || n_experts > 65535)
+        return KQ_ERR_ARG;
+    int st = check_device();
+    if (st) return st;
+    return to_status(launch_moe_group(ids, n_pairs, n_experts, counts, offsets, perm, nullptr,
+                                      KQ_F32, 0, (cudaStream_t)stream));
+}
+
+int kq_validate(int type, const void *w, int64_t rows, int64_t k, int64_t *first_bad_block,
+                void *stream) {
+    int64_t rb;
+    int st = check_weights(type, w, rows, k, &rb);
+    if (st) return st;
+    if (first_bad_block == nullptr) return KQ_ERR_ARG;
+    *first_bad_block = -1;
+    if (type != KQ_TQ1_G128) return KQ_OK;
+    if ((st = check_device())) return st;
+    static std::mutex mu;  // the scan result lives in one device word
+    std::lock_guard<std::mutex> g(mu);
+    cudaStream_t s = (cudaStream_t)stream;
+    const unsigned long long none = ~0ull;
+    unsigned long long got = none;
+    if (cudaMemcpyToSymbolAsync(g_scan_first_bad, &none, sizeof(none), 0,
+                                cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return KQ_ERR_CUDA;
+    unsigned long long *dev_word = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&dev_word), g_scan_first_bad) != cudaSuccess)
+        return KQ_ERR_CUDA;
+    if (launch_tq1_scan(w, rows * (k / 128), dev_word, s) != cudaSuccess) return KQ_ERR_CUDA;
+    if (cudaMemcpyFromSymbolAsync(&got, g_scan_first_bad, sizeof(got), 0, cudaMemcpyDeviceToHost,
+                                  s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return KQ_ERR_CUDA;
+    *first_bad_block = (got == none) ? -1 : (int64_t)got;
+    return KQ_OK;
+}
+
+int kq_device_status(void *stream) {
+    int st = check_device();
+    if (st) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned int word = 0, zero = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KQ_ERR_CUDA;
+    if (cudaMemcpyFromSymbolAsync(&word, g_error_word, sizeof(word), 0, cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaMemcpyToSymbolAsync(g_error_word, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return KQ_ERR_CUDA;
+    if (word & ERR_TIMEOUT) return KQ_ERR_DEVICE_TIMEOUT;
+    if (word & ERR_BAD_ID) return KQ_ERR_DEVICE;
+    return KQ_OK;
+}
+
+const char *kq_status_string(int status) {
+    switch (status) {
+    case KQ_OK: return "ok";
+    case KQ_ERR_ARG: return "invalid argument (null pointer, non-positive dimension or top_k)";
+    case KQ_ERR_TYPE: return "unknown codec";
+    case KQ_ERR_SHAPE: return "K is not a multiple of the block size, or bad stride";
+    case KQ_ERR_DTYPE: return "unsupported dtype";
+    case KQ_ERR_ALIGN: return "pointer is not 16-byte aligned";
+    case KQ_ERR_OVERFLOW: return "size overflow";
+    case KQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case KQ_ERR_CUDA: return "CUDA runtime error";
+    case KQ_ERR_DEVICE: return "device reported an out-of-range expert id";
+    case KQ_ERR_DEVICE_TIMEOUT: return "a bounded device wait timed out";
+    case KQ_ERR_UNSUPPORTED: return "unsupported device or path for these arguments";
+    default: return "unknown status";
+    }
+}
+
+}  // extern "C"

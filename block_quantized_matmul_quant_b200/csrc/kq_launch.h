@@ -1,0 +1,49 @@
+// kq_launch.h -- internal launcher declarations (host side).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kq {
+
+struct IdArgs {
+    int type;
+    const void *w;
+    int64_t n_experts, n, k, expert_stride;
+    const void *x;
+    int x_dtype;
+    int64_t n_tokens, top_k;
+    void *y;
+    int y_dtype;
+    const int32_t *counts, *offsets, *perm;  // grouping (device)
+    const int32_t *tiles;                    // tensor-core tile list (device)
+    const int32_t *n_tiles;                  // its length (device)
+};
+
+cudaError_t launch_dequant(int type, const void *w, int64_t rows, int64_t k, void *out, int dt,
+                           cudaStream_t s);
+cudaError_t launch_simple_matmul(int type, const void *w, int64_t n, int64_t k, const void *x,
+                                 int xdt, int64_t m, void *y, int ydt, cudaStream_t s);
+cudaError_t launch_tq1_scan(const void *w, int64_t blocks, unsigned long long *first_bad,
+                            cudaStream_t s);
+cudaError_t launch_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_experts,
+                             int32_t *counts, int32_t *offsets, int32_t *perm, void *y,
+                             int y_dtype, int64_t n, cudaStream_t s);
+cudaError_t launch_simple_id(const IdArgs &a, cudaStream_t s);
+
+// Bandwidth kernels (kq_gemv.cu).  Return cudaErrorNotSupported when the
+// shape is outside what the kernel serves.
+bool gemv_supported(int type, int64_t n, int64_t k, int x_dtype, int64_t m);
+// const_w: weights are not written by earlier work on the stream, so the
+// kernel may prefetch them before the preceding kernel completes (PDL).
+cudaError_t launch_gemv(int type, const void *w, int64_t n, int64_t k, const void *x, int xdt,
+                        int64_t m, void *y, int ydt, bool const_w, cudaStream_t s);
+bool gemv_id_supported(int type, int64_t k, int x_dtype);
+cudaError_t launch_gemv_id(const IdArgs &a, cudaStream_t s);
+
+// Tensor-core kernels (kq_gemm_sm100.cu).
+bool gemm_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype);
+cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const void *x, int64_t m,
+                        void *y, int ydt, cudaStream_t s);
+
+}  // namespace kq

@@ -1,0 +1,189 @@
+// kq_moe.cu -- expert grouping and the plain expert-indexed product.
+//
+// Grouping (mlx-kquant `expert_tile_map`, mlx-native map0 schedule): the
+// (token, slot) pairs are grouped by expert id on the device -- per-expert
+// counts, their exclusive prefix sum, and the pair indices of each expert in
+// ascending order (a stable sort).  No host synchronisation: ids may come
+// from earlier GPU work.  Invalid ids (outside [0, E)) write a NaN output
+// row and set the sticky device error word (mlx-native
+// `quantized_matmul_id_ggml`: invalid routing metadata reads no expert
+// weights and writes a non-finite poison sentinel).
+#include "kq_decode.cuh"
+#include "kq_launch.h"
+
+namespace kq {
+
+constexpr int GROUP_THREADS = 1024;
+
+// One CTA.  Warp w owns experts w, w + 32, ...; it scans the ids in order,
+// so each expert's pair list comes out ascending.
+__global__ void __launch_bounds__(GROUP_THREADS) moe_group_kernel(
+    const int32_t *__restrict__ ids, int n_pairs, int n_experts, int32_t *__restrict__ counts,
+    int32_t *__restrict__ offsets, int32_t *__restrict__ perm, void *y, int y_dtype, int64_t n,
+    unsigned int *err) {
+    extern __shared__ int s_off[];  // n_experts + 1
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    __shared__ int s_bad;
+    if (threadIdx.x == 0) s_bad = 0;
+    __syncthreads();
+    // validation (+ poison rows)
+    for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
+        const int e = ids[p];
+        if (e < 0 || e >= n_experts) {
+            s_bad = 1;
+            if (y != nullptr) {
+                if (y_dtype == KQ_F32) {
+                    float *yr = static_cast<float *>(y) + (int64_t)p * n;
+                    for (int64_t j = 0; j < n; ++j) yr[j] = __int_as_float(0x7fc00000);
+                } else {
+                    __nv_bfloat16 *yr = static_cast<__nv_bfloat16 *>(y) + (int64_t)p * n;
+                    for (int64_t j = 0; j < n; ++j) yr[j] = __ushort_as_bfloat16((unsigned short)0x7fc0);
+                }
+            }
+        }
+    }
+    // pass 1: counts
+    for (int e = warp; e < n_experts; e += nwarps) {
+        int cnt = 0;
+        for (int base = 0; base < n_pairs; base += 32) {
+            const int p = base + lane;
+            const bool hit = p < n_pairs && ids[p] == e;
+            cnt += __popc(__ballot_sync(0xffffffffu, hit));
+        }
+        if (lane == 0) s_off[e] = cnt;
+    }
+    __syncthreads();
+    // exclusive scan by warp 0, 32 experts at a time
+    if (warp == 0) {
+        int carry = 0;
+        for (int base = 0; base < n_experts; base += 32) {
+            const int e = base + lane;
+            const int c = e < n_experts ? s_off[e] : 0;
+            int incl = c;
+            #pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            if (e < n_experts) {
+                counts[e] = c;
+                s_off[e] = carry + incl - c;
+            }
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) s_off[n_experts] = carry;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e <= n_experts; e += blockDim.x) offsets[e] = s_off[e];
+    // pass 2: stable scatter
+    const unsigned lt = (1u << lane) - 1u;
+    for (int e = warp; e < n_experts; e += nwarps) {
+        int pos = s_off[e];
+        for (int base = 0; base < n_pairs; base += 32) {
+            const int p = base + lane;
+            const bool hit = p < n_pairs && ids[p] == e;
+            const unsigned mask = __ballot_sync(0xffffffffu, hit);
+            if (hit) perm[pos + __popc(mask & lt)] = p;
+            pos += __popc(mask);
+        }
+    }
+    for (int p = s_off[n_experts] + threadIdx.x; p < n_pairs; p += blockDim.x) perm[p] = -1;
+    if (threadIdx.x == 0 && s_bad) atomicOr(err, ERR_BAD_ID);
+}
+
+cudaError_t launch_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_experts,
+                             int32_t *counts, int32_t *offsets, int32_t *perm, void *y,
+                             int y_dtype, int64_t n, cudaStream_t s) {
+    const size_t smem = sizeof(int) * (size_t)(n_experts + 1);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(moe_group_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    moe_group_kernel<<<1, GROUP_THREADS, smem, s>>>(ids, (int)n_pairs, (int)n_experts, counts,
+                                                     offsets, perm, y, y_dtype, n, error_word());
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- plain grouped product
+// Grid (ceil(n / 8), n_experts): warp = one weight row of expert e; it walks
+// the pairs routed to e four at a time.
+template <int TYPE, typename XT, typename YT>
+__global__ void __launch_bounds__(256) simple_id_kernel(
+    const uint8_t *__restrict__ w, int64_t n, int64_t k, int64_t expert_stride,
+    const XT *__restrict__ x, int top_k, const int32_t *__restrict__ counts,
+    const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm, YT *__restrict__ y) {
+    using G = Geom<TYPE>;
+    using U = Unit<TYPE>;
+    constexpr int TB = 4;
+    const int e = blockIdx.y;
+    const int cnt = counts[e];
+    if (cnt == 0) return;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = blockIdx.x * 8LL + (threadIdx.x >> 5);
+    if (row >= n) return;
+    const int64_t nb = k / G::QK;
+    const uint8_t *wr = w + e * expert_stride + row * nb * G::BB;
+    const int32_t *plist = perm + offsets[e];
+    const int64_t units = nb * U::PER_BLOCK;
+    for (int c0 = 0; c0 < cnt; c0 += TB) {
+        int pr[TB];
+        #pragma unroll
+        for (int t = 0; t < TB; ++t) pr[t] = (c0 + t < cnt) ? plist[c0 + t] : -1;
+        float acc[TB] = {0.f, 0.f, 0.f, 0.f};
+        for (int64_t i = lane; i < units; i += 32) {
+            const int64_t bi = i / U::PER_BLOCK;
+            const int u = (int)(i % U::PER_BLOCK);
+            float wv[8];
+            U::decode(wr + bi * G::BB, u, wv);
+            const int64_t col = bi * G::QK + 8 * u;
+            #pragma unroll
+            for (int t = 0; t < TB; ++t) {
+                if (pr[t] >= 0) {
+                    float xv[8];
+                    load_x8(x + (int64_t)(pr[t] / top_k) * k + col, xv);
+                    #pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[t] = fmaf(wv[j], xv[j], acc[t]);
+                }
+            }
+        }
+        #pragma unroll
+        for (int t = 0; t < TB; ++t) {
+            float v = acc[t];
+            #pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0 && pr[t] >= 0) store_out(y + (int64_t)pr[t] * n + row, v);
+        }
+    }
+}
+
+template <int TYPE, typename XT, typename YT>
+static cudaError_t simple_id_t(const IdArgs &a, cudaStream_t s) {
+    dim3 grid((unsigned)((a.n + 7) / 8), (unsigned)a.n_experts);
+    simple_id_kernel<TYPE, XT, YT><<<grid, 256, 0, s>>>(
+        static_cast<const uint8_t *>(a.w), a.n, a.k, a.expert_stride,
+        static_cast<const XT *>(a.x), (int)a.top_k, a.counts, a.offsets, a.perm,
+        static_cast<YT *>(a.y));
+    return cudaGetLastError();
+}
+
+template <int TYPE>
+static cudaError_t simple_id_xy(const IdArgs &a, cudaStream_t s) {
+    if (a.x_dtype == KQ_F32) {
+        if (a.y_dtype == KQ_F32) return simple_id_t<TYPE, float, float>(a, s);
+        return simple_id_t<TYPE, float, __nv_bfloat16>(a, s);
+    }
+    if (a.y_dtype == KQ_F32) return simple_id_t<TYPE, __nv_bfloat16, float>(a, s);
+    return simple_id_t<TYPE, __nv_bfloat16, __nv_bfloat16>(a, s);
+}
+
+cudaError_t launch_simple_id(const IdArgs &a, cudaStream_t s) {
+    switch (a.type) {
+    case KQ_Q8_0: return simple_id_xy<KQ_Q8_0>(a, s);
+    case KQ_Q4_K: return simple_id_xy<KQ_Q4_K>(a, s);
+    case KQ_Q2_K: return simple_id_xy<KQ_Q2_K>(a, s);
+    default: return simple_id_xy<KQ_TQ1_G128>(a, s);
+    }
+}
+
+}  // namespace kq

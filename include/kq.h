@@ -1,0 +1,202 @@
+/*
+ * kq.h -- C ABI of libkq: matrix products against block-quantized
+ *         (GGUF-style) weights on NVIDIA B200 (sm_100a).
+ *
+ * The library decodes the weight blocks on the fly inside its CUDA kernels.
+ * Codecs: Q8_0, Q4_K, Q2_K (GGML block formats) and TQ1_G128 (28-byte,
+ * 128-weight ternary blocks).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  * Pointers named `w`, `x`, `y`, `out`, `ids`, `workspace` are DEVICE
+ *    pointers (memory of the current CUDA device, allocated by the caller).
+ *    Pointers named `first_bad_block` are HOST pointers.  The caller owns all
+ *    memory; no call allocates device memory.
+ *  * `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *    enqueue work on it and return without synchronizing, except where a
+ *    call says it synchronizes.
+ *  * Weights are row-major: row n of a [N, K] weight is (K / QK) consecutive
+ *    wire blocks, kq_row_bytes(type, K) bytes, rows packed back to back
+ *    (the mlx-kquant `quantized_matmul` layout, w laid out [N, K] with the
+ *    byte-packed last dimension).  Activations x are row-major [M, K],
+ *    outputs y row-major [M, N]; all contiguous.
+ *  * Alignment: w, x, y, out, ids and workspace must be 16-byte aligned.
+ *  * Return value: KQ_OK (0) or a negative KQ_ERR_* code.  Every argument is
+ *    validated on the host before anything is enqueued, so an error return
+ *    means no work was launched (no partial output).
+ *  * Floating-point dtypes: KQ_F32, KQ_BF16 (and KQ_F16 for kq_dequantize's
+ *    output).  Accumulation is always fp32.
+ */
+#ifndef KQ_H
+#define KQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KQ_API __attribute__((visibility("default")))
+#else
+#define KQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- codecs (GGML type numbers where GGML has one) ---- */
+#define KQ_Q8_0     8     /* 34 B / 32 w:  fp16 d, int8 q[32]; w = d*q            */
+#define KQ_Q2_K     10    /* 84 B / 256 w: scales[16], qs[64], fp16 d, fp16 dmin   */
+#define KQ_Q4_K     12    /* 144 B / 256 w: fp16 d, fp16 dmin, scales[12], qs[128] */
+#define KQ_TQ1_G128 1001  /* 28 B / 128 w: 25 full trit bytes, tail byte, fp16 scale */
+
+/* ---- dtypes ---- */
+#define KQ_F32  0
+#define KQ_BF16 1
+#define KQ_F16  2
+
+/* ---- status codes ---- */
+#define KQ_OK                   0
+#define KQ_ERR_ARG             -1   /* null pointer, zero/negative dim, top_k not in 1..E */
+#define KQ_ERR_TYPE            -2   /* unknown codec                                  */
+#define KQ_ERR_SHAPE           -3   /* K not a multiple of the block size, bad stride  */
+#define KQ_ERR_DTYPE           -4   /* unsupported dtype for this argument             */
+#define KQ_ERR_ALIGN           -5   /* pointer not 16-byte aligned                     */
+#define KQ_ERR_OVERFLOW        -6   /* a byte or element count overflows int64 / int32 */
+#define KQ_ERR_WORKSPACE       -7   /* workspace null or smaller than required         */
+#define KQ_ERR_CUDA            -8   /* a CUDA runtime call failed                      */
+#define KQ_ERR_DEVICE          -9   /* device-side error word was set (bad expert id)  */
+#define KQ_ERR_DEVICE_TIMEOUT  -10  /* a bounded device-side wait gave up              */
+#define KQ_ERR_UNSUPPORTED     -11  /* current device is not sm_100 / path unavailable */
+
+/* ---- matmul paths (kq_matmul_ex / kq_matmul_id_ex) ---- */
+#define KQ_PATH_AUTO     0  /* dispatch by shape (the default of kq_matmul)          */
+#define KQ_PATH_SIMPLE   1  /* plain CUDA-core kernel, any codec/shape               */
+#define KQ_PATH_GEMV     2  /* bandwidth kernel: weights decoded in registers         */
+#define KQ_PATH_GEMM     3  /* TMA + tcgen05 tensor-core kernel (bf16 x only)         */
+/* Flag OR-ed into `path`: the caller guarantees that no work enqueued earlier
+ * on the stream writes the weight bytes (they are constant, as model weights
+ * are).  The kernel may then start streaming weights before the preceding
+ * kernel has finished (programmatic dependent launch); x is still read only
+ * after the preceding work completes. */
+#define KQ_FLAG_CONST_WEIGHTS 0x100
+
+/* Weights per block and bytes per block of a codec; 0 for an unknown codec. */
+KQ_API int kq_block_weights(int type);
+KQ_API int kq_block_bytes(int type);
+/* Bytes of one weight row of length k; -1 if k is not a multiple of the
+ * block size or the codec is unknown. */
+KQ_API int64_t kq_row_bytes(int type, int64_t k);
+
+/*
+ * kq_dequantize -- decode weights to floats.
+ * Defines: mlx-kquant bindings.cpp `dequantize(w, scales, kquant_type, dtype)`
+ * (wire bytes -> float array; the K-quant scales live inside w).
+ *   w       [rows, kq_row_bytes(type, k)] u8 wire blocks (device)
+ *   out     [rows, k] of out_dtype (KQ_F32, KQ_BF16 or KQ_F16) (device)
+ * The fp32 result is bit-exact: each weight is the codec definition's IEEE
+ * fp32 operation sequence (products exact, one rounding at the final
+ * subtraction).  bf16/f16 outputs are that fp32 value rounded to nearest even.
+ * TQ1_G128 bytes above the legal maximum (242 full, 26 tail) decode to zero.
+ */
+KQ_API int kq_dequantize(int type, const void *w, int64_t rows, int64_t k,
+                  void *out, int out_dtype, void *stream);
+
+/*
+ * kq_matmul -- y = x @ dequant(w)^T.
+ * Defines: mlx-kquant bindings.cpp `quantized_matmul(x, w, scales,
+ * kquant_type, transpose=True)`: `x @ dequant(w)` with w laid out [N, K].
+ *   w  [n, kq_row_bytes(type, k)] u8 (device)
+ *   x  [m, k] of x_dtype (KQ_F32 or KQ_BF16) (device)
+ *   y  [m, n] of y_dtype (KQ_F32 or KQ_BF16) (device), fully overwritten
+ *   y[i][j] = sum_k dequant(w)[j][k] * x[i][k], fp32 accumulation.
+ * Small m runs the bandwidth-bound kernel that decodes weights in
+ * registers; large m with bf16 x runs the tensor-core kernel, which rounds
+ * decoded weights to bf16 before the bf16 x bf16 -> fp32 MMA.
+ */
+KQ_API int kq_matmul(int type, const void *w, int64_t n, int64_t k,
+              const void *x, int x_dtype, int64_t m,
+              void *y, int y_dtype, void *stream);
+
+/* kq_matmul with an explicit path (KQ_PATH_*); KQ_ERR_UNSUPPORTED if the
+ * path cannot serve these arguments (e.g. KQ_PATH_GEMM with fp32 x). */
+KQ_API int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k,
+                 const void *x, int x_dtype, int64_t m,
+                 void *y, int y_dtype, int path, void *stream);
+
+/*
+ * kq_matmul_id -- expert-indexed (mixture-of-experts) product.
+ * Defines: mlx-native 0.21.0 quantized_matmul_id_ggml.rs (module doc and
+ * `quantized_matmul_id_ggml`): for every token t and slot s,
+ *   e = ids[t][s];  y[t][s][j] = sum_k dequant(w_e)[j][k] * x[t][k].
+ * Same operation as mlx-kquant `gather_qmm` with rhs_indices = ids.
+ *   w    expert stack; expert e's [n, kq_row_bytes(type, k)] rows start at
+ *        w + e * expert_stride bytes (expert_stride >= n * row bytes,
+ *        a multiple of 16) (device)
+ *   x    [n_tokens, k] of x_dtype (KQ_F32 or KQ_BF16) (device)
+ *   ids  [n_tokens, top_k] int32 (device; may be produced by earlier work
+ *        on the same stream -- the host never reads it)
+ *   y    [n_tokens, top_k, n] of y_dtype (KQ_F32 or KQ_BF16) (device)
+ *   workspace  device scratch of at least
+ *        kq_matmul_id_workspace_bytes(n_tokens, top_k, n_experts) bytes,
+ *        owned by the caller; its contents are overwritten.  Calls that
+ *        share one workspace must be ordered on the GPU (one stream).
+ * Duplicate ids within a token are legal.  An id outside [0, n_experts)
+ * reads no weights, writes NaN to its whole output row and sets the
+ * device error word (see kq_device_status); the other rows are exact.
+ * Tokens routed to one expert are grouped before the decode, so each hit
+ * expert's weights are streamed once per group of tokens; the result of a
+ * (t, s) row does not depend on the other tokens' ids.
+ */
+KQ_API size_t kq_matmul_id_workspace_bytes(int64_t n_tokens, int64_t top_k, int64_t n_experts);
+KQ_API int kq_matmul_id(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
+                 int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
+                 const int32_t *ids, int64_t top_k, void *y, int y_dtype,
+                 void *workspace, size_t workspace_bytes, void *stream);
+/* kq_matmul_id with an explicit path: KQ_PATH_SIMPLE, KQ_PATH_GEMV (grouped
+ * mat-vec) or KQ_PATH_GEMM (grouped tensor-core GEMM, bf16 x only). */
+KQ_API int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
+                    int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
+                    const int32_t *ids, int64_t top_k, void *y, int y_dtype,
+                    void *workspace, size_t workspace_bytes, int path, void *stream);
+
+/*
+ * kq_moe_group -- the grouping step of kq_matmul_id, exposed for testing.
+ * Defines: mlx-kquant bindings.cpp `expert_tile_map` and mlx-native's map0
+ * schedule (per-expert routed counts and routed-token lists, built on the
+ * device without a host sync).
+ *   ids      [n_tokens * top_k] int32 (device)
+ *   counts   [n_experts] int32 out: pairs routed to each expert (device)
+ *   offsets  [n_experts + 1] int32 out: exclusive prefix sum of counts (device)
+ *   perm     [n_tokens * top_k] int32 out: pair indices p = t*top_k + s
+ *            grouped by expert, ascending p inside each expert (a stable
+ *            sort by expert id); pairs with an invalid id are left out and
+ *            the tail perm[offsets[n_experts] ..] is set to -1 (device)
+ * Sets the device error word if any id is outside [0, n_experts).
+ */
+KQ_API int kq_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_experts,
+                 int32_t *counts, int32_t *offsets, int32_t *perm, void *stream);
+
+/*
+ * kq_validate -- scan TQ1_G128 weights for bytes above the legal maximum
+ * (ternel_packed_model.py: MAX_FULL_CODE_BYTE = 242, MAX_TAIL_CODE_BYTE = 26).
+ * SYNCHRONIZES `stream`.  *first_bad_block (host) receives the row-major index
+ * of the first block holding an illegal byte, or -1.  Other codecs have no
+ * illegal byte patterns and report -1.
+ */
+KQ_API int kq_validate(int type, const void *w, int64_t rows, int64_t k,
+                int64_t *first_bad_block, void *stream);
+
+/*
+ * kq_device_status -- SYNCHRONIZES `stream`, then returns and clears the
+ * current device's sticky error word: KQ_OK, KQ_ERR_DEVICE (an expert id was
+ * out of range in some call since the last check) or KQ_ERR_DEVICE_TIMEOUT.
+ */
+KQ_API int kq_device_status(void *stream);
+
+/* Static description of a status code. */
+KQ_API const char *kq_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KQ_H */

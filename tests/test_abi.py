@@ -1,0 +1,83 @@
+"""The C-ABI library loads and exports every symbol include/kq.h declares.
+Runs without a GPU: only calls that do not touch a device are made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    import block_quantized_matmul_quant_b200 as kq
+
+    kq.ensure_built()
+    return kq.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "kq.h")).read()
+    return re.findall(r"KQ_API\s+[\w\s\*]+?\b(kq_\w+)\s*\(", src)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for required in ("kq_dequantize", "kq_matmul", "kq_matmul_id", "kq_device_status",
+                     "kq_validate", "kq_row_bytes", "kq_matmul_id_workspace_bytes"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_block_geometry_and_row_bytes(L):
+    assert (L.kq_block_weights(8), L.kq_block_bytes(8)) == (32, 34)
+    assert (L.kq_block_weights(12), L.kq_block_bytes(12)) == (256, 144)
+    assert (L.kq_block_weights(10), L.kq_block_bytes(10)) == (256, 84)
+    assert (L.kq_block_weights(1001), L.kq_block_bytes(1001)) == (128, 28)
+    assert L.kq_block_weights(3) == 0
+    assert L.kq_row_bytes(12, 4096) == 2304
+    assert L.kq_row_bytes(1001, 17408) == 3808
+    assert L.kq_row_bytes(8, 1024) == 1088
+    assert L.kq_row_bytes(12, 100) == -1
+
+
+def test_status_strings(L):
+    for st in range(0, -12, -1):
+        assert L.kq_status_string(st)
+    assert b"unknown" in L.kq_status_string(-99)
+
+
+def test_workspace_size(L):
+    b = L.kq_matmul_id_workspace_bytes(32, 6, 64)
+    assert b >= 4 * (64 + 65 + 192) and b % 256 == 0
+    assert L.kq_matmul_id_workspace_bytes(0, 6, 64) == 0
+
+
+def test_argument_errors_before_any_launch(L):
+    # All of these fail host validation, before the device is queried.
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)   # never dereferenced
+    assert L.kq_matmul(12, None, 4, 256, fake, 1, 1, fake, 0, None) == -1          # null w
+    assert L.kq_matmul(12, fake, 4, 100, fake, 1, 1, fake, 0, None) == -3          # K % 256
+    assert L.kq_matmul(77, fake, 4, 256, fake, 1, 1, fake, 0, None) == -2          # codec
+    assert L.kq_matmul(12, vp((1 << 20) + 8), 4, 256, fake, 1, 1, fake, 0, None) == -5  # align
+    assert L.kq_matmul(12, fake, 4, 256, fake, 7, 1, fake, 0, None) == -4          # dtype
+    assert L.kq_matmul(12, fake, 0, 256, fake, 1, 1, fake, 0, None) == -1          # n = 0
+    assert L.kq_dequantize(1001, fake, 2, 130, fake, 0, None) == -3
+    ws = L.kq_matmul_id_workspace_bytes(4, 2, 3)
+    # top_k > n_experts
+    assert L.kq_matmul_id(12, fake, 3, 8, 256, 8 * 144, fake, 1, 4, fake, 4, fake, 0, fake, ws,
+                          None) == -1
+    # expert stride smaller than one expert
+    assert L.kq_matmul_id(12, fake, 3, 8, 256, 144, fake, 1, 4, fake, 2, fake, 0, fake, ws,
+                          None) == -3
+    # workspace too small
+    assert L.kq_matmul_id(12, fake, 3, 8, 256, 8 * 144, fake, 1, 4, fake, 2, fake, 0, fake, 16,
+                          None) == -7
+    # overflow of n * row bytes
+    assert L.kq_matmul(12, fake, 1 << 60, 256, fake, 1, 1, fake, 0, None) == -6

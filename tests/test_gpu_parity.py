@@ -1,0 +1,265 @@
+"""Parity of the CUDA path with the CPU oracle (needs a B200).
+
+Small cases span several CTAs / tiles and a ragged tail; the five measured
+workloads run at full size in the launch configuration the benchmark times,
+compared on all outputs (or on sampled weight rows where the oracle would
+take long).  Decode is compared bit for bit; products by the normwise row
+error of tests/kqtest.py.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from kqtest import BF16_OUT, FP32_PATH_TOL, GEMV_TOL, TOL, row_rel_err, to_device_w, to_device_x
+
+pytestmark = pytest.mark.gpu
+
+CODECS = [synth.Q8_0, synth.Q2_K, synth.Q4_K, synth.TQ1_G128]
+
+
+def rng(seed):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+# ---------------------------------------------------------------- dequantize
+
+@pytest.mark.parametrize("codec", CODECS)
+@pytest.mark.parametrize("rows,nblocks", [(1, 1), (37, 3), (300, 8)])
+def test_dequantize_bit_exact(kq, codec, rows, nblocks):
+    import torch
+
+    k = synth.geometry(codec)[0] * nblocks
+    w = synth.gen_weights(codec, rows, k, rng(rows + codec))
+    ref = oracle.decode_f32(codec, w, k)
+    got = kq.dequantize(to_device_w(w), codec, k).cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    for dt in (torch.bfloat16, torch.float16):
+        g = kq.dequantize(to_device_w(w), codec, k, dtype=dt).cpu()
+        r = torch.from_numpy(ref).to(dt)   # round-to-nearest-even of the fp32 decode
+        assert torch.equal(g.view(torch.int16), r.view(torch.int16))
+
+
+def test_dequantize_illegal_tq1_bytes_and_validate(kq):
+    w = synth.gen_weights(synth.TQ1_G128, 5, 384, rng(1))
+    w[3, 28 + 7] = 250        # full byte of block 1, row 3
+    w[4, 2 * 28 + 25] = 200   # tail byte of block 2, row 4
+    ref = oracle.decode_f32(synth.TQ1_G128, w, 384)
+    got = kq.dequantize(to_device_w(w), synth.TQ1_G128, 384).cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    assert np.all(got[3, 128 + 35:128 + 40] == 0)
+    assert kq.validate(to_device_w(w), synth.TQ1_G128, 384) == oracle.tq1_first_illegal(w, 384) == 3 * 3 + 1
+    ok = synth.gen_weights(synth.TQ1_G128, 5, 384, rng(2))
+    assert kq.validate(to_device_w(ok), synth.TQ1_G128, 384) == -1
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_dequantize_full_workload_weights(kq, name):
+    wl = synth.WORKLOADS[name]
+    w, _, _ = synth.make_inputs(wl)
+    w = w.reshape(-1, synth.row_bytes(wl.codec, wl.k))
+    ref = oracle.decode_f32(wl.codec, w, wl.k)
+    got = kq.dequantize(to_device_w(w), wl.codec, wl.k).cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+# ---------------------------------------------------------------- matmul
+
+def _paths(kq):
+    return {"simple": kq.PATH_SIMPLE, "gemv": kq.PATH_GEMV, "gemm": kq.PATH_GEMM}
+
+
+@pytest.mark.parametrize("codec", CODECS)
+@pytest.mark.parametrize("xdt", ["f32", "bf16"])
+@pytest.mark.parametrize("m", [1, 3, 8, 19])
+def test_matmul_simple_path(kq, codec, xdt, m):
+    import torch
+
+    qk = synth.geometry(codec)[0]
+    k = qk * (3 if qk == 256 else 9)
+    n = 261
+    r = rng(100 + m + codec)
+    w = synth.gen_weights(codec, n, k, r)
+    x = synth.gen_x(m, k, xdt, r)
+    ref = oracle.matmul(codec, w, k, x)
+    for ydt in (torch.float32, torch.bfloat16):
+        y = kq.matmul(to_device_w(w), codec, to_device_x(x, xdt), out_dtype=ydt,
+                      path=kq.PATH_SIMPLE).float().cpu().numpy()
+        err = row_rel_err(y, ref)
+        if ydt == torch.float32:
+            assert err <= FP32_PATH_TOL
+        else:
+            assert err <= TOL[xdt] + BF16_OUT
+
+
+GEMV_CASES = [
+    # (n, k, m): several CTAs, ragged row counts, 1..32+ blocks per row
+    (300, 256, 1), (1000, 1024, 1), (4099, 4096, 1), (777, 2048, 2), (513, 4096, 3),
+    (1500, 9216, 1), (640, 8192, 4), (257, 4096, 8), (5, 512, 5), (2000, 11008 // 256 * 256, 1),
+]
+
+
+@pytest.mark.parametrize("n,k,m", GEMV_CASES)
+@pytest.mark.parametrize("xdt", ["f32", "bf16"])
+def test_matmul_gemv_q4_k(kq, n, k, m, xdt):
+    import torch
+
+    r = rng(n + k + m)
+    w = synth.gen_weights(synth.Q4_K, n, k, r)
+    x = synth.gen_x(m, k, xdt, r)
+    ref = oracle.matmul(synth.Q4_K, w, k, x, threads=8)
+    wd, xd = to_device_w(w), to_device_x(x, xdt)
+    for flags in (False, True):
+        y = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV, const_weights=flags).cpu().numpy()
+        err = row_rel_err(y, ref)
+        assert err <= GEMV_TOL, err
+    yb = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV, out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert row_rel_err(yb, ref) <= TOL[xdt] + BF16_OUT
+
+
+def test_matmul_gemv_deterministic(kq):
+    r = rng(7)
+    w = synth.gen_weights(synth.Q4_K, 4096, 4096, r)
+    x = synth.gen_x(1, 4096, "bf16", r)
+    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    a = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV).cpu().numpy()
+    b = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV).cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+def test_matmul_unit_vector_selects_column(kq):
+    # x = e_j  =>  y = column j of the decoded weights (exactly, in fp32).
+    k, n = 1024, 333
+    w = synth.gen_weights(synth.Q4_K, n, k, rng(8))
+    dec = oracle.decode_f32(synth.Q4_K, w, k)
+    x = np.zeros((2, k), np.float32)
+    x[0, 5] = 1.0
+    x[1, 1000] = 1.0
+    for path in (kq.PATH_SIMPLE, kq.PATH_GEMV):
+        y = kq.matmul(to_device_w(w), synth.Q4_K, to_device_x(x, "f32"), path=path).cpu().numpy()
+        # one nonzero activation: both paths are exact up to fp32 rounding
+        np.testing.assert_allclose(y[0], dec[:, 5], rtol=1e-5, atol=1e-6)
+        np.testing.assert_allclose(y[1], dec[:, 1000], rtol=1e-5, atol=1e-6)
+
+
+# ---------------------------------------------------------------- workloads at full size
+
+def _workload_check(kq, name, sample_rows=None):
+    import torch
+
+    wl = synth.WORKLOADS[name]
+    w, x, ids = synth.make_inputs(wl)
+    if wl.kind == "moe":
+        ydt = torch.float32 if wl.y_dtype == "f32" else torch.bfloat16
+        y = kq.matmul_id(to_device_w(w), wl.codec, to_device_x(x, wl.x_dtype),
+                         torch.from_numpy(ids).cuda(), out_dtype=ydt).float().cpu().numpy()
+        ref = oracle.matmul_id(wl.codec, w, wl.k, x, ids)
+        return row_rel_err(y, ref)
+    ydt = torch.float32 if wl.y_dtype == "f32" else torch.bfloat16
+    y = kq.matmul(to_device_w(w), wl.codec, to_device_x(x, wl.x_dtype), out_dtype=ydt,
+                  const_weights=True).float().cpu().numpy()
+    if sample_rows is None:
+        ref = oracle.matmul(wl.codec, w, wl.k, x, threads=8)
+        return row_rel_err(y, ref)
+    rows = np.unique(np.concatenate([sample_rows, [0, wl.n - 1]]))
+    ref = oracle.matmul(wl.codec, w[rows], wl.k, x, threads=8)   # [m, len(rows)]
+    return row_rel_err(y[:, rows], ref)
+
+
+@pytest.mark.parametrize("name", ["q8_0_gemv_256x1024", "q4_k_gemv_4096x4096",
+                                  "tq1_g128_gemv_5120x17408", "moe_q4_k_e64_1408x2048_t32_top6"])
+def test_workload_full_size(kq, name):
+    wl = synth.WORKLOADS[name]
+    err = _workload_check(kq, name)
+    assert err <= TOL[wl.x_dtype], err
+
+
+def test_workload_prefill_gemm_sampled_rows(kq):
+    wl = synth.WORKLOADS["q4_k_gemm_512x11008x4096"]
+    # rows at tile boundaries plus a random sample
+    rows = np.concatenate([np.arange(0, wl.n, 997), [127, 128, 255, 256, 11007 - 128],
+                           rng(3).integers(0, wl.n, 40)])
+    err = _workload_check(kq, wl.name, sample_rows=rows)
+    assert err <= TOL[wl.x_dtype], err
+
+
+# ---------------------------------------------------------------- expert-indexed
+
+def _stable_group(ids, e):
+    flat = ids.reshape(-1)
+    valid = (flat >= 0) & (flat < e)
+    counts = np.bincount(flat[valid], minlength=e)
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    order = np.argsort(np.where(valid, flat, e), kind="stable")[: valid.sum()]
+    return counts, offsets, order
+
+
+@pytest.mark.parametrize("t,top_k,e", [(32, 6, 64), (7, 3, 5), (100, 8, 16), (1, 1, 1), (300, 2, 40)])
+def test_moe_group_exact(kq, t, top_k, e):
+    import torch
+
+    ids = synth.gen_ids(t, top_k, e, rng(t))
+    counts, offsets, perm = kq.moe_group(torch.from_numpy(ids).cuda(), e)
+    c, o, p = _stable_group(ids, e)
+    assert np.array_equal(counts.cpu().numpy(), c)
+    assert np.array_equal(offsets.cpu().numpy(), o)
+    assert np.array_equal(perm.cpu().numpy(), p)
+    assert kq.device_status() == 0
+
+
+@pytest.mark.parametrize("codec", CODECS)
+@pytest.mark.parametrize("path", ["simple", "auto"])
+def test_matmul_id_small(kq, codec, path):
+    import torch
+
+    qk = synth.geometry(codec)[0]
+    k = qk * (2 if qk == 256 else 8)
+    e, n, t, top_k = 5, 70, 7, 3
+    r = rng(codec)
+    w = synth.gen_weights(codec, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, "bf16", r)
+    ids = synth.gen_ids(t, top_k, e, r)
+    ids[2, 1] = ids[2, 0]            # duplicate ids in a token are legal
+    ref = oracle.matmul_id(codec, w, k, x, ids)
+    p = {"simple": kq.PATH_SIMPLE, "auto": kq.PATH_AUTO}[path]
+    y = kq.matmul_id(to_device_w(w), codec, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
+                     path=p).cpu().numpy()
+    assert row_rel_err(y, ref) <= FP32_PATH_TOL
+    assert kq.device_status() == 0
+
+
+def test_matmul_id_bad_ids_poison_rows(kq):
+    import torch
+
+    e, n, k, t = 4, 33, 512, 5
+    r = rng(11)
+    w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, "f32", r)
+    ids = synth.gen_ids(t, 2, e, r)
+    ids[1, 0] = 4
+    ids[3, 1] = -7
+    y = kq.matmul_id(to_device_w(w), synth.Q4_K, to_device_x(x, "f32"), torch.from_numpy(ids).cuda()
+                     ).cpu().numpy()
+    ref = oracle.matmul_id(synth.Q4_K, w, k, x, ids)
+    assert np.all(np.isnan(y[1, 0])) and np.all(np.isnan(y[3, 1]))
+    good = ~np.isnan(ref[..., 0])
+    assert row_rel_err(y[good], ref[good]) <= FP32_PATH_TOL
+    assert kq.device_status() == -9    # KQ_ERR_DEVICE, then cleared
+    assert kq.device_status() == 0
+
+
+# ---------------------------------------------------------------- errors on device arguments
+
+def test_error_codes(kq):
+    import torch
+
+    w = to_device_w(synth.gen_weights(synth.Q4_K, 8, 512, rng(1)))
+    xf = torch.zeros((1, 512), dtype=torch.float32, device="cuda")
+    with pytest.raises(kq.KQError) as ei:
+        kq.matmul(w, synth.Q4_K, xf, path=kq.PATH_GEMM)       # tensor-core path needs bf16 x
+    assert ei.value.status == -11
+    bad_out = torch.empty((1, 9), device="cuda")[:, 1:]        # 4-byte offset
+    with pytest.raises(kq.KQError) as ei:
+        kq.matmul(w, synth.Q4_K, xf, out=bad_out, path=kq.PATH_SIMPLE)
+    assert ei.value.status == -5
+    assert kq.device_status() == 0
