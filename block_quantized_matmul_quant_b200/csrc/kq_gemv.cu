@@ -74,7 +74,7 @@ __device__ __forceinline__ int dp2a_hi(int a, uint32_t b, int c) {
 }
 
 // Byte i (0..3) of w as an exact float.
-__device__ __forceinline__ float byte_f(uint32_t w, int i) {
+[[maybe_unused]] __device__ __forceinline__ float byte_f(uint32_t w, int i) {
     return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | (uint32_t)i)) - 8388608.0f;
 }
 

@@ -1,13 +1,14 @@
 // kq_ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, bulk and
 // tensor (TMA) copies, programmatic dependent launch, packed fp32 math.
-// Every wait on an mbarrier is bounded: after `KQ_SPIN_LIMIT` polls it
-// gives up, sets the device error word and reports failure to the caller.
+// Every wait on an mbarrier is bounded: after `KQ_SPIN_LIMIT` polls (each
+// suspending at most ~1 us, so a few seconds at most) it gives up, sets the
+// device error word and reports failure to the caller.
 #pragma once
 
 #include "kq_common.cuh"
 
 #ifndef KQ_SPIN_LIMIT
-#define KQ_SPIN_LIMIT (1u << 26)
+#define KQ_SPIN_LIMIT (1u << 22)
 #endif
 
 namespace kq {
@@ -55,6 +56,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
     for (uint32_t i = 0; i < KQ_SPIN_LIMIT; ++i)
         if (mbar_try_wait(bar, parity)) return true;
+    atomicOr(err, ERR_TIMEOUT);
+    return false;
+}
+
+// Non-blocking poll of a phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded busy wait for a single latency-critical thread (an MMA or TMA
+// issuer): it resumes the moment the phase completes instead of sleeping.
+// About 2^28 polls (well under a minute) before it gives up like mbar_wait.
+__device__ __forceinline__ bool mbar_spin(uint64_t *bar, uint32_t parity, unsigned int *err) {
+    for (uint32_t i = 0; i < (KQ_SPIN_LIMIT << 6); ++i)
+        if (mbar_test_wait(bar, parity)) return true;
     atomicOr(err, ERR_TIMEOUT);
     return false;
 }

@@ -142,6 +142,51 @@ def test_matmul_unit_vector_selects_column(kq):
         np.testing.assert_allclose(y[1], dec[:, 1000], rtol=1e-5, atol=1e-6)
 
 
+GEMM_CASES = [
+    # (n, k, m): one tile, ragged rows / tokens, several waves of tiles
+    (128, 256, 16), (300, 512, 19), (261, 768, 33), (1000, 1024, 64), (777, 2048, 100),
+    (4096, 4096, 128), (2000, 4096, 300), (2752, 4096, 512), (640, 8192, 1024),
+]
+
+
+def _bf16_weight_reference(w, k, x):
+    """x @ bf16(decode_f32(w))^T in fp64: what the tensor-core path computes up
+    to fp32 accumulation (weights rounded to nearest-even bf16)."""
+    import torch
+
+    dec = oracle.decode_f32(synth.Q4_K, w, k)
+    wb = torch.from_numpy(dec).to(torch.bfloat16).to(torch.float64).numpy()
+    return x.astype(np.float64) @ wb.T
+
+
+@pytest.mark.parametrize("n,k,m", GEMM_CASES)
+def test_matmul_gemm_q4_k(kq, n, k, m):
+    import torch
+
+    r = rng(1000 + n + k + m)
+    w = synth.gen_weights(synth.Q4_K, n, k, r)
+    x = synth.gen_x(m, k, "bf16", r)
+    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    y = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMM).cpu().numpy()
+    ref = oracle.matmul(synth.Q4_K, w, k, x, threads=8)
+    assert row_rel_err(y, ref) <= TOL["bf16"]
+    # tight: equal to the bf16-rounded-weight product up to fp32 accumulation
+    assert row_rel_err(y, _bf16_weight_reference(w, k, x)) <= FP32_PATH_TOL
+    yb = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMM, out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert row_rel_err(yb, ref) <= TOL["bf16"] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+def test_matmul_gemm_deterministic(kq):
+    r = rng(17)
+    w = synth.gen_weights(synth.Q4_K, 1500, 4096, r)
+    x = synth.gen_x(200, 4096, "bf16", r)
+    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    a = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMM).cpu().numpy()
+    b = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMM).cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
 # ---------------------------------------------------------------- workloads at full size
 
 def _workload_check(kq, name, sample_rows=None):
