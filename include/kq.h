@@ -160,6 +160,33 @@ KQ_API int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n
                     void *workspace, size_t workspace_bytes, int path, void *stream);
 
 /*
+ * kq_matmul_id_noalloc -- kq_matmul_id for callers that cannot allocate
+ * device memory.  (The pages have no counterpart of this call.)
+ * Some callers are handed only their input and output buffers and have no
+ * device allocator of their own -- a plugin running inside another
+ * framework's execution plan, or a host language that cannot call
+ * cudaMalloc -- so they cannot provide kq_matmul_id's workspace.  This call
+ * takes the same arguments minus the workspace and computes the same result
+ * with the same kernels, using a scratch array built into the library:
+ *   * The array holds 256 KiB; a request whose
+ *     kq_matmul_id_workspace_bytes(n_tokens, top_k, n_experts) exceeds it is
+ *     rejected with KQ_ERR_WORKSPACE before any work is enqueued.
+ *   * Every GPU that loads the library keeps the array until the process
+ *     exits.  The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   * Every call shares the one array: calls that overlap on the GPU (on
+ *     different streams, or from different host threads) race and give
+ *     wrong results.  Order them on one stream.  The array keeps the last
+ *     call's contents; nothing in it needs to start at zero.
+ *   * Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ */
+KQ_API int kq_matmul_id_noalloc(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
+                                int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
+                                const int32_t *ids, int64_t top_k, void *y, int y_dtype,
+                                void *stream);
+
+/*
  * kq_moe_group -- the grouping step of kq_matmul_id, exposed for testing.
  * Defines: mlx-kquant bindings.cpp `expert_tile_map` and mlx-native's map0
  * schedule (per-expert routed counts and routed-token lists, built on the
