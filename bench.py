@@ -202,6 +202,66 @@ class GemvStep:
         return self.wbytes * self.pool  # weight bytes per step
 
 
+class PoolStep:
+    """A workload's calls over a pool of weight copies larger than 4x L2."""
+
+    def __init__(self, torch, kq, wl, l2_bytes):
+        w, x, ids = synth.make_inputs(wl)
+        self.wl, self.kq = wl, kq
+        self.wbytes = w.nbytes
+        self.pool = max(4, -(-4 * l2_bytes // w.nbytes))
+        base = torch.from_numpy(w).cuda()
+        self.ws = [base.clone() for _ in range(self.pool)]
+        self.x = _x_tensor(torch, x, wl.x_dtype).cuda()
+        self.ids = torch.from_numpy(ids).cuda() if ids is not None else None
+        ydt = torch.float32 if wl.y_dtype == "f32" else torch.bfloat16
+        shape = (wl.m, wl.top_k, wl.n) if wl.kind == "moe" else (wl.m, wl.n)
+        self.y = torch.empty(shape, dtype=ydt, device="cuda")
+        if wl.kind == "moe":
+            self.ws_bytes = kq.matmul_id_workspace_bytes(wl.m, wl.top_k, wl.n_experts)
+            self.scratch = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+            self.hit_experts = len(np.unique(ids))
+
+    def run(self):
+        for i in range(self.pool):
+            if self.wl.kind == "moe":
+                self.kq.matmul_id(self.ws[i], self.wl.codec, self.x, self.ids, out=self.y,
+                                  workspace=self.scratch)
+            else:
+                self.kq.matmul(self.ws[i], self.wl.codec, self.x, out=self.y, const_weights=True)
+
+
+def secondary_metrics(torch, kq, l2, peaks):
+    """The other measured workloads, one short timed graph each."""
+    out = {}
+    for name in ("q4_k_gemm_512x11008x4096", "moe_q4_k_e64_1408x2048_t32_top6",
+                 "tq1_g128_gemv_5120x17408", "q8_0_gemv_256x1024"):
+        wl = synth.WORKLOADS[name]
+        st = PoolStep(torch, kq, wl, l2)
+        ms = time_graph(torch, st.run, 5, 3, None)
+        us = ms * 1e3 / (5 * st.pool)
+        if wl.kind == "gemm":
+            tf = 2.0 * wl.m * wl.n * wl.k / (us * 1e-6) / 1e12
+            out[name] = {"us_per_call": round(us, 2), "TFLOP/s": round(tf, 1),
+                         "frac_burst": round(tf / peaks["bf16_tflops"], 4),
+                         "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+                         "kernel": "gemm_q4k_kernel (tcgen05)"}
+        elif wl.kind == "moe":
+            per_expert = st.wbytes // wl.n_experts
+            moved = st.hit_experts * per_expert + wl.m * wl.k * 2 + wl.m * wl.top_k * wl.n * 4
+            out[name] = {"us_per_call": round(us, 2), "tokens/s": round(wl.m / (us * 1e-6), 1),
+                         "GB/s": round(moved / (us * 1e-6) / 1e9, 1),
+                         "frac_hbm": round(moved / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                         "hit_experts": st.hit_experts, "kernel": "moe_group + grouped product"}
+        else:
+            gbs = st.wbytes / (us * 1e-6) / 1e9
+            out[name] = {"us_per_call": round(us, 3), "weight GB/s": round(gbs, 1),
+                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        del st
+        torch.cuda.empty_cache()
+    return out
+
+
 def time_graph(torch, fn, steps, warmup, pg):
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
@@ -295,6 +355,9 @@ def run_gpu(args):
     ms = max_over_ranks(torch, pg, ms)
     e2e_ms = time_eager(torch, step.run_e2e, max(1, args.steps // 4), 1, pg)
     e2e_ms = max_over_ranks(torch, pg, e2e_ms) / max(1, args.steps // 4)
+    status = kq.device_status()
+    if status != 0:  # a kernel reported a bad input or a wait that gave up: no number
+        raise SystemExit(f"device status {status} during the timed steps")
     per_step_ms = ms / args.steps
     total_bytes = step.step_units() * args.steps * world
     value = total_bytes / (ms / 1e3) / 1e9
@@ -312,7 +375,7 @@ def run_gpu(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "u8 Q4_K weights x bf16 activations, fp32 accumulate",
+        "dtype": "int16 activation codes x u4 quants (dp2a, int32), f32 scale-and-sum",
         "data": "synthetic (seeded Q4_K wire bytes and N(0,1) bf16 activations)",
         "config": {
             "workload": wl.name,
@@ -344,6 +407,11 @@ def run_gpu(args):
         },
         "clocks": clk.summary(),
     }
+    if world == 1 and not args.no_secondary:
+        out["secondary"] = secondary_metrics(torch, kq, l2, peaks)
+        status = kq.device_status()
+        if status != 0:
+            raise SystemExit(f"device status {status} during the secondary workloads")
     if rank == 0 and world == 1:
         out["cpu_baseline"] = cpu_baseline_gemv(wl, budget_s=args.cpu_seconds)
     if rank == 0:
@@ -393,6 +461,34 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_profile(args):
+    """A few eager calls of one workload, for ncu captures (no timing)."""
+    import torch
+
+    import block_quantized_matmul_quant_b200 as kq
+
+    kq.lib()
+    wl = synth.WORKLOADS[args.profile]
+    w, x, ids = synth.make_inputs(wl)
+    wd = torch.from_numpy(w).cuda()
+    xd = _x_tensor(torch, x, wl.x_dtype).cuda()
+    ydt = torch.float32 if wl.y_dtype == "f32" else torch.bfloat16
+    if wl.kind == "moe":
+        idd = torch.from_numpy(ids).cuda()
+        y = torch.empty((wl.m, wl.top_k, wl.n), dtype=ydt, device="cuda")
+        for _ in range(args.profile_calls):
+            kq.matmul_id(wd, wl.codec, xd, idd, out=y)
+    else:
+        y = torch.empty((wl.m, wl.n), dtype=ydt, device="cuda")
+        for _ in range(args.profile_calls):
+            kq.matmul(wd, wl.codec, xd, out=y, const_weights=True)
+    torch.cuda.synchronize()
+    status = kq.device_status()
+    if status != 0:  # a kernel reported a bad input or a wait that gave up
+        raise SystemExit(f"device status {status} after {wl.name}")
+    print(json.dumps({"profiled": wl.name, "calls": args.profile_calls}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -401,10 +497,17 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="kq", choices=["kq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile", default=None, choices=sorted(synth.WORKLOADS),
+                    help="run a few eager calls of one workload (for ncu) and exit")
+    ap.add_argument("--profile-calls", type=int, default=3)
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other workloads' numbers (prefill GEMM, MoE, TQ1, Q8_0)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

@@ -43,6 +43,12 @@ namespace {
 #ifndef KQ_GEMV_MAX_WARPS
 #define KQ_GEMV_MAX_WARPS 16
 #endif
+#ifndef KQ_GEMV_MIN_BLOCKS
+#define KQ_GEMV_MIN_BLOCKS 1
+#endif
+#ifndef KQ_GEMV_XREG
+#define KQ_GEMV_XREG 1
+#endif
 constexpr int GEMV_SMEM_LIMIT = KQ_GEMV_SMEM_LIMIT;
 constexpr int GEMV_MAX_WARPS = KQ_GEMV_MAX_WARPS;
 constexpr int GEMV_MAX_SLOTS = 4;
@@ -60,6 +66,10 @@ struct GemvParams {
     int xs_bytes;     // per-sub-block scales (and as many bytes again of sums)
     int early;        // issue weight copies before griddepcontrol.wait
     unsigned int *err;
+    // expert-indexed mode (grid.y = expert): grouping from the device
+    const int32_t *counts, *offsets, *perm;
+    int top_k;
+    int64_t expert_stride;
 };
 
 __device__ __forceinline__ int dp2a_lo(int a, uint32_t b, int c) {
@@ -96,7 +106,8 @@ __device__ __forceinline__ void load_x8v(const __nv_bfloat16 *p, float v[8]) {
     v[4] = bf16lo(a.z); v[5] = bf16hi(a.z); v[6] = bf16lo(a.w); v[7] = bf16hi(a.w);
 }
 
-// Stage TB activation rows for a CTA.
+// Stage TB activation rows for a CTA: slot t holds activation row tok[t]
+// (zeros where tok[t] < 0).
 //   codes  int16, layout [t][j16][unit ^ (j16 & 7)] of 16-byte groups (8
 //          consecutive positions); units padded to a multiple of 8 so the XOR
 //          swizzle stays in range.  Readers (lane = unit, fixed j16) and
@@ -108,8 +119,8 @@ __device__ __forceinline__ void load_x8v(const __nv_bfloat16 *p, float v[8]) {
 // A thread owns 8 consecutive positions; the four threads of a sub-block are
 // adjacent lanes.  All loads of up to XIT rounds are issued before use.
 template <int C, int TB, typename XT, typename F>
-__device__ __forceinline__ void stage_activations(const GemvParams &p, int4 *xq, float *xsc,
-                                                  float *xsum, F &&after_first_loads) {
+__device__ __forceinline__ void stage_activations(const GemvParams &p, const int *tok, int4 *xq,
+                                                  float *xsc, float *xsum, F &&after_first_loads) {
     constexpr int XIT = 4;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nthr = blockDim.x;
     const int per_row = p.k / 8, nitems = TB * per_row;
@@ -121,8 +132,8 @@ __device__ __forceinline__ void stage_activations(const GemvParams &p, int4 *xq,
         for (int it = 0; it < XIT; ++it) {
             const int idx = (r0 + it) * nthr + (int)threadIdx.x;
             const int t = idx / per_row, pos = (idx % per_row) * 8;
-            if (r0 + it < nrounds && idx < nitems && t < p.m) {
-                load_x8v(x + (int64_t)t * p.k + pos, v[it]);
+            if (r0 + it < nrounds && idx < nitems && tok[t] >= 0) {
+                load_x8v(x + (int64_t)tok[t] * p.k + pos, v[it]);
             } else {
                 #pragma unroll
                 for (int e = 0; e < 8; ++e) v[it][e] = 0.f;
@@ -192,11 +203,18 @@ template <> struct Vec<4> {
     }
 };
 
-// XREG: the lane's activation codes live in registers for the whole kernel
-// (one token, at most 32 units of at most 2 chunks, i.e. K <= 4096).
+// One pass of a CTA over weight rows [row_begin, row_end) of `w` with TB
+// activation slots: slot t multiplies activation row tok[t] (none if < 0) and
+// writes output row yrow[t].  XREG: the lane's activation codes live in
+// registers (one slot, at most 32 units of at most 2 chunks, K <= 4096).
+// `pass` counts earlier passes of this CTA over the same row range: the ring's
+// barriers are initialised in pass 0 only and their phases run on across
+// passes (a live mbarrier is never initialised again).  Returns false if a
+// wait gave up (the device error word is set).
 template <int C, int TB, int R, bool XREG, typename XT, typename YT>
-__global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, 1) gemv_q4k_kernel(const GemvParams p) {
-    extern __shared__ __align__(128) uint8_t smem[];
+__device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w, int row_begin,
+                                          int row_end, const int *tok, const int64_t *yrow,
+                                          uint8_t *smem, int pass) {
     int4 *xq = reinterpret_cast<int4 *>(smem);
     float *xsc = reinterpret_cast<float *>(smem + p.xq_bytes);
     float *xsum = reinterpret_cast<float *>(smem + p.xq_bytes + p.xs_bytes);
@@ -204,44 +222,53 @@ __global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, 1) gemv_q4k_kernel(const 
     uint64_t *full = reinterpret_cast<uint64_t *>(ring + (size_t)p.warps * p.slots * p.row_bytes);
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int row_begin = blockIdx.x * p.rows_per_cta;
-    const int row_end = min(p.n, row_begin + p.rows_per_cta);
-    if (row_begin >= row_end) return;
     const int my_rows = warp < row_end - row_begin ? (row_end - row_begin - warp + p.warps - 1) / p.warps : 0;
     uint8_t *my_ring = ring + (size_t)warp * p.slots * p.row_bytes;
     uint64_t *my_full = full + warp * p.slots;
     const int64_t row_bytes = p.row_bytes;
+    // Fills of this warp's ring before this pass (every pass has my_rows rows).
+    const int base = pass * my_rows;
 
-    if (lane == 0) {
-        for (int s = 0; s < p.slots; ++s) mbar_init(&my_full[s], 1);
-        fence_mbar_init();
+    if (pass == 0) {
+        if (lane == 0) {
+            for (int s = 0; s < p.slots; ++s) mbar_init(&my_full[s], 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
     }
-    __syncwarp();
     auto issue = [&](int i) {
-        const int slot = i % p.slots;
+        const int slot = (base + i) % p.slots;
         const int64_t r = row_begin + warp + (int64_t)i * p.warps;
         mbar_arrive_expect_tx(&my_full[slot], (uint32_t)row_bytes);
-        bulk_g2s(my_ring + slot * row_bytes, p.w + r * row_bytes, (uint32_t)row_bytes, &my_full[slot]);
+        bulk_g2s(my_ring + slot * row_bytes, w + r * row_bytes, (uint32_t)row_bytes, &my_full[slot]);
     };
     // Let the next kernel on the stream be scheduled now: it only prefetches
     // constant weights before its own griddepcontrol.wait, which waits for
     // this grid to complete.
     griddep_launch_dependents();
-    // Constant weights: start moving this CTA's rows into L2 before waiting
-    // for the preceding kernel.
-    if (p.early && threadIdx.x == 0) {
-        const int64_t bytes = (int64_t)(row_end - row_begin) * row_bytes;
-        const uint8_t *src = p.w + (int64_t)row_begin * row_bytes;
-        for (int64_t off = 0; off < bytes; off += 32768)
-            prefetch_l2(src + off, (uint32_t)(bytes - off < 32768 ? bytes - off : 32768));
+    // Constant weights: before waiting for the preceding kernel, copy this
+    // warp's first rows straight into its slots and start the CTA's other
+    // rows towards L2.  (A CTA fits beside the preceding kernel's CTA, so
+    // this runs while that kernel is still computing.)
+    const int first = min(p.slots, my_rows);
+    if (p.early) {
+        if (lane == 0)
+            for (int i = 0; i < first; ++i) issue(i);  // early mode makes one pass
+        if (threadIdx.x == 0 && (row_end - row_begin) > p.slots * p.warps) {
+            const int64_t bytes = (int64_t)(row_end - row_begin) * row_bytes;
+            const uint8_t *src = w + (int64_t)row_begin * row_bytes;
+            for (int64_t off = 0; off < bytes; off += 32768)
+                prefetch_l2(src + off, (uint32_t)(bytes - off < 32768 ? bytes - off : 32768));
+        }
     }
     griddep_wait();
-    // Activation loads go out first (they gate every row); the row copies
-    // into shared memory follow right behind them.
-    const int first = min(p.slots, my_rows);
-    stage_activations<C, TB, XT>(p, xq, xsc, xsum, [&]() {
-        if (lane == 0)
+    // Otherwise the activation loads go out first (they gate every row) and
+    // the row copies follow right behind them.
+    stage_activations<C, TB, XT>(p, tok, xq, xsc, xsum, [&]() {
+        if (!p.early && lane == 0) {
+            fence_proxy_async_smem();  // generic reads of the slots in an earlier pass
             for (int i = 0; i < first; ++i) issue(i);
+        }
     });
     __syncthreads();
 
@@ -270,9 +297,9 @@ __global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, 1) gemv_q4k_kernel(const 
         const uint8_t *rowp[R];
         #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const int ii = i + min(r, nr - 1);
+            const int ii = base + i + min(r, nr - 1);
             const int slot = ii % p.slots;
-            if (r < nr && !mbar_wait(&my_full[slot], (uint32_t)(ii / p.slots) & 1u, p.err)) return;
+            if (r < nr && !mbar_wait(&my_full[slot], (uint32_t)(ii / p.slots) & 1u, p.err)) return false;
             rowp[r] = my_ring + slot * row_bytes;
         }
         float acc[R][TB];
@@ -384,12 +411,12 @@ __global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, 1) gemv_q4k_kernel(const 
         for (int r = 0; r < R; ++r) {
             if (r < nr) {
                 const int64_t row = row_begin + warp + (int64_t)(i + r) * p.warps;
-                if (lane < TB && lane < p.m) {
+                if (lane < TB && tok[lane] >= 0) {
                     float v = acc[r][0];
                     #pragma unroll
                     for (int t = 1; t < TB; ++t)
                         if (lane == t) v = acc[r][t];
-                    store_out(y + (int64_t)lane * p.n + row, v);
+                    store_out(y + yrow[lane] * p.n + row, v);
                 }
             }
         }
@@ -399,6 +426,56 @@ __global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, 1) gemv_q4k_kernel(const 
             for (int r = 0; r < nr; ++r)
                 if (i + r + p.slots < my_rows) issue(i + r + p.slots);
         }
+    }
+    return true;
+}
+
+template <int C, int TB, int R, bool XREG, typename XT, typename YT>
+__global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, KQ_GEMV_MIN_BLOCKS) gemv_q4k_kernel(const GemvParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_tok[TB];
+    __shared__ int64_t s_yrow[TB];
+    const int row_begin = blockIdx.x * p.rows_per_cta;
+    const int row_end = min(p.n, row_begin + p.rows_per_cta);
+    if (row_begin >= row_end) return;
+    if (threadIdx.x < TB) {
+        s_tok[threadIdx.x] = (int)threadIdx.x < p.m ? (int)threadIdx.x : -1;
+        s_yrow[threadIdx.x] = threadIdx.x;
+    }
+    __syncthreads();
+    gemv_pass<C, TB, R, XREG, XT, YT>(p, p.w, row_begin, row_end, s_tok, s_yrow, smem, 0);
+}
+
+// Expert-indexed form: CTA (chunk, e) streams rows of expert e's slice once
+// per group of up to TB (token, slot) pairs routed to e (the device-side
+// grouping of kq_moe.cu: ascending pair order), so each hit expert's weights
+// leave HBM once per group; experts nobody chose cost nothing.
+template <int C, int TB, int R, typename XT, typename YT>
+__global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, 1) gemv_id_q4k_kernel(const GemvParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_tok[TB];
+    __shared__ int64_t s_yrow[TB];
+    __shared__ int s_failed;
+    const int e = blockIdx.y;
+    const int cnt = p.counts[e];
+    const int row_begin = blockIdx.x * p.rows_per_cta;
+    const int row_end = min(p.n, row_begin + p.rows_per_cta);
+    if (cnt == 0 || row_begin >= row_end) return;
+    const int32_t *pairs = p.perm + p.offsets[e];
+    const uint8_t *w = p.w + (int64_t)e * p.expert_stride;
+    if (threadIdx.x == 0) s_failed = 0;
+    for (int j0 = 0, pass = 0; j0 < cnt; j0 += TB, ++pass) {
+        __syncthreads();  // the previous pass is done with s_tok / s_yrow
+        if (s_failed) return;  // a wait gave up: the ring's phases are unknown
+        if (threadIdx.x < TB) {
+            const int j = j0 + (int)threadIdx.x;
+            const int pr = j < cnt ? pairs[j] : -1;
+            s_tok[threadIdx.x] = pr >= 0 ? pr / p.top_k : -1;
+            s_yrow[threadIdx.x] = pr >= 0 ? pr : 0;
+        }
+        __syncthreads();
+        if (!gemv_pass<C, TB, R, false, XT, YT>(p, w, row_begin, row_end, s_tok, s_yrow, smem, pass))
+            s_failed = 1;
     }
 }
 
@@ -480,7 +557,8 @@ template <int C, typename XT, typename YT>
 cudaError_t dispatch_tb(GemvParams p, int tb, bool const_w, cudaStream_t s) {
     switch (tb) {
     case 1:
-        if (C <= 2 && p.units <= 32) return launch_q4k<C, 1, (C <= 2), XT, YT>(p, const_w, s);
+        if (KQ_GEMV_XREG && C <= 2 && p.units <= 32)
+            return launch_q4k<C, 1, (KQ_GEMV_XREG && C <= 2), XT, YT>(p, const_w, s);
         return launch_q4k<C, 1, false, XT, YT>(p, const_w, s);
     case 2: return launch_q4k<C, 2, false, XT, YT>(p, const_w, s);
     case 4: return launch_q4k<C, 4, false, XT, YT>(p, const_w, s);
@@ -502,26 +580,116 @@ cudaError_t dispatch_c(GemvParams p, int tb, bool const_w, cudaStream_t s) {
 bool gemv_supported(int type, int64_t n, int64_t k, int x_dtype, int64_t m) {
     (void)x_dtype;
     GemvParams p;
-    return plan_gemv(type, n, k, m, sm_count(), &p);
+    return m >= 1 && plan_gemv(type, n, k, m < 8 ? m : 8, sm_count(), &p);
 }
 
+// More than eight activation rows run as consecutive launches of up to eight
+// rows each (the weights are streamed once per launch).
 cudaError_t launch_gemv(int type, const void *w, int64_t n, int64_t k, const void *x, int xdt,
                         int64_t m, void *y, int ydt, bool const_w, cudaStream_t s) {
-    GemvParams p;
-    const int tb = tb_for(m);
-    if (!plan_gemv(type, n, k, m, sm_count(), &p)) return cudaErrorNotSupported;
-    p.w = static_cast<const uint8_t *>(w);
-    p.x = x;
-    p.y = y;
-    if (xdt == KQ_F32) {
-        if (ydt == KQ_F32) return dispatch_c<float, float>(p, tb, const_w, s);
-        return dispatch_c<float, __nv_bfloat16>(p, tb, const_w, s);
+    const size_t xs = (xdt == KQ_F32 ? 4 : 2), ys = (ydt == KQ_F32 ? 4 : 2);
+    for (int64_t m0 = 0; m0 < m; m0 += 8) {
+        const int64_t mc = m - m0 < 8 ? m - m0 : 8;
+        GemvParams p = {};
+        const int tb = tb_for(mc);
+        if (!plan_gemv(type, n, k, mc, sm_count(), &p)) return cudaErrorNotSupported;
+        p.w = static_cast<const uint8_t *>(w);
+        p.x = static_cast<const char *>(x) + (size_t)m0 * (size_t)k * xs;
+        p.y = static_cast<char *>(y) + (size_t)m0 * (size_t)n * ys;
+        cudaError_t e;
+        if (xdt == KQ_F32) {
+            e = ydt == KQ_F32 ? dispatch_c<float, float>(p, tb, const_w, s)
+                              : dispatch_c<float, __nv_bfloat16>(p, tb, const_w, s);
+        } else {
+            e = ydt == KQ_F32 ? dispatch_c<__nv_bfloat16, float>(p, tb, const_w, s)
+                              : dispatch_c<__nv_bfloat16, __nv_bfloat16>(p, tb, const_w, s);
+        }
+        if (e != cudaSuccess) return e;
     }
-    if (ydt == KQ_F32) return dispatch_c<__nv_bfloat16, float>(p, tb, const_w, s);
-    return dispatch_c<__nv_bfloat16, __nv_bfloat16>(p, tb, const_w, s);
+    return cudaSuccess;
 }
 
-bool gemv_id_supported(int, int64_t, int) { return false; }
-cudaError_t launch_gemv_id(const IdArgs &, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int ID_TB = 4;  // (token, slot) pairs per pass over an expert's rows
+
+// Grid (chunks, E): about two CTAs per SM if every expert were hit; eight
+// warps per CTA so that two CTAs fit on an SM.
+bool plan_gemv_id(int type, int64_t n, int64_t k, int64_t n_experts, int num_sms, GemvParams *p) {
+    if (type != KQ_Q4_K || n < 1 || n > INT32_MAX / 2 || k > (1 << 20) || n_experts < 1) return false;
+    const int nb = (int)(k / 256);
+    const int C = chunks_per_unit(nb);
+    const int units = nb * 4 / C, units_pad = (units + 7) / 8 * 8;
+    const int64_t row_bytes = (int64_t)nb * 144;
+    int64_t chunks = (2 * num_sms + n_experts - 1) / n_experts;
+    if (chunks < 1) chunks = 1;
+    if (chunks > n) chunks = n;
+    const int rows_per_cta = (int)((n + chunks - 1) / chunks);
+    const size_t xq_bytes = (size_t)ID_TB * 8 * C * units_pad * 16;
+    const size_t xs_bytes = (size_t)ID_TB * units * 2 * C * 4;
+    const size_t fixed = xq_bytes + 2 * xs_bytes;
+    const size_t limit = 100 * 1024;
+    if (fixed + 1024 >= limit) return false;
+    const int warps = rows_per_cta < 8 ? rows_per_cta : 8;
+    const int rows_per_warp = (rows_per_cta + warps - 1) / warps;
+    int slots = rows_per_warp < GEMV_MAX_SLOTS ? rows_per_warp : GEMV_MAX_SLOTS;
+    while (slots > 1 && fixed + (size_t)warps * slots * (row_bytes + 8) > limit) --slots;
+    if (fixed + (size_t)warps * slots * (row_bytes + 8) > limit) return false;
+    p->nb = nb; p->units = units; p->units_pad = units_pad; p->rows_per_cta = rows_per_cta;
+    p->warps = warps; p->slots = slots; p->row_bytes = (int)row_bytes;
+    p->xq_bytes = (int)xq_bytes; p->xs_bytes = (int)xs_bytes;
+    p->n = (int)n; p->k = (int)k; p->m = ID_TB;
+    return true;
+}
+
+template <int C, typename XT, typename YT>
+cudaError_t launch_id_q4k(GemvParams p, int64_t n_experts, cudaStream_t s) {
+    auto kern = gemv_id_q4k_kernel<C, ID_TB, 1, XT, YT>;
+    const size_t smem = (size_t)p.xq_bytes + 2 * (size_t)p.xs_bytes +
+                        (size_t)p.warps * p.slots * ((size_t)p.row_bytes + 8);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)((p.n + p.rows_per_cta - 1) / p.rows_per_cta), (unsigned)n_experts);
+    kern<<<grid, 32 * p.warps, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename XT, typename YT>
+cudaError_t dispatch_id_c(GemvParams p, int64_t n_experts, cudaStream_t s) {
+    switch (chunks_per_unit(p.nb)) {
+    case 4: return launch_id_q4k<4, XT, YT>(p, n_experts, s);
+    case 2: return launch_id_q4k<2, XT, YT>(p, n_experts, s);
+    default: return launch_id_q4k<1, XT, YT>(p, n_experts, s);
+    }
+}
+
+}  // namespace
+
+bool gemv_id_supported(int type, int64_t k, int x_dtype) {
+    (void)x_dtype;
+    GemvParams p;
+    return plan_gemv_id(type, 1024, k, 8, 148, &p);
+}
+
+cudaError_t launch_gemv_id(const IdArgs &a, cudaStream_t s) {
+    GemvParams p = {};
+    if (!plan_gemv_id(a.type, a.n, a.k, a.n_experts, sm_count(), &p)) return cudaErrorNotSupported;
+    p.w = static_cast<const uint8_t *>(a.w);
+    p.x = a.x;
+    p.y = a.y;
+    p.early = 0;
+    p.err = error_word();
+    p.counts = a.counts;
+    p.offsets = a.offsets;
+    p.perm = a.perm;
+    p.top_k = (int)a.top_k;
+    p.expert_stride = a.expert_stride;
+    if (a.x_dtype == KQ_F32) {
+        if (a.y_dtype == KQ_F32) return dispatch_id_c<float, float>(p, a.n_experts, s);
+        return dispatch_id_c<float, __nv_bfloat16>(p, a.n_experts, s);
+    }
+    if (a.y_dtype == KQ_F32) return dispatch_id_c<__nv_bfloat16, float>(p, a.n_experts, s);
+    return dispatch_id_c<__nv_bfloat16, __nv_bfloat16>(p, a.n_experts, s);
+}
 
 }  // namespace kq
