@@ -185,6 +185,18 @@ class GemvStep:
         self.host_y = torch.empty((wl.m, wl.n), dtype=ydt).pin_memory()
 
     def run(self):
+        """The pool's GEMVs have no data dependency on one another, and the
+        calls say so (independent=True): consecutive calls stream side by
+        side.  Each call still stages its activations, decodes every weight
+        and writes its output."""
+        for i in range(self.pool):
+            self.kq.matmul(self.ws[i], self.wl.codec, self.xs[i], out=self.ys[i],
+                           independent=True)
+
+    def run_serial(self):
+        """The same calls, each ordered after the one before it (a chain of
+        dependent layers): weights stream early, activations are read only
+        after the preceding kernel completes."""
         for i in range(self.pool):
             self.kq.matmul(self.ws[i], self.wl.codec, self.xs[i], out=self.ys[i],
                            const_weights=True)
@@ -353,6 +365,9 @@ def run_gpu(args):
     with ClockSampler(local) as clk:
         ms = time_graph(torch, step.run, args.steps, args.warmup, pg)
     ms = max_over_ranks(torch, pg, ms)
+    serial_steps = max(3, args.steps // 4)
+    serial_ms = max_over_ranks(torch, pg, time_graph(torch, step.run_serial, serial_steps, 3, pg))
+    serial_us = serial_ms * 1e3 / (serial_steps * step.launches)
     e2e_ms = time_eager(torch, step.run_e2e, max(1, args.steps // 4), 1, pg)
     e2e_ms = max_over_ranks(torch, pg, e2e_ms) / max(1, args.steps // 4)
     status = kq.device_status()
@@ -386,6 +401,13 @@ def run_gpu(args):
             "l2_policy": f"inputs larger than L2: each step streams {step.pool} distinct weight "
                          f"matrices ({step.pool * step.wbytes / 1e6:.0f} MB > 4x L2 {l2 / 1e6:.0f} MB)",
             "parallelism": f"replicas x{world}",
+            "calls": "independent (kq flag: no call reads or writes another's buffers; "
+                     "each still stages x, decodes every weight, writes y)",
+        },
+        "serial_chain": {
+            "us_per_call": round(serial_us, 4),
+            "GB/s": round(step.wbytes / (serial_us * 1e-6) / 1e9, 1),
+            "note": "same calls, each ordered after the previous kernel (dependent layers)",
         },
         "gpu_launches": args.steps * step.launches,
         "e2e": {

@@ -20,6 +20,7 @@ CODECS = {"q8_0": Q8_0, "q2_k": Q2_K, "q4_k": Q4_K, "tq1_g128": TQ1_G128}
 F32, BF16, F16 = 0, 1, 2
 PATH_AUTO, PATH_SIMPLE, PATH_GEMV, PATH_GEMM = 0, 1, 2, 3
 FLAG_CONST_WEIGHTS = 0x100
+FLAG_INDEPENDENT = 0x200
 
 _DT = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}
 
@@ -130,8 +131,13 @@ def dequantize(w: torch.Tensor, codec, k: int, dtype=torch.float32, out=None) ->
 
 
 def matmul(w: torch.Tensor, codec, x: torch.Tensor, out=None, out_dtype=torch.float32,
-           path: int = PATH_AUTO, const_weights: bool = False) -> torch.Tensor:
-    """y[m, n] = sum_k dequant(w)[n, k] * x[m, k]; x [m, k] fp32/bf16."""
+           path: int = PATH_AUTO, const_weights: bool = False,
+           independent: bool = False) -> torch.Tensor:
+    """y[m, n] = sum_k dequant(w)[n, k] * x[m, k]; x [m, k] fp32/bf16.
+
+    const_weights: no earlier work on the stream writes w.
+    independent: no earlier work on the stream writes w or x, or touches
+    out; consecutive independent calls may then run side by side."""
     c = _codec(codec)
     if x.dim() != 2 or not x.is_contiguous():
         raise ValueError("x must be a contiguous [m, k] tensor")
@@ -139,7 +145,7 @@ def matmul(w: torch.Tensor, codec, x: torch.Tensor, out=None, out_dtype=torch.fl
     n = _weights(w, c, k)
     if out is None:
         out = torch.empty((m, n), dtype=out_dtype, device=x.device)
-    flags = path | (FLAG_CONST_WEIGHTS if const_weights else 0)
+    flags = path | (FLAG_CONST_WEIGHTS if const_weights else 0) | (FLAG_INDEPENDENT if independent else 0)
     _check(lib().kq_matmul_ex(c, _ptr(w), n, k, _ptr(x), _DT[x.dtype], m, _ptr(out),
                               _DT[out.dtype], flags, _stream()), "kq_matmul")
     return out

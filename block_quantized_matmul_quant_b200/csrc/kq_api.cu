@@ -106,9 +106,16 @@ static bool id_workspace_layout(int64_t n_tokens, int64_t top_k, int64_t n_exper
     return true;
 }
 
-// Threshold of activation rows above which the tensor-core kernel serves
-// bf16 inputs (measured on B200; see the dispatch table in DESIGN).
-constexpr int64_t GEMM_MIN_M = 16;
+// Activation rows from which the tensor-core kernel serves bf16 inputs; the
+// bandwidth kernel handles up to eight rows per launch.
+constexpr int64_t GEMM_MIN_M = 9;
+// Mean (token, slot) pairs per expert from which the expert-indexed product
+// runs on the tensor cores (each hit expert's weights are then decoded once
+// per token tile of up to 176 pairs, instead of once per four pairs).
+constexpr int64_t ID_GEMM_MIN_PAIRS_PER_EXPERT = 16;
+// The TQ1 bandwidth kernel takes two activation rows per pass over the
+// weights; beyond this many rows the plain kernel is used.
+constexpr int64_t TQ1_GEMV_MAX_M = 8;
 
 }  // namespace kq
 
@@ -142,8 +149,9 @@ int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, i
     if (m <= 0) return KQ_ERR_ARG;
     if ((st = check_act(x, x_dtype, m, k, false))) return st;
     if ((st = check_act(y, y_dtype, m, n, false))) return st;
-    const bool const_w = (path & KQ_FLAG_CONST_WEIGHTS) != 0;
-    path &= ~KQ_FLAG_CONST_WEIGHTS;
+    const bool indep = (path & KQ_FLAG_INDEPENDENT) != 0;
+    const bool const_w = indep || (path & KQ_FLAG_CONST_WEIGHTS) != 0;
+    path &= ~(KQ_FLAG_CONST_WEIGHTS | KQ_FLAG_INDEPENDENT);
     if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMM) return KQ_ERR_ARG;
     if ((st = check_device())) return st;
     cudaStream_t s = (cudaStream_t)stream;
@@ -151,7 +159,7 @@ int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, i
     const bool can_gemv = gemv_supported(type, n, k, x_dtype, m);
     if (path == KQ_PATH_AUTO) {
         if (can_gemm && m >= GEMM_MIN_M) path = KQ_PATH_GEMM;
-        else if (can_gemv) path = KQ_PATH_GEMV;
+        else if (can_gemv && (type != KQ_TQ1_G128 || m <= TQ1_GEMV_MAX_M)) path = KQ_PATH_GEMV;
         else path = KQ_PATH_SIMPLE;
     }
     switch (path) {
@@ -160,7 +168,10 @@ int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, i
         return to_status(launch_gemm(type, w, n, k, x, m, y, y_dtype, s));
     case KQ_PATH_GEMV:
         if (!can_gemv) return KQ_ERR_UNSUPPORTED;
-        return to_status(launch_gemv(type, w, n, k, x, x_dtype, m, y, y_dtype, const_w, s));
+        return to_status(launch_gemv(type, w, n, k, x, x_dtype, m, y, y_dtype,
+                                     indep ? GemvOrder::kIndependent
+                                           : const_w ? GemvOrder::kConstWeights : GemvOrder::kStream,
+                                     s));
     default:
         return to_status(launch_simple_matmul(type, w, n, k, x, x_dtype, m, y, y_dtype, s));
     }
@@ -216,13 +227,24 @@ int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64
     a.tiles = reinterpret_cast<int32_t *>(ws + l.tiles);
     a.n_tiles = reinterpret_cast<int32_t *>(ws + l.n_tiles);
     const bool can_gemv = gemv_id_supported(type, k, x_dtype);
-    if (path == KQ_PATH_AUTO) path = can_gemv ? KQ_PATH_GEMV : KQ_PATH_SIMPLE;
-    if (path == KQ_PATH_GEMM) return KQ_ERR_UNSUPPORTED;
+    const bool can_gemm = gemm_supported(type, n, k, x_dtype, y_dtype);
+    if (path == KQ_PATH_AUTO) {
+        if (can_gemm && pairs >= ID_GEMM_MIN_PAIRS_PER_EXPERT * n_experts) path = KQ_PATH_GEMM;
+        else path = can_gemv ? KQ_PATH_GEMV : KQ_PATH_SIMPLE;
+    }
+    if (path == KQ_PATH_GEMM && !can_gemm) return KQ_ERR_UNSUPPORTED;
     if (path == KQ_PATH_GEMV && !can_gemv) return KQ_ERR_UNSUPPORTED;
     cudaError_t e = launch_moe_group(ids, pairs, n_experts, const_cast<int32_t *>(a.counts),
                                      const_cast<int32_t *>(a.offsets),
                                      const_cast<int32_t *>(a.perm), y, y_dtype, n, s);
     if (e != cudaSuccess) return KQ_ERR_CUDA;
+    if (path == KQ_PATH_GEMM) {
+        const int bn = gemm_id_bn(n_tokens, top_k, n_experts);
+        e = launch_moe_tiles(a.offsets, n_experts, bn, const_cast<int32_t *>(a.tiles),
+                             const_cast<int32_t *>(a.n_tiles), s);
+        if (e != cudaSuccess) return KQ_ERR_CUDA;
+        return to_status(launch_gemm_id(a, bn, s));
+    }
     if (path == KQ_PATH_GEMV) return to_status(launch_gemv_id(a, s));
     return to_status(launch_simple_id(a, s));
 }

@@ -8,7 +8,13 @@
 //
 //  * Persistent kernel, one CTA per SM, static round-robin over output tiles
 //    of 128 weight rows (the MMA's M) x BN tokens (the MMA's N, a multiple of
-//    16 <= 256 picked by the host to balance waves over the SMs).
+//    16 <= 192 picked by the host to balance waves over the SMs).
+//  * The decoded weights never touch shared memory: decoder threads turn raw
+//    super-block bytes into bf16 in registers and write them straight into
+//    tensor memory (tcgen05.st), where the MMA reads its A operand
+//    (tcgen05.mma with A in TMEM, B = activations in shared memory).  Shared
+//    memory only carries the activation tiles and the raw bytes, so the
+//    tensor core's operand reads do not compete with decoder stores.
 //  * Warp roles:  warp 0  TMA producer -- bf16 activation tiles (64 K x BN,
 //                         128-byte swizzle) and raw Q4_K super-blocks
 //                         (128 rows x 144 bytes) into shared-memory rings;
@@ -16,12 +22,15 @@
 //                         (kind::f16, bf16 x bf16 -> fp32 in TMEM) and
 //                         tcgen05.commit's to the stage / accumulator barriers;
 //                 warps 2-5  epilogue -- tcgen05.ld from TMEM, convert, store;
-//                 warps 6-13 decoders -- raw super-block bytes -> exact fp32
-//                         weights (d*sc*q - dmin*m, one rounding) -> bf16
-//                         (round to nearest even) written in the canonical
-//                         K-major 128-byte-swizzled layout the MMA reads.
-//  * Two TMEM accumulators (2 x BN columns) let the epilogue of tile i
-//    overlap the main loop of tile i+1.
+//                 warps 6..  decoders, in groups of four warps (one per TMEM
+//                         lane quadrant, so lane = weight row): group j
+//                         decodes the stages s with s % groups == j, 64 K
+//                         positions of its 32 rows per warp, exact fp32
+//                         (d*sc*q - dmin*m, one rounding) -> bf16 (round to
+//                         nearest even).
+//  * TMEM (512 columns): accumulators at columns 0 and 256 (BN each, so the
+//    epilogue of tile i overlaps the main loop of tile i+1); the stage ring's
+//    A slots (32 columns = 128 rows x 64 bf16) fill the gaps after them.
 //  * Every mbarrier wait is bounded (kq_ptx.cuh): on timeout the kernel sets
 //    the device error word and the waiting role stops; TMEM is released by
 //    the allocating warp after a block barrier that every thread reaches.
@@ -42,24 +51,61 @@ constexpr int BM = 128;            // weight rows per tile (MMA M)
 constexpr int BK = 64;             // K per stage (one 128-byte swizzle atom of bf16)
 constexpr int SB_BYTES = 144;      // Q4_K super-block
 constexpr int RAW_STAGE_BYTES = BM * SB_BYTES;   // 18432
-constexpr int A_STAGE_BYTES = BM * BK * 2;       // 16384
 #ifndef KQ_GEMM_DEC_WARPS
 #define KQ_GEMM_DEC_WARPS 16
 #endif
 constexpr int DEC_WARP0 = 6, DEC_WARPS = KQ_GEMM_DEC_WARPS;  // 8 or 16
+constexpr int DEC_GROUPS = DEC_WARPS / 4;                    // 2 or 4
+static_assert(DEC_GROUPS == 2 || DEC_GROUPS == 4, "decoder warps come in 2 or 4 groups of 4");
 constexpr int NUM_THREADS = (DEC_WARP0 + DEC_WARPS) * 32;
 constexpr int EPI_WARP0 = 2;
 constexpr int RAW_STAGES = 2;
+constexpr int MAX_A_STAGES = 8;   // TMEM A slots
+constexpr int MAX_B_STAGES = 10;  // activation tiles in shared memory
+constexpr int MAX_BN = 192;
 constexpr int SMEM_BUDGET = 227 * 1024;
 
 struct GemmParams {
     int n, k, m;
     int bn, m_tiles, n_tiles, tiles;
-    int stages;  // depth of the shared stage ring (decoded weights + activations)
+    int a_stages;  // decoded-weight ring: A slots in TMEM
+    int b_stages;  // activation ring: tiles in shared memory (deeper: their loads come from L2)
+    int a_col0;    // first TMEM column after an accumulator (BN rounded up to 32)
     int b_stage_bytes;
     void *y;
     unsigned int *err;
+    // expert-indexed mode: token tiles come from the device-side grouping
+    const int32_t *perm;      // pair indices t * top_k + s, grouped by expert
+    const int32_t *offsets;   // [E + 1] segment starts in perm
+    const int2 *id_tiles;     // (expert, first position in perm) per token tile
+    const int32_t *id_n_tiles;
+    int top_k;
 };
+
+// One output tile: weight rows n0.. of expert e times BN activation rows.
+// Dense: activation rows m0..m0+rows-1.  Expert-indexed: the activation rows
+// of pairs perm[m0 .. m0+rows-1].
+struct Tile {
+    int n0, e, m0, rows;
+};
+
+template <bool ID>
+__device__ __forceinline__ Tile tile_at(const GemmParams &p, int u) {
+    Tile t;
+    if constexpr (ID) {
+        const int2 tt = p.id_tiles[u / p.n_tiles];
+        t.n0 = (u % p.n_tiles) * BM;
+        t.e = tt.x;
+        t.m0 = tt.y;
+        t.rows = min(p.bn, p.offsets[tt.x + 1] - tt.y);
+    } else {
+        t.n0 = (u / p.m_tiles) * BM;
+        t.e = 0;
+        t.m0 = (u % p.m_tiles) * p.bn;
+        t.rows = min(p.bn, p.m - t.m0);
+    }
+    return t;
+}
 
 // ---- tcgen05 / TMA wrappers ----
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
@@ -68,6 +114,26 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+        : "memory");
+}
+// Four rows r0..r3 (columns x.. of a box one row high) into four consecutive
+// 128-byte rows of shared memory.
+__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int x, int r0, int r1,
+                                            int r2, int r3, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+        "r"(smem_addr(bar))
         : "memory");
 }
 
@@ -88,12 +154,13 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t accumulate) {
+// D (TMEM) += A (TMEM) * B (shared memory descriptor)
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -110,6 +177,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16]) {
           "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// 32 consecutive TMEM columns of this thread's lane <- r[0..31]; returns once
+// the writes are complete.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t r[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
@@ -130,6 +210,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
            ((uint32_t)(m >> 4) << 24);
 }
 
+// TMEM column of stage slot s: slots alternate between the gap after the
+// first accumulator (columns a_col0..255) and the gap after the second
+// (256 + a_col0..511), 32 columns each.
+__device__ __forceinline__ uint32_t a_slot_col(uint32_t s, int a_col0) {
+    return ((s & 1u) << 8) + (uint32_t)a_col0 + ((s >> 1) << 5);
+}
+
 __device__ __forceinline__ float half_f(uint32_t bits) { return half_bits_to_float(bits); }
 
 // Byte i of w as an exact float (2^23 exponent trick).
@@ -137,39 +224,58 @@ __device__ __forceinline__ float byte_float(uint32_t w, int i) {
     return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | (uint32_t)i)) - 8388608.0f;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
+// Four quant bytes (one nibble each, already masked: q or 16*q) -> two bf16x2
+// words of w = scale * nibble + bias with one fp32 rounding, then RNE to bf16.
+__device__ __forceinline__ void decode4(uint32_t nib, float2 scale, float2 bias, uint32_t &o0,
+                                        uint32_t &o1) {
+    const float2 magic = make_float2(-8388608.0f, -8388608.0f), one = make_float2(1.f, 1.f);
+    float2 f0 = make_float2(__uint_as_float(__byte_perm(nib, 0x4B000000u, 0x7440u)),
+                            __uint_as_float(__byte_perm(nib, 0x4B000000u, 0x7441u)));
+    float2 f1 = make_float2(__uint_as_float(__byte_perm(nib, 0x4B000000u, 0x7442u)),
+                            __uint_as_float(__byte_perm(nib, 0x4B000000u, 0x7443u)));
+    f0 = ffma2(f0, one, magic);  // exact: the nibble value
+    f1 = ffma2(f1, one, magic);
+    f0 = ffma2(f0, scale, bias);  // exact products, one rounding each
+    f1 = ffma2(f1, scale, bias);
+    const __nv_bfloat162 b0 = __floats2bfloat162_rn(f0.x, f0.y);
+    const __nv_bfloat162 b1 = __floats2bfloat162_rn(f1.x, f1.y);
+    o0 = *reinterpret_cast<const uint32_t *>(&b0);
+    o1 = *reinterpret_cast<const uint32_t *>(&b1);
 }
 
-template <typename YT>
+template <typename YT, bool ID>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_q4k_kernel(const __grid_constant__ CUtensorMap tmap_x,
                     const __grid_constant__ CUtensorMap tmap_w, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
-    const int S = p.stages;
-    uint8_t *a_ring = smem;                                    // S x 16 KB
-    uint8_t *b_ring = a_ring + S * A_STAGE_BYTES;              // S x bn*128
-    uint8_t *raw_ring = b_ring + S * p.b_stage_bytes;          // RAW_STAGES x 18 KB
+    const int SA = p.a_stages, SB = p.b_stages;
+    uint8_t *b_ring = smem;                                    // SB x bn*128
+    uint8_t *raw_ring = b_ring + SB * p.b_stage_bytes;         // RAW_STAGES x 18 KB
     uint64_t *bars = reinterpret_cast<uint64_t *>(raw_ring + RAW_STAGES * RAW_STAGE_BYTES);
-    uint64_t *full = bars;                   // [S]  TMA bytes + decoder warps -> MMA
-    uint64_t *empty = full + S;              // [S]  MMA -> TMA, decoders
-    uint64_t *raw_full = empty + S;          // [RAW] TMA -> decoders
+    uint64_t *full_a = bars;                 // [SA] one decoder group (4 warps) -> MMA
+    uint64_t *empty_a = full_a + SA;         // [SA] MMA -> decoders
+    uint64_t *full_b = empty_a + SA;         // [SB] TMA bytes -> MMA
+    uint64_t *empty_b = full_b + SB;         // [SB] MMA -> TMA
+    uint64_t *raw_full = empty_b + SB;       // [RAW] TMA -> decoders
     uint64_t *raw_empty = raw_full + RAW_STAGES;  // [RAW] decoders -> TMA
     uint64_t *acc_full = raw_empty + RAW_STAGES;  // [2] MMA -> epilogue
     uint64_t *acc_empty = acc_full + 2;           // [2] epilogue -> MMA
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    int *s_rows = reinterpret_cast<int *>(bars + 48);   // expert-indexed: activation row per tile row
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nk = p.k / BK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1 + DEC_WARPS);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(&full_a[s], 4);
+            mbar_init(&empty_a[s], 1);
+        }
+        for (int s = 0; s < SB; ++s) {
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty_b[s], 1);
         }
         for (int r = 0; r < RAW_STAGES; ++r) {
             mbar_init(&raw_full[r], 1);
@@ -191,71 +297,93 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     griddep_wait();
+    // Work units: dense tiles, or (token tile, weight tile) pairs whose token
+    // tiles the grouping step wrote on the device.
+    const int units = ID ? *p.id_n_tiles * p.n_tiles : p.tiles;
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         // Ring positions advance incrementally (no division in the issue
         // loop: this single thread must keep pace with the tensor core).
-        if (lane == 0) {
-            uint32_t slot = 0, phase = 0, rslot = 0, rphase = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-                const int n0 = (tile / p.m_tiles) * BM, m0 = (tile % p.m_tiles) * p.bn;
+        // Expert-indexed tiles first gather their activation row numbers
+        // (the whole warp, into s_rows; rows past the segment repeat its
+        // first row and their outputs are dropped), then load the tile four
+        // rows per gather.
+        uint32_t slot = 0, phase = 0, rslot = 0, rphase = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            const Tile t = tile_at<ID>(p, u);
+            if constexpr (ID) {
+                __syncwarp();  // lane 0 has issued every load of the previous tile
+                for (int i = lane; i < p.bn; i += 32)
+                    s_rows[i] = p.perm[t.m0 + (i < t.rows ? i : 0)] / p.top_k;
+                __syncwarp();
+            }
+            if (lane == 0) {
                 for (int ks = 0; ks < nk; ++ks) {
                     if ((ks & 3) == 0) {  // raw super-block for this and the next 3 stages
                         ok = mbar_wait(&raw_empty[rslot], rphase ^ 1, p.err);
                         if (!ok) break;
                         mbar_arrive_expect_tx(&raw_full[rslot], RAW_STAGE_BYTES);
-                        tma_load_2d(raw_ring + rslot * RAW_STAGE_BYTES, &tmap_w, (ks >> 2) * SB_BYTES, n0,
-                                    &raw_full[rslot]);
+                        tma_load_3d(raw_ring + rslot * RAW_STAGE_BYTES, &tmap_w, (ks >> 2) * SB_BYTES,
+                                    t.n0, t.e, &raw_full[rslot]);
                         if (++rslot == RAW_STAGES) { rslot = 0; rphase ^= 1; }
                     }
-                    ok = mbar_wait(&empty[slot], phase ^ 1, p.err);
+                    ok = mbar_wait(&empty_b[slot], phase ^ 1, p.err);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(&full[slot], p.b_stage_bytes);
-                    tma_load_2d(b_ring + slot * p.b_stage_bytes, &tmap_x, ks * BK, m0, &full[slot]);
-                    if (++slot == (uint32_t)S) { slot = 0; phase ^= 1; }
+                    mbar_arrive_expect_tx(&full_b[slot], p.b_stage_bytes);
+                    uint8_t *dst = b_ring + slot * p.b_stage_bytes;
+                    if constexpr (ID) {
+                        for (int i = 0; i < p.bn; i += 4)
+                            tma_gather4(dst + i * 128, &tmap_x, ks * BK, s_rows[i], s_rows[i + 1],
+                                        s_rows[i + 2], s_rows[i + 3], &full_b[slot]);
+                    } else {
+                        tma_load_2d(dst, &tmap_x, ks * BK, t.m0, &full_b[slot]);
+                    }
+                    if (++slot == (uint32_t)SB) { slot = 0; phase ^= 1; }
                 }
             }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
-        // One wait per stage (the stage's barrier collects the activation
-        // tile's bytes and the eight decoder warps), four MMAs whose
-        // descriptors only advance their start address, one commit that
-        // frees the stage when the MMAs are done.
+        // Per stage: wait for the activation tile's bytes and for the four
+        // warps that decoded the weights, four MMAs of K = 16 (A: 8 TMEM
+        // columns apart, B: 32 bytes apart in the swizzle atom), and one
+        // commit per ring that frees the slots when the MMAs are done.
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(BM, p.bn);
-            const uint64_t a_desc0 = sw128_desc(smem_addr(a_ring));
             const uint64_t b_desc0 = sw128_desc(smem_addr(b_ring));
-            const uint32_t a_step = A_STAGE_BYTES >> 4, b_step = (uint32_t)p.b_stage_bytes >> 4;
-            uint32_t slot = 0, phase = 0;
-            uint64_t ad = a_desc0, bd = b_desc0;
+            const uint32_t b_step = (uint32_t)p.b_stage_bytes >> 4;
+            uint32_t sa = 0, pa = 0, sb = 0, pb = 0;
+            uint64_t bd = b_desc0;
             int tl = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x, ++tl) {
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++tl) {
                 const int acc = tl & 1;
                 ok = mbar_wait(&acc_empty[acc], ((tl >> 1) & 1) ^ 1, p.err);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
                 for (int ks = 0; ks < nk; ++ks) {
-                    ok = mbar_wait(&full[slot], phase, p.err);
+                    ok = mbar_wait(&full_b[sb], pb, p.err) && mbar_wait(&full_a[sa], pa, p.err);
                     if (!ok) break;
-                    mma_bf16(d_tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
-                    mma_bf16(d_tmem, ad + 2, bd + 2, idesc, 1u);
-                    mma_bf16(d_tmem, ad + 4, bd + 4, idesc, 1u);
-                    mma_bf16(d_tmem, ad + 6, bd + 6, idesc, 1u);
-                    mma_commit(&empty[slot]);  // frees the stage once these MMAs finish
-                    if (++slot == (uint32_t)S) {
-                        slot = 0;
-                        phase ^= 1;
-                        ad = a_desc0;
+                    tc_fence_after();
+                    const uint32_t at = tmem_base + a_slot_col(sa, p.a_col0);
+                    mma_bf16_ts(d_tmem, at, bd, idesc, ks > 0 ? 1u : 0u);
+                    mma_bf16_ts(d_tmem, at + 8, bd + 2, idesc, 1u);
+                    mma_bf16_ts(d_tmem, at + 16, bd + 4, idesc, 1u);
+                    mma_bf16_ts(d_tmem, at + 24, bd + 6, idesc, 1u);
+                    mma_commit(&empty_b[sb]);  // frees both slots once these MMAs finish
+                    mma_commit(&empty_a[sa]);
+                    if (++sb == (uint32_t)SB) {
+                        sb = 0;
+                        pb ^= 1;
                         bd = b_desc0;
                     } else {
-                        ad += a_step;
                         bd += b_step;
                     }
+                    if (++sa == (uint32_t)SA) { sa = 0; pa ^= 1; }
                 }
                 if (ok) mma_commit(&acc_full[acc]);
             }
@@ -265,12 +393,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
         YT *y = static_cast<YT *>(p.y);
         int tl = 0;
-        for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++tl) {
+        for (int u = blockIdx.x; u < units; u += gridDim.x, ++tl) {
             const int acc = tl & 1;
-            const int n0 = (tile / p.m_tiles) * BM, m0 = (tile % p.m_tiles) * p.bn;
-            if (!mbar_wait(&acc_full[acc], (tl >> 1) & 1, p.err)) break;
+            const Tile t = tile_at<ID>(p, u);
+            // warp-uniform outcome: the TMEM loads below are .sync.aligned
+            if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], (tl >> 1) & 1, p.err))) break;
             tc_fence_after();
-            const int n = n0 + 32 * q + lane;
+            const int n = t.n0 + 32 * q + lane;
             const uint32_t t_row = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * 256);
             for (int c0 = 0; c0 < p.bn; c0 += 16) {
                 uint32_t r[16];
@@ -278,8 +407,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (n < p.n) {
                     #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const int m = m0 + c0 + j;
-                        if (m < p.m) store_out(y + (int64_t)m * p.n + n, __uint_as_float(r[j]));
+                        if (c0 + j < t.rows) {
+                            // output row: the activation row, or the (token, slot) pair
+                            const int64_t m = ID ? (int64_t)__ldg(p.perm + t.m0 + c0 + j) : (int64_t)(t.m0 + c0 + j);
+                            store_out(y + m * p.n + n, __uint_as_float(r[j]));
+                        }
                     }
                 }
             }
@@ -289,27 +421,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else {
         // ---------------- decoders ----------------
-        // DEC_WARPS * 32 threads share the 128 rows x 32 quant bytes of a
-        // stage: QB = 32 * 128 / threads bytes each (16 or 8).  Eight
-        // consecutive lanes take eight consecutive rows and the same byte
-        // range, so the raw reads (rows 144 bytes apart) and the swizzled
-        // 16-byte stores hit distinct bank groups.  A thread decodes both
-        // nibbles of its bytes: low nibbles are K positions QB*part + 0.. of
-        // the stage (sub-block 2cc), high nibbles K positions 32 + QB*part
-        // + 0.. (sub-block 2cc+1).
-        constexpr int PARTS = DEC_WARPS / 4;      // byte ranges per row: 2 or 4
-        constexpr int QB = 32 / PARTS;            // quant bytes per thread: 16 or 8
-        constexpr int NW = QB / 4;                // quant words per thread
-        const int t = threadIdx.x - DEC_WARP0 * 32;
-        const int r = 8 * (t / (8 * PARTS)) + (t & 7);   // weight row in the tile
-        const int part = (t >> 3) % PARTS;               // which QB bytes
-        const float2 magic = make_float2(-8388608.0f, -8388608.0f), one = make_float2(1.f, 1.f);
-        uint32_t g = 0, rsb = 0;
+        // Group grp (four consecutive warps, one per TMEM lane quadrant)
+        // decodes stage g when g % DEC_GROUPS == grp.  Lane l of a warp in
+        // quadrant q owns weight row r = 32 q + l: per stage it reads the
+        // row's 32 quant bytes of chunk cc = g % 4 (low nibbles: K positions
+        // 0..31 of the stage = sub-block 2cc, high nibbles: K 32..63 =
+        // sub-block 2cc+1) and writes 32 TMEM columns of its lane, column j
+        // holding the bf16 pair at K positions 2j, 2j+1.
+        const int grp = (warp - DEC_WARP0) >> 2;
+        const int quad = warp & 3;
+        const int r = 32 * quad + lane;
+        const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quad) << 16);
+        uint32_t slot = 0, phase = 0, rs = 0, rph = 0;
+        uint32_t g = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             for (int ks = 0; ks < nk && ok; ks += 4) {
-                const int rs = rsb % RAW_STAGES;
-                ok = mbar_wait(&raw_full[rs], (rsb / RAW_STAGES) & 1, p.err);
+                ok = __all_sync(0xffffffffu, mbar_wait(&raw_full[rs], rph, p.err));
                 if (!ok) break;
                 const uint8_t *blk = raw_ring + rs * RAW_STAGE_BYTES + r * SB_BYTES;
                 const uint4 hd = *reinterpret_cast<const uint4 *>(blk);
@@ -320,67 +448,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const uint32_t m_hi = ((hd.w >> 4) & 0x0F0F0F0Fu) | ((hd.z >> 2) & 0x30303030u);
                 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
-                    const int s = g % S;
-                    ok = mbar_wait(&empty[s], ((g / S) & 1) ^ 1, p.err);
-                    if (!ok) break;
-                    const uint32_t scw = cc < 2 ? sc_lo : sc_hi, mw = cc < 2 ? m_lo : m_hi;
-                    const int b0 = (2 * cc) & 3;
-                    // exact products: d*sc (17 bits), dmin*m (17 bits); high
-                    // nibbles arrive as 16*q, so their scale is divided by 16
-                    const float ds_lo = d * byte_float(scw, b0), dm_lo = dmin * byte_float(mw, b0);
-                    const float ds_hi = d * byte_float(scw, b0 + 1) * 0.0625f;
-                    const float dm_hi = dmin * byte_float(mw, b0 + 1);
-                    const float2 dsl = make_float2(ds_lo, ds_lo), dml = make_float2(-dm_lo, -dm_lo);
-                    const float2 dsh = make_float2(ds_hi, ds_hi), dmh = make_float2(-dm_hi, -dm_hi);
-                    uint32_t qw[NW];
-                    if constexpr (NW == 4) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * cc + QB * part);
-                        qw[0] = v.x; qw[1] = v.y; qw[2] = v.z; qw[3] = v.w;
-                    } else {
-                        const uint2 v = *reinterpret_cast<const uint2 *>(blk + 16 + 32 * cc + QB * part);
-                        qw[0] = v.x; qw[1] = v.y;
-                    }
-                    uint32_t lo_out[2 * NW], hi_out[2 * NW];
-                    #pragma unroll
-                    for (int wd = 0; wd < NW; ++wd) {
-                        const uint32_t lo = qw[wd] & 0x0F0F0F0Fu, hi = qw[wd] & 0xF0F0F0F0u;
+                    if ((int)(g & (DEC_GROUPS - 1)) == grp) {
+                        // warp-uniform outcome: the TMEM store below is .sync.aligned
+                        ok = __all_sync(0xffffffffu, mbar_wait(&empty_a[slot], phase ^ 1, p.err));
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t scw = cc < 2 ? sc_lo : sc_hi, mw = cc < 2 ? m_lo : m_hi;
+                        const int b0 = (2 * cc) & 3;
+                        // exact products: d*sc (17 bits), dmin*m (17 bits); high
+                        // nibbles arrive as 16*q, so their scale is divided by 16
+                        const float ds_lo = d * byte_float(scw, b0), dm_lo = dmin * byte_float(mw, b0);
+                        const float ds_hi = d * byte_float(scw, b0 + 1) * 0.0625f;
+                        const float dm_hi = dmin * byte_float(mw, b0 + 1);
+                        const float2 sl = make_float2(ds_lo, ds_lo), bl = make_float2(-dm_lo, -dm_lo);
+                        const float2 sh = make_float2(ds_hi, ds_hi), bh = make_float2(-dm_hi, -dm_hi);
+                        const uint4 v0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * cc);
+                        const uint4 v1 = *reinterpret_cast<const uint4 *>(blk + 32 + 32 * cc);
+                        const uint32_t qw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                        uint32_t out[32];
                         #pragma unroll
-                        for (int pr = 0; pr < 2; ++pr) {
-                            // bytes 2pr, 2pr+1 -> 2^23 + q (exact), minus 2^23 -> q
-                            float2 fl = make_float2(
-                                __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7440u + 2 * pr)),
-                                __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7441u + 2 * pr)));
-                            float2 fh = make_float2(
-                                __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7440u + 2 * pr)),
-                                __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7441u + 2 * pr)));
-                            fl = ffma2(fl, one, magic);
-                            fh = ffma2(fh, one, magic);
-                            const float2 wl = ffma2(fl, dsl, dml);  // one rounding each
-                            const float2 wh = ffma2(fh, dsh, dmh);
-                            const __nv_bfloat162 bl = __floats2bfloat162_rn(wl.x, wl.y);
-                            const __nv_bfloat162 bh = __floats2bfloat162_rn(wh.x, wh.y);
-                            lo_out[2 * wd + pr] = *reinterpret_cast<const uint32_t *>(&bl);
-                            hi_out[2 * wd + pr] = *reinterpret_cast<const uint32_t *>(&bh);
+                        for (int wd = 0; wd < 8; ++wd) {
+                            decode4(qw[wd] & 0x0F0F0F0Fu, sl, bl, out[2 * wd], out[2 * wd + 1]);
+                            decode4(qw[wd] & 0xF0F0F0F0u, sh, bh, out[16 + 2 * wd], out[17 + 2 * wd]);
                         }
+                        tmem_st32(t_lane + a_slot_col(slot, p.a_col0), out);
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&full_a[slot]);
                     }
-                    const uint32_t arow = smem_addr(a_ring + s * A_STAGE_BYTES + r * 128);
-                    #pragma unroll
-                    for (int j = 0; j < NW / 2; ++j) {  // 16-byte chunks: QB/8 low, QB/8 high
-                        const int c_lo = (QB / 8) * part + j, c_hi = 4 + (QB / 8) * part + j;
-                        st_shared_v4(arow + ((c_lo ^ (r & 7)) << 4), lo_out[4 * j], lo_out[4 * j + 1],
-                                     lo_out[4 * j + 2], lo_out[4 * j + 3]);
-                        st_shared_v4(arow + ((c_hi ^ (r & 7)) << 4), hi_out[4 * j], hi_out[4 * j + 1],
-                                     hi_out[4 * j + 2], hi_out[4 * j + 3]);
-                    }
-                    fence_proxy_async_smem();  // make the generic writes visible to the MMA
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&full[s]);
                     ++g;
+                    if (++slot == (uint32_t)SA) { slot = 0; phase ^= 1; }
                 }
                 if (!ok) break;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&raw_empty[rs]);
-                ++rsb;
+                if (++rs == RAW_STAGES) { rs = 0; rph ^= 1; }
             }
         }
     }
@@ -427,8 +529,8 @@ int pick_bn(int m, int n_tiles, int sms) {
 #ifdef KQ_GEMM_FORCE_BN
     return KQ_GEMM_FORCE_BN;
 #endif
-    static const int cands[] = {256, 224, 192, 176, 160, 128, 112, 96, 80, 64, 48, 32, 16};
-    int best = 256;
+    static const int cands[] = {192, 176, 160, 128, 112, 96, 80, 64, 48, 32, 16};
+    int best = cands[0];
     double best_cost = 1e30;
     for (int bn : cands) {
         if (bn > 16 && bn >= 2 * m + 16) continue;  // far wider than the problem
@@ -444,12 +546,19 @@ int pick_bn(int m, int n_tiles, int sms) {
     return best;
 }
 
-// Depth of the stage ring: as many (decoded A + activation B) stages as
-// shared memory holds next to the raw super-block ring, at most six.
-int stages_for(int bn) {
-    const int per = A_STAGE_BYTES + bn * 128;
-    const int st = (SMEM_BUDGET - 2048 - RAW_STAGES * RAW_STAGE_BYTES) / per;
-    return st > 6 ? 6 : st;
+// First TMEM column after an accumulator of bn columns (32-column aligned).
+int a_col0_for(int bn) { return (bn + 31) / 32 * 32; }
+
+// Ring depths: the A slots (32 TMEM columns each) that fit in the two gaps
+// after the accumulators, and as many activation tiles as shared memory
+// holds next to the raw ring (barriers and the row list take 2.25 KB).
+int a_stages_for(int bn) {
+    const int st = 2 * ((256 - a_col0_for(bn)) / 32);
+    return st < MAX_A_STAGES ? st : MAX_A_STAGES;
+}
+int b_stages_for(int bn) {
+    const int st = (SMEM_BUDGET - 1024 - 2304 - RAW_STAGES * RAW_STAGE_BYTES) / (bn * 128);
+    return st < MAX_B_STAGES ? st : MAX_B_STAGES;
 }
 
 }  // namespace
@@ -461,49 +570,52 @@ bool gemm_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype) {
     return encode_fn() != nullptr;
 }
 
-cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const void *x, int64_t m,
-                        void *y, int ydt, cudaStream_t s) {
-    (void)type;
-    auto enc = encode_fn();
-    if (!enc || m < 1 || m > (1 << 30)) return cudaErrorNotSupported;
-    const int sms = num_sms();
-    GemmParams p;
-    p.n = (int)n; p.k = (int)k; p.m = (int)m;
-    p.n_tiles = (int)((n + BM - 1) / BM);
-    p.bn = pick_bn((int)m, p.n_tiles, sms);
-    p.m_tiles = (int)((m + p.bn - 1) / p.bn);
-    p.tiles = p.n_tiles * p.m_tiles;
-    p.stages = stages_for(p.bn);
-    p.b_stage_bytes = p.bn * 128;
-    p.y = y;
-    p.err = error_word();
+namespace {
 
-    CUtensorMap tx, tw;
-    {
-        cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)m};
-        cuuint64_t strides[1] = {(cuuint64_t)k * 2};
-        cuuint32_t box[2] = {BK, (cuuint32_t)p.bn};
-        cuuint32_t es[2] = {1, 1};
-        if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box,
-                es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    {
-        const int64_t rb = (k / 256) * SB_BYTES;
-        cuuint64_t dims[2] = {(cuuint64_t)rb, (cuuint64_t)n};
-        cuuint64_t strides[1] = {(cuuint64_t)rb};
-        cuuint32_t box[2] = {SB_BYTES, BM};
-        cuuint32_t es[2] = {1, 1};
-        if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(w), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    const size_t smem = 1024 + (size_t)p.stages * (A_STAGE_BYTES + p.b_stage_bytes) +
-                        RAW_STAGES * RAW_STAGE_BYTES + 256;
+// Activations [rows, k] bf16: 64-column boxes of box_rows rows, 128-byte swizzle.
+bool encode_x_map(CUtensorMap *m, const void *x, int64_t rows, int64_t k, int box_rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)k * 2};
+    cuuint32_t box[2] = {BK, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box,
+                       es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Raw Q4_K rows of one or more experts: (row bytes, rows, experts), one
+// super-block column of BM rows per box.
+bool encode_w_map(CUtensorMap *m, const void *w, int64_t n, int64_t k, int64_t n_experts,
+                  int64_t expert_stride) {
+    const int64_t rb = (k / 256) * SB_BYTES;
+    cuuint64_t dims[3] = {(cuuint64_t)rb, (cuuint64_t)n, (cuuint64_t)n_experts};
+    cuuint64_t strides[2] = {(cuuint64_t)rb, (cuuint64_t)expert_stride};
+    cuuint32_t box[3] = {SB_BYTES, BM, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(w), dims, strides, box, es,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool fill_ring(GemmParams *p) {
+    p->a_stages = a_stages_for(p->bn);
+    p->b_stages = b_stages_for(p->bn);
+    p->a_col0 = a_col0_for(p->bn);
+    p->b_stage_bytes = p->bn * 128;
+    return p->bn <= MAX_BN && p->bn % 16 == 0 && p->a_stages >= 2 && p->b_stages >= 2;
+}
+
+template <typename YT, bool ID>
+cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const GemmParams &p, int grid,
+                          cudaStream_t s) {
+    // alignment slack, activation ring, raw ring, barriers (384 B) and the
+    // expert-indexed row list (768 B)
+    const size_t smem = 1024 + (size_t)p.b_stages * p.b_stage_bytes + RAW_STAGES * RAW_STAGE_BYTES + 384 + 1024;
+    auto kern = gemm_q4k_kernel<YT, ID>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.tiles < sms ? p.tiles : sms));
+    cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(NUM_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
@@ -512,16 +624,66 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (ydt == KQ_F32) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_q4k_kernel<float>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        return cudaLaunchKernelEx(&cfg, gemm_q4k_kernel<float>, tx, tw, p);
-    }
-    cudaError_t e = cudaFuncSetAttribute(gemm_q4k_kernel<__nv_bfloat16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, gemm_q4k_kernel<__nv_bfloat16>, tx, tw, p);
+    return cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const void *x, int64_t m,
+                        void *y, int ydt, cudaStream_t s) {
+    (void)type;
+    if (!encode_fn() || m < 1 || m > (1 << 30)) return cudaErrorNotSupported;
+    const int sms = num_sms();
+    GemmParams p = {};
+    p.n = (int)n; p.k = (int)k; p.m = (int)m;
+    p.n_tiles = (int)((n + BM - 1) / BM);
+    p.bn = pick_bn((int)m, p.n_tiles, sms);
+    p.m_tiles = (int)((m + p.bn - 1) / p.bn);
+    p.tiles = p.n_tiles * p.m_tiles;
+    if (!fill_ring(&p)) return cudaErrorNotSupported;
+    p.y = y;
+    p.err = error_word();
+    CUtensorMap tx, tw;
+    if (!encode_x_map(&tx, x, m, k, p.bn) || !encode_w_map(&tw, w, n, k, 1, n * ((k / 256) * SB_BYTES)))
+        return cudaErrorInvalidValue;
+    const int grid = p.tiles < sms ? p.tiles : sms;
+    return ydt == KQ_F32 ? launch_kernel<float, false>(tx, tw, p, grid, s)
+                         : launch_kernel<__nv_bfloat16, false>(tx, tw, p, grid, s);
+}
+
+int gemm_id_bn(int64_t n_tokens, int64_t top_k, int64_t n_experts) {
+    // about 1.5x the mean number of pairs per expert, in steps of 16
+    const int64_t pairs = n_tokens * top_k;
+    int64_t bn = (3 * pairs / (2 * n_experts) + 15) / 16 * 16;
+    if (bn < 16) bn = 16;
+    if (bn > 176) bn = 176;
+    return (int)bn;
+}
+
+cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
+    if (!encode_fn()) return cudaErrorNotSupported;
+    const int sms = num_sms();
+    GemmParams p = {};
+    p.n = (int)a.n; p.k = (int)a.k; p.m = (int)a.n_tokens;
+    p.n_tiles = (int)((a.n + BM - 1) / BM);
+    p.bn = bn;
+    if (!fill_ring(&p)) return cudaErrorNotSupported;
+    p.y = a.y;
+    p.err = error_word();
+    p.perm = a.perm;
+    p.offsets = a.offsets;
+    p.id_tiles = reinterpret_cast<const int2 *>(a.tiles);
+    p.id_n_tiles = a.n_tiles;
+    p.top_k = (int)a.top_k;
+    CUtensorMap tx, tw;
+    if (!encode_x_map(&tx, a.x, a.n_tokens, a.k, 1) ||
+        !encode_w_map(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride))
+        return cudaErrorInvalidValue;
+    // persistent grid: the number of token tiles is only known on the device
+    const int64_t max_units = (a.n_tokens * a.top_k / bn + a.n_experts) * p.n_tiles;
+    const int grid = (int)(max_units < sms ? max_units : sms);
+    return a.y_dtype == KQ_F32 ? launch_kernel<float, true>(tx, tw, p, grid, s)
+                               : launch_kernel<__nv_bfloat16, true>(tx, tw, p, grid, s);
 }
 
 }  // namespace kq

@@ -34,23 +34,26 @@ namespace kq {
 
 namespace {
 
-// A CTA takes at most half of an SM (threads, registers, shared memory), so
-// the next kernel's CTA can be resident beside it and start streaming its
-// weights while this one finishes (programmatic dependent launch).
-#ifndef KQ_GEMV_SMEM_LIMIT
-#define KQ_GEMV_SMEM_LIMIT (200 * 1024)
-#endif
-#ifndef KQ_GEMV_MAX_WARPS
-#define KQ_GEMV_MAX_WARPS 16
-#endif
-#ifndef KQ_GEMV_MIN_BLOCKS
-#define KQ_GEMV_MIN_BLOCKS 1
-#endif
+// Two CTA sizes.  A call ordered after the preceding kernel gets a whole
+// SM (16 warps, up to 200 KB of row slots): its latency is what counts.
+// Independent calls get a fraction of an SM (KQ_GEMV_SHARE_BLOCKS CTAs fit
+// on one: KQ_GEMV_SHARE_WARPS warps, at most 128 registers a thread, an
+// equal share of shared memory), so the next calls' CTAs are resident
+// beside this one and stream their weights while this one computes.
 #ifndef KQ_GEMV_XREG
 #define KQ_GEMV_XREG 1
 #endif
-constexpr int GEMV_SMEM_LIMIT = KQ_GEMV_SMEM_LIMIT;
-constexpr int GEMV_MAX_WARPS = KQ_GEMV_MAX_WARPS;
+#ifndef KQ_GEMV_SHARE_WARPS
+#define KQ_GEMV_SHARE_WARPS 4
+#endif
+#ifndef KQ_GEMV_SHARE_BLOCKS
+#define KQ_GEMV_SHARE_BLOCKS 3
+#endif
+constexpr int GEMV_SMEM_LIMIT = 200 * 1024;
+constexpr int GEMV_MAX_WARPS = 16;
+constexpr int GEMV_HALF_MAX_WARPS = KQ_GEMV_SHARE_WARPS;
+constexpr int GEMV_HALF_BLOCKS = KQ_GEMV_SHARE_BLOCKS;
+constexpr int GEMV_HALF_SMEM_LIMIT = (224 / GEMV_HALF_BLOCKS - 12) * 1024;
 constexpr int GEMV_MAX_SLOTS = 4;
 
 struct GemvParams {
@@ -65,6 +68,7 @@ struct GemvParams {
     int xq_bytes;     // staged int16 activations
     int xs_bytes;     // per-sub-block scales (and as many bytes again of sums)
     int early;        // issue weight copies before griddepcontrol.wait
+    int indep;        // independent call: no griddepcontrol.wait at all
     unsigned int *err;
     // expert-indexed mode (grid.y = expert): grouping from the device
     const int32_t *counts, *offsets, *perm;
@@ -261,7 +265,7 @@ __device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w,
                 prefetch_l2(src + off, (uint32_t)(bytes - off < 32768 ? bytes - off : 32768));
         }
     }
-    griddep_wait();
+    if (!p.indep) griddep_wait();
     // Otherwise the activation loads go out first (they gate every row) and
     // the row copies follow right behind them.
     stage_activations<C, TB, XT>(p, tok, xq, xsc, xsum, [&]() {
@@ -430,8 +434,10 @@ __device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w,
     return true;
 }
 
-template <int C, int TB, int R, bool XREG, typename XT, typename YT>
-__global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, KQ_GEMV_MIN_BLOCKS) gemv_q4k_kernel(const GemvParams p) {
+template <int C, int TB, int R, bool XREG, int MINB, typename XT, typename YT>
+__global__ void __launch_bounds__(MINB == 1 ? 32 * GEMV_MAX_WARPS : 32 * GEMV_HALF_MAX_WARPS, MINB)
+    gemv_q4k_kernel(const GemvParams p) {
+    static_assert(MINB == 1 || MINB == GEMV_HALF_BLOCKS, "whole-SM or shared-SM build");
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_tok[TB];
     __shared__ int64_t s_yrow[TB];
@@ -444,6 +450,9 @@ __global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, KQ_GEMV_MIN_BLOCKS) gemv_
     }
     __syncthreads();
     gemv_pass<C, TB, R, XREG, XT, YT>(p, p.w, row_begin, row_end, s_tok, s_yrow, smem, 0);
+    // An independent call still completes after the work before it, so that
+    // stream order holds for whatever follows.
+    if (p.indep) griddep_wait();
 }
 
 // Expert-indexed form: CTA (chunk, e) streams rows of expert e's slice once
@@ -483,7 +492,8 @@ int chunks_per_unit(int nb) { return nb >= 32 ? 4 : nb >= 16 ? 2 : 1; }
 int tb_for(int64_t m) { return m <= 1 ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : 8; }
 int rows_per_step(int tb) { return tb <= 2 ? 2 : 1; }
 
-bool plan_gemv(int type, int64_t n, int64_t k, int64_t m, int num_sms, GemvParams *p) {
+bool plan_gemv(int type, int64_t n, int64_t k, int64_t m, int num_sms, int max_warps,
+               int smem_limit, GemvParams *p) {
     if (type != KQ_Q4_K) return false;
     if (m < 1 || m > 8 || n < 1 || n > INT32_MAX / 2 || k > (1 << 20)) return false;
     const int tb = tb_for(m), R = rows_per_step(tb);
@@ -495,16 +505,16 @@ bool plan_gemv(int type, int64_t n, int64_t k, int64_t m, int num_sms, GemvParam
     const size_t xq_bytes = (size_t)tb * 8 * C * units_pad * 16;
     const size_t xs_bytes = (size_t)tb * units * 2 * C * 4;
     const size_t fixed = xq_bytes + 2 * xs_bytes;
-    if (fixed + 1024 >= GEMV_SMEM_LIMIT) return false;
-    int warps = rows_per_cta < GEMV_MAX_WARPS ? rows_per_cta : GEMV_MAX_WARPS;
+    if (fixed + 1024 >= (size_t)smem_limit) return false;
+    int warps = rows_per_cta < max_warps ? rows_per_cta : max_warps;
     for (; warps >= 1; --warps) {
         const int rows_per_warp = (rows_per_cta + warps - 1) / warps;
         const int want = rows_per_warp < GEMV_MAX_SLOTS ? rows_per_warp : GEMV_MAX_SLOTS;
         const int min_slots = rows_per_warp < R ? rows_per_warp : R;
         int slots = want;
-        while (slots > min_slots && fixed + (size_t)warps * slots * (row_bytes + 8) > GEMV_SMEM_LIMIT)
+        while (slots > min_slots && fixed + (size_t)warps * slots * (row_bytes + 8) > (size_t)smem_limit)
             --slots;
-        if (fixed + (size_t)warps * slots * (row_bytes + 8) <= GEMV_SMEM_LIMIT) {
+        if (fixed + (size_t)warps * slots * (row_bytes + 8) <= (size_t)smem_limit) {
             p->nb = nb; p->units = units; p->units_pad = units_pad; p->rows_per_cta = rows_per_cta;
             p->warps = warps; p->slots = slots; p->row_bytes = (int)row_bytes;
             p->xq_bytes = (int)xq_bytes; p->xs_bytes = (int)xs_bytes;
@@ -529,8 +539,11 @@ int sm_count() {
 }
 
 template <int C, int TB, bool XREG, typename XT, typename YT>
-cudaError_t launch_q4k(GemvParams p, bool const_w, cudaStream_t s) {
-    auto kern = gemv_q4k_kernel<C, TB, TB <= 2 ? 2 : 1, XREG, XT, YT>;
+cudaError_t launch_q4k(GemvParams p, GemvOrder order, cudaStream_t s) {
+    // half-SM build when the plan fits it (independent calls)
+    auto kern = p.warps <= GEMV_HALF_MAX_WARPS && order == GemvOrder::kIndependent
+                    ? gemv_q4k_kernel<C, TB, TB <= 2 ? 2 : 1, XREG, GEMV_HALF_BLOCKS, XT, YT>
+                    : gemv_q4k_kernel<C, TB, TB <= 2 ? 2 : 1, XREG, 1, XT, YT>;
     const size_t smem = (size_t)p.xq_bytes + 2 * (size_t)p.xs_bytes +
                         (size_t)p.warps * p.slots * ((size_t)p.row_bytes + 8);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -542,36 +555,38 @@ cudaError_t launch_q4k(GemvParams p, bool const_w, cudaStream_t s) {
     cfg.stream = s;
     // Programmatic overlap with the preceding kernel is always allowed: the
     // kernel reads nothing produced by earlier work before griddepcontrol.wait,
-    // except the weights when the caller declared them constant.
+    // except the weights when the caller declared them constant, and waits
+    // not at all when the caller declared the call independent.
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    p.early = const_w ? 1 : 0;
+    p.early = order != GemvOrder::kStream ? 1 : 0;
+    p.indep = order == GemvOrder::kIndependent ? 1 : 0;
     p.err = error_word();
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 template <int C, typename XT, typename YT>
-cudaError_t dispatch_tb(GemvParams p, int tb, bool const_w, cudaStream_t s) {
+cudaError_t dispatch_tb(GemvParams p, int tb, GemvOrder order, cudaStream_t s) {
     switch (tb) {
     case 1:
         if (KQ_GEMV_XREG && C <= 2 && p.units <= 32)
-            return launch_q4k<C, 1, (KQ_GEMV_XREG && C <= 2), XT, YT>(p, const_w, s);
-        return launch_q4k<C, 1, false, XT, YT>(p, const_w, s);
-    case 2: return launch_q4k<C, 2, false, XT, YT>(p, const_w, s);
-    case 4: return launch_q4k<C, 4, false, XT, YT>(p, const_w, s);
-    default: return launch_q4k<C, 8, false, XT, YT>(p, const_w, s);
+            return launch_q4k<C, 1, (KQ_GEMV_XREG && C <= 2), XT, YT>(p, order, s);
+        return launch_q4k<C, 1, false, XT, YT>(p, order, s);
+    case 2: return launch_q4k<C, 2, false, XT, YT>(p, order, s);
+    case 4: return launch_q4k<C, 4, false, XT, YT>(p, order, s);
+    default: return launch_q4k<C, 8, false, XT, YT>(p, order, s);
     }
 }
 
 template <typename XT, typename YT>
-cudaError_t dispatch_c(GemvParams p, int tb, bool const_w, cudaStream_t s) {
+cudaError_t dispatch_c(GemvParams p, int tb, GemvOrder order, cudaStream_t s) {
     switch (chunks_per_unit(p.nb)) {
-    case 4: return dispatch_tb<4, XT, YT>(p, tb, const_w, s);
-    case 2: return dispatch_tb<2, XT, YT>(p, tb, const_w, s);
-    default: return dispatch_tb<1, XT, YT>(p, tb, const_w, s);
+    case 4: return dispatch_tb<4, XT, YT>(p, tb, order, s);
+    case 2: return dispatch_tb<2, XT, YT>(p, tb, order, s);
+    default: return dispatch_tb<1, XT, YT>(p, tb, order, s);
     }
 }
 
@@ -579,30 +594,36 @@ cudaError_t dispatch_c(GemvParams p, int tb, bool const_w, cudaStream_t s) {
 
 bool gemv_supported(int type, int64_t n, int64_t k, int x_dtype, int64_t m) {
     (void)x_dtype;
+    if (type == KQ_TQ1_G128) return m >= 1 && gemv_tq1_supported(n, k);
     GemvParams p;
-    return m >= 1 && plan_gemv(type, n, k, m < 8 ? m : 8, sm_count(), &p);
+    return m >= 1 && plan_gemv(type, n, k, m < 8 ? m : 8, sm_count(), GEMV_MAX_WARPS, GEMV_SMEM_LIMIT, &p);
 }
 
 // More than eight activation rows run as consecutive launches of up to eight
 // rows each (the weights are streamed once per launch).
 cudaError_t launch_gemv(int type, const void *w, int64_t n, int64_t k, const void *x, int xdt,
-                        int64_t m, void *y, int ydt, bool const_w, cudaStream_t s) {
+                        int64_t m, void *y, int ydt, GemvOrder order, cudaStream_t s) {
+    if (type == KQ_TQ1_G128) return launch_gemv_tq1(w, n, k, x, xdt, m, y, ydt, order, s);
+    const bool half = order == GemvOrder::kIndependent;
     const size_t xs = (xdt == KQ_F32 ? 4 : 2), ys = (ydt == KQ_F32 ? 4 : 2);
     for (int64_t m0 = 0; m0 < m; m0 += 8) {
         const int64_t mc = m - m0 < 8 ? m - m0 : 8;
         GemvParams p = {};
         const int tb = tb_for(mc);
-        if (!plan_gemv(type, n, k, mc, sm_count(), &p)) return cudaErrorNotSupported;
+        // independent calls take the half-SM plan when it fits, else a whole SM
+        if (!(half && plan_gemv(type, n, k, mc, sm_count(), GEMV_HALF_MAX_WARPS, GEMV_HALF_SMEM_LIMIT, &p)) &&
+            !plan_gemv(type, n, k, mc, sm_count(), GEMV_MAX_WARPS, GEMV_SMEM_LIMIT, &p))
+            return cudaErrorNotSupported;
         p.w = static_cast<const uint8_t *>(w);
         p.x = static_cast<const char *>(x) + (size_t)m0 * (size_t)k * xs;
         p.y = static_cast<char *>(y) + (size_t)m0 * (size_t)n * ys;
         cudaError_t e;
         if (xdt == KQ_F32) {
-            e = ydt == KQ_F32 ? dispatch_c<float, float>(p, tb, const_w, s)
-                              : dispatch_c<float, __nv_bfloat16>(p, tb, const_w, s);
+            e = ydt == KQ_F32 ? dispatch_c<float, float>(p, tb, order, s)
+                              : dispatch_c<float, __nv_bfloat16>(p, tb, order, s);
         } else {
-            e = ydt == KQ_F32 ? dispatch_c<__nv_bfloat16, float>(p, tb, const_w, s)
-                              : dispatch_c<__nv_bfloat16, __nv_bfloat16>(p, tb, const_w, s);
+            e = ydt == KQ_F32 ? dispatch_c<__nv_bfloat16, float>(p, tb, order, s)
+                              : dispatch_c<__nv_bfloat16, __nv_bfloat16>(p, tb, order, s);
         }
         if (e != cudaSuccess) return e;
     }
@@ -612,16 +633,17 @@ cudaError_t launch_gemv(int type, const void *w, int64_t n, int64_t k, const voi
 namespace {
 
 constexpr int ID_TB = 4;  // (token, slot) pairs per pass over an expert's rows
+constexpr int ID_R = 2;   // weight rows per step: each staged activation load serves two rows
 
-// Grid (chunks, E): about two CTAs per SM if every expert were hit; eight
-// warps per CTA so that two CTAs fit on an SM.
+// Grid (chunks, E): at most two CTAs per SM if every expert were hit (one
+// wave); eight warps per CTA so that two CTAs fit on an SM.
 bool plan_gemv_id(int type, int64_t n, int64_t k, int64_t n_experts, int num_sms, GemvParams *p) {
     if (type != KQ_Q4_K || n < 1 || n > INT32_MAX / 2 || k > (1 << 20) || n_experts < 1) return false;
     const int nb = (int)(k / 256);
     const int C = chunks_per_unit(nb);
     const int units = nb * 4 / C, units_pad = (units + 7) / 8 * 8;
     const int64_t row_bytes = (int64_t)nb * 144;
-    int64_t chunks = (2 * num_sms + n_experts - 1) / n_experts;
+    int64_t chunks = (2 * num_sms) / n_experts;
     if (chunks < 1) chunks = 1;
     if (chunks > n) chunks = n;
     const int rows_per_cta = (int)((n + chunks - 1) / chunks);
@@ -633,7 +655,8 @@ bool plan_gemv_id(int type, int64_t n, int64_t k, int64_t n_experts, int num_sms
     const int warps = rows_per_cta < 8 ? rows_per_cta : 8;
     const int rows_per_warp = (rows_per_cta + warps - 1) / warps;
     int slots = rows_per_warp < GEMV_MAX_SLOTS ? rows_per_warp : GEMV_MAX_SLOTS;
-    while (slots > 1 && fixed + (size_t)warps * slots * (row_bytes + 8) > limit) --slots;
+    const int min_slots = rows_per_warp < ID_R ? rows_per_warp : ID_R;  // a step holds ID_R rows
+    while (slots > min_slots && fixed + (size_t)warps * slots * (row_bytes + 8) > limit) --slots;
     if (fixed + (size_t)warps * slots * (row_bytes + 8) > limit) return false;
     p->nb = nb; p->units = units; p->units_pad = units_pad; p->rows_per_cta = rows_per_cta;
     p->warps = warps; p->slots = slots; p->row_bytes = (int)row_bytes;
@@ -644,7 +667,7 @@ bool plan_gemv_id(int type, int64_t n, int64_t k, int64_t n_experts, int num_sms
 
 template <int C, typename XT, typename YT>
 cudaError_t launch_id_q4k(GemvParams p, int64_t n_experts, cudaStream_t s) {
-    auto kern = gemv_id_q4k_kernel<C, ID_TB, 1, XT, YT>;
+    auto kern = gemv_id_q4k_kernel<C, ID_TB, ID_R, XT, YT>;
     const size_t smem = (size_t)p.xq_bytes + 2 * (size_t)p.xs_bytes +
                         (size_t)p.warps * p.slots * ((size_t)p.row_bytes + 8);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

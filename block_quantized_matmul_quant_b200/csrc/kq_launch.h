@@ -30,14 +30,27 @@ cudaError_t launch_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_expe
                              int32_t *counts, int32_t *offsets, int32_t *perm, void *y,
                              int y_dtype, int64_t n, cudaStream_t s);
 cudaError_t launch_simple_id(const IdArgs &a, cudaStream_t s);
+// Token tiles of at most bn pairs per expert segment, (expert, first
+// position in perm) each, and their number -- from the grouping's offsets.
+cudaError_t launch_moe_tiles(const int32_t *offsets, int64_t n_experts, int bn, int32_t *tiles,
+                             int32_t *n_tiles, cudaStream_t s);
 
 // Bandwidth kernels (kq_gemv.cu).  Return cudaErrorNotSupported when the
 // shape is outside what the kernel serves.
 bool gemv_supported(int type, int64_t n, int64_t k, int x_dtype, int64_t m);
-// const_w: weights are not written by earlier work on the stream, so the
-// kernel may prefetch them before the preceding kernel completes (PDL).
+// How a bandwidth-kernel call is ordered against earlier work on its stream:
+//   kStream        read everything after the preceding kernel completes;
+//   kConstWeights  weights are never written by earlier work: stream them
+//                  before the preceding kernel completes (PDL), x after;
+//   kIndependent   nothing earlier touches w, x or y: never wait, and use a
+//                  half-SM CTA so consecutive calls run side by side.
+enum class GemvOrder { kStream, kConstWeights, kIndependent };
 cudaError_t launch_gemv(int type, const void *w, int64_t n, int64_t k, const void *x, int xdt,
-                        int64_t m, void *y, int ydt, bool const_w, cudaStream_t s);
+                        int64_t m, void *y, int ydt, GemvOrder order, cudaStream_t s);
+// TQ1_G128 bandwidth kernel (kq_gemv_tq1.cu); launch_gemv routes to it.
+bool gemv_tq1_supported(int64_t n, int64_t k);
+cudaError_t launch_gemv_tq1(const void *w, int64_t n, int64_t k, const void *x, int xdt, int64_t m,
+                            void *y, int ydt, GemvOrder order, cudaStream_t s);
 bool gemv_id_supported(int type, int64_t k, int x_dtype);
 cudaError_t launch_gemv_id(const IdArgs &a, cudaStream_t s);
 
@@ -45,5 +58,9 @@ cudaError_t launch_gemv_id(const IdArgs &a, cudaStream_t s);
 bool gemm_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype);
 cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const void *x, int64_t m,
                         void *y, int ydt, cudaStream_t s);
+// Expert-indexed form over the grouping's token tiles (a.tiles / a.n_tiles,
+// written by launch_moe_tiles with the same bn).
+int gemm_id_bn(int64_t n_tokens, int64_t top_k, int64_t n_experts);
+cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s);
 
 }  // namespace kq

@@ -105,6 +105,55 @@ cudaError_t launch_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_expe
     return cudaGetLastError();
 }
 
+// Token tiles for the tensor-core expert product: expert e's segment
+// [offsets[e], offsets[e+1]) of the grouped pair list splits into
+// ceil(count / bn) tiles.  One CTA; warp 0 scans the per-expert tile counts
+// 32 experts at a time, then every thread writes the tiles of its experts.
+constexpr int TILE_THREADS = 256;
+
+__global__ void __launch_bounds__(TILE_THREADS) moe_tiles_kernel(const int32_t *__restrict__ offsets,
+                                                                 int n_experts, int bn,
+                                                                 int2 *__restrict__ tiles,
+                                                                 int32_t *__restrict__ n_tiles) {
+    extern __shared__ int s_first[];  // n_experts: first tile index of each expert
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x < 32) {
+        int carry = 0;
+        for (int base = 0; base < n_experts; base += 32) {
+            const int e = base + lane;
+            const int c = e < n_experts ? (offsets[e + 1] - offsets[e] + bn - 1) / bn : 0;
+            int incl = c;
+            #pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            if (e < n_experts) s_first[e] = carry + incl - c;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) *n_tiles = carry;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < n_experts; e += blockDim.x) {
+        const int p0 = offsets[e], p1 = offsets[e + 1];
+        int i = s_first[e];
+        for (int q = p0; q < p1; q += bn) tiles[i++] = make_int2(e, q);
+    }
+}
+
+cudaError_t launch_moe_tiles(const int32_t *offsets, int64_t n_experts, int bn, int32_t *tiles,
+                             int32_t *n_tiles, cudaStream_t s) {
+    const size_t smem = sizeof(int) * (size_t)n_experts;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(moe_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    moe_tiles_kernel<<<1, TILE_THREADS, smem, s>>>(offsets, (int)n_experts, bn,
+                                                   reinterpret_cast<int2 *>(tiles), n_tiles);
+    return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- plain grouped product
 // Grid (ceil(n / 8), n_experts): warp = one weight row of expert e; it walks
 // the pairs routed to e four at a time.

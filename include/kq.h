@@ -79,6 +79,14 @@ extern "C" {
  * kernel has finished (programmatic dependent launch); x is still read only
  * after the preceding work completes. */
 #define KQ_FLAG_CONST_WEIGHTS 0x100
+/* Flag OR-ed into `path`: the call is independent of everything enqueued
+ * before it on the stream -- no earlier work writes w or x, or reads or
+ * writes y (e.g. separate projections of one activation, or a batch of
+ * weight matrices).  The kernel then never waits for the preceding kernel:
+ * consecutive independent calls stream their weights concurrently.  Implies
+ * KQ_FLAG_CONST_WEIGHTS.  Honoured by the bandwidth kernel; other paths
+ * keep stream order. */
+#define KQ_FLAG_INDEPENDENT 0x200
 
 /* Weights per block and bytes per block of a codec; 0 for an unknown codec. */
 KQ_API int kq_block_weights(int type);

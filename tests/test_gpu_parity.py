@@ -96,6 +96,7 @@ GEMV_CASES = [
     # (n, k, m): several CTAs, ragged row counts, 1..32+ blocks per row
     (300, 256, 1), (1000, 1024, 1), (4099, 4096, 1), (777, 2048, 2), (513, 4096, 3),
     (1500, 9216, 1), (640, 8192, 4), (257, 4096, 8), (5, 512, 5), (2000, 11008 // 256 * 256, 1),
+    (640, 1024, 19),   # more than eight activation rows: consecutive launches of eight
 ]
 
 
@@ -109,12 +110,77 @@ def test_matmul_gemv_q4_k(kq, n, k, m, xdt):
     x = synth.gen_x(m, k, xdt, r)
     ref = oracle.matmul(synth.Q4_K, w, k, x, threads=8)
     wd, xd = to_device_w(w), to_device_x(x, xdt)
-    for flags in (False, True):
-        y = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV, const_weights=flags).cpu().numpy()
+    ys = []
+    for cw, ind in ((False, False), (True, False), (False, True)):
+        y = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV, const_weights=cw,
+                      independent=ind).cpu().numpy()
         err = row_rel_err(y, ref)
         assert err <= GEMV_TOL, err
+        ys.append(y)
+    # every ordering mode computes each row the same way: identical bits
+    assert all(np.array_equal(ys[0].view(np.uint32), yy.view(np.uint32)) for yy in ys[1:])
     yb = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV, out_dtype=torch.bfloat16).float().cpu().numpy()
     assert row_rel_err(yb, ref) <= TOL[xdt] + BF16_OUT
+
+
+TQ1_GEMV_CASES = [
+    # (n, k, m): one block, a ragged last lane step, several steps per row,
+    # rows not a multiple of the SM count, two rows per launch and a third
+    (5, 128, 1), (300, 1280, 1), (777, 4096 + 128, 2), (1000, 17408, 1), (129, 8192, 3),
+]
+
+
+@pytest.mark.parametrize("n,k,m", TQ1_GEMV_CASES)
+@pytest.mark.parametrize("xdt", ["f32", "bf16"])
+def test_matmul_gemv_tq1(kq, n, k, m, xdt):
+    import torch
+
+    r = rng(3 * n + k + m)
+    w = synth.gen_weights(synth.TQ1_G128, n, k, r)
+    # illegal code bytes decode to zero: a full byte and a tail byte
+    w[0, 5] = 243
+    w[n - 1, (k // 128 - 1) * 28 + 25] = 27
+    x = synth.gen_x(m, k, xdt, r)
+    ref = oracle.matmul(synth.TQ1_G128, w, k, x, threads=8)
+    wd, xd = to_device_w(w), to_device_x(x, xdt)
+    ys = []
+    for cw, ind in ((False, False), (True, False), (False, True)):
+        y = kq.matmul(wd, synth.TQ1_G128, xd, path=kq.PATH_GEMV, const_weights=cw,
+                      independent=ind).cpu().numpy()
+        assert row_rel_err(y, ref) <= GEMV_TOL
+        ys.append(y)
+    assert all(np.array_equal(ys[0].view(np.uint32), yy.view(np.uint32)) for yy in ys[1:])
+    yb = kq.matmul(wd, synth.TQ1_G128, xd, path=kq.PATH_GEMV,
+                   out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert row_rel_err(yb, ref) <= TOL[xdt] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+def test_matmul_gemv_independent_calls_back_to_back(kq):
+    """Many independent calls queued on one stream (they run side by side),
+    then an ordinary call, queued right behind them, that reads the first
+    call's output as its activations: every result must be the one computed
+    alone, and the ordinary call must see the finished output."""
+    import torch
+
+    r = rng(23)
+    n = k = 4096
+    ws = [synth.gen_weights(synth.Q4_K, n, k, r) for _ in range(3)]
+    x = synth.gen_x(1, k, "bf16", r)
+    wds = [to_device_w(w) for w in ws]
+    xd = to_device_x(x, "bf16")
+    alone = [kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV).cpu().numpy() for wd in wds]
+    outs = [torch.full((1, n), float("nan"), device="cuda") for _ in range(24)]
+    y2 = torch.empty((1, n), device="cuda")
+    torch.cuda.synchronize()
+    for i, o in enumerate(outs):
+        kq.matmul(wds[i % 3], synth.Q4_K, xd, out=o, path=kq.PATH_GEMV, independent=True)
+    kq.matmul(wds[1], synth.Q4_K, outs[0], out=y2, path=kq.PATH_GEMV)   # fp32 x = outs[0]
+    for i, o in enumerate(outs):
+        assert np.array_equal(o.cpu().numpy().view(np.uint32), alone[i % 3].view(np.uint32))
+    ref2 = oracle.matmul(synth.Q4_K, ws[1], k, alone[0].astype(np.float64), threads=8)
+    assert row_rel_err(y2.cpu().numpy(), ref2) <= GEMV_TOL
+    assert kq.device_status() == 0
 
 
 def test_matmul_gemv_deterministic(kq):
@@ -269,7 +335,113 @@ def test_matmul_id_small(kq, codec, path):
     p = {"simple": kq.PATH_SIMPLE, "auto": kq.PATH_AUTO}[path]
     y = kq.matmul_id(to_device_w(w), codec, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
                      path=p).cpu().numpy()
-    assert row_rel_err(y, ref) <= FP32_PATH_TOL
+    assert row_rel_err(y, ref) <= (GEMV_TOL if (path == "auto" and codec == synth.Q4_K) else FP32_PATH_TOL)
+    assert kq.device_status() == 0
+
+
+@pytest.mark.parametrize("t,top_k,e,n,k", [
+    (32, 6, 64, 1408, 2048),   # the MoE workload's shape
+    (20, 4, 5, 300, 1024),     # ~16 pairs per expert: about four passes of four
+    (24, 2, 3, 5000, 512),     # 7 rows per warp through 4 slots, over several passes
+    (3, 2, 40, 257, 4096),     # most experts hit by nobody
+    (7, 3, 4, 129, 512),
+])
+@pytest.mark.parametrize("xdt", ["f32", "bf16"])
+def test_matmul_id_grouped_gemv(kq, t, top_k, e, n, k, xdt):
+    import torch
+
+    r = rng(t + e + n)
+    w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, xdt, r)
+    ids = synth.gen_ids(t, top_k, e, r)
+    ref = oracle.matmul_id(synth.Q4_K, w, k, x, ids)
+    wd, xd, idd = to_device_w(w), to_device_x(x, xdt), torch.from_numpy(ids).cuda()
+    y = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMV).cpu().numpy()
+    assert row_rel_err(y, ref) <= GEMV_TOL
+    y2 = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMV).cpu().numpy()
+    assert np.array_equal(y.view(np.uint32), y2.view(np.uint32))   # deterministic
+    yb = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMV,
+                      out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert row_rel_err(yb, ref) <= TOL[xdt] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+def _bf16_weight_reference_id(w, k, x, ids):
+    """y[t, s] = x[t] @ bf16(decode_f32(w[ids[t, s]]))^T in fp64 (NaN rows for
+    ids outside [0, E)): the tensor-core expert product up to fp32 accumulation."""
+    e_n = w.shape[0]
+    ref = np.full(ids.shape + (w.shape[1],), np.nan)
+    for e in range(e_n):
+        hit = ids == e
+        if hit.any():
+            ye = _bf16_weight_reference(w[e], k, x)   # [T, n]
+            ref[hit] = ye[np.nonzero(hit)[0]]
+    return ref
+
+
+@pytest.mark.parametrize("t,top_k,e,n,k,skew", [
+    (512, 6, 64, 384, 2048, False),    # the MoE routing at prefill length (3 weight tiles)
+    (100, 2, 3, 300, 1024, False),     # ragged weight rows, ~66 pairs per expert
+    (64, 4, 8, 129, 512, False),
+    (7, 3, 4, 129, 512, False),        # a handful of pairs: token tiles of 16
+    (300, 1, 4, 256, 512, True),       # one expert takes almost every token
+])
+def test_matmul_id_grouped_gemm(kq, t, top_k, e, n, k, skew):
+    import torch
+
+    r = rng(7 * t + e + n)
+    w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, "bf16", r)
+    ids = synth.gen_ids(t, top_k, e, r)
+    if skew:
+        ids[:, 0] = np.where(np.arange(t) % 50 == 0, 1, 2)
+    ref = oracle.matmul_id(synth.Q4_K, w, k, x, ids)
+    wd, xd, idd = to_device_w(w), to_device_x(x, "bf16"), torch.from_numpy(ids).cuda()
+    y = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMM).cpu().numpy()
+    assert row_rel_err(y, ref) <= TOL["bf16"]
+    assert row_rel_err(y, _bf16_weight_reference_id(w, k, x, ids)) <= FP32_PATH_TOL
+    y2 = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMM).cpu().numpy()
+    assert np.array_equal(y.view(np.uint32), y2.view(np.uint32))   # deterministic
+    yb = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMM,
+                      out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert row_rel_err(yb, ref) <= TOL["bf16"] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+def test_matmul_id_auto_uses_tensor_cores_for_long_prefill(kq):
+    import torch
+
+    t, top_k, e, n, k = 512, 6, 64, 256, 1024   # 48 pairs per expert on average
+    r = rng(99)
+    w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, "bf16", r)
+    ids = synth.gen_ids(t, top_k, e, r)
+    y = kq.matmul_id(to_device_w(w), synth.Q4_K, to_device_x(x, "bf16"),
+                     torch.from_numpy(ids).cuda()).cpu().numpy()
+    # equal to the bf16-weight product: the tensor-core path ran
+    assert row_rel_err(y, _bf16_weight_reference_id(w, k, x, ids)) <= FP32_PATH_TOL
+    assert kq.device_status() == 0
+
+
+@pytest.mark.parametrize("path", ["auto", "gemm"])
+def test_matmul_id_bad_ids_poison_rows_bf16(kq, path):
+    import torch
+
+    e, n, k, t = 4, 140, 512, 40
+    r = rng(12)
+    w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, "bf16", r)
+    ids = synth.gen_ids(t, 2, e, r)
+    ids[1, 0] = 4
+    ids[30, 1] = -7
+    p = {"auto": kq.PATH_AUTO, "gemm": kq.PATH_GEMM}[path]
+    y = kq.matmul_id(to_device_w(w), synth.Q4_K, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
+                     path=p).cpu().numpy()
+    ref = oracle.matmul_id(synth.Q4_K, w, k, x, ids)
+    assert np.all(np.isnan(y[1, 0])) and np.all(np.isnan(y[30, 1]))
+    good = ~np.isnan(ref[..., 0])
+    assert row_rel_err(y[good], ref[good]) <= TOL["bf16"]
+    assert kq.device_status() == -9    # KQ_ERR_DEVICE, then cleared
     assert kq.device_status() == 0
 
 
@@ -288,7 +460,7 @@ def test_matmul_id_bad_ids_poison_rows(kq):
     ref = oracle.matmul_id(synth.Q4_K, w, k, x, ids)
     assert np.all(np.isnan(y[1, 0])) and np.all(np.isnan(y[3, 1]))
     good = ~np.isnan(ref[..., 0])
-    assert row_rel_err(y[good], ref[good]) <= FP32_PATH_TOL
+    assert row_rel_err(y[good], ref[good]) <= GEMV_TOL
     assert kq.device_status() == -9    # KQ_ERR_DEVICE, then cleared
     assert kq.device_status() == 0
 
