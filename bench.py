@@ -229,6 +229,9 @@ class PoolStep:
         ydt = torch.float32 if wl.y_dtype == "f32" else torch.bfloat16
         shape = (wl.m, wl.top_k, wl.n) if wl.kind == "moe" else (wl.m, wl.n)
         self.y = torch.empty(shape, dtype=ydt, device="cuda")
+        # independent calls must not share an output buffer
+        self.ys = [torch.empty(shape, dtype=ydt, device="cuda") for _ in range(self.pool)] \
+            if wl.kind == "gemv" else None
         if wl.kind == "moe":
             self.ws_bytes = kq.matmul_id_workspace_bytes(wl.m, wl.top_k, wl.n_experts)
             self.scratch = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
@@ -239,6 +242,9 @@ class PoolStep:
             if self.wl.kind == "moe":
                 self.kq.matmul_id(self.ws[i], self.wl.codec, self.x, self.ids, out=self.y,
                                   workspace=self.scratch)
+            elif self.wl.kind == "gemv":
+                # the pool's calls are unrelated, as in the headline step
+                self.kq.matmul(self.ws[i], self.wl.codec, self.x, out=self.ys[i], independent=True)
             else:
                 self.kq.matmul(self.ws[i], self.wl.codec, self.x, out=self.y, const_weights=True)
 

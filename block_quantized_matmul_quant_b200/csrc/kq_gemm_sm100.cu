@@ -64,6 +64,10 @@ constexpr int MAX_A_STAGES = 8;   // TMEM A slots
 constexpr int MAX_B_STAGES = 10;  // activation tiles in shared memory
 constexpr int MAX_BN = 192;
 constexpr int SMEM_BUDGET = 227 * 1024;
+// Epilogue staging: each epilogue warp owns two buffers of one 16-token x
+// 32-row output chunk, written to global memory by TMA stores.
+constexpr int EPI_CHUNK_M = 16, EPI_CHUNK_N = 32;
+constexpr int EPI_STAGE_BYTES = 2 * 4 * EPI_CHUNK_M * EPI_CHUNK_N * 4;  // 2 buffers x 4 warps, f32 size
 
 struct GemmParams {
     int n, k, m;
@@ -74,6 +78,7 @@ struct GemmParams {
     int b_stage_bytes;
     void *y;
     unsigned int *err;
+    int y_tma;     // dense output through TMA stores (tmap_y) instead of per-element stores
     // expert-indexed mode: token tiles come from the device-side grouping
     const int32_t *perm;      // pair indices t * top_k + s, grouped by expert
     const int32_t *offsets;   // [E + 1] segment starts in perm
@@ -125,6 +130,19 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
         : "memory");
 }
+// Shared memory -> global tile store (bulk group), and its completion waits.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_addr(src))
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_le1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Four rows r0..r3 (columns x.. of a box one row high) into four consecutive
 // 128-byte rows of shared memory.
 __device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int x, int r0, int r1,
@@ -246,14 +264,16 @@ __device__ __forceinline__ void decode4(uint32_t nib, float2 scale, float2 bias,
 template <typename YT, bool ID>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_q4k_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                    const __grid_constant__ CUtensorMap tmap_w, const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmap_w,
+                    const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     const int SA = p.a_stages, SB = p.b_stages;
     uint8_t *b_ring = smem;                                    // SB x bn*128
     uint8_t *raw_ring = b_ring + SB * p.b_stage_bytes;         // RAW_STAGES x 18 KB
-    uint64_t *bars = reinterpret_cast<uint64_t *>(raw_ring + RAW_STAGES * RAW_STAGE_BYTES);
+    uint8_t *epi_stage = raw_ring + RAW_STAGES * RAW_STAGE_BYTES;  // EPI_STAGE_BYTES
+    uint64_t *bars = reinterpret_cast<uint64_t *>(epi_stage + EPI_STAGE_BYTES);
     uint64_t *full_a = bars;                 // [SA] one decoder group (4 warps) -> MMA
     uint64_t *empty_a = full_a + SA;         // [SA] MMA -> decoders
     uint64_t *full_b = empty_a + SA;         // [SB] TMA bytes -> MMA
@@ -291,6 +311,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (warp == 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+        if (p.y_tma)
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_y)) : "memory");
     }
     tc_fence_before();
     __syncthreads();
@@ -390,8 +412,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else if (warp < EPI_WARP0 + 4) {
         // ---------------- epilogue ----------------
+        // Warp q drains TMEM lanes 32q..32q+31 (weight rows n0+32q..) 16
+        // tokens at a time.  Dense outputs go through shared memory: the
+        // chunk is written as [16 tokens][32 rows] and one TMA store moves it
+        // (two buffers per warp, so converting the next chunk overlaps the
+        // store of this one).  Expert-indexed outputs scatter rows and are
+        // stored element by element.
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
         YT *y = static_cast<YT *>(p.y);
+        YT *stage = reinterpret_cast<YT *>(epi_stage) + (size_t)(warp - EPI_WARP0) * 2 * EPI_CHUNK_M * EPI_CHUNK_N;
+        int sbuf = 0;
         int tl = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x, ++tl) {
             const int acc = tl & 1;
@@ -404,7 +434,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int c0 = 0; c0 < p.bn; c0 += 16) {
                 uint32_t r[16];
                 tmem_ld16(t_row + (uint32_t)c0, r);
-                if (n < p.n) {
+                if (!ID && p.y_tma) {
+                    if (c0 >= t.rows) continue;   // tokens past the end: nothing to store
+                    if (lane == 0) bulk_wait_read_le1();   // this buffer's previous store has read it
+                    __syncwarp();
+                    YT *buf = stage + sbuf * EPI_CHUNK_M * EPI_CHUNK_N;
+                    #pragma unroll
+                    for (int j = 0; j < 16; ++j) store_out(buf + j * EPI_CHUNK_N + lane, __uint_as_float(r[j]));
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    // the map clips rows past n and tokens past m
+                    if (lane == 0 && t.n0 + 32 * q < p.n) tma_store_2d(&tmap_y, buf, t.n0 + 32 * q, t.m0 + c0);
+                    sbuf ^= 1;
+                } else if (n < p.n) {
                     #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         if (c0 + j < t.rows) {
@@ -419,6 +461,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[acc]);
         }
+        if (lane == 0) bulk_wait_all();   // stores have read shared memory before the CTA exits
     } else {
         // ---------------- decoders ----------------
         // Group grp (four consecutive warps, one per TMEM lane quadrant)
@@ -523,12 +566,17 @@ int num_sms() {
     return cached[dev];
 }
 
-// Choose BN (tokens per tile) minimising rounds * BN over the SMs, with a
-// small charge per extra token tile (each one re-decodes the weight tile).
+// Choose BN (tokens per tile).  A stage of a tile costs about the larger of
+// its MMAs (4 x BN/2 cycles for 128 x BN x 64) and the decode of its 128 x 64
+// weights, which does not shrink with BN (about 400 cycles, measured): the
+// cost of a shape is rounds of tiles over the SMs x that per-stage cost, so
+// extra token tiles (each one decodes its weight tile again) must buy fewer
+// rounds.  Ties go to the narrower tile.
 int pick_bn(int m, int n_tiles, int sms) {
 #ifdef KQ_GEMM_FORCE_BN
     return KQ_GEMM_FORCE_BN;
 #endif
+    constexpr double DECODE_CYCLES_PER_STAGE = 400.0, MMA_FIXED = 48.0;
     static const int cands[] = {192, 176, 160, 128, 112, 96, 80, 64, 48, 32, 16};
     int best = cands[0];
     double best_cost = 1e30;
@@ -537,8 +585,10 @@ int pick_bn(int m, int n_tiles, int sms) {
         const int mt = (m + bn - 1) / bn;
         const long tiles = (long)mt * n_tiles;
         const long rounds = (tiles + sms - 1) / sms;
-        const double cost = (double)rounds * (bn + 24);  // 24 ~ per-tile fixed cost in token units
-        if (cost < best_cost) {
+        const double stage = 2.0 * bn + MMA_FIXED > DECODE_CYCLES_PER_STAGE ? 2.0 * bn + MMA_FIXED
+                                                                           : DECODE_CYCLES_PER_STAGE;
+        const double cost = (double)rounds * stage;
+        if (cost <= best_cost) {
             best_cost = cost;
             best = bn;
         }
@@ -557,7 +607,7 @@ int a_stages_for(int bn) {
     return st < MAX_A_STAGES ? st : MAX_A_STAGES;
 }
 int b_stages_for(int bn) {
-    const int st = (SMEM_BUDGET - 1024 - 2304 - RAW_STAGES * RAW_STAGE_BYTES) / (bn * 128);
+    const int st = (SMEM_BUDGET - 1024 - 2304 - RAW_STAGES * RAW_STAGE_BYTES - EPI_STAGE_BYTES) / (bn * 128);
     return st < MAX_B_STAGES ? st : MAX_B_STAGES;
 }
 
@@ -583,6 +633,21 @@ bool encode_x_map(CUtensorMap *m, const void *x, int64_t rows, int64_t k, int bo
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Dense output [m, n] of 2- or 4-byte elements: boxes of 32 rows (n) x 16
+// tokens (m) for the epilogue's stores.  false if the row pitch is not a
+// multiple of 16 bytes (the epilogue then stores element by element).
+bool encode_y_map(CUtensorMap *mp, void *y, int64_t m, int64_t n, int ydt) {
+    const int es = ydt == KQ_F32 ? 4 : 2;
+    if ((n * es) % 16) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)n, (cuuint64_t)m};
+    cuuint64_t strides[1] = {(cuuint64_t)(n * es)};
+    cuuint32_t box[2] = {EPI_CHUNK_N, EPI_CHUNK_M};
+    cuuint32_t estr[2] = {1, 1};
+    return encode_fn()(mp, ydt == KQ_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                       y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Raw Q4_K rows of one or more experts: (row bytes, rows, experts), one
 // super-block column of BM rows per box.
 bool encode_w_map(CUtensorMap *m, const void *w, int64_t n, int64_t k, int64_t n_experts,
@@ -606,11 +671,12 @@ bool fill_ring(GemmParams *p) {
 }
 
 template <typename YT, bool ID>
-cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const GemmParams &p, int grid,
-                          cudaStream_t s) {
-    // alignment slack, activation ring, raw ring, barriers (384 B) and the
-    // expert-indexed row list (768 B)
-    const size_t smem = 1024 + (size_t)p.b_stages * p.b_stage_bytes + RAW_STAGES * RAW_STAGE_BYTES + 384 + 1024;
+cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CUtensorMap &ty,
+                          const GemmParams &p, int grid, cudaStream_t s) {
+    // alignment slack, activation ring, raw ring, epilogue staging, barriers
+    // (384 B) and the expert-indexed row list (768 B)
+    const size_t smem = 1024 + (size_t)p.b_stages * p.b_stage_bytes + RAW_STAGES * RAW_STAGE_BYTES +
+                        EPI_STAGE_BYTES + 384 + 1024;
     auto kern = gemm_q4k_kernel<YT, ID>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -624,7 +690,7 @@ cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const Ge
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+    return cudaLaunchKernelEx(&cfg, kern, tx, tw, ty, p);
 }
 
 }  // namespace
@@ -643,12 +709,14 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
     if (!fill_ring(&p)) return cudaErrorNotSupported;
     p.y = y;
     p.err = error_word();
-    CUtensorMap tx, tw;
+    CUtensorMap tx, tw, ty;
     if (!encode_x_map(&tx, x, m, k, p.bn) || !encode_w_map(&tw, w, n, k, 1, n * ((k / 256) * SB_BYTES)))
         return cudaErrorInvalidValue;
+    p.y_tma = encode_y_map(&ty, y, m, n, ydt) ? 1 : 0;
+    if (!p.y_tma) ty = tx;   // unused
     const int grid = p.tiles < sms ? p.tiles : sms;
-    return ydt == KQ_F32 ? launch_kernel<float, false>(tx, tw, p, grid, s)
-                         : launch_kernel<__nv_bfloat16, false>(tx, tw, p, grid, s);
+    return ydt == KQ_F32 ? launch_kernel<float, false>(tx, tw, ty, p, grid, s)
+                         : launch_kernel<__nv_bfloat16, false>(tx, tw, ty, p, grid, s);
 }
 
 int gemm_id_bn(int64_t n_tokens, int64_t top_k, int64_t n_experts) {
@@ -682,8 +750,8 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     // persistent grid: the number of token tiles is only known on the device
     const int64_t max_units = (a.n_tokens * a.top_k / bn + a.n_experts) * p.n_tiles;
     const int grid = (int)(max_units < sms ? max_units : sms);
-    return a.y_dtype == KQ_F32 ? launch_kernel<float, true>(tx, tw, p, grid, s)
-                               : launch_kernel<__nv_bfloat16, true>(tx, tw, p, grid, s);
+    return a.y_dtype == KQ_F32 ? launch_kernel<float, true>(tx, tw, tx, p, grid, s)
+                               : launch_kernel<__nv_bfloat16, true>(tx, tw, tx, p, grid, s);
 }
 
 }  // namespace kq

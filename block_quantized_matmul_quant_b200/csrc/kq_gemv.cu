@@ -255,23 +255,33 @@ __device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w,
     // rows towards L2.  (A CTA fits beside the preceding kernel's CTA, so
     // this runs while that kernel is still computing.)
     const int first = min(p.slots, my_rows);
-    if (p.early) {
-        if (lane == 0)
-            for (int i = 0; i < first; ++i) issue(i);  // early mode makes one pass
+    auto prefetch_rest = [&]() {  // rows beyond the ring's first fill, towards L2
         if (threadIdx.x == 0 && (row_end - row_begin) > p.slots * p.warps) {
             const int64_t bytes = (int64_t)(row_end - row_begin) * row_bytes;
             const uint8_t *src = w + (int64_t)row_begin * row_bytes;
             for (int64_t off = 0; off < bytes; off += 32768)
                 prefetch_l2(src + off, (uint32_t)(bytes - off < 32768 ? bytes - off : 32768));
         }
+    };
+    // An ordered call with constant weights issues its row copies before
+    // waiting for the preceding kernel (early mode makes one pass).
+    const bool copies_first = p.early && !p.indep;
+    if (copies_first) {
+        if (lane == 0)
+            for (int i = 0; i < first; ++i) issue(i);
+        prefetch_rest();
     }
     if (!p.indep) griddep_wait();
-    // Otherwise the activation loads go out first (they gate every row) and
-    // the row copies follow right behind them.
+    // Otherwise the activation loads go out first (they gate every row; an
+    // independent call's are ready at once) and the row copies follow right
+    // behind them.
     stage_activations<C, TB, XT>(p, tok, xq, xsc, xsum, [&]() {
-        if (!p.early && lane == 0) {
-            fence_proxy_async_smem();  // generic reads of the slots in an earlier pass
-            for (int i = 0; i < first; ++i) issue(i);
+        if (!copies_first) {
+            if (lane == 0) {
+                fence_proxy_async_smem();  // generic reads of the slots in an earlier pass
+                for (int i = 0; i < first; ++i) issue(i);
+            }
+            if (p.indep) prefetch_rest();
         }
     });
     __syncthreads();
@@ -458,9 +468,12 @@ __global__ void __launch_bounds__(MINB == 1 ? 32 * GEMV_MAX_WARPS : 32 * GEMV_HA
 // Expert-indexed form: CTA (chunk, e) streams rows of expert e's slice once
 // per group of up to TB (token, slot) pairs routed to e (the device-side
 // grouping of kq_moe.cu: ascending pair order), so each hit expert's weights
-// leave HBM once per group; experts nobody chose cost nothing.
+// leave HBM once per group; experts nobody chose cost nothing.  A pass takes
+// four pairs while three or more remain, else exactly the one or two left:
+// the dot-product work follows the pairs actually routed.
 template <int C, int TB, int R, typename XT, typename YT>
 __global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, 1) gemv_id_q4k_kernel(const GemvParams p) {
+    static_assert(TB == 4, "passes of 4, 2 or 1 pairs share the 4-slot staging layout");
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_tok[TB];
     __shared__ int64_t s_yrow[TB];
@@ -473,18 +486,24 @@ __global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, 1) gemv_id_q4k_kernel(con
     const int32_t *pairs = p.perm + p.offsets[e];
     const uint8_t *w = p.w + (int64_t)e * p.expert_stride;
     if (threadIdx.x == 0) s_failed = 0;
-    for (int j0 = 0, pass = 0; j0 < cnt; j0 += TB, ++pass) {
+    for (int j0 = 0, pass = 0; j0 < cnt; ++pass) {
+        const int rem = cnt - j0;
+        const int tb = rem >= 3 ? 4 : rem;   // pairs this pass (block-uniform)
         __syncthreads();  // the previous pass is done with s_tok / s_yrow
         if (s_failed) return;  // a wait gave up: the ring's phases are unknown
         if (threadIdx.x < TB) {
             const int j = j0 + (int)threadIdx.x;
-            const int pr = j < cnt ? pairs[j] : -1;
+            const int pr = (int)threadIdx.x < tb && j < cnt ? pairs[j] : -1;
             s_tok[threadIdx.x] = pr >= 0 ? pr / p.top_k : -1;
             s_yrow[threadIdx.x] = pr >= 0 ? pr : 0;
         }
         __syncthreads();
-        if (!gemv_pass<C, TB, R, false, XT, YT>(p, w, row_begin, row_end, s_tok, s_yrow, smem, pass))
-            s_failed = 1;
+        bool ok;
+        if (tb == 4) ok = gemv_pass<C, 4, R, false, XT, YT>(p, w, row_begin, row_end, s_tok, s_yrow, smem, pass);
+        else if (tb == 2) ok = gemv_pass<C, 2, R, false, XT, YT>(p, w, row_begin, row_end, s_tok, s_yrow, smem, pass);
+        else ok = gemv_pass<C, 1, R, false, XT, YT>(p, w, row_begin, row_end, s_tok, s_yrow, smem, pass);
+        if (!ok) s_failed = 1;
+        j0 += tb;
     }
 }
 

@@ -17,8 +17,9 @@
 //    so a lane reads the five activations of a byte with one 128-bit load.
 //  * A 256-entry table in shared memory maps a code byte to its five digits
 //    minus one as signed bytes (d0-1 .. d3-1 | d4-1, 0, 0, 0); illegal bytes
-//    map to zeros.  The table is replicated once per lane, so the 32 lanes'
-//    lookups of arbitrary bytes never share a bank.
+//    map to zeros.  A 64-bit load is served per half-warp, so the table is
+//    replicated 16 times (lane l reads copy l % 16) and the lookups of
+//    arbitrary bytes never share a bank.
 //  * dp2a multiplies two 16-bit activations by two signed trits and
 //    accumulates in int32 (|sum| < 2^21 per block: exact), then one fp32
 //    multiply by s * scale per block.
@@ -36,8 +37,9 @@ namespace {
 constexpr int TQ_BB = 28;            // bytes per block
 constexpr int TQ_QK = 128;           // weights per block
 constexpr int TQ_REC = 27;           // 16-byte activation records per block (26 used, odd stride)
-constexpr int TQ_WARPS = 16;
-constexpr int TQ_TABLE_BYTES = 256 * 32 * 8;
+constexpr int TQ_WARPS = 32;
+constexpr int TQ_COPIES = 16;
+constexpr int TQ_TABLE_BYTES = 256 * TQ_COPIES * 8;
 constexpr int TQ_SMEM_LIMIT = 220 * 1024;
 
 struct Tq1Params {
@@ -81,7 +83,7 @@ __device__ __forceinline__ uint2 trit_entry(uint32_t p) {
 template <int TB, typename XT, typename YT>
 __global__ void __launch_bounds__(32 * TQ_WARPS, 1) gemv_tq1_kernel(const Tq1Params p) {
     extern __shared__ __align__(16) uint8_t smem[];
-    uint2 *table = reinterpret_cast<uint2 *>(smem);                              // [256][32]
+    uint2 *table = reinterpret_cast<uint2 *>(smem);                              // [256][16]
     uint4 *xrec = reinterpret_cast<uint4 *>(smem + TQ_TABLE_BYTES);              // [TB][nb][27]
     float *xs = reinterpret_cast<float *>(smem + TQ_TABLE_BYTES + (size_t)TB * p.nb * TQ_REC * 16);  // [TB][nb]
 
@@ -105,11 +107,11 @@ __global__ void __launch_bounds__(32 * TQ_WARPS, 1) gemv_tq1_kernel(const Tq1Par
     };
     if (p.early) prefetch_rows();
 
-    // trit table: thread t fills entry t's 32 lane copies, copy (c + t) % 32
-    // at step c, so a warp's 32 stores fall in distinct banks
+    // trit table: thread t fills entry t's copies, copy (c + t) % 16 at
+    // step c, so a half-warp's stores fall in distinct banks
     for (int e = threadIdx.x; e < 256; e += blockDim.x) {
         const uint2 v = trit_entry((uint32_t)e);
-        for (int c = 0; c < 32; ++c) table[e * 32 + ((c + e) & 31)] = v;
+        for (int c = 0; c < TQ_COPIES; ++c) table[e * TQ_COPIES + ((c + e) & (TQ_COPIES - 1))] = v;
     }
     // zero the activation records (their pad halves stay zero)
     {
@@ -149,8 +151,8 @@ __global__ void __launch_bounds__(32 * TQ_WARPS, 1) gemv_tq1_kernel(const Tq1Par
     }
     __syncthreads();
 
-    // ---- rows: warp w takes rows w, w + 16, ...; lane l takes blocks l, l + 32, ...
-    const uint2 *tab = table + lane;
+    // ---- rows: warp w takes rows w, w + TQ_WARPS, ...; lane l takes blocks l, l + 32, ...
+    const uint2 *tab = table + (lane & (TQ_COPIES - 1));
     const int steps_per_row = (p.nb + 31) / 32;
     const int my_rows = warp < row_end - row_begin ? (row_end - row_begin - warp + TQ_WARPS - 1) / TQ_WARPS : 0;
     const int nsteps = my_rows * steps_per_row;
@@ -176,25 +178,26 @@ __global__ void __launch_bounds__(32 * TQ_WARPS, 1) gemv_tq1_kernel(const Tq1Par
         load_step(s + 1, nxt);
         const int b = (s % steps_per_row) * 32 + lane;
         const int bb = b < p.nb ? b : 0;
-        int ia[TB];
+        int ia[TB][2];   // two chains per row: even and odd code bytes
         #pragma unroll
-        for (int t = 0; t < TB; ++t) ia[t] = 0;
+        for (int t = 0; t < TB; ++t) ia[t][0] = ia[t][1] = 0;
         #pragma unroll
         for (int j = 0; j < 26; ++j) {
             uint32_t code = __byte_perm(cur[j >> 2], 0u, 0x4440u | (uint32_t)(j & 3));
             if (j == 25 && code > 26u) code = 255u;   // illegal tail byte: all digits read as zero weight
-            const uint2 tv = tab[code * 32];
+            const uint2 tv = tab[code * TQ_COPIES];
             #pragma unroll
             for (int t = 0; t < TB; ++t) {
                 const uint4 xv = xrec[((size_t)t * p.nb + bb) * TQ_REC + j];
-                int a = dp2a_lo_ss((int)xv.x, (int)tv.x, ia[t]);
+                int a = dp2a_lo_ss((int)xv.x, (int)tv.x, ia[t][j & 1]);
                 a = dp2a_hi_ss((int)xv.y, (int)tv.x, a);
-                ia[t] = dp2a_lo_ss((int)xv.z, (int)tv.y, a);
+                ia[t][j & 1] = dp2a_lo_ss((int)xv.z, (int)tv.y, a);
             }
         }
         const float scale = half_bits_to_float(cur[6] >> 16);
         #pragma unroll
-        for (int t = 0; t < TB; ++t) acc[t] = fmaf((float)ia[t], scale * xs[t * p.nb + bb], acc[t]);
+        for (int t = 0; t < TB; ++t)
+            acc[t] = fmaf((float)(ia[t][0] + ia[t][1]), scale * xs[t * p.nb + bb], acc[t]);
         if ((s + 1) % steps_per_row == 0) {   // row done (warp-uniform)
             const int r = row_begin + warp + (s / steps_per_row) * TQ_WARPS;
             #pragma unroll
