@@ -15,14 +15,15 @@
 //    (tcgen05.mma with A in TMEM, B = activations in shared memory).  Shared
 //    memory only carries the activation tiles and the raw bytes, so the
 //    tensor core's operand reads do not compete with decoder stores.
-//  * Warp roles:  warp 0  TMA producer -- bf16 activation tiles (64 K x BN,
-//                         128-byte swizzle) and raw Q4_K super-blocks
-//                         (128 rows x 144 bytes) into shared-memory rings;
+//  * Warp roles:  warp 0  TMA producer of bf16 activation tiles (64 K x BN,
+//                         128-byte swizzle) into a shared-memory ring;
+//                 warp 6  TMA producer of raw Q4_K super-blocks (128 rows x
+//                         144 bytes) into their own ring;
 //                 warp 1  MMA issuer -- one thread issues tcgen05.mma
 //                         (kind::f16, bf16 x bf16 -> fp32 in TMEM) and
 //                         tcgen05.commit's to the stage / accumulator barriers;
 //                 warps 2-5  epilogue -- tcgen05.ld from TMEM, convert, store;
-//                 warps 6..  decoders, in groups of four warps (one per TMEM
+//                 warps 7..  decoders, in groups of four warps (one per TMEM
 //                         lane quadrant, so lane = weight row): group j
 //                         decodes the stages s with s % groups == j, 64 K
 //                         positions of its 32 rows per warp, exact fp32
@@ -54,14 +55,15 @@ constexpr int RAW_STAGE_BYTES = BM * SB_BYTES;   // 18432
 #ifndef KQ_GEMM_DEC_WARPS
 #define KQ_GEMM_DEC_WARPS 16
 #endif
-constexpr int DEC_WARP0 = 6, DEC_WARPS = KQ_GEMM_DEC_WARPS;  // 8 or 16
+constexpr int RAW_WARP = 6;  // raw super-block producer
+constexpr int DEC_WARP0 = 7, DEC_WARPS = KQ_GEMM_DEC_WARPS;  // 8 or 16
 constexpr int DEC_GROUPS = DEC_WARPS / 4;                    // 2 or 4
 static_assert(DEC_GROUPS == 2 || DEC_GROUPS == 4, "decoder warps come in 2 or 4 groups of 4");
 constexpr int NUM_THREADS = (DEC_WARP0 + DEC_WARPS) * 32;
 constexpr int EPI_WARP0 = 2;
-constexpr int RAW_STAGES = 2;
+constexpr int MAX_RAW_STAGES = 8;
 constexpr int MAX_A_STAGES = 8;   // TMEM A slots
-constexpr int MAX_B_STAGES = 10;  // activation tiles in shared memory
+constexpr int MAX_B_STAGES = 32;  // activation tiles in shared memory
 constexpr int MAX_BN = 192;
 constexpr int SMEM_BUDGET = 227 * 1024;
 // Epilogue staging: each epilogue warp owns two buffers of one 16-token x
@@ -74,6 +76,7 @@ struct GemmParams {
     int bn, m_tiles, n_tiles, tiles;
     int a_stages;  // decoded-weight ring: A slots in TMEM
     int b_stages;  // activation ring: tiles in shared memory (deeper: their loads come from L2)
+    int raw_stages;  // raw super-block ring (each slot: 128 rows x 144 bytes, 4 stages of K)
     int a_col0;    // first TMEM column after an accumulator (BN rounded up to 32)
     int b_stage_bytes;
     void *y;
@@ -210,6 +213,23 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t r[32]) 
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// A warp's wait on an mbarrier phase, with one outcome for the whole warp.
+// KQ_GEMM_LANE0_WAIT: lane 0 alone polls and the warp follows it (the
+// barrier sees one poller instead of 32); otherwise every lane polls.
+#ifndef KQ_GEMM_LANE0_WAIT
+#define KQ_GEMM_LANE0_WAIT 0
+#endif
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
+#if KQ_GEMM_LANE0_WAIT
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err);
+    __syncwarp();
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+#else
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, err));
+#endif
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (SBO), leading offset 16 bytes, sm_100 descriptor version 1.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -228,11 +248,20 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
            ((uint32_t)(m >> 4) << 24);
 }
 
-// TMEM column of stage slot s: slots alternate between the gap after the
-// first accumulator (columns a_col0..255) and the gap after the second
-// (256 + a_col0..511), 32 columns each.
+// TMEM accumulators: two (columns 0 and 256; the epilogue of one tile
+// overlaps the next tile's main loop) or, as a build option, one (more A
+// slots; measured slower).
+#ifndef KQ_GEMM_ACC_BUFS
+#define KQ_GEMM_ACC_BUFS 2
+#endif
+constexpr int ACC_BUFS = KQ_GEMM_ACC_BUFS;
+static_assert(ACC_BUFS == 1 || ACC_BUFS == 2, "one or two accumulators");
+
+// TMEM column of stage slot s, 32 columns each.  Two accumulators: slots
+// alternate between the gap after the first (a_col0..255) and the gap after
+// the second (256 + a_col0..511).  One accumulator: slots follow it.
 __device__ __forceinline__ uint32_t a_slot_col(uint32_t s, int a_col0) {
-    return ((s & 1u) << 8) + (uint32_t)a_col0 + ((s >> 1) << 5);
+    return ACC_BUFS == 2 ? ((s & 1u) << 8) + (uint32_t)a_col0 + ((s >> 1) << 5) : (uint32_t)a_col0 + (s << 5);
 }
 
 __device__ __forceinline__ float half_f(uint32_t bits) { return half_bits_to_float(bits); }
@@ -269,21 +298,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
-    const int SA = p.a_stages, SB = p.b_stages;
+    const int SA = p.a_stages, SB = p.b_stages, SR = p.raw_stages;
     uint8_t *b_ring = smem;                                    // SB x bn*128
-    uint8_t *raw_ring = b_ring + SB * p.b_stage_bytes;         // RAW_STAGES x 18 KB
-    uint8_t *epi_stage = raw_ring + RAW_STAGES * RAW_STAGE_BYTES;  // EPI_STAGE_BYTES
+    uint8_t *raw_ring = b_ring + SB * p.b_stage_bytes;         // SR x 18 KB
+    uint8_t *epi_stage = raw_ring + SR * RAW_STAGE_BYTES;      // EPI_STAGE_BYTES
     uint64_t *bars = reinterpret_cast<uint64_t *>(epi_stage + EPI_STAGE_BYTES);
     uint64_t *full_a = bars;                 // [SA] one decoder group (4 warps) -> MMA
     uint64_t *empty_a = full_a + SA;         // [SA] MMA -> decoders
     uint64_t *full_b = empty_a + SA;         // [SB] TMA bytes -> MMA
     uint64_t *empty_b = full_b + SB;         // [SB] MMA -> TMA
     uint64_t *raw_full = empty_b + SB;       // [RAW] TMA -> decoders
-    uint64_t *raw_empty = raw_full + RAW_STAGES;  // [RAW] decoders -> TMA
-    uint64_t *acc_full = raw_empty + RAW_STAGES;  // [2] MMA -> epilogue
+    uint64_t *raw_empty = raw_full + SR;     // [RAW] decoders -> TMA
+    uint64_t *acc_full = raw_empty + SR;     // [2] MMA -> epilogue
     uint64_t *acc_empty = acc_full + 2;           // [2] epilogue -> MMA
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
-    int *s_rows = reinterpret_cast<int *>(bars + 48);   // expert-indexed: activation row per tile row
+    int *s_rows = reinterpret_cast<int *>(bars + 128);  // expert-indexed: activation row per tile row
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nk = p.k / BK;
@@ -297,7 +326,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&full_b[s], 1);
             mbar_init(&empty_b[s], 1);
         }
-        for (int r = 0; r < RAW_STAGES; ++r) {
+        for (int r = 0; r < SR; ++r) {
             mbar_init(&raw_full[r], 1);
             mbar_init(&raw_empty[r], DEC_WARPS);
         }
@@ -323,15 +352,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // tiles the grouping step wrote on the device.
     const int units = ID ? *p.id_n_tiles * p.n_tiles : p.tiles;
 
-    if (warp == 0) {
-        // ---------------- TMA producer ----------------
+    if (warp == RAW_WARP) {
+        // ---------------- raw super-block producer ----------------
+        // Runs ahead of the decoders by the whole raw ring, independently of
+        // the activation ring (narrow token tiles stream fresh weights).
+        if (lane == 0) {
+            uint32_t rslot = 0, rphase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                const Tile t = tile_at<ID>(p, u);
+                for (int ks = 0; ks < nk; ks += 4) {
+                    ok = mbar_wait(&raw_empty[rslot], rphase ^ 1, p.err);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&raw_full[rslot], RAW_STAGE_BYTES);
+                    tma_load_3d(raw_ring + rslot * RAW_STAGE_BYTES, &tmap_w, (ks >> 2) * SB_BYTES, t.n0, t.e,
+                                &raw_full[rslot]);
+                    if (++rslot == (uint32_t)SR) { rslot = 0; rphase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 0) {
+        // ---------------- activation producer ----------------
         // Ring positions advance incrementally (no division in the issue
         // loop: this single thread must keep pace with the tensor core).
         // Expert-indexed tiles first gather their activation row numbers
         // (the whole warp, into s_rows; rows past the segment repeat its
         // first row and their outputs are dropped), then load the tile four
         // rows per gather.
-        uint32_t slot = 0, phase = 0, rslot = 0, rphase = 0;
+        uint32_t slot = 0, phase = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             const Tile t = tile_at<ID>(p, u);
@@ -343,14 +391,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             if (lane == 0) {
                 for (int ks = 0; ks < nk; ++ks) {
-                    if ((ks & 3) == 0) {  // raw super-block for this and the next 3 stages
-                        ok = mbar_wait(&raw_empty[rslot], rphase ^ 1, p.err);
-                        if (!ok) break;
-                        mbar_arrive_expect_tx(&raw_full[rslot], RAW_STAGE_BYTES);
-                        tma_load_3d(raw_ring + rslot * RAW_STAGE_BYTES, &tmap_w, (ks >> 2) * SB_BYTES,
-                                    t.n0, t.e, &raw_full[rslot]);
-                        if (++rslot == RAW_STAGES) { rslot = 0; rphase ^= 1; }
-                    }
                     ok = mbar_wait(&empty_b[slot], phase ^ 1, p.err);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&full_b[slot], p.b_stage_bytes);
@@ -382,8 +422,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int tl = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++tl) {
-                const int acc = tl & 1;
-                ok = mbar_wait(&acc_empty[acc], ((tl >> 1) & 1) ^ 1, p.err);
+                const int acc = tl % ACC_BUFS;
+                ok = mbar_wait(&acc_empty[acc], ((tl / ACC_BUFS) & 1) ^ 1, p.err);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
@@ -424,10 +464,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int sbuf = 0;
         int tl = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x, ++tl) {
-            const int acc = tl & 1;
+            const int acc = tl % ACC_BUFS;
             const Tile t = tile_at<ID>(p, u);
             // warp-uniform outcome: the TMEM loads below are .sync.aligned
-            if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], (tl >> 1) & 1, p.err))) break;
+            if (!warp_wait(&acc_full[acc], (tl / ACC_BUFS) & 1, p.err)) break;
             tc_fence_after();
             const int n = t.n0 + 32 * q + lane;
             const uint32_t t_row = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * 256);
@@ -480,7 +520,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             for (int ks = 0; ks < nk && ok; ks += 4) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&raw_full[rs], rph, p.err));
+                ok = warp_wait(&raw_full[rs], rph, p.err);
                 if (!ok) break;
                 const uint8_t *blk = raw_ring + rs * RAW_STAGE_BYTES + r * SB_BYTES;
                 const uint4 hd = *reinterpret_cast<const uint4 *>(blk);
@@ -493,7 +533,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int cc = 0; cc < 4; ++cc) {
                     if ((int)(g & (DEC_GROUPS - 1)) == grp) {
                         // warp-uniform outcome: the TMEM store below is .sync.aligned
-                        ok = __all_sync(0xffffffffu, mbar_wait(&empty_a[slot], phase ^ 1, p.err));
+                        ok = warp_wait(&empty_a[slot], phase ^ 1, p.err);
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t scw = cc < 2 ? sc_lo : sc_hi, mw = cc < 2 ? m_lo : m_hi;
@@ -525,7 +565,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (!ok) break;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&raw_empty[rs]);
-                if (++rs == RAW_STAGES) { rs = 0; rph ^= 1; }
+                if (++rs == (uint32_t)SR) { rs = 0; rph ^= 1; }
             }
         }
     }
@@ -603,12 +643,23 @@ int a_col0_for(int bn) { return (bn + 31) / 32 * 32; }
 // after the accumulators, and as many activation tiles as shared memory
 // holds next to the raw ring (barriers and the row list take 2.25 KB).
 int a_stages_for(int bn) {
-    const int st = 2 * ((256 - a_col0_for(bn)) / 32);
+    const int st = ACC_BUFS == 2 ? 2 * ((256 - a_col0_for(bn)) / 32) : (512 - a_col0_for(bn)) / 32;
     return st < MAX_A_STAGES ? st : MAX_A_STAGES;
 }
+// Shared memory: activation ring first (up to ten stages next to KQ_GEMM_MIN_RAW raw
+// slots), then as many raw slots as the rest holds (up to eight: narrow
+// token tiles stream fresh weights, whose HBM latency needs depth).
+constexpr int SMEM_RINGS = SMEM_BUDGET - 1024 - 2560 - EPI_STAGE_BYTES;  // less alignment, barriers, rows, epilogue
+#ifndef KQ_GEMM_MIN_RAW
+#define KQ_GEMM_MIN_RAW 2
+#endif
 int b_stages_for(int bn) {
-    const int st = (SMEM_BUDGET - 1024 - 2304 - RAW_STAGES * RAW_STAGE_BYTES - EPI_STAGE_BYTES) / (bn * 128);
+    const int st = (SMEM_RINGS - KQ_GEMM_MIN_RAW * RAW_STAGE_BYTES) / (bn * 128);
     return st < MAX_B_STAGES ? st : MAX_B_STAGES;
+}
+int raw_stages_for(int bn, int b_stages) {
+    const int st = (SMEM_RINGS - b_stages * bn * 128) / RAW_STAGE_BYTES;
+    return st < MAX_RAW_STAGES ? st : MAX_RAW_STAGES;
 }
 
 }  // namespace
@@ -665,9 +716,10 @@ bool encode_w_map(CUtensorMap *m, const void *w, int64_t n, int64_t k, int64_t n
 bool fill_ring(GemmParams *p) {
     p->a_stages = a_stages_for(p->bn);
     p->b_stages = b_stages_for(p->bn);
+    p->raw_stages = raw_stages_for(p->bn, p->b_stages);
     p->a_col0 = a_col0_for(p->bn);
     p->b_stage_bytes = p->bn * 128;
-    return p->bn <= MAX_BN && p->bn % 16 == 0 && p->a_stages >= 2 && p->b_stages >= 2;
+    return p->bn <= MAX_BN && p->bn % 16 == 0 && p->a_stages >= 2 && p->b_stages >= 2 && p->raw_stages >= 2;
 }
 
 template <typename YT, bool ID>
@@ -675,8 +727,8 @@ cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CU
                           const GemmParams &p, int grid, cudaStream_t s) {
     // alignment slack, activation ring, raw ring, epilogue staging, barriers
     // (384 B) and the expert-indexed row list (768 B)
-    const size_t smem = 1024 + (size_t)p.b_stages * p.b_stage_bytes + RAW_STAGES * RAW_STAGE_BYTES +
-                        EPI_STAGE_BYTES + 384 + 1024;
+    const size_t smem = 1024 + (size_t)p.b_stages * p.b_stage_bytes + (size_t)p.raw_stages * RAW_STAGE_BYTES +
+                        EPI_STAGE_BYTES + 2560;
     auto kern = gemm_q4k_kernel<YT, ID>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

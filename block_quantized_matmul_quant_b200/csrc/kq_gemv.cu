@@ -43,6 +43,9 @@ namespace {
 #ifndef KQ_GEMV_XREG
 #define KQ_GEMV_XREG 1
 #endif
+#ifndef KQ_GEMV_LANE0_WAIT
+#define KQ_GEMV_LANE0_WAIT 0
+#endif
 #ifndef KQ_GEMV_SHARE_WARPS
 #define KQ_GEMV_SHARE_WARPS 4
 #endif
@@ -53,8 +56,13 @@ constexpr int GEMV_SMEM_LIMIT = 200 * 1024;
 constexpr int GEMV_MAX_WARPS = 16;
 constexpr int GEMV_HALF_MAX_WARPS = KQ_GEMV_SHARE_WARPS;
 constexpr int GEMV_HALF_BLOCKS = KQ_GEMV_SHARE_BLOCKS;
-constexpr int GEMV_HALF_SMEM_LIMIT = (224 / GEMV_HALF_BLOCKS - 12) * 1024;
+// An SM has 228 KB of shared memory and reserves 1 KB per resident CTA;
+// leave 256 B for the kernel's static arrays.
+constexpr int GEMV_HALF_SMEM_LIMIT = 233472 / GEMV_HALF_BLOCKS - 1024 - 256;
 constexpr int GEMV_MAX_SLOTS = 4;
+// Slots a warp of a shared-SM CTA keeps in flight (more, measured, is slower:
+// fewer CTAs fit side by side).
+constexpr int GEMV_HALF_MAX_SLOTS = 4;
 
 struct GemvParams {
     const uint8_t *w;
@@ -313,7 +321,18 @@ __device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w,
         for (int r = 0; r < R; ++r) {
             const int ii = base + i + min(r, nr - 1);
             const int slot = ii % p.slots;
-            if (r < nr && !mbar_wait(&my_full[slot], (uint32_t)(ii / p.slots) & 1u, p.err)) return false;
+            if (r < nr) {
+#if KQ_GEMV_LANE0_WAIT
+                // lane 0 polls, the warp follows it
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait(&my_full[slot], (uint32_t)(ii / p.slots) & 1u, p.err);
+                __syncwarp();
+                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return false;
+#else
+                if (!__all_sync(0xffffffffu, mbar_wait(&my_full[slot], (uint32_t)(ii / p.slots) & 1u, p.err)))
+                    return false;
+#endif
+            }
             rowp[r] = my_ring + slot * row_bytes;
         }
         float acc[R][TB];
@@ -512,7 +531,7 @@ int tb_for(int64_t m) { return m <= 1 ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : 8; }
 int rows_per_step(int tb) { return tb <= 2 ? 2 : 1; }
 
 bool plan_gemv(int type, int64_t n, int64_t k, int64_t m, int num_sms, int max_warps,
-               int smem_limit, GemvParams *p) {
+               int smem_limit, int max_slots, GemvParams *p) {
     if (type != KQ_Q4_K) return false;
     if (m < 1 || m > 8 || n < 1 || n > INT32_MAX / 2 || k > (1 << 20)) return false;
     const int tb = tb_for(m), R = rows_per_step(tb);
@@ -528,7 +547,7 @@ bool plan_gemv(int type, int64_t n, int64_t k, int64_t m, int num_sms, int max_w
     int warps = rows_per_cta < max_warps ? rows_per_cta : max_warps;
     for (; warps >= 1; --warps) {
         const int rows_per_warp = (rows_per_cta + warps - 1) / warps;
-        const int want = rows_per_warp < GEMV_MAX_SLOTS ? rows_per_warp : GEMV_MAX_SLOTS;
+        const int want = rows_per_warp < max_slots ? rows_per_warp : max_slots;
         const int min_slots = rows_per_warp < R ? rows_per_warp : R;
         int slots = want;
         while (slots > min_slots && fixed + (size_t)warps * slots * (row_bytes + 8) > (size_t)smem_limit)
@@ -566,6 +585,9 @@ cudaError_t launch_q4k(GemvParams p, GemvOrder order, cudaStream_t s) {
     const size_t smem = (size_t)p.xq_bytes + 2 * (size_t)p.xs_bytes +
                         (size_t)p.warps * p.slots * ((size_t)p.row_bytes + 8);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // the whole shared-memory carveout, so that the shared-SM CTAs fit side by side
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((p.n + p.rows_per_cta - 1) / p.rows_per_cta));
@@ -615,7 +637,8 @@ bool gemv_supported(int type, int64_t n, int64_t k, int x_dtype, int64_t m) {
     (void)x_dtype;
     if (type == KQ_TQ1_G128) return m >= 1 && gemv_tq1_supported(n, k);
     GemvParams p;
-    return m >= 1 && plan_gemv(type, n, k, m < 8 ? m : 8, sm_count(), GEMV_MAX_WARPS, GEMV_SMEM_LIMIT, &p);
+    return m >= 1 && plan_gemv(type, n, k, m < 8 ? m : 8, sm_count(), GEMV_MAX_WARPS, GEMV_SMEM_LIMIT,
+                               GEMV_MAX_SLOTS, &p);
 }
 
 // More than eight activation rows run as consecutive launches of up to eight
@@ -630,8 +653,9 @@ cudaError_t launch_gemv(int type, const void *w, int64_t n, int64_t k, const voi
         GemvParams p = {};
         const int tb = tb_for(mc);
         // independent calls take the half-SM plan when it fits, else a whole SM
-        if (!(half && plan_gemv(type, n, k, mc, sm_count(), GEMV_HALF_MAX_WARPS, GEMV_HALF_SMEM_LIMIT, &p)) &&
-            !plan_gemv(type, n, k, mc, sm_count(), GEMV_MAX_WARPS, GEMV_SMEM_LIMIT, &p))
+        if (!(half && plan_gemv(type, n, k, mc, sm_count(), GEMV_HALF_MAX_WARPS, GEMV_HALF_SMEM_LIMIT,
+                                GEMV_HALF_MAX_SLOTS, &p)) &&
+            !plan_gemv(type, n, k, mc, sm_count(), GEMV_MAX_WARPS, GEMV_SMEM_LIMIT, GEMV_MAX_SLOTS, &p))
             return cudaErrorNotSupported;
         p.w = static_cast<const uint8_t *>(w);
         p.x = static_cast<const char *>(x) + (size_t)m0 * (size_t)k * xs;
