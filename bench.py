@@ -508,8 +508,9 @@ def run_profile(args):
             kq.matmul_id(wd, wl.codec, xd, idd, out=y)
     else:
         y = torch.empty((wl.m, wl.n), dtype=ydt, device="cuda")
+        indep = args.profile_mode == "independent"
         for _ in range(args.profile_calls):
-            kq.matmul(wd, wl.codec, xd, out=y, const_weights=True)
+            kq.matmul(wd, wl.codec, xd, out=y, const_weights=not indep, independent=indep)
     torch.cuda.synchronize()
     status = kq.device_status()
     if status != 0:  # a kernel reported a bad input or a wait that gave up
@@ -528,6 +529,8 @@ def main():
     ap.add_argument("--profile", default=None, choices=sorted(synth.WORKLOADS),
                     help="run a few eager calls of one workload (for ncu) and exit")
     ap.add_argument("--profile-calls", type=int, default=3)
+    ap.add_argument("--profile-mode", default="independent", choices=["independent", "const"],
+                    help="GEMV call ordering in --profile (the headline step uses independent calls)")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the other workloads' numbers (prefill GEMM, MoE, TQ1, Q8_0)")
     args = ap.parse_args()
