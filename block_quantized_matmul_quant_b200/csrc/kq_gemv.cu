@@ -62,7 +62,20 @@ constexpr int GEMV_HALF_SMEM_LIMIT = 233472 / GEMV_HALF_BLOCKS - 1024 - 256;
 constexpr int GEMV_MAX_SLOTS = 4;
 // Slots a warp of a shared-SM CTA keeps in flight (more, measured, is slower:
 // fewer CTAs fit side by side).
-constexpr int GEMV_HALF_MAX_SLOTS = 4;
+#ifndef KQ_GEMV_SHARE_SLOTS
+#define KQ_GEMV_SHARE_SLOTS 4
+#endif
+constexpr int GEMV_HALF_MAX_SLOTS = KQ_GEMV_SHARE_SLOTS;
+// Independent calls spread over (SMs / KQ_GEMV_SHARE_GRID_DIV) CTAs.
+// When an independent call's CTA asks L2 for the rows beyond its ring's first
+// fill: 0 after its first activation loads, 1 before them, 2 never (measured
+// fastest: the ring alone keeps enough bytes in flight).
+#ifndef KQ_GEMV_PREFETCH_MODE
+#define KQ_GEMV_PREFETCH_MODE 2
+#endif
+#ifndef KQ_GEMV_SHARE_GRID_DIV
+#define KQ_GEMV_SHARE_GRID_DIV 2
+#endif
 
 struct GemvParams {
     const uint8_t *w;
@@ -279,6 +292,9 @@ __device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w,
             for (int i = 0; i < first; ++i) issue(i);
         prefetch_rest();
     }
+#if KQ_GEMV_PREFETCH_MODE == 1
+    if (p.indep) prefetch_rest();
+#endif
     if (!p.indep) griddep_wait();
     // Otherwise the activation loads go out first (they gate every row; an
     // independent call's are ready at once) and the row copies follow right
@@ -289,7 +305,9 @@ __device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w,
                 fence_proxy_async_smem();  // generic reads of the slots in an earlier pass
                 for (int i = 0; i < first; ++i) issue(i);
             }
+#if KQ_GEMV_PREFETCH_MODE == 0
             if (p.indep) prefetch_rest();
+#endif
         }
     });
     __syncthreads();
@@ -653,8 +671,8 @@ cudaError_t launch_gemv(int type, const void *w, int64_t n, int64_t k, const voi
         GemvParams p = {};
         const int tb = tb_for(mc);
         // independent calls take the half-SM plan when it fits, else a whole SM
-        if (!(half && plan_gemv(type, n, k, mc, sm_count(), GEMV_HALF_MAX_WARPS, GEMV_HALF_SMEM_LIMIT,
-                                GEMV_HALF_MAX_SLOTS, &p)) &&
+        if (!(half && plan_gemv(type, n, k, mc, sm_count() / KQ_GEMV_SHARE_GRID_DIV, GEMV_HALF_MAX_WARPS,
+                                GEMV_HALF_SMEM_LIMIT, GEMV_HALF_MAX_SLOTS, &p)) &&
             !plan_gemv(type, n, k, mc, sm_count(), GEMV_MAX_WARPS, GEMV_SMEM_LIMIT, GEMV_MAX_SLOTS, &p))
             return cudaErrorNotSupported;
         p.w = static_cast<const uint8_t *>(w);
