@@ -347,7 +347,10 @@ __device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w,
                 __syncwarp();
                 if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return false;
 #else
-                if (!__all_sync(0xffffffffu, mbar_wait(&my_full[slot], (uint32_t)(ii / p.slots) & 1u, p.err)))
+                // a landed row costs one non-blocking poll (measured faster than
+                // going straight to the suspending wait)
+                const uint32_t par = (uint32_t)(ii / p.slots) & 1u;
+                if (!__all_sync(0xffffffffu, mbar_test_wait(&my_full[slot], par) || mbar_wait(&my_full[slot], par, p.err)))
                     return false;
 #endif
             }

@@ -52,14 +52,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait; returns false (and flags the device error word) on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
-    for (uint32_t i = 0; i < KQ_SPIN_LIMIT; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    atomicOr(err, ERR_TIMEOUT);
-    return false;
-}
-
 // Non-blocking poll of a phase.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
@@ -71,6 +63,24 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+
+// Bounded wait; returns false (and flags the device error word) on timeout.
+// KQ_WAIT_FASTPATH: one non-blocking poll first, so that a phase which has
+// already completed costs no suspend-capable wait.
+#ifndef KQ_WAIT_FASTPATH
+#define KQ_WAIT_FASTPATH 0
+#endif
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
+#if KQ_WAIT_FASTPATH
+    if (mbar_test_wait(bar, parity)) return true;
+#endif
+    for (uint32_t i = 0; i < KQ_SPIN_LIMIT; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    atomicOr(err, ERR_TIMEOUT);
+    return false;
+}
+
+
 
 // Bounded busy wait for a single latency-critical thread (an MMA or TMA
 // issuer): it resumes the moment the phase completes instead of sleeping.
