@@ -49,7 +49,7 @@ namespace kq {
 namespace {
 
 constexpr int BM = 128;            // weight rows per tile (MMA M)
-constexpr int BK = 64;             // K per stage (one 128-byte swizzle atom of bf16)
+constexpr int BK = 64;             // K per swizzle atom (128 bytes of bf16); a stage holds CPS atoms
 constexpr int SB_BYTES = 144;      // Q4_K super-block
 constexpr int RAW_STAGE_BYTES = BM * SB_BYTES;   // 18432
 #ifndef KQ_GEMM_DEC_WARPS
@@ -257,11 +257,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
 constexpr int ACC_BUFS = KQ_GEMM_ACC_BUFS;
 static_assert(ACC_BUFS == 1 || ACC_BUFS == 2, "one or two accumulators");
 
-// TMEM column of stage slot s, 32 columns each.  Two accumulators: slots
-// alternate between the gap after the first (a_col0..255) and the gap after
-// the second (256 + a_col0..511).  One accumulator: slots follow it.
+// TMEM column of stage slot s, 32 columns per 64 K of the stage (CPS of
+// them).  Two accumulators: slots alternate between the gap after the first
+// (a_col0..255) and the gap after the second (256 + a_col0..511).  One
+// accumulator: slots follow it.
+template <int CPS>
 __device__ __forceinline__ uint32_t a_slot_col(uint32_t s, int a_col0) {
-    return ACC_BUFS == 2 ? ((s & 1u) << 8) + (uint32_t)a_col0 + ((s >> 1) << 5) : (uint32_t)a_col0 + (s << 5);
+    return ACC_BUFS == 2 ? ((s & 1u) << 8) + (uint32_t)a_col0 + (s >> 1) * (32u * CPS)
+                         : (uint32_t)a_col0 + s * (32u * CPS);
 }
 
 __device__ __forceinline__ float half_f(uint32_t bits) { return half_bits_to_float(bits); }
@@ -290,7 +293,9 @@ __device__ __forceinline__ void decode4(uint32_t nib, float2 scale, float2 bias,
     o1 = *reinterpret_cast<const uint32_t *>(&b1);
 }
 
-template <typename YT, bool ID>
+// CPS: 64-K swizzle atoms per pipeline stage (1, or 2 for narrow token tiles,
+// which halves the per-K barrier traffic of the single MMA thread).
+template <typename YT, bool ID, int CPS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_q4k_kernel(const __grid_constant__ CUtensorMap tmap_x,
                     const __grid_constant__ CUtensorMap tmap_w,
@@ -315,7 +320,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int *s_rows = reinterpret_cast<int *>(bars + 128);  // expert-indexed: activation row per tile row
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nk = p.k / BK;
+    constexpr int SPS = 4 / CPS;           // stages per raw super-block (256 K)
+    const int nk = p.k / (BK * CPS);       // stages per tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SA; ++s) {
@@ -361,11 +367,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
                 const Tile t = tile_at<ID>(p, u);
-                for (int ks = 0; ks < nk; ks += 4) {
+                for (int sb = 0; sb < p.k / 256; ++sb) {
                     ok = mbar_wait(&raw_empty[rslot], rphase ^ 1, p.err);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&raw_full[rslot], RAW_STAGE_BYTES);
-                    tma_load_3d(raw_ring + rslot * RAW_STAGE_BYTES, &tmap_w, (ks >> 2) * SB_BYTES, t.n0, t.e,
+                    tma_load_3d(raw_ring + rslot * RAW_STAGE_BYTES, &tmap_w, sb * SB_BYTES, t.n0, t.e,
                                 &raw_full[rslot]);
                     if (++rslot == (uint32_t)SR) { rslot = 0; rphase ^= 1; }
                 }
@@ -394,13 +400,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     ok = mbar_wait(&empty_b[slot], phase ^ 1, p.err);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&full_b[slot], p.b_stage_bytes);
-                    uint8_t *dst = b_ring + slot * p.b_stage_bytes;
-                    if constexpr (ID) {
-                        for (int i = 0; i < p.bn; i += 4)
-                            tma_gather4(dst + i * 128, &tmap_x, ks * BK, s_rows[i], s_rows[i + 1],
-                                        s_rows[i + 2], s_rows[i + 3], &full_b[slot]);
-                    } else {
-                        tma_load_2d(dst, &tmap_x, ks * BK, t.m0, &full_b[slot]);
+                    #pragma unroll
+                    for (int c = 0; c < CPS; ++c) {   // one 64-K atom (bn rows x 128 B) each
+                        uint8_t *dst = b_ring + slot * p.b_stage_bytes + c * p.bn * 128;
+                        const int kx = (ks * CPS + c) * BK;
+                        if constexpr (ID) {
+                            for (int i = 0; i < p.bn; i += 4)
+                                tma_gather4(dst + i * 128, &tmap_x, kx, s_rows[i], s_rows[i + 1], s_rows[i + 2],
+                                            s_rows[i + 3], &full_b[slot]);
+                        } else {
+                            tma_load_2d(dst, &tmap_x, kx, t.m0, &full_b[slot]);
+                        }
                     }
                     if (++slot == (uint32_t)SB) { slot = 0; phase ^= 1; }
                 }
@@ -431,11 +441,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     ok = mbar_wait(&full_b[sb], pb, p.err) && mbar_wait(&full_a[sa], pa, p.err);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t at = tmem_base + a_slot_col(sa, p.a_col0);
-                    mma_bf16_ts(d_tmem, at, bd, idesc, ks > 0 ? 1u : 0u);
-                    mma_bf16_ts(d_tmem, at + 8, bd + 2, idesc, 1u);
-                    mma_bf16_ts(d_tmem, at + 16, bd + 4, idesc, 1u);
-                    mma_bf16_ts(d_tmem, at + 24, bd + 6, idesc, 1u);
+                    const uint32_t at = tmem_base + a_slot_col<CPS>(sa, p.a_col0);
+                    #pragma unroll
+                    for (int c = 0; c < CPS; ++c) {
+                        const uint64_t bc = bd + (uint64_t)(c * ((p.bn * 128) >> 4));
+                        mma_bf16_ts(d_tmem, at + 32 * c, bc, idesc, (ks > 0 || c > 0) ? 1u : 0u);
+                        mma_bf16_ts(d_tmem, at + 32 * c + 8, bc + 2, idesc, 1u);
+                        mma_bf16_ts(d_tmem, at + 32 * c + 16, bc + 4, idesc, 1u);
+                        mma_bf16_ts(d_tmem, at + 32 * c + 24, bc + 6, idesc, 1u);
+                    }
                     mma_commit(&empty_b[sb]);  // frees both slots once these MMAs finish
                     mma_commit(&empty_a[sa]);
                     if (++sb == (uint32_t)SB) {
@@ -519,7 +533,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t g = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-            for (int ks = 0; ks < nk && ok; ks += 4) {
+            for (int sb = 0; sb < p.k / 256 && ok; ++sb) {
                 ok = warp_wait(&raw_full[rs], rph, p.err);
                 if (!ok) break;
                 const uint8_t *blk = raw_ring + rs * RAW_STAGE_BYTES + r * SB_BYTES;
@@ -530,12 +544,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const uint32_t sc_hi = (hd.w & 0x0F0F0F0Fu) | ((hd.y >> 2) & 0x30303030u);
                 const uint32_t m_hi = ((hd.w >> 4) & 0x0F0F0F0Fu) | ((hd.z >> 2) & 0x30303030u);
                 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                for (int st = 0; st < SPS; ++st) {
                     if ((int)(g & (DEC_GROUPS - 1)) == grp) {
-                        // warp-uniform outcome: the TMEM store below is .sync.aligned
+                        // warp-uniform outcome: the TMEM stores below are .sync.aligned
                         ok = warp_wait(&empty_a[slot], phase ^ 1, p.err);
                         if (!ok) break;
                         tc_fence_after();
+                      #pragma unroll
+                      for (int c = 0; c < CPS; ++c) {
+                        const int cc = st * CPS + c;   // 64-K chunk of the super-block
                         const uint32_t scw = cc < 2 ? sc_lo : sc_hi, mw = cc < 2 ? m_lo : m_hi;
                         const int b0 = (2 * cc) & 3;
                         // exact products: d*sc (17 bits), dmin*m (17 bits); high
@@ -554,7 +571,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             decode4(qw[wd] & 0x0F0F0F0Fu, sl, bl, out[2 * wd], out[2 * wd + 1]);
                             decode4(qw[wd] & 0xF0F0F0F0u, sh, bh, out[16 + 2 * wd], out[17 + 2 * wd]);
                         }
-                        tmem_st32(t_lane + a_slot_col(slot, p.a_col0), out);
+                        tmem_st32(t_lane + a_slot_col<CPS>(slot, p.a_col0) + 32 * c, out);
+                      }
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&full_a[slot]);
@@ -642,8 +660,8 @@ int a_col0_for(int bn) { return (bn + 31) / 32 * 32; }
 // Ring depths: the A slots (32 TMEM columns each) that fit in the two gaps
 // after the accumulators, and as many activation tiles as shared memory
 // holds next to the raw ring (barriers and the row list take 2.25 KB).
-int a_stages_for(int bn) {
-    const int st = ACC_BUFS == 2 ? 2 * ((256 - a_col0_for(bn)) / 32) : (512 - a_col0_for(bn)) / 32;
+int a_stages_for(int bn, int cps) {
+    const int st = ACC_BUFS == 2 ? 2 * ((256 - a_col0_for(bn)) / (32 * cps)) : (512 - a_col0_for(bn)) / (32 * cps);
     return st < MAX_A_STAGES ? st : MAX_A_STAGES;
 }
 // Shared memory: activation ring first (up to ten stages next to KQ_GEMM_MIN_RAW raw
@@ -653,12 +671,12 @@ constexpr int SMEM_RINGS = SMEM_BUDGET - 1024 - 2560 - EPI_STAGE_BYTES;  // less
 #ifndef KQ_GEMM_MIN_RAW
 #define KQ_GEMM_MIN_RAW 2
 #endif
-int b_stages_for(int bn) {
-    const int st = (SMEM_RINGS - KQ_GEMM_MIN_RAW * RAW_STAGE_BYTES) / (bn * 128);
+int b_stages_for(int b_stage_bytes) {
+    const int st = (SMEM_RINGS - KQ_GEMM_MIN_RAW * RAW_STAGE_BYTES) / b_stage_bytes;
     return st < MAX_B_STAGES ? st : MAX_B_STAGES;
 }
-int raw_stages_for(int bn, int b_stages) {
-    const int st = (SMEM_RINGS - b_stages * bn * 128) / RAW_STAGE_BYTES;
+int raw_stages_for(int b_stage_bytes, int b_stages) {
+    const int st = (SMEM_RINGS - b_stages * b_stage_bytes) / RAW_STAGE_BYTES;
     return st < MAX_RAW_STAGES ? st : MAX_RAW_STAGES;
 }
 
@@ -713,23 +731,27 @@ bool encode_w_map(CUtensorMap *m, const void *w, int64_t n, int64_t k, int64_t n
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool fill_ring(GemmParams *p) {
-    p->a_stages = a_stages_for(p->bn);
-    p->b_stages = b_stages_for(p->bn);
-    p->raw_stages = raw_stages_for(p->bn, p->b_stages);
+// 64-K atoms per stage: two for narrow token tiles (their MMAs are short, so
+// the single MMA thread's per-stage waits and commits dominate), else one.
+int cps_for(int bn) { return bn <= 64 ? 2 : 1; }
+
+bool fill_ring(GemmParams *p, int cps) {
+    p->b_stage_bytes = p->bn * 128 * cps;
+    p->a_stages = a_stages_for(p->bn, cps);
+    p->b_stages = b_stages_for(p->b_stage_bytes);
+    p->raw_stages = raw_stages_for(p->b_stage_bytes, p->b_stages);
     p->a_col0 = a_col0_for(p->bn);
-    p->b_stage_bytes = p->bn * 128;
     return p->bn <= MAX_BN && p->bn % 16 == 0 && p->a_stages >= 2 && p->b_stages >= 2 && p->raw_stages >= 2;
 }
 
-template <typename YT, bool ID>
+template <typename YT, bool ID, int CPS>
 cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CUtensorMap &ty,
                           const GemmParams &p, int grid, cudaStream_t s) {
     // alignment slack, activation ring, raw ring, epilogue staging, barriers
     // (384 B) and the expert-indexed row list (768 B)
     const size_t smem = 1024 + (size_t)p.b_stages * p.b_stage_bytes + (size_t)p.raw_stages * RAW_STAGE_BYTES +
                         EPI_STAGE_BYTES + 2560;
-    auto kern = gemm_q4k_kernel<YT, ID>;
+    auto kern = gemm_q4k_kernel<YT, ID, CPS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -758,7 +780,8 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
     p.bn = pick_bn((int)m, p.n_tiles, sms);
     p.m_tiles = (int)((m + p.bn - 1) / p.bn);
     p.tiles = p.n_tiles * p.m_tiles;
-    if (!fill_ring(&p)) return cudaErrorNotSupported;
+    const int cps = cps_for(p.bn);
+    if (!fill_ring(&p, cps)) return cudaErrorNotSupported;
     p.y = y;
     p.err = error_word();
     CUtensorMap tx, tw, ty;
@@ -767,8 +790,11 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
     p.y_tma = encode_y_map(&ty, y, m, n, ydt) ? 1 : 0;
     if (!p.y_tma) ty = tx;   // unused
     const int grid = p.tiles < sms ? p.tiles : sms;
-    return ydt == KQ_F32 ? launch_kernel<float, false>(tx, tw, ty, p, grid, s)
-                         : launch_kernel<__nv_bfloat16, false>(tx, tw, ty, p, grid, s);
+    if (cps == 2)
+        return ydt == KQ_F32 ? launch_kernel<float, false, 2>(tx, tw, ty, p, grid, s)
+                             : launch_kernel<__nv_bfloat16, false, 2>(tx, tw, ty, p, grid, s);
+    return ydt == KQ_F32 ? launch_kernel<float, false, 1>(tx, tw, ty, p, grid, s)
+                         : launch_kernel<__nv_bfloat16, false, 1>(tx, tw, ty, p, grid, s);
 }
 
 int gemm_id_bn(int64_t n_tokens, int64_t top_k, int64_t n_experts) {
@@ -787,7 +813,8 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     p.n = (int)a.n; p.k = (int)a.k; p.m = (int)a.n_tokens;
     p.n_tiles = (int)((a.n + BM - 1) / BM);
     p.bn = bn;
-    if (!fill_ring(&p)) return cudaErrorNotSupported;
+    const int cps = cps_for(bn);
+    if (!fill_ring(&p, cps)) return cudaErrorNotSupported;
     p.y = a.y;
     p.err = error_word();
     p.perm = a.perm;
@@ -802,8 +829,11 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     // persistent grid: the number of token tiles is only known on the device
     const int64_t max_units = (a.n_tokens * a.top_k / bn + a.n_experts) * p.n_tiles;
     const int grid = (int)(max_units < sms ? max_units : sms);
-    return a.y_dtype == KQ_F32 ? launch_kernel<float, true>(tx, tw, tx, p, grid, s)
-                               : launch_kernel<__nv_bfloat16, true>(tx, tw, tx, p, grid, s);
+    if (cps == 2)
+        return a.y_dtype == KQ_F32 ? launch_kernel<float, true, 2>(tx, tw, tx, p, grid, s)
+                                   : launch_kernel<__nv_bfloat16, true, 2>(tx, tw, tx, p, grid, s);
+    return a.y_dtype == KQ_F32 ? launch_kernel<float, true, 1>(tx, tw, tx, p, grid, s)
+                               : launch_kernel<__nv_bfloat16, true, 1>(tx, tw, tx, p, grid, s);
 }
 
 }  // namespace kq
