@@ -330,11 +330,19 @@ def time_eager(torch, fn, steps, warmup, pg):
 
 
 def max_over_ranks(torch, pg, v):
+    """The slowest rank's time: every rank's replica must finish."""
     if pg is None:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank_step, steps, world, ms):
+    """Whole-job rate: the units every replica processed over the slowest
+    rank's time (weak scaling: each rank streams its own pool)."""
+    return units_per_rank_step * steps * world / (ms / 1e3)
 
 
 def cpu_baseline_gemv(wl, budget_s=10.0):
@@ -380,8 +388,7 @@ def run_gpu(args):
     if status != 0:  # a kernel reported a bad input or a wait that gave up: no number
         raise SystemExit(f"device status {status} during the timed steps")
     per_step_ms = ms / args.steps
-    total_bytes = step.step_units() * args.steps * world
-    value = total_bytes / (ms / 1e3) / 1e9
+    value = job_throughput(step.step_units(), args.steps, world, ms) / 1e9
     launch_us = ms * 1e3 / (args.steps * step.launches)
     achieved = step.algo_bytes_per_launch / (launch_us * 1e-6) / 1e9
     traffic = measured_traffic("gemv_q4k_4096x4096", ["kq_gemv.cu", "kq_ptx.cuh", "kq_common.cuh"])
