@@ -23,10 +23,13 @@
 //  * dp2a multiplies two 16-bit activations by two signed trits and
 //    accumulates in int32 (|sum| < 2^21 per block: exact), then one fp32
 //    multiply by s * scale per block.
+//  * A warp takes two weight rows at a time, so one activation-record load
+//    serves both (the shared-memory instruction queue is the limit: per code
+//    byte one record load and one table load per row before).
 //  * Weights are read straight from global memory, one block (28 bytes) per
-//    lane, with the next block's words loaded before the current one is
-//    used; each CTA first asks L2 to prefetch its whole row range, so the
-//    stream runs at HBM speed while the lanes compute.
+//    lane and row, with the next blocks' words loaded before the current
+//    ones are used; each CTA first asks L2 to prefetch its whole row range,
+//    so the stream runs at HBM speed while the lanes compute.
 #include "kq_ptx.cuh"
 #include "kq_launch.h"
 
@@ -37,7 +40,7 @@ namespace {
 constexpr int TQ_BB = 28;            // bytes per block
 constexpr int TQ_QK = 128;           // weights per block
 constexpr int TQ_REC = 27;           // 16-byte activation records per block (26 used, odd stride)
-constexpr int TQ_WARPS = 32;
+constexpr int TQ_WARPS = 16;
 constexpr int TQ_COPIES = 16;
 constexpr int TQ_TABLE_BYTES = 256 * TQ_COPIES * 8;
 constexpr int TQ_SMEM_LIMIT = 220 * 1024;
@@ -151,66 +154,94 @@ __global__ void __launch_bounds__(32 * TQ_WARPS, 1) gemv_tq1_kernel(const Tq1Par
     }
     __syncthreads();
 
-    // ---- rows: warp w takes rows w, w + TQ_WARPS, ...; lane l takes blocks l, l + 32, ...
+    // ---- rows: warp w takes rows w, w + TQ_WARPS, ... two at a time (one
+    // activation record load serves both); lane l takes blocks l, l + 32, ...
     const uint2 *tab = table + (lane & (TQ_COPIES - 1));
     const int steps_per_row = (p.nb + 31) / 32;
     const int my_rows = warp < row_end - row_begin ? (row_end - row_begin - warp + TQ_WARPS - 1) / TQ_WARPS : 0;
-    const int nsteps = my_rows * steps_per_row;
-    auto load_step = [&](int s, uint32_t wv[7]) {
-        const int r = row_begin + warp + (s / steps_per_row) * TQ_WARPS;
+    const int npairs = (my_rows + 1) / 2;
+    const int nsteps = npairs * steps_per_row;
+    auto load_step = [&](int s, uint32_t wv[2][7]) {
+        const int pr = s / steps_per_row;
         const int b = (s % steps_per_row) * 32 + lane;
-        if (s < nsteps && b < p.nb) {
-            const uint32_t *src = reinterpret_cast<const uint32_t *>(p.w + (int64_t)r * row_bytes + (int64_t)b * TQ_BB);
-            #pragma unroll
-            for (int j = 0; j < 7; ++j) wv[j] = __ldg(src + j);
-        } else {
-            #pragma unroll
-            for (int j = 0; j < 7; ++j) wv[j] = 0u;   // scale 0: contributes nothing
+        #pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int i = 2 * pr + h;
+            if (s < nsteps && i < my_rows && b < p.nb) {
+                const int r = row_begin + warp + i * TQ_WARPS;
+                const uint32_t *src =
+                    reinterpret_cast<const uint32_t *>(p.w + (int64_t)r * row_bytes + (int64_t)b * TQ_BB);
+                #pragma unroll
+                for (int j = 0; j < 7; ++j) wv[h][j] = __ldg(src + j);
+            } else {
+                #pragma unroll
+                for (int j = 0; j < 7; ++j) wv[h][j] = 0u;
+            }
         }
     };
     YT *y = static_cast<YT *>(p.y);
-    uint32_t cur[7], nxt[7];
+    uint32_t cur[2][7], nxt[2][7];
     load_step(0, cur);
-    float acc[TB];
+    float acc[2][TB];
     #pragma unroll
-    for (int t = 0; t < TB; ++t) acc[t] = 0.f;
+    for (int h = 0; h < 2; ++h)
+        #pragma unroll
+        for (int t = 0; t < TB; ++t) acc[h][t] = 0.f;
     for (int s = 0; s < nsteps; ++s) {
         load_step(s + 1, nxt);
         const int b = (s % steps_per_row) * 32 + lane;
         const int bb = b < p.nb ? b : 0;
-        int ia[TB][2];   // two chains per row: even and odd code bytes
+        int ia[2][TB][2];
         #pragma unroll
-        for (int t = 0; t < TB; ++t) ia[t][0] = ia[t][1] = 0;
+        for (int h = 0; h < 2; ++h)
+            #pragma unroll
+            for (int t = 0; t < TB; ++t) ia[h][t][0] = ia[h][t][1] = 0;
         #pragma unroll
         for (int j = 0; j < 26; ++j) {
-            uint32_t code = __byte_perm(cur[j >> 2], 0u, 0x4440u | (uint32_t)(j & 3));
-            if (j == 25 && code > 26u) code = 255u;   // illegal tail byte: all digits read as zero weight
-            const uint2 tv = tab[code * TQ_COPIES];
+            uint2 tv[2];
+            #pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t code = __byte_perm(cur[h][j >> 2], 0u, 0x4440u | (uint32_t)(j & 3));
+                if (j == 25 && code > 26u) code = 255u;
+                tv[h] = tab[code * TQ_COPIES];
+            }
             #pragma unroll
             for (int t = 0; t < TB; ++t) {
                 const uint4 xv = xrec[((size_t)t * p.nb + bb) * TQ_REC + j];
-                int a = dp2a_lo_ss((int)xv.x, (int)tv.x, ia[t][j & 1]);
-                a = dp2a_hi_ss((int)xv.y, (int)tv.x, a);
-                ia[t][j & 1] = dp2a_lo_ss((int)xv.z, (int)tv.y, a);
-            }
-        }
-        const float scale = half_bits_to_float(cur[6] >> 16);
-        #pragma unroll
-        for (int t = 0; t < TB; ++t)
-            acc[t] = fmaf((float)(ia[t][0] + ia[t][1]), scale * xs[t * p.nb + bb], acc[t]);
-        if ((s + 1) % steps_per_row == 0) {   // row done (warp-uniform)
-            const int r = row_begin + warp + (s / steps_per_row) * TQ_WARPS;
-            #pragma unroll
-            for (int t = 0; t < TB; ++t) {
-                float v = acc[t];
                 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0) store_out(y + (int64_t)t * p.n + r, v);
-                acc[t] = 0.f;
+                for (int h = 0; h < 2; ++h) {
+                    int a = dp2a_lo_ss((int)xv.x, (int)tv[h].x, ia[h][t][j & 1]);
+                    a = dp2a_hi_ss((int)xv.y, (int)tv[h].x, a);
+                    ia[h][t][j & 1] = dp2a_lo_ss((int)xv.z, (int)tv[h].y, a);
+                }
             }
         }
         #pragma unroll
-        for (int j = 0; j < 7; ++j) cur[j] = nxt[j];
+        for (int h = 0; h < 2; ++h) {
+            const float scale = half_bits_to_float(cur[h][6] >> 16);
+            #pragma unroll
+            for (int t = 0; t < TB; ++t)
+                acc[h][t] = fmaf((float)(ia[h][t][0] + ia[h][t][1]), scale * xs[t * p.nb + bb], acc[h][t]);
+        }
+        if ((s + 1) % steps_per_row == 0) {
+            const int pr = s / steps_per_row;
+            #pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int i = 2 * pr + h;
+                #pragma unroll
+                for (int t = 0; t < TB; ++t) {
+                    float v = acc[h][t];
+                    #pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                    if (lane == 0 && i < my_rows) store_out(y + (int64_t)t * p.n + row_begin + warp + i * TQ_WARPS, v);
+                    acc[h][t] = 0.f;
+                }
+            }
+        }
+        #pragma unroll
+        for (int h = 0; h < 2; ++h)
+            #pragma unroll
+            for (int j = 0; j < 7; ++j) cur[h][j] = nxt[h][j];
     }
     if (p.indep) griddep_wait();   // complete after the work before it (stream order)
 }
