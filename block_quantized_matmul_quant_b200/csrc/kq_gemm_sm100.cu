@@ -213,21 +213,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t r[32]) 
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// A warp's wait on an mbarrier phase, with one outcome for the whole warp.
-// KQ_GEMM_LANE0_WAIT: lane 0 alone polls and the warp follows it (the
-// barrier sees one poller instead of 32); otherwise every lane polls.
-#ifndef KQ_GEMM_LANE0_WAIT
-#define KQ_GEMM_LANE0_WAIT 0
-#endif
+// A warp's wait on an mbarrier phase, with one outcome for the whole warp
+// (every lane polls: measured faster than lane 0 polling alone).
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
-#if KQ_GEMM_LANE0_WAIT
-    bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err);
-    __syncwarp();
-    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-#else
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, err));
-#endif
 }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups

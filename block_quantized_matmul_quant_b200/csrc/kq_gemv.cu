@@ -43,9 +43,6 @@ namespace {
 #ifndef KQ_GEMV_XREG
 #define KQ_GEMV_XREG 1
 #endif
-#ifndef KQ_GEMV_LANE0_WAIT
-#define KQ_GEMV_LANE0_WAIT 0
-#endif
 #ifndef KQ_GEMV_SHARE_WARPS
 #define KQ_GEMV_SHARE_WARPS 4
 #endif
@@ -67,12 +64,6 @@ constexpr int GEMV_MAX_SLOTS = 4;
 #endif
 constexpr int GEMV_HALF_MAX_SLOTS = KQ_GEMV_SHARE_SLOTS;
 // Independent calls spread over (SMs / KQ_GEMV_SHARE_GRID_DIV) CTAs.
-// When an independent call's CTA asks L2 for the rows beyond its ring's first
-// fill: 0 after its first activation loads, 1 before them, 2 never (measured
-// fastest: the ring alone keeps enough bytes in flight).
-#ifndef KQ_GEMV_PREFETCH_MODE
-#define KQ_GEMV_PREFETCH_MODE 2
-#endif
 #ifndef KQ_GEMV_SHARE_GRID_DIV
 #define KQ_GEMV_SHARE_GRID_DIV 2
 #endif
@@ -292,22 +283,16 @@ __device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w,
             for (int i = 0; i < first; ++i) issue(i);
         prefetch_rest();
     }
-#if KQ_GEMV_PREFETCH_MODE == 1
-    if (p.indep) prefetch_rest();
-#endif
     if (!p.indep) griddep_wait();
     // Otherwise the activation loads go out first (they gate every row; an
     // independent call's are ready at once) and the row copies follow right
-    // behind them.
+    // behind them.  An independent call asks L2 for nothing more: its ring
+    // keeps enough bytes in flight (an L2 prefetch of its rows, before or
+    // after staging, measured slower).
     stage_activations<C, TB, XT>(p, tok, xq, xsc, xsum, [&]() {
-        if (!copies_first) {
-            if (lane == 0) {
-                fence_proxy_async_smem();  // generic reads of the slots in an earlier pass
-                for (int i = 0; i < first; ++i) issue(i);
-            }
-#if KQ_GEMV_PREFETCH_MODE == 0
-            if (p.indep) prefetch_rest();
-#endif
+        if (!copies_first && lane == 0) {
+            fence_proxy_async_smem();  // generic reads of the slots in an earlier pass
+            for (int i = 0; i < first; ++i) issue(i);
         }
     });
     __syncthreads();
@@ -340,19 +325,11 @@ __device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w,
             const int ii = base + i + min(r, nr - 1);
             const int slot = ii % p.slots;
             if (r < nr) {
-#if KQ_GEMV_LANE0_WAIT
-                // lane 0 polls, the warp follows it
-                bool ok = true;
-                if (lane == 0) ok = mbar_wait(&my_full[slot], (uint32_t)(ii / p.slots) & 1u, p.err);
-                __syncwarp();
-                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return false;
-#else
                 // a landed row costs one non-blocking poll (measured faster than
-                // going straight to the suspending wait)
+                // going straight to the suspending wait); one outcome per warp
                 const uint32_t par = (uint32_t)(ii / p.slots) & 1u;
                 if (!__all_sync(0xffffffffu, mbar_test_wait(&my_full[slot], par) || mbar_wait(&my_full[slot], par, p.err)))
                     return false;
-#endif
             }
             rowp[r] = my_ring + slot * row_bytes;
         }

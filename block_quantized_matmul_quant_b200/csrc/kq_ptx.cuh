@@ -65,15 +65,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Bounded wait; returns false (and flags the device error word) on timeout.
-// KQ_WAIT_FASTPATH: one non-blocking poll first, so that a phase which has
-// already completed costs no suspend-capable wait.
-#ifndef KQ_WAIT_FASTPATH
-#define KQ_WAIT_FASTPATH 0
-#endif
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
-#if KQ_WAIT_FASTPATH
-    if (mbar_test_wait(bar, parity)) return true;
-#endif
     for (uint32_t i = 0; i < KQ_SPIN_LIMIT; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     atomicOr(err, ERR_TIMEOUT);
