@@ -154,6 +154,9 @@ KQ_API int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k,
  * Tokens routed to one expert are grouped before the decode, so each hit
  * expert's weights are streamed once per group of tokens; the result of a
  * (t, s) row does not depend on the other tokens' ids.
+ * Paths: Q4_K with bf16 x runs the grouped tensor-core GEMM (weights
+ * rounded to bf16, like kq_matmul's GEMM); Q4_K with fp32 x the grouped
+ * mat-vec (exact fp32 weights); other codecs the plain grouped kernel.
  */
 KQ_API size_t kq_matmul_id_workspace_bytes(int64_t n_tokens, int64_t top_k, int64_t n_experts);
 KQ_API int kq_matmul_id(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,

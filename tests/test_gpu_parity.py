@@ -183,6 +183,41 @@ def test_matmul_gemv_independent_calls_back_to_back(kq):
     assert kq.device_status() == 0
 
 
+def test_independent_flag_on_other_paths_keeps_stream_order(kq):
+    """The flag is honoured by the bandwidth kernels only; the plain and the
+    tensor-core kernels keep stream order and give their usual result."""
+    import torch
+
+    r = rng(31)
+    n, k, m = 300, 1024, 20
+    w = synth.gen_weights(synth.Q4_K, n, k, r)
+    x = synth.gen_x(m, k, "bf16", r)
+    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    ref = oracle.matmul(synth.Q4_K, w, k, x, threads=8)
+    for path in (kq.PATH_SIMPLE, kq.PATH_GEMM):
+        a = kq.matmul(wd, synth.Q4_K, xd, path=path).cpu().numpy()
+        b = kq.matmul(wd, synth.Q4_K, xd, path=path, independent=True).cpu().numpy()
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+        assert row_rel_err(b, ref) <= TOL["bf16"]
+    assert kq.device_status() == 0
+
+
+def test_tq1_auto_beyond_eight_rows_uses_the_plain_kernel(kq):
+    r = rng(32)
+    n, k, m = 100, 1280, 11
+    w = synth.gen_weights(synth.TQ1_G128, n, k, r)
+    x = synth.gen_x(m, k, "f32", r)
+    ref = oracle.matmul(synth.TQ1_G128, w, k, x, threads=8)
+    wd, xd = to_device_w(w), to_device_x(x, "f32")
+    y = kq.matmul(wd, synth.TQ1_G128, xd).cpu().numpy()
+    ys = kq.matmul(wd, synth.TQ1_G128, xd, path=kq.PATH_SIMPLE).cpu().numpy()
+    assert np.array_equal(y.view(np.uint32), ys.view(np.uint32))   # the plain kernel served it
+    assert row_rel_err(y, ref) <= FP32_PATH_TOL
+    yg = kq.matmul(wd, synth.TQ1_G128, xd, path=kq.PATH_GEMV).cpu().numpy()   # six launches of two rows
+    assert row_rel_err(yg, ref) <= GEMV_TOL
+    assert kq.device_status() == 0
+
+
 def test_matmul_gemv_deterministic(kq):
     r = rng(7)
     w = synth.gen_weights(synth.Q4_K, 4096, 4096, r)
