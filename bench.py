@@ -53,11 +53,38 @@ def load_peaks():
                 "source": "fallback"}
 
 
-def kernel_source_hash(names):
+def strip_comments(src: str) -> str:
+    """C/C++ source without comments and whitespace (the code a capture ran)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        if src.startswith("//", i):
+            i = src.find("\n", i)
+            i = n if i < 0 else i
+        elif src.startswith("/*", i):
+            i = src.find("*/", i + 2)
+            i = n if i < 0 else i + 2
+        elif src[i] in "\"'":
+            q, j = src[i], i + 1
+            while j < n and src[j] != q:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(src[i])
+            i += 1
+    return "".join("".join(out).split())
+
+
+def kernel_source_hash(names, read=None):
+    """Hash of the kernel sources' code (comments and whitespace ignored)."""
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "block_quantized_matmul_quant_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        if read is None:
+            with open(os.path.join(ROOT, "block_quantized_matmul_quant_b200", "csrc", n)) as f:
+                text = f.read()
+        else:
+            text = read(n)
+        h.update(strip_comments(text).encode())
     return h.hexdigest()[:16]
 
 

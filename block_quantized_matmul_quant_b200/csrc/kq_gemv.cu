@@ -5,16 +5,20 @@
 // `kernel_mul_mv_q8_0_f32` and mlx-native's `kernel_mul_mv_id_*` family).
 //
 // B200 design
-//  * Grid = one CTA per SM.  A CTA owns a contiguous range of weight rows;
-//    warp w of the CTA owns rows w, w + W, w + 2W, ... of that range and
-//    streams them through a private ring of shared-memory row slots with
-//    cp.async.bulk copies (one per row, completion counted on one mbarrier
-//    per slot).  Each warp starts on its first row as soon as that row has
-//    landed; the ring keeps the next rows in flight without registers.
+//  * A CTA owns a contiguous range of weight rows; warp w of the CTA owns
+//    rows w, w + W, w + 2W, ... of that range and streams them through a
+//    private ring of shared-memory row slots with cp.async.bulk copies (one
+//    per row, completion counted on one mbarrier per slot).  Each warp starts
+//    on its first row as soon as that row has landed; the ring keeps the
+//    next rows in flight without registers.
+//  * Two CTA shapes.  A call ordered after the preceding kernel: one CTA per
+//    SM, 16 warps (its latency is what counts).  A call declared independent
+//    of earlier work: a third of an SM per CTA (4 warps) on half as many
+//    CTAs as SMs, so three calls stream side by side on every SM.
 //  * Activations are staged once per CTA as 16-bit fixed point per 32-wide
-//    sub-block: x ~= s * xq with s a power of two chosen from the
-//    sub-block's largest |x| (|xq| <= 32767, error <= 2^-15 of that maximum,
-//    exact for bf16 inputs whose exponent is within 7 of the maximum's), plus
+//    sub-block: x ~= s * xq with s = 2^(e-13), e = floor(log2) of the
+//    sub-block's largest |x| (|xq| < 2^14, error <= 2^-14 of that maximum,
+//    exact for bf16 inputs whose exponent is within 6 of the maximum's), plus
 //    the fp32 sum of the sub-block.  The mlx-kquant pages ship int8
 //    activation kernels for the same reason (arm64 NEON int8 GEMV); 16 bits
 //    keep the error near 1e-5, far inside the 2e-3 / 1e-2 bars.
@@ -26,7 +30,9 @@
 //    turns the integer sums into the product; every 32-weight sum fits int32.
 //  * Programmatic dependent launch: activations are read after
 //    griddepcontrol.wait.  When the caller declares the weights constant the
-//    row copies are issued before it, overlapping the previous kernel.
+//    row copies are issued before it, overlapping the previous kernel; an
+//    independent call never waits before its work and waits once at its end,
+//    so that it completes after the work before it.
 #include "kq_ptx.cuh"
 #include "kq_launch.h"
 
