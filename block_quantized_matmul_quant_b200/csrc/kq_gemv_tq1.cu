@@ -29,7 +29,9 @@
 //  * Weights are read straight from global memory, one block (28 bytes) per
 //    lane and row, with the next blocks' words loaded before the current
 //    ones are used; each CTA first asks L2 to prefetch its whole row range,
-//    so the stream runs at HBM speed while the lanes compute.
+//    so the weights are on chip when the lanes reach them.  The lanes'
+//    shared-memory loads, not the weight stream, bound the kernel (about a
+//    sixth of the copy bandwidth).
 #include "kq_ptx.cuh"
 #include "kq_launch.h"
 
