@@ -505,6 +505,28 @@ def test_matmul_id_bad_ids_poison_rows(kq):
     assert kq.device_status() == 0
 
 
+@pytest.mark.parametrize("xdt,path", [("f32", "auto"), ("bf16", "auto"), ("bf16", "gemm"), ("f32", "simple")])
+def test_matmul_id_all_ids_invalid(kq, xdt, path):
+    """No valid pair: the grouping leaves every expert empty (zero token
+    tiles for the tensor-core path, zero passes for the grouped GEMV), every
+    output row is the poison sentinel and the error word is set once."""
+    import torch
+
+    e, n, k, t, top_k = 3, 140, 512, 24, 2
+    r = rng(13)
+    w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, xdt, r)
+    ids = np.where(np.arange(t * top_k).reshape(t, top_k) % 2 == 0, e, -1).astype(np.int32)
+    p = {"auto": kq.PATH_AUTO, "gemm": kq.PATH_GEMM, "simple": kq.PATH_SIMPLE}[path]
+    y = kq.matmul_id(to_device_w(w), synth.Q4_K, to_device_x(x, xdt), torch.from_numpy(ids).cuda(),
+                     path=p).float().cpu().numpy()
+    assert y.shape == (t, top_k, n)
+    assert np.all(np.isnan(y))
+    assert np.all(np.isnan(oracle.matmul_id(synth.Q4_K, w, k, x, ids)))
+    assert kq.device_status() == -9
+    assert kq.device_status() == 0
+
+
 # ---------------------------------------------------------------- errors on device arguments
 
 def test_error_codes(kq):
