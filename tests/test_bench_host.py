@@ -53,3 +53,26 @@ def test_committed_traffic_entries_are_well_formed():
             continue
         assert len(e["source_hash"]) == 16
         assert e["dram_bytes_per_launch"] > 0
+
+
+def test_reference_arm_prints_one_contract_line(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+
+    class A:
+        workload = "q4_k_gemv_4096x4096"
+        steps, warmup = 1, 0
+
+    bench.run_reference(A())
+    lines = capsys.readouterr().out.strip().splitlines()
+    assert len(lines) == 1
+    r = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config"):
+        assert key in r
+    assert r["impl"] == "reference" and r["value"] > 0 and r["higher_is_better"] is True
+    assert r["config"]["workload"] == "q4_k_gemv_4096x4096"
+    cb = r["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == r["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert r["e2e"] == {"value": r["value"], "unit": r["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
