@@ -285,26 +285,33 @@ def secondary_metrics(torch, kq, l2, peaks):
         st = PoolStep(torch, kq, wl, l2)
         ms = time_graph(torch, st.run, 5, 3, None)
         us = ms * 1e3 / (5 * st.pool)
-        if wl.kind == "gemm":
-            tf = 2.0 * wl.m * wl.n * wl.k / (us * 1e-6) / 1e12
-            out[name] = {"us_per_call": round(us, 2), "TFLOP/s": round(tf, 1),
-                         "frac_burst": round(tf / peaks["bf16_tflops"], 4),
-                         "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
-                         "kernel": "gemm_q4k_kernel (tcgen05)"}
-        elif wl.kind == "moe":
-            per_expert = st.wbytes // wl.n_experts
-            moved = st.hit_experts * per_expert + wl.m * wl.k * 2 + wl.m * wl.top_k * wl.n * 4
-            out[name] = {"us_per_call": round(us, 2), "tokens/s": round(wl.m / (us * 1e-6), 1),
-                         "GB/s": round(moved / (us * 1e-6) / 1e9, 1),
-                         "frac_hbm": round(moved / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
-                         "hit_experts": st.hit_experts, "kernel": "moe_group + grouped product"}
-        else:
-            gbs = st.wbytes / (us * 1e-6) / 1e9
-            out[name] = {"us_per_call": round(us, 3), "weight GB/s": round(gbs, 1),
-                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        out[name] = secondary_entry(wl, us, st.wbytes, getattr(st, "hit_experts", 0), peaks)
         del st
         torch.cuda.empty_cache()
     return out
+
+
+def secondary_entry(wl, us, wbytes, hit_experts, peaks):
+    """One secondary workload's figures from its time per call."""
+    if wl.kind == "gemm":
+        tf = 2.0 * wl.m * wl.n * wl.k / (us * 1e-6) / 1e12
+        return {"us_per_call": round(us, 2), "TFLOP/s": round(tf, 1),
+                "frac_burst": round(tf / peaks["bf16_tflops"], 4),
+                "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+                "kernel": "gemm_q4k_kernel (tcgen05)"}
+    if wl.kind == "moe":
+        per_expert = wbytes // wl.n_experts
+        moved = hit_experts * per_expert + wl.m * wl.k * 2 + wl.m * wl.top_k * wl.n * 4
+        # consecutive calls share the ids and use different expert stacks:
+        # a gate projection followed by an up projection
+        return {"us_per_call": round(us, 2), "gate_up_pair_us": round(2 * us, 2),
+                "tokens/s": round(wl.m / (us * 1e-6), 1),
+                "GB/s": round(moved / (us * 1e-6) / 1e9, 1),
+                "frac_hbm": round(moved / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                "hit_experts": hit_experts, "kernel": "moe_group + grouped product"}
+    gbs = wbytes / (us * 1e-6) / 1e9
+    return {"us_per_call": round(us, 3), "weight GB/s": round(gbs, 1),
+            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
 
 
 def time_graph(torch, fn, steps, warmup, pg):

@@ -76,3 +76,52 @@ def test_reference_arm_prints_one_contract_line(monkeypatch, capsys):
     assert cb["kind"] == "oracle" and cb["value"] == r["value"] and cb["cores"] >= 1 and cb["sample"]
     assert r["e2e"] == {"value": r["value"], "unit": r["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+PEAKS = {"hbm_gbs": 6468.0, "bf16_tflops": 1644.2, "bf16_tflops_sustained": 1385.2}
+
+
+def test_secondary_entry_figures():
+    import synth
+
+    g = bench.secondary_entry(synth.WORKLOADS["q4_k_gemm_512x11008x4096"], 67.2, 0, 0, PEAKS)
+    tf = 2 * 512 * 11008 * 4096 / 67.2e-6 / 1e12
+    assert g["TFLOP/s"] == round(tf, 1)
+    assert g["frac_burst"] == round(tf / 1644.2, 4) and g["frac_sustained"] == round(tf / 1385.2, 4)
+
+    wl = synth.WORKLOADS["moe_q4_k_e64_1408x2048_t32_top6"]
+    wbytes = 64 * 1408 * (2048 // 256) * 144
+    m = bench.secondary_entry(wl, 83.0, wbytes, 63, PEAKS)
+    moved = 63 * 1408 * 8 * 144 + 32 * 2048 * 2 + 32 * 6 * 1408 * 4
+    assert moved == 103_399_424
+    assert m["GB/s"] == round(moved / 83.0e-6 / 1e9, 1)
+    assert m["gate_up_pair_us"] == 166.0 and m["tokens/s"] == round(32 / 83.0e-6, 1)
+
+    v = bench.secondary_entry(synth.WORKLOADS["tq1_g128_gemv_5120x17408"], 17.9, 19_496_960, 0, PEAKS)
+    assert v["weight GB/s"] == round(19_496_960 / 17.9e-6 / 1e9, 1)
+    assert v["frac_hbm"] == round(19_496_960 / 17.9e-6 / 1e9 / 6468.0, 4)
+
+
+def test_secondary_metrics_call_site(monkeypatch):
+    """The timed loop's bookkeeping (time per call from the graph time) with
+    the GPU parts replaced by stand-ins."""
+    import types
+
+    class FakeStep:
+        def __init__(self, torch, kq, wl, l2):
+            self.wl, self.pool, self.wbytes = wl, 8, 1_000_000
+            if wl.kind == "moe":
+                self.hit_experts = 63
+
+        def run(self):
+            pass
+
+    monkeypatch.setattr(bench, "PoolStep", FakeStep)
+    monkeypatch.setattr(bench, "time_graph", lambda torch, fn, steps, warmup, pg: 0.4)  # ms per 5 steps
+    fake_torch = types.SimpleNamespace(cuda=types.SimpleNamespace(empty_cache=lambda: None))
+    out = bench.secondary_metrics(fake_torch, None, 0, PEAKS)
+    assert set(out) == {"q4_k_gemm_512x11008x4096", "moe_q4_k_e64_1408x2048_t32_top6",
+                        "tq1_g128_gemv_5120x17408", "q8_0_gemv_256x1024"}
+    us = 0.4 * 1e3 / (5 * 8)
+    assert out["q8_0_gemv_256x1024"]["us_per_call"] == round(us, 3)
+    assert out["moe_q4_k_e64_1408x2048_t32_top6"]["hit_experts"] == 63
