@@ -50,6 +50,9 @@
  *            Q2_K, 84 B / 256 w: 16 scale/min bytes @0 (low nibble scale,
  *              high nibble min), 64 quant bytes @16 (four 2-bit quants each),
  *              fp16 d @80, fp16 dmin @82;  w = float(d)*sc*q - float(dmin)*m.
+ *          Parity unpinned against an external GGUF file (none is at hand):
+ *          the tests pin these two decoders to blocks built by packers written
+ *          separately from this file, field by field.
  *
  * Products in the fp32 decode are exact (at most 21 significant bits), so the
  * one rounding is the final subtraction; the decode result is unique.
