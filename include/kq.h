@@ -22,8 +22,11 @@
  *    outputs y row-major [M, N]; all contiguous.
  *  * Alignment: w, x, y, out, ids and workspace must be 16-byte aligned.
  *  * Return value: KQ_OK (0) or a negative KQ_ERR_* code.  Every argument is
- *    validated on the host before anything is enqueued, so an error return
- *    means no work was launched (no partial output).
+ *    validated on the host before anything is enqueued, so an argument error
+ *    means no work was launched (no partial output).  KQ_ERR_CUDA (a failed
+ *    launch) from a call made of several kernels (kq_matmul_id: grouping,
+ *    then the product) may follow the launch of its earlier kernels; the
+ *    output is then unspecified.
  *  * Floating-point dtypes: KQ_F32, KQ_BF16 (and KQ_F16 for kq_dequantize's
  *    output).  Accumulation is always fp32.
  */

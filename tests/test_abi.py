@@ -81,3 +81,29 @@ def test_argument_errors_before_any_launch(L):
                           None) == -7
     # overflow of n * row bytes
     assert L.kq_matmul(12, fake, 1 << 60, 256, fake, 1, 1, fake, 0, None) == -6
+
+
+def test_more_argument_errors_before_any_launch(L):
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)
+    odd = vp((1 << 20) + 4)
+    assert L.kq_matmul(12, fake, 4, 256, fake, 1, 0, fake, 0, None) == -1          # m = 0
+    assert L.kq_matmul(12, fake, 4, 256, None, 1, 1, fake, 0, None) == -1          # null x
+    assert L.kq_matmul(12, fake, 4, 256, fake, 1, 1, None, 0, None) == -1          # null y
+    assert L.kq_matmul(12, fake, 4, 256, fake, 1, 1, odd, 0, None) == -5           # y alignment
+    assert L.kq_matmul_ex(12, fake, 4, 256, fake, 1, 1, fake, 0, 7, None) == -1    # unknown path
+    assert L.kq_dequantize(12, fake, 2, 256, fake, 9, None) == -4                  # out dtype
+    ws = L.kq_matmul_id_workspace_bytes(4, 2, 3)
+
+    def mid(n_experts=3, stride=8 * 144, ids=fake, top_k=2, work=fake, wsb=ws, path=0):
+        return L.kq_matmul_id_ex(12, fake, n_experts, 8, 256, stride, fake, 1, 4, ids, top_k, fake, 0,
+                                 work, wsb, path, None)
+
+    assert mid(stride=8 * 144 + 8) == -3             # expert stride not a multiple of 16
+    assert mid(ids=None) == -1
+    assert mid(ids=odd) == -5
+    assert mid(top_k=0) == -1
+    assert mid(n_experts=70000, top_k=2) == -1       # beyond the grid's expert dimension
+    assert mid(work=None) == -7
+    assert mid(work=odd) == -5
+    assert mid(path=9) == -1
