@@ -25,8 +25,9 @@
  *    validated on the host before anything is enqueued, so an argument error
  *    means no work was launched (no partial output).  KQ_ERR_CUDA (a failed
  *    launch) from a call made of several kernels (kq_matmul_id: grouping,
- *    then the product) may follow the launch of its earlier kernels; the
- *    output is then unspecified.
+ *    then the product; the bandwidth kernel: one launch per eight activation
+ *    rows) may follow the launch of its earlier kernels; the output is then
+ *    unspecified.
  *  * Floating-point dtypes: KQ_F32, KQ_BF16 (and KQ_F16 for kq_dequantize's
  *    output).  Accumulation is always fp32.
  */
