@@ -1,5 +1,6 @@
 // kq_api.cu -- the C ABI (include/kq.h): argument validation, dispatch and
 // the device status word.  All validation happens before any launch.
+#include <atomic>
 #include <mutex>
 #include <string.h>
 
@@ -11,17 +12,39 @@ namespace kq {
 __device__ unsigned long long g_scan_first_bad;
 __device__ unsigned int g_error_word = 0;
 
-// Device address of this device's error word (cached per device ordinal).
-unsigned int *error_word() {
-    static unsigned int *cache[64];
+// Per-device host caches below are atomics: calls may come from several
+// host threads, and each thread that finds an entry empty stores the same
+// value.
+static int current_device() {
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    if (cache[dev] == nullptr) {
+    return dev >= 0 && dev < 64 ? dev : 0;
+}
+
+// Device address of this device's error word (cached per device ordinal).
+unsigned int *error_word() {
+    static std::atomic<unsigned int *> cache[64];
+    const int dev = current_device();
+    unsigned int *w = cache[dev].load(std::memory_order_relaxed);
+    if (w == nullptr) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_error_word) == cudaSuccess) cache[dev] = static_cast<unsigned int *>(p);
+        if (cudaGetSymbolAddress(&p, g_error_word) == cudaSuccess) {
+            w = static_cast<unsigned int *>(p);
+            cache[dev].store(w, std::memory_order_relaxed);
+        }
     }
-    return cache[dev];
+    return w;
+}
+
+int sm_count() {
+    static std::atomic<int> cache[64];
+    const int dev = current_device();
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        cache[dev].store(v, std::memory_order_relaxed);
+    }
+    return v;
 }
 
 static int block_weights(int type) {
@@ -48,18 +71,20 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // Current device must be sm_100 (B200); cached per device ordinal.
 static int check_device() {
-    static int cache[64];  // 0 unknown, 1 ok, -1 not sm_100
+    static std::atomic<int> cache[64];  // 0 unknown, 1 ok, -1 not sm_100
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return KQ_ERR_CUDA;
     if (dev < 0 || dev >= 64) return KQ_ERR_UNSUPPORTED;
-    if (cache[dev] == 0) {
+    int c = cache[dev].load(std::memory_order_relaxed);
+    if (c == 0) {
         int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
             return KQ_ERR_CUDA;
-        cache[dev] = (major == 10 && minor == 0) ? 1 : -1;
+        c = (major == 10 && minor == 0) ? 1 : -1;
+        cache[dev].store(c, std::memory_order_relaxed);
     }
-    return cache[dev] == 1 ? KQ_OK : KQ_ERR_UNSUPPORTED;
+    return c == 1 ? KQ_OK : KQ_ERR_UNSUPPORTED;
 }
 
 static int to_status(cudaError_t e) { return e == cudaSuccess ? KQ_OK : KQ_ERR_CUDA; }

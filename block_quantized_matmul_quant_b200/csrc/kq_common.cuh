@@ -22,6 +22,8 @@ template <> struct Geom<KQ_TQ1_G128> { static constexpr int QK = 128; static con
 // (error_word() on the host), since each translation unit is compiled
 // without relocatable device code.
 unsigned int *error_word();
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count();
 constexpr unsigned ERR_BAD_ID = 1u;
 constexpr unsigned ERR_TIMEOUT = 2u;
 

@@ -600,18 +600,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-int num_sms() {
-    static int cached[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    if (!cached[dev]) {
-        int v = 0;
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-        cached[dev] = v > 0 ? v : 148;
-    }
-    return cached[dev];
-}
 
 // Choose BN (tokens per tile).  A stage of a tile costs about the larger of
 // its MMAs (4 x BN/2 cycles for 128 x BN x 64) and the decode of its 128 x 64
@@ -762,7 +750,7 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
                         void *y, int ydt, cudaStream_t s) {
     (void)type;
     if (!encode_fn() || m < 1 || m > (1 << 30)) return cudaErrorNotSupported;
-    const int sms = num_sms();
+    const int sms = sm_count();
     GemmParams p = {};
     p.n = (int)n; p.k = (int)k; p.m = (int)m;
     p.n_tiles = (int)((n + BM - 1) / BM);
@@ -797,7 +785,7 @@ int gemm_id_bn(int64_t n_tokens, int64_t top_k, int64_t n_experts) {
 
 cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     if (!encode_fn()) return cudaErrorNotSupported;
-    const int sms = num_sms();
+    const int sms = sm_count();
     GemmParams p = {};
     p.n = (int)a.n; p.k = (int)a.k; p.m = (int)a.n_tokens;
     p.n_tiles = (int)((a.n + BM - 1) / BM);

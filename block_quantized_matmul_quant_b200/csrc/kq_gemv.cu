@@ -570,19 +570,6 @@ bool plan_gemv(int type, int64_t n, int64_t k, int64_t m, int num_sms, int max_w
     return false;
 }
 
-int sm_count() {
-    static int cached[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    if (cached[dev] == 0) {
-        int v = 0;
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-        cached[dev] = v > 0 ? v : 148;
-    }
-    return cached[dev];
-}
-
 template <int C, int TB, bool XREG, typename XT, typename YT>
 cudaError_t launch_q4k(GemvParams p, GemvOrder order, cudaStream_t s) {
     // half-SM build when the plan fits it (independent calls)

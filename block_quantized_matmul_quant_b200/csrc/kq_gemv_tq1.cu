@@ -279,18 +279,6 @@ cudaError_t launch_tq1_tb(const Tq1Params &p, int xdt, int ydt, cudaStream_t s) 
                          : launch_tq1_t<TB, __nv_bfloat16, __nv_bfloat16>(p, s);
 }
 
-int tq1_sms() {
-    static int cached[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    if (!cached[dev]) {
-        int v = 0;
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-        cached[dev] = v > 0 ? v : 148;
-    }
-    return cached[dev];
-}
 
 }  // namespace
 
@@ -307,7 +295,7 @@ cudaError_t launch_gemv_tq1(const void *w, int64_t n, int64_t k, const void *x, 
     const int nb = (int)(k / TQ_QK);
     const int tb_max = tq1_smem_bytes(2, nb) <= (size_t)TQ_SMEM_LIMIT ? 2 : 1;
     const size_t xs = (xdt == KQ_F32 ? 4 : 2), ys = (ydt == KQ_F32 ? 4 : 2);
-    const int sms = tq1_sms();
+    const int sms = sm_count();
     for (int64_t m0 = 0; m0 < m; m0 += tb_max) {
         const int tb = (int)(m - m0 < tb_max ? m - m0 : tb_max);
         Tq1Params p = {};
