@@ -2,7 +2,8 @@
 
 Argument marshalling only: every step of the computation runs in the CUDA
 kernels of ``libkq.so`` (built in-tree from ``csrc/`` by ``_build.py``).  torch
-supplies device memory and the current stream.  There is no CPU fallback:
+supplies device memory and the current stream; each buffer's shape, dtype,
+layout and device are checked here, since the C ABI receives bare pointers.  There is no CPU fallback:
 when the library is missing or the device is not an sm_100 GPU the calls
 raise.
 """
@@ -110,9 +111,34 @@ def row_bytes(codec, k: int) -> int:
     return int(lib().kq_row_bytes(_codec(codec), int(k)))
 
 
+def _on_current_device(name: str, t: torch.Tensor):
+    # the library works on the current CUDA device; its pointers must live there
+    if not t.is_cuda or t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} must be a CUDA tensor on the current device, not {t.device}")
+
+
+def _check_tensor(name: str, t: torch.Tensor, shape, dtypes, device):
+    """The C ABI takes plain pointers, so sizes are checked here: a buffer of
+    the wrong shape would be read or written past its end."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}; expected one of {sorted(map(str, dtypes))}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the weights on {device}")
+
+
+_ACT = (torch.float32, torch.bfloat16)
+
+
 def _weights(w: torch.Tensor, codec: int, k: int):
     if w.dtype != torch.uint8 or not w.is_contiguous() or not w.is_cuda:
         raise ValueError("w must be a contiguous uint8 CUDA tensor of wire blocks")
+    _on_current_device("w", w)
     rb = row_bytes(codec, k)
     if rb <= 0 or w.numel() % rb:
         raise ValueError(f"w holds {w.numel()} bytes, not a whole number of {rb}-byte rows")
@@ -125,6 +151,7 @@ def dequantize(w: torch.Tensor, codec, k: int, dtype=torch.float32, out=None) ->
     rows = _weights(w, c, k)
     if out is None:
         out = torch.empty((rows, k), dtype=dtype, device=w.device)
+    _check_tensor("out", out, (rows, k), tuple(_DT), w.device)
     _check(lib().kq_dequantize(c, _ptr(w), rows, k, _ptr(out), _DT[out.dtype], _stream()),
            "kq_dequantize")
     return out
@@ -143,8 +170,10 @@ def matmul(w: torch.Tensor, codec, x: torch.Tensor, out=None, out_dtype=torch.fl
         raise ValueError("x must be a contiguous [m, k] tensor")
     m, k = x.shape
     n = _weights(w, c, k)
+    _check_tensor("x", x, (m, k), _ACT, w.device)
     if out is None:
         out = torch.empty((m, n), dtype=out_dtype, device=x.device)
+    _check_tensor("out", out, (m, n), _ACT, w.device)
     flags = path | (FLAG_CONST_WEIGHTS if const_weights else 0) | (FLAG_INDEPENDENT if independent else 0)
     _check(lib().kq_matmul_ex(c, _ptr(w), n, k, _ptr(x), _DT[x.dtype], m, _ptr(out),
                               _DT[out.dtype], flags, _stream()), "kq_matmul")
@@ -160,20 +189,31 @@ def matmul_id(w: torch.Tensor, codec, x: torch.Tensor, ids: torch.Tensor, out=No
     """y[t, s, n] = sum_k dequant(w[ids[t, s]])[n, k] * x[t, k].
     w: [E, n, row_bytes] uint8; x: [T, k]; ids: [T, top_k] int32."""
     c = _codec(codec)
-    if w.dim() != 3:
-        raise ValueError("w must be [n_experts, n, row_bytes]")
+    if w.dim() != 3 or w.dtype != torch.uint8:
+        raise ValueError("w must be uint8 [n_experts, n, row_bytes]")
     e, n, rb = w.shape
+    if x.dim() != 2:
+        raise ValueError("x must be [n_tokens, k]")
     t, k = x.shape
     if rb != row_bytes(c, k):
         raise ValueError("w's last dimension does not match k")
-    if ids.dtype != torch.int32 or ids.dim() != 2 or ids.shape[0] != t:
+    # rows of one expert packed back to back; experts w.stride(0) bytes apart
+    if w.stride(2) != 1 or w.stride(1) != rb:
+        raise ValueError("each expert's rows must be packed back to back")
+    _on_current_device("w", w)
+    _check_tensor("x", x, (t, k), _ACT, w.device)
+    if ids.dim() != 2:
         raise ValueError("ids must be int32 [n_tokens, top_k]")
     top_k = ids.shape[1]
+    _check_tensor("ids", ids, (t, top_k), (torch.int32,), w.device)
     if out is None:
         out = torch.empty((t, top_k, n), dtype=out_dtype, device=x.device)
+    _check_tensor("out", out, (t, top_k, n), _ACT, w.device)
     need = matmul_id_workspace_bytes(t, top_k, e)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or workspace.device != w.device:
+        raise ValueError("workspace must be a contiguous uint8 tensor on the weights' device")
     _check(lib().kq_matmul_id_ex(c, _ptr(w), e, n, k, w.stride(0), _ptr(x), _DT[x.dtype], t,
                                  _ptr(ids), top_k, _ptr(out), _DT[out.dtype], _ptr(workspace),
                                  workspace.numel(), path, _stream()), "kq_matmul_id")
@@ -182,6 +222,9 @@ def matmul_id(w: torch.Tensor, codec, x: torch.Tensor, ids: torch.Tensor, out=No
 
 def moe_group(ids: torch.Tensor, n_experts: int):
     """(counts [E], offsets [E+1], perm [P]) of the device-side expert grouping."""
+    if ids.dtype != torch.int32:
+        raise ValueError("ids must be int32")
+    _on_current_device("ids", ids)
     ids = ids.contiguous().view(-1)
     p = ids.numel()
     counts = torch.empty(n_experts, dtype=torch.int32, device=ids.device)

@@ -542,3 +542,24 @@ def test_error_codes(kq):
         kq.matmul(w, synth.Q4_K, xf, out=bad_out, path=kq.PATH_SIMPLE)
     assert ei.value.status == -5
     assert kq.device_status() == 0
+
+
+def test_binding_rejects_wrong_buffers_before_any_launch(kq):
+    """Buffers whose size the C ABI cannot see are checked by the binding."""
+    import torch
+
+    w = to_device_w(synth.gen_weights(synth.Q4_K, 8, 512, rng(2)))
+    x = torch.zeros((2, 512), dtype=torch.bfloat16, device="cuda")
+    for bad in (torch.empty((2, 7), device="cuda"), torch.empty((8, 2), device="cuda").t(),
+                torch.empty((2, 8), dtype=torch.float64, device="cuda")):
+        with pytest.raises(ValueError):
+            kq.matmul(w, synth.Q4_K, x, out=bad)
+    with pytest.raises(ValueError):
+        kq.dequantize(w, synth.Q4_K, 512, out=torch.empty((8, 256), device="cuda"))
+    we = w.view(2, 4, -1)
+    ids = torch.zeros((2, 1), dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError):
+        kq.matmul_id(we, synth.Q4_K, x, ids, out=torch.empty((2, 1, 3), device="cuda"))
+    with pytest.raises(ValueError):
+        kq.matmul_id(we, synth.Q4_K, x, ids.to(torch.int64))
+    assert kq.device_status() == 0
