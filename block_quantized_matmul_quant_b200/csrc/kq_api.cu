@@ -290,6 +290,9 @@ int kq_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_experts, int32_t
     if (!ids || !counts || !offsets || !perm) return KQ_ERR_ARG;
     if (n_pairs <= 0 || n_pairs > INT32_MAX || n_experts <= 0 || n_experts > 65535)
         return KQ_ERR_ARG;
+    auto aligned4 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; };
+    if (!aligned16(ids) || !aligned4(counts) || !aligned4(offsets) || !aligned4(perm))
+        return KQ_ERR_ALIGN;
     int st = check_device();
     if (st) return st;
     return to_status(launch_moe_group(ids, n_pairs, n_experts, counts, offsets, perm, nullptr,

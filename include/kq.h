@@ -213,7 +213,9 @@ KQ_API int kq_matmul_id_noalloc(int type, const void *w, int64_t n_experts, int6
  *            grouped by expert, ascending p inside each expert (a stable
  *            sort by expert id); pairs with an invalid id are left out and
  *            the tail perm[offsets[n_experts] ..] is set to -1 (device)
- * Sets the device error word if any id is outside [0, n_experts).
+ * ids must be 16-byte aligned (KQ_ERR_ALIGN otherwise), counts, offsets and
+ * perm 4-byte aligned.  Sets the device error word if any id is outside
+ * [0, n_experts).
  */
 KQ_API int kq_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_experts,
                  int32_t *counts, int32_t *offsets, int32_t *perm, void *stream);

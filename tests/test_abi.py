@@ -107,3 +107,13 @@ def test_more_argument_errors_before_any_launch(L):
     assert mid(work=None) == -7
     assert mid(work=odd) == -5
     assert mid(path=9) == -1
+
+
+def test_moe_group_argument_errors(L):
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)
+    assert L.kq_moe_group(None, 8, 4, fake, fake, fake, None) == -1
+    assert L.kq_moe_group(fake, 0, 4, fake, fake, fake, None) == -1
+    assert L.kq_moe_group(fake, 8, 70000, fake, fake, fake, None) == -1
+    assert L.kq_moe_group(vp((1 << 20) + 4), 8, 4, fake, fake, fake, None) == -5   # ids alignment
+    assert L.kq_moe_group(fake, 8, 4, vp((1 << 20) + 2), fake, fake, None) == -5   # counts alignment
