@@ -600,7 +600,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-
 // Choose BN (tokens per tile).  A stage of a tile costs about the larger of
 // its MMAs (4 x BN/2 cycles for 128 x BN x 64) and the decode of its 128 x 64
 // weights, which does not shrink with BN (about 400 cycles, measured): the

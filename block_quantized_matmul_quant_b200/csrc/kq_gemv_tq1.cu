@@ -279,7 +279,6 @@ cudaError_t launch_tq1_tb(const Tq1Params &p, int xdt, int ydt, cudaStream_t s) 
                          : launch_tq1_t<TB, __nv_bfloat16, __nv_bfloat16>(p, s);
 }
 
-
 }  // namespace
 
 bool gemv_tq1_supported(int64_t n, int64_t k) {
