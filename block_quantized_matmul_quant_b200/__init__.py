@@ -3,9 +3,9 @@
 Argument marshalling only: every step of the computation runs in the CUDA
 kernels of ``libkq.so`` (built in-tree from ``csrc/`` by ``_build.py``).  torch
 supplies device memory and the current stream; each buffer's shape, dtype,
-layout and device are checked here, since the C ABI receives bare pointers.  There is no CPU fallback:
-when the library is missing or the device is not an sm_100 GPU the calls
-raise.
+layout and device are checked here, since the C ABI receives bare pointers.
+There is no CPU fallback: when the library is missing or the device is not
+an sm_100 GPU the calls raise.
 """
 from __future__ import annotations
 
