@@ -125,3 +125,21 @@ def test_secondary_metrics_call_site(monkeypatch):
     us = 0.4 * 1e3 / (5 * 8)
     assert out["q8_0_gemv_256x1024"]["us_per_call"] == round(us, 3)
     assert out["moe_q4_k_e64_1408x2048_t32_top6"]["hit_experts"] == 63
+
+
+def test_clock_summary_reads_sampled_lines():
+    cs = bench.ClockSampler(0)
+    cs.lines = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1900, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1950, 1965, 800.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+        "0, [N/A], 1965, 1, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    s = cs.summary()
+    assert s["sm_mhz"] == 1950 and s["sm_max_mhz"] == 1965 and s["samples"] == 3
+    assert s["reasons"] == ["sw_power_cap"]
+    cs.lines = ["0, 1965, 1965, 700, 0x8, Active, Not Active, Not Active, Not Active"]
+    assert cs.summary()["reasons"] == ["hw_slowdown"]
+    cs.lines = []
+    assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
