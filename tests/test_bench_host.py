@@ -143,3 +143,14 @@ def test_clock_summary_reads_sampled_lines():
     assert cs.summary()["reasons"] == ["hw_slowdown"]
     cs.lines = []
     assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+
+
+def test_clocks_rejected_rules():
+    ok = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert not bench.clocks_rejected(ok)
+    assert not bench.clocks_rejected({"sm_mhz": 1300.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]})
+    assert bench.clocks_rejected({"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["hw_slowdown"]})
+    assert bench.clocks_rejected({"sm_mhz": 1900.0, "sm_max_mhz": 1965.0,
+                                  "reasons": ["sw_power_cap", "sw_thermal_slowdown"]})
+    assert bench.clocks_rejected({"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "reasons": []})   # stuck low
+    assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]})
