@@ -148,6 +148,11 @@ class ClockSampler:
             if len(parts) < 9:
                 continue
             try:
+                if int(parts[4], 16) & 1:   # GPU idle: not a sample under load
+                    continue
+            except ValueError:
+                pass
+            try:
                 sm.append(float(parts[1]))
                 mx.append(float(parts[2]))
             except ValueError:

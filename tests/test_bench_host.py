@@ -154,3 +154,14 @@ def test_clocks_rejected_rules():
                                   "reasons": ["sw_power_cap", "sw_thermal_slowdown"]})
     assert bench.clocks_rejected({"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "reasons": []})   # stuck low
     assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]})
+
+
+def test_clock_summary_skips_idle_samples():
+    cs = bench.ClockSampler(0)
+    cs.lines = [
+        "0, 345, 1965, 120.0, 0x0000000000000001, Not Active, Not Active, Not Active, Not Active",
+        "0, 1965, 1965, 900.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+    ]
+    s = cs.summary()
+    assert s["samples"] == 1 and s["sm_mhz"] == 1965
+    assert not bench.clocks_rejected(s)
