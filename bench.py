@@ -141,37 +141,41 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                if int(parts[4], 16) & 1:   # GPU idle: not a sample under load
-                    continue
-            except ValueError:
-                pass
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                sm, mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+            try:
+                idle = bool(int(parts[4], 16) & 1)   # the GPU-idle reason bit
+            except ValueError:
+                idle = False
+            rows.append((sm, mx, idle, parts[5:9]))
+        busy = [r for r in rows if not r[2]]
+        use = busy or rows   # samples under load; all of them if none was
+        if not use:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = {n for r in use for n, v in zip(names, r[3]) if v.lower() == "active"}
+        out = {"sm_mhz": statistics.median(r[0] for r in use), "sm_max_mhz": max(r[1] for r in use),
+               "reasons": sorted(reasons), "samples": len(use)}
+        if not busy:
+            out["idle_samples_only"] = True
+        return out
 
 
 def clocks_rejected(summary):
     """A timed region sampled under a hardware or thermal slowdown, or with
-    the SM clock stuck well below its maximum and no reason given (a clock
-    lock left by someone else), is measured again once."""
+    the SM clock stuck well below its maximum under load and no reason given
+    (a clock lock left by someone else), is measured again once."""
     if {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"} & set(summary.get("reasons", [])):
         return True
+    if summary.get("idle_samples_only"):
+        return False
     sm, mx = summary.get("sm_mhz"), summary.get("sm_max_mhz")
     return bool(sm and mx and sm < 0.8 * mx and not summary.get("reasons"))
 

@@ -165,3 +165,11 @@ def test_clock_summary_skips_idle_samples():
     s = cs.summary()
     assert s["samples"] == 1 and s["sm_mhz"] == 1965
     assert not bench.clocks_rejected(s)
+
+
+def test_clock_summary_with_idle_samples_only():
+    cs = bench.ClockSampler(0)
+    cs.lines = ["0, 120, 1965, 100.0, 0x0000000000000001, Not Active, Not Active, Not Active, Not Active"] * 3
+    s = cs.summary()
+    assert s["idle_samples_only"] is True and s["sm_mhz"] == 120 and s["samples"] == 3
+    assert not bench.clocks_rejected(s)   # idle clocks say nothing about a lock
