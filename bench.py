@@ -213,7 +213,7 @@ class GemvStep:
         w, x, _ = synth.make_inputs(wl)
         self.wl = wl
         self.wbytes = w.nbytes
-        self.pool = max(8, -(-4 * l2_bytes // w.nbytes))
+        self.pool = pool_size(w.nbytes, l2_bytes)
         base = torch.from_numpy(w).cuda()
         # replicas of the seeded matrix: distinct HBM addresses, same values
         self.ws = [base.clone() for _ in range(self.pool)]
@@ -398,24 +398,69 @@ def job_throughput(units_per_rank_step, steps, world, ms):
     return units_per_rank_step * steps * world / (ms / 1e3)
 
 
-def cpu_baseline_gemv(wl, budget_s=10.0):
-    """The oracle as it stands, on the host's cores, over whole GEMVs of the
-    workload repeated until ~budget_s of CPU work; GB/s of weight bytes."""
+def _time_oracle_gemvs(wl, w, x, threads, budget_s):
     import oracle
 
-    w, x, _ = synth.make_inputs(wl)
-    cores = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
     n = 0
     while True:
-        oracle.matmul(wl.codec, w, wl.k, x, threads=cores)
+        oracle.matmul(wl.codec, w, wl.k, x, threads=threads)
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 10000:
-            break
+            return n, el
+
+
+def cpu_baseline_gemv(wl, budget_s=10.0):
+    """The oracle as it stands, on the host's cores, over whole GEMVs of the
+    workload repeated until ~budget_s of CPU work; GB/s of weight bytes.  It
+    runs on every core of the process's affinity set, and once more on a
+    single thread for a third of the budget."""
+    w, x, _ = synth.make_inputs(wl)
+    cores = len(os.sched_getaffinity(0))
+    n, el = _time_oracle_gemvs(wl, w, x, cores, budget_s)
+    n1, el1 = _time_oracle_gemvs(wl, w, x, 1, budget_s / 3)
+    name = f"{wl.n}x{wl.k} {synth.CODEC_NAMES[wl.codec]}"
     return {"value": w.nbytes * n / el / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} whole {wl.n}x{wl.k} {synth.CODEC_NAMES[wl.codec]} GEMVs (fp64 accumulate) "
-                      f"in {el:.1f} s on {cores} threads"}
+            "sample": f"{n} whole {name} GEMVs (fp64 accumulate) in {el:.1f} s on {cores} threads",
+            "single_thread": {"value": w.nbytes * n1 / el1 / 1e9, "unit": "GB/s", "cores": 1,
+                              "sample": f"{n1} whole {name} GEMVs in {el1:.1f} s on one thread"}}
+
+
+def headline_config(wl, wbytes, pool, l2, world):
+    """The `config` object of the bench line; both arms print the same one."""
+    return {
+        "workload": wl.name,
+        "weights": f"{wl.n}x{wl.k} {synth.CODEC_NAMES[wl.codec].upper()} ({wbytes} B)",
+        "x": f"{wl.x_dtype} [{wl.m},{wl.k}]",
+        "y": f"{wl.y_dtype} [{wl.m},{wl.n}]",
+        "pool_matrices_per_step": pool,
+        "l2_policy": f"inputs larger than L2: each step streams {pool} distinct weight "
+                     f"matrices ({pool * wbytes / 1e6:.0f} MB > 4x L2 {l2 / 1e6:.0f} MB)",
+        "parallelism": f"replicas x{world}",
+        "calls": "independent (kq flag: no call reads or writes another's buffers; "
+                 "each still stages x, decodes every weight, writes y)",
+    }
+
+
+def pool_size(wbytes, l2):
+    """Distinct weight matrices per step: at least four times the L2 cache."""
+    return max(8, -(-4 * l2 // wbytes))
+
+
+# B200 L2 as the CUDA runtime reports it; used only when no device is visible.
+B200_L2_BYTES = 132644864
+
+
+def l2_bytes(local=0):
+    try:
+        import torch
+
+        if torch.cuda.is_available():
+            return int(torch.cuda.get_device_properties(local).L2_cache_size)
+    except Exception:
+        pass
+    return B200_L2_BYTES
 
 
 def run_gpu(args):
@@ -426,7 +471,7 @@ def run_gpu(args):
     wl = synth.WORKLOADS[args.workload]
     if wl.kind != "gemv":
         raise SystemExit("the bench's headline step is the decode GEMV workload")
-    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    l2 = l2_bytes(local)
     step = GemvStep(torch, kq, wl, l2)
     peaks = load_peaks()
     for attempt in range(2):
@@ -464,18 +509,7 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "int16 activation codes x u4 quants (dp2a, int32), f32 scale-and-sum",
         "data": "synthetic (seeded Q4_K wire bytes and N(0,1) bf16 activations)",
-        "config": {
-            "workload": wl.name,
-            "weights": f"{wl.n}x{wl.k} Q4_K ({step.wbytes} B)",
-            "x": f"bf16 [{wl.m},{wl.k}]",
-            "y": f"{wl.y_dtype} [{wl.m},{wl.n}]",
-            "pool_matrices_per_step": step.pool,
-            "l2_policy": f"inputs larger than L2: each step streams {step.pool} distinct weight "
-                         f"matrices ({step.pool * step.wbytes / 1e6:.0f} MB > 4x L2 {l2 / 1e6:.0f} MB)",
-            "parallelism": f"replicas x{world}",
-            "calls": "independent (kq flag: no call reads or writes another's buffers; "
-                     "each still stages x, decodes every weight, writes y)",
-        },
+        "config": headline_config(wl, step.wbytes, step.pool, l2, world),
         "serial_chain": {
             "us_per_call": round(serial_us, 4),
             "GB/s": round(step.wbytes / (serial_us * 1e-6) / 1e9, 1),
@@ -525,6 +559,8 @@ def run_reference(args):
 
     wl = synth.WORKLOADS[args.workload]
     w, x, _ = synth.make_inputs(wl)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    l2 = l2_bytes()
     cores = len(os.sched_getaffinity(0))
     for _ in range(args.warmup):
         oracle.matmul(wl.codec, w, wl.k, x, threads=cores)
@@ -538,7 +574,7 @@ def run_reference(args):
         "metric": "Q4_K GEMV weight GB/s",
         "value": round(value, 4),
         "unit": "GB/s",
-        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(el * 1e3 / args.steps, 4),
@@ -547,7 +583,7 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "u8 Q4_K weights, fp64 accumulate",
         "data": "synthetic",
-        "config": {"workload": wl.name, "weights": f"{wl.n}x{wl.k} Q4_K", "x": f"bf16 [{wl.m},{wl.k}]"},
+        "config": headline_config(wl, w.nbytes, pool_size(w.nbytes, l2), l2, world),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": f"one whole {wl.n}x{wl.k} GEMV per step on {cores} threads"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,

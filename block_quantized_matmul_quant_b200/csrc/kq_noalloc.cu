@@ -10,12 +10,16 @@
 //
 // The array is a file-scope __device__ object of KQ_NOALLOC_SCRATCH_BYTES
 // bytes: every GPU that loads the library holds it until the process exits.
-// In host code the array's name is only a host-side stand-in, so the device
-// address is looked up with cudaGetSymbolAddress -- once per device, with
-// that device current, on the first call made on it -- and passed on as the
-// workspace of the ordinary kq_matmul_id path.  Nothing here allocates.
-#include <mutex>
-
+// In host code the array's name is only a host-side stand-in, so its device
+// address is looked up with cudaGetSymbolAddress on every call, with the
+// calling device current, and passed on as the workspace of the ordinary
+// kq_matmul_id path.  Looking it up each time (a table lookup in the CUDA
+// runtime, no allocation) keeps the address right for the context that is
+// current now: an address cached from an earlier context (one destroyed by
+// cudaDeviceReset and created again) could point at memory the module no
+// longer owns.  The first call on a device is the set-up: it loads the
+// library's device code on that device (lazy module loading) and so should
+// come before any stream capture.  Nothing here allocates.
 #include "kq_common.cuh"
 
 namespace {
@@ -24,23 +28,11 @@ constexpr size_t KQ_NOALLOC_SCRATCH_BYTES = 256 * 1024;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[KQ_NOALLOC_SCRATCH_BYTES];
 
-constexpr int MAX_DEVICES = 64;
-std::mutex g_mu;
-void *g_scratch_addr[MAX_DEVICES];
-
-// Device address of this device's scratch array (looked up on first use).
+// Device address of the scratch array in the current device's context.
 int scratch_for_current_device(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return KQ_ERR_CUDA;
-    if (dev < 0 || dev >= MAX_DEVICES) return KQ_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-            return KQ_ERR_CUDA;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KQ_ERR_CUDA;
+    *out = p;
     return KQ_OK;
 }
 

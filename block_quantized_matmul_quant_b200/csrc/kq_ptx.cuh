@@ -72,18 +72,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
     return false;
 }
 
-
-
-// Bounded busy wait for a single latency-critical thread (an MMA or TMA
-// issuer): it resumes the moment the phase completes instead of sleeping.
-// About 2^28 polls (well under a minute) before it gives up like mbar_wait.
-__device__ __forceinline__ bool mbar_spin(uint64_t *bar, uint32_t parity, unsigned int *err) {
-    for (uint32_t i = 0; i < (KQ_SPIN_LIMIT << 6); ++i)
-        if (mbar_test_wait(bar, parity)) return true;
-    atomicOr(err, ERR_TIMEOUT);
-    return false;
-}
-
 // Contiguous global -> shared bulk copy; completion counted on `bar`.
 // dst, src 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {

@@ -187,9 +187,11 @@ KQ_API int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n
  *     kq_matmul_id_workspace_bytes(n_tokens, top_k, n_experts) exceeds it is
  *     rejected with KQ_ERR_WORKSPACE before any work is enqueued.
  *   * Every GPU that loads the library keeps the array until the process
- *     exits.  The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     exits.  Each call looks up the array's device address in the current
+ *     device's context (cudaGetSymbolAddress), so the address stays valid
+ *     after that context is destroyed and created again.  The first call on
+ *     a device is its set-up: it loads the library's device code there (lazy
+ *     module loading), so make that first call before any stream capture.
  *   * Every call shares the one array: calls that overlap on the GPU (on
  *     different streams, or from different host threads) race and give
  *     wrong results.  Order them on one stream.  The array keeps the last

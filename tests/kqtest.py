@@ -11,7 +11,7 @@ import numpy as np
 TOL = {"f32": 2e-3, "bf16": 1e-2}
 FP32_PATH_TOL = 1e-4
 # The bandwidth kernel rounds activations to 16-bit fixed point per 32-wide
-# sub-block (error <= 2^-15 of the sub-block's max |x| per element, random
+# sub-block (error <= 2^-14 of the sub-block's max |x| per element, random
 # in sign): the row error is ~3e-5 of the row norm for N(0,1) activations;
 # 3e-4 leaves a 10x margin and still catches any decode slip.
 GEMV_TOL = 3e-4

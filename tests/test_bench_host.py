@@ -72,6 +72,12 @@ def test_reference_arm_prints_one_contract_line(monkeypatch, capsys):
         assert key in r
     assert r["impl"] == "reference" and r["value"] > 0 and r["higher_is_better"] is True
     assert r["config"]["workload"] == "q4_k_gemv_4096x4096"
+    # the same config object the GPU arm prints for this workload and world size
+    wl = bench.synth.WORKLOADS["q4_k_gemv_4096x4096"]
+    wbytes = wl.weight_bytes()
+    l2 = bench.l2_bytes()
+    assert r["config"] == bench.headline_config(wl, wbytes, bench.pool_size(wbytes, l2), l2, 1)
+    assert r["config"]["pool_matrices_per_step"] == 57 or l2 != bench.B200_L2_BYTES
     cb = r["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == r["value"] and cb["cores"] >= 1 and cb["sample"]
     assert r["e2e"] == {"value": r["value"], "unit": r["unit"], "h2d_bytes_per_step": 0,
