@@ -134,13 +134,14 @@ static bool id_workspace_layout(int64_t n_tokens, int64_t top_k, int64_t n_exper
 // Activation rows from which the tensor-core kernel serves bf16 inputs; the
 // bandwidth kernel handles up to eight rows per launch.
 constexpr int64_t GEMM_MIN_M = 9;
-// Mean (token, slot) pairs per expert from which the expert-indexed product
-// runs on the tensor cores (each hit expert's weights are then decoded once
-// per token tile of up to 176 pairs, instead of once per pass of four).
-// Measured on B200 with 64 experts of 1408 x 2048, top-6: already faster
-// at 3 pairs per expert (32 tokens: 101 vs 109 us; 128 tokens: 134 vs
-// 313 us), so every bf16 Q4_K request takes it.
-constexpr int64_t ID_GEMM_MIN_PAIRS_PER_EXPERT = 0;
+// Mean (token, slot) pairs per expert above which the expert-indexed
+// product runs on the tensor cores (each hit expert's weights are then
+// decoded once per token tile of up to 176 pairs); at or below it the
+// bandwidth kernel streams each hit expert's rows once per four pairs.
+// Measured on B200, 64 experts of 1408 x 2048, top-6, bf16 (us per call,
+// bandwidth vs tensor-core kernel): 8 tokens 47 vs 55, 32 tokens 96 vs 84,
+// 64 tokens 147 vs 85, 128 tokens 259 vs 113.
+constexpr int64_t ID_GEMV_MAX_PAIRS_PER_EXPERT = 1;
 // The TQ1 bandwidth kernel takes two activation rows per pass over the
 // weights; beyond this many rows the plain kernel is used.
 constexpr int64_t TQ1_GEMV_MAX_M = 8;
@@ -254,10 +255,10 @@ int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64
     a.perm = reinterpret_cast<int32_t *>(ws + l.perm);
     a.tiles = reinterpret_cast<int32_t *>(ws + l.tiles);
     a.n_tiles = reinterpret_cast<int32_t *>(ws + l.n_tiles);
-    const bool can_gemv = gemv_id_supported(type, k, x_dtype);
+    const bool can_gemv = moe_gemv_supported(type, n, k, n_experts);
     const bool can_gemm = gemm_supported(type, n, k, x_dtype, y_dtype);
     if (path == KQ_PATH_AUTO) {
-        if (can_gemm && pairs >= ID_GEMM_MIN_PAIRS_PER_EXPERT * n_experts) path = KQ_PATH_GEMM;
+        if (can_gemm && (!can_gemv || pairs > ID_GEMV_MAX_PAIRS_PER_EXPERT * n_experts)) path = KQ_PATH_GEMM;
         else path = can_gemv ? KQ_PATH_GEMV : KQ_PATH_SIMPLE;
     }
     if (path == KQ_PATH_GEMM && !can_gemm) return KQ_ERR_UNSUPPORTED;
@@ -273,7 +274,7 @@ int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64
         if (e != cudaSuccess) return KQ_ERR_CUDA;
         return to_status(launch_gemm_id(a, bn, s));
     }
-    if (path == KQ_PATH_GEMV) return to_status(launch_gemv_id(a, s));
+    if (path == KQ_PATH_GEMV) return to_status(launch_moe_gemv(a, s));
     return to_status(launch_simple_id(a, s));
 }
 

@@ -2,7 +2,7 @@
 //
 // y[t][n] = sum_k dequant(w)[n][k] * x[t][k] for t < m <= 8: the qmv case of
 // mlx-kquant `quantized_matmul` (the pages' Metal forms are ds4's
-// `kernel_mul_mv_q8_0_f32` and mlx-native's `kernel_mul_mv_id_*` family).
+// `kernel_mul_mv_q8_0_f32`; the expert-indexed form lives in kq_moe_gemv.cu).
 //
 // B200 design
 //  * A CTA owns a contiguous range of weight rows; warp w of the CTA owns
@@ -88,10 +88,6 @@ struct GemvParams {
     int early;        // issue weight copies before griddepcontrol.wait
     int indep;        // independent call: no griddepcontrol.wait at all
     unsigned int *err;
-    // expert-indexed mode (grid.y = expert): grouping from the device
-    const int32_t *counts, *offsets, *perm;
-    int top_k;
-    int64_t expert_stride;
 };
 
 __device__ __forceinline__ int dp2a_lo(int a, uint32_t b, int c) {
@@ -488,48 +484,6 @@ __global__ void __launch_bounds__(MINB == 1 ? 32 * GEMV_MAX_WARPS : 32 * GEMV_HA
     if (p.indep) griddep_wait();
 }
 
-// Expert-indexed form: CTA (chunk, e) streams rows of expert e's slice once
-// per group of up to TB (token, slot) pairs routed to e (the device-side
-// grouping of kq_moe.cu: ascending pair order), so each hit expert's weights
-// leave HBM once per group; experts nobody chose cost nothing.  A pass takes
-// four pairs while three or more remain, else exactly the one or two left:
-// the dot-product work follows the pairs actually routed.
-template <int C, int TB, int R, typename XT, typename YT>
-__global__ void __launch_bounds__(32 * GEMV_MAX_WARPS, 1) gemv_id_q4k_kernel(const GemvParams p) {
-    static_assert(TB == 4, "passes of 4, 2 or 1 pairs share the 4-slot staging layout");
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int s_tok[TB];
-    __shared__ int64_t s_yrow[TB];
-    __shared__ int s_failed;
-    const int e = blockIdx.y;
-    const int cnt = p.counts[e];
-    const int row_begin = blockIdx.x * p.rows_per_cta;
-    const int row_end = min(p.n, row_begin + p.rows_per_cta);
-    if (cnt == 0 || row_begin >= row_end) return;
-    const int32_t *pairs = p.perm + p.offsets[e];
-    const uint8_t *w = p.w + (int64_t)e * p.expert_stride;
-    if (threadIdx.x == 0) s_failed = 0;
-    for (int j0 = 0, pass = 0; j0 < cnt; ++pass) {
-        const int rem = cnt - j0;
-        const int tb = rem >= 3 ? 4 : rem;   // pairs this pass (block-uniform)
-        __syncthreads();  // the previous pass is done with s_tok / s_yrow
-        if (s_failed) return;  // a wait gave up: the ring's phases are unknown
-        if (threadIdx.x < TB) {
-            const int j = j0 + (int)threadIdx.x;
-            const int pr = (int)threadIdx.x < tb && j < cnt ? pairs[j] : -1;
-            s_tok[threadIdx.x] = pr >= 0 ? pr / p.top_k : -1;
-            s_yrow[threadIdx.x] = pr >= 0 ? pr : 0;
-        }
-        __syncthreads();
-        bool ok;
-        if (tb == 4) ok = gemv_pass<C, 4, R, false, XT, YT>(p, w, row_begin, row_end, s_tok, s_yrow, smem, pass);
-        else if (tb == 2) ok = gemv_pass<C, 2, R, false, XT, YT>(p, w, row_begin, row_end, s_tok, s_yrow, smem, pass);
-        else ok = gemv_pass<C, 1, R, false, XT, YT>(p, w, row_begin, row_end, s_tok, s_yrow, smem, pass);
-        if (!ok) s_failed = 1;
-        j0 += tb;
-    }
-}
-
 int chunks_per_unit(int nb) { return nb >= 32 ? 4 : nb >= 16 ? 2 : 1; }
 int tb_for(int64_t m) { return m <= 1 ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : 8; }
 #ifndef KQ_GEMV_ROWS_PER_STEP_1
@@ -671,91 +625,6 @@ cudaError_t launch_gemv(int type, const void *w, int64_t n, int64_t k, const voi
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
-}
-
-namespace {
-
-constexpr int ID_TB = 4;  // (token, slot) pairs per pass over an expert's rows
-constexpr int ID_R = 2;   // weight rows per step: each staged activation load serves two rows
-
-// Grid (chunks, E): at most two CTAs per SM if every expert were hit (one
-// wave); eight warps per CTA so that two CTAs fit on an SM.
-bool plan_gemv_id(int type, int64_t n, int64_t k, int64_t n_experts, int num_sms, GemvParams *p) {
-    if (type != KQ_Q4_K || n < 1 || n > INT32_MAX / 2 || k > (1 << 20) || n_experts < 1) return false;
-    const int nb = (int)(k / 256);
-    const int C = chunks_per_unit(nb);
-    const int units = nb * 4 / C, units_pad = (units + 7) / 8 * 8;
-    const int64_t row_bytes = (int64_t)nb * 144;
-    int64_t chunks = (2 * num_sms) / n_experts;
-    if (chunks < 1) chunks = 1;
-    if (chunks > n) chunks = n;
-    const int rows_per_cta = (int)((n + chunks - 1) / chunks);
-    const size_t xq_bytes = (size_t)ID_TB * 8 * C * units_pad * 16;
-    const size_t xs_bytes = (size_t)ID_TB * units * 2 * C * 4;
-    const size_t fixed = xq_bytes + 2 * xs_bytes;
-    const size_t limit = 100 * 1024;
-    if (fixed + 1024 >= limit) return false;
-    const int warps = rows_per_cta < 8 ? rows_per_cta : 8;
-    const int rows_per_warp = (rows_per_cta + warps - 1) / warps;
-    int slots = rows_per_warp < GEMV_MAX_SLOTS ? rows_per_warp : GEMV_MAX_SLOTS;
-    const int min_slots = rows_per_warp < ID_R ? rows_per_warp : ID_R;  // a step holds ID_R rows
-    while (slots > min_slots && fixed + (size_t)warps * slots * (row_bytes + 8) > limit) --slots;
-    if (fixed + (size_t)warps * slots * (row_bytes + 8) > limit) return false;
-    p->nb = nb; p->units = units; p->units_pad = units_pad; p->rows_per_cta = rows_per_cta;
-    p->warps = warps; p->slots = slots; p->row_bytes = (int)row_bytes;
-    p->xq_bytes = (int)xq_bytes; p->xs_bytes = (int)xs_bytes;
-    p->n = (int)n; p->k = (int)k; p->m = ID_TB;
-    return true;
-}
-
-template <int C, typename XT, typename YT>
-cudaError_t launch_id_q4k(GemvParams p, int64_t n_experts, cudaStream_t s) {
-    auto kern = gemv_id_q4k_kernel<C, ID_TB, ID_R, XT, YT>;
-    const size_t smem = (size_t)p.xq_bytes + 2 * (size_t)p.xs_bytes +
-                        (size_t)p.warps * p.slots * ((size_t)p.row_bytes + 8);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)((p.n + p.rows_per_cta - 1) / p.rows_per_cta), (unsigned)n_experts);
-    kern<<<grid, 32 * p.warps, smem, s>>>(p);
-    return cudaGetLastError();
-}
-
-template <typename XT, typename YT>
-cudaError_t dispatch_id_c(GemvParams p, int64_t n_experts, cudaStream_t s) {
-    switch (chunks_per_unit(p.nb)) {
-    case 4: return launch_id_q4k<4, XT, YT>(p, n_experts, s);
-    case 2: return launch_id_q4k<2, XT, YT>(p, n_experts, s);
-    default: return launch_id_q4k<1, XT, YT>(p, n_experts, s);
-    }
-}
-
-}  // namespace
-
-bool gemv_id_supported(int type, int64_t k, int x_dtype) {
-    (void)x_dtype;
-    GemvParams p;
-    return plan_gemv_id(type, 1024, k, 8, 148, &p);
-}
-
-cudaError_t launch_gemv_id(const IdArgs &a, cudaStream_t s) {
-    GemvParams p = {};
-    if (!plan_gemv_id(a.type, a.n, a.k, a.n_experts, sm_count(), &p)) return cudaErrorNotSupported;
-    p.w = static_cast<const uint8_t *>(a.w);
-    p.x = a.x;
-    p.y = a.y;
-    p.early = 0;
-    p.err = error_word();
-    p.counts = a.counts;
-    p.offsets = a.offsets;
-    p.perm = a.perm;
-    p.top_k = (int)a.top_k;
-    p.expert_stride = a.expert_stride;
-    if (a.x_dtype == KQ_F32) {
-        if (a.y_dtype == KQ_F32) return dispatch_id_c<float, float>(p, a.n_experts, s);
-        return dispatch_id_c<float, __nv_bfloat16>(p, a.n_experts, s);
-    }
-    if (a.y_dtype == KQ_F32) return dispatch_id_c<__nv_bfloat16, float>(p, a.n_experts, s);
-    return dispatch_id_c<__nv_bfloat16, __nv_bfloat16>(p, a.n_experts, s);
 }
 
 }  // namespace kq

@@ -51,8 +51,10 @@ cudaError_t launch_gemv(int type, const void *w, int64_t n, int64_t k, const voi
 bool gemv_tq1_supported(int64_t n, int64_t k);
 cudaError_t launch_gemv_tq1(const void *w, int64_t n, int64_t k, const void *x, int xdt, int64_t m,
                             void *y, int ydt, GemvOrder order, cudaStream_t s);
-bool gemv_id_supported(int type, int64_t k, int x_dtype);
-cudaError_t launch_gemv_id(const IdArgs &a, cudaStream_t s);
+// Expert-indexed bandwidth kernel (kq_moe_gemv.cu): Q4_K, few pairs per
+// expert; runs after launch_moe_group on the same stream.
+bool moe_gemv_supported(int type, int64_t n, int64_t k, int64_t n_experts);
+cudaError_t launch_moe_gemv(const IdArgs &a, cudaStream_t s);
 
 // Tensor-core kernels (kq_gemm_sm100.cu).
 bool gemm_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype);

@@ -72,6 +72,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
     return false;
 }
 
+// Bounded wait that polls without suspending: a non-blocking test, then a
+// short sleep.  For phases completed by other threads' arrivals, where a
+// suspended try_wait can stay asleep up to its whole time hint after the
+// phase completes.  Gives up after about as long as mbar_wait.
+__device__ __forceinline__ bool mbar_wait_poll(uint64_t *bar, uint32_t parity, unsigned int *err) {
+    for (uint32_t i = 0; i < (KQ_SPIN_LIMIT << 4); ++i) {
+        if (mbar_test_wait(bar, parity)) return true;
+        __nanosleep(32);
+    }
+    atomicOr(err, ERR_TIMEOUT);
+    return false;
+}
+
 // Contiguous global -> shared bulk copy; completion counted on `bar`.
 // dst, src 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {

@@ -124,9 +124,14 @@ def test_matmul_gemv_q4_k(kq, n, k, m, xdt):
 
 
 TQ1_GEMV_CASES = [
-    # (n, k, m): one block, a ragged last lane step, several steps per row,
-    # rows not a multiple of the SM count, two rows per launch and a third
-    (5, 128, 1), (300, 1280, 1), (777, 4096 + 128, 2), (1000, 17408, 1), (129, 8192, 3),
+    # table kernel (rows not a multiple of 16 bytes): one block, a ragged
+    # last lane step, several steps per row, two rows per launch and a third
+    (5, 128, 1), (300, 1280, 1), (777, 4096 + 128, 2),
+    # split kernel (K a multiple of 512): 4 to 192 blocks a row (136 row
+    # groups down to 2), rows not a multiple of the groups or the SM count,
+    # ring slots reused within a CTA, one launch per activation row
+    (1000, 17408, 1), (129, 8192, 3), (300, 512, 1), (2000, 5120, 2), (17, 24576, 1),
+    (5120, 17408, 1), (4001, 4096, 1),
 ]
 
 
@@ -153,6 +158,29 @@ def test_matmul_gemv_tq1(kq, n, k, m, xdt):
     yb = kq.matmul(wd, synth.TQ1_G128, xd, path=kq.PATH_GEMV,
                    out_dtype=torch.bfloat16).float().cpu().numpy()
     assert row_rel_err(yb, ref) <= TOL[xdt] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+@pytest.mark.parametrize("codec,n,k", [(synth.TQ1_G128, 300, 2048), (synth.TQ1_G128, 200, 1280)])
+def test_matmul_gemv_nonfinite_activations(kq, codec, n, k):
+    """An infinite and a NaN activation: the fixed-point kernels compute such
+    a call exactly in fp32, so each output is NaN, +-inf or finite as in the
+    IEEE product (the fp64 oracle), and the finite outputs stay in tolerance."""
+    r = rng(41 + n)
+    w = synth.gen_weights(codec, n, k, r)
+    x = synth.gen_x(3, k, "f32", r)
+    x[0, 7] = np.inf           # row 0: one +inf
+    x[1, k - 3] = -np.inf      # row 1: one -inf and one NaN
+    x[1, 11] = np.nan
+    ref = oracle.matmul(codec, w, k, x, threads=8)
+    y = kq.matmul(to_device_w(w), codec, to_device_x(x, "f32"), path=kq.PATH_GEMV).cpu().numpy()
+    assert np.array_equal(np.isnan(y), np.isnan(ref))
+    assert np.array_equal(np.isposinf(y), np.isposinf(ref))
+    assert np.array_equal(np.isneginf(y), np.isneginf(ref))
+    assert np.isnan(ref[1]).all() and np.isinf(ref[0]).any()
+    fin = np.isfinite(ref)
+    assert row_rel_err(y[2:], ref[2:]) <= GEMV_TOL      # the finite row
+    assert np.allclose(y[fin], ref[fin], rtol=1e-3, atol=1e-3 * np.abs(ref[2]).max())
     assert kq.device_status() == 0
 
 
@@ -371,9 +399,11 @@ def test_matmul_id_small(kq, codec, path):
     y = kq.matmul_id(to_device_w(w), codec, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
                      path=p).cpu().numpy()
     if path == "auto" and codec == synth.Q4_K:
-        # bf16 Q4_K requests run the grouped tensor-core product: bf16 weights
-        assert row_rel_err(y, ref) <= TOL["bf16"]
-        assert row_rel_err(y, _bf16_weight_reference_id(w, k, x, ids)) <= FP32_PATH_TOL
+        # few pairs per expert: the grouped bandwidth kernel (16-bit codes)
+        assert row_rel_err(y, ref) <= GEMV_TOL
+        yg = kq.matmul_id(to_device_w(w), codec, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
+                          path=kq.PATH_GEMV).cpu().numpy()
+        assert np.array_equal(y.view(np.uint32), yg.view(np.uint32))
     else:
         assert row_rel_err(y, ref) <= FP32_PATH_TOL
     assert kq.device_status() == 0
@@ -381,10 +411,12 @@ def test_matmul_id_small(kq, codec, path):
 
 @pytest.mark.parametrize("t,top_k,e,n,k", [
     (32, 6, 64, 1408, 2048),   # the MoE workload's shape
-    (20, 4, 5, 300, 1024),     # ~16 pairs per expert: about four passes of four
-    (24, 2, 3, 5000, 512),     # 7 rows per warp through 4 slots, over several passes
-    (3, 2, 40, 257, 4096),     # most experts hit by nobody
+    (20, 4, 5, 300, 1024),     # ~16 pairs per expert: four rounds of four
+    (24, 2, 3, 5000, 512),     # half the lanes of a group idle, many tiles, ring slots reused
+    (3, 2, 40, 257, 4096),     # most experts hit by nobody; four warps a row group
     (7, 3, 4, 129, 512),
+    (11, 3, 6, 333, 1280),     # 40 sub-blocks a row (a group of two warps, 24 lanes idle), ragged tiles
+    (64, 8, 16, 96, 2048),     # 32 pairs per expert: eight rounds
 ])
 @pytest.mark.parametrize("xdt", ["f32", "bf16"])
 def test_matmul_id_grouped_gemv(kq, t, top_k, e, n, k, xdt):
@@ -403,6 +435,36 @@ def test_matmul_id_grouped_gemv(kq, t, top_k, e, n, k, xdt):
     yb = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMV,
                       out_dtype=torch.bfloat16).float().cpu().numpy()
     assert row_rel_err(yb, ref) <= TOL[xdt] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+def test_matmul_id_grouped_gemv_skewed_and_nonfinite(kq):
+    """One expert takes most pairs (several rounds), experts with a single
+    pair; then an infinite and a NaN activation: the rounds that stage them
+    run exactly in fp32, so every output is NaN, +-inf or finite as in the
+    IEEE product."""
+    import torch
+
+    t, top_k, e, n, k = 40, 2, 6, 200, 1024
+    r = rng(77)
+    w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, "f32", r)
+    ids = synth.gen_ids(t, top_k, e, r)
+    ids[:, 0] = np.where(np.arange(t) % 13 == 0, 5, 1)
+    wd, idd = to_device_w(w), torch.from_numpy(ids).cuda()
+    ref = oracle.matmul_id(synth.Q4_K, w, k, x, ids)
+    y = kq.matmul_id(wd, synth.Q4_K, to_device_x(x, "f32"), idd, path=kq.PATH_GEMV).cpu().numpy()
+    assert row_rel_err(y, ref) <= GEMV_TOL
+    x[3, 17] = np.inf
+    x[9, 1000] = np.nan
+    x[9, 5] = -np.inf
+    ref = oracle.matmul_id(synth.Q4_K, w, k, x, ids)
+    y = kq.matmul_id(wd, synth.Q4_K, to_device_x(x, "f32"), idd, path=kq.PATH_GEMV).cpu().numpy()
+    assert np.array_equal(np.isnan(y), np.isnan(ref))
+    assert np.array_equal(np.isposinf(y), np.isposinf(ref))
+    assert np.array_equal(np.isneginf(y), np.isneginf(ref))
+    fin = np.isfinite(ref).all(axis=2)
+    assert row_rel_err(y[fin], ref[fin]) <= GEMV_TOL
     assert kq.device_status() == 0
 
 
