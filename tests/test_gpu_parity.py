@@ -399,11 +399,13 @@ def test_matmul_id_small(kq, codec, path):
     y = kq.matmul_id(to_device_w(w), codec, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
                      path=p).cpu().numpy()
     if path == "auto" and codec == synth.Q4_K:
-        # few pairs per expert: the grouped bandwidth kernel (16-bit codes)
-        assert row_rel_err(y, ref) <= GEMV_TOL
-        yg = kq.matmul_id(to_device_w(w), codec, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
-                          path=kq.PATH_GEMV).cpu().numpy()
-        assert np.array_equal(y.view(np.uint32), yg.view(np.uint32))
+        # bf16 Q4_K: the dispatch picks the grouped bandwidth kernel or the
+        # grouped tensor-core kernel by pairs per expert; the result is one
+        # of the two, bit for bit, within the bf16 contract
+        assert row_rel_err(y, ref) <= TOL["bf16"]
+        outs = [kq.matmul_id(to_device_w(w), codec, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
+                             path=pp).cpu().numpy() for pp in (kq.PATH_GEMV, kq.PATH_GEMM)]
+        assert any(np.array_equal(y.view(np.uint32), o.view(np.uint32)) for o in outs)
     else:
         assert row_rel_err(y, ref) <= FP32_PATH_TOL
     assert kq.device_status() == 0
