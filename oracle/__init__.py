@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "kq_oracle.c")
 _LIB = os.path.join(_HERE, "libkq_oracle.so")
 
-Q8_0, Q2_K, Q4_K, TQ1_G128 = 8, 10, 12, 1001
+Q8_0, Q2_K, Q4_K, Q5_K, Q6_K, TQ1_G128 = 8, 10, 12, 13, 14, 1001
 
 
 def build(force: bool = False) -> str:
@@ -54,6 +54,8 @@ def _load():
         lib.kqo_matmul_id.argtypes = [ctypes.c_int, u8p, i64, i64, i64, i64, i64, f64p, i64,
                                       i32p, i64, f64p]
         lib.kqo_matmul_id.restype = ctypes.c_int
+        lib.kqo_get_rows.argtypes = [ctypes.c_int, u8p, i64, i64, i64, i32p, i64, f32p]
+        lib.kqo_get_rows.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -134,3 +136,16 @@ def matmul_id(codec: int, w: np.ndarray, k: int, x: np.ndarray, ids: np.ndarray)
     if st:
         raise ValueError(f"oracle matmul_id failed ({st})")
     return y
+
+
+def get_rows(codec: int, w: np.ndarray, k: int, ids: np.ndarray) -> np.ndarray:
+    """out[t] = fp32 decode of row ids[t] of w; ids outside the table give
+    an all-zero row.  w: [rows, row_bytes] u8; ids: int32 [T]."""
+    w = _as_rows(w, codec, k)
+    ids = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
+    out = np.empty((ids.size, k), dtype=np.float32)
+    st = _load().kqo_get_rows(codec, _ptr(w, ctypes.c_uint8), w.shape[0], k, w.shape[1],
+                              _ptr(ids, ctypes.c_int32), ids.size, _ptr(out, ctypes.c_float))
+    if st:
+        raise ValueError(f"oracle get_rows failed ({st})")
+    return out

@@ -50,6 +50,8 @@
  *            Q2_K, 84 B / 256 w: 16 scale/min bytes @0 (low nibble scale,
  *              high nibble min), 64 quant bytes @16 (four 2-bit quants each),
  *              fp16 d @80, fp16 dmin @82;  w = float(d)*sc*q - float(dmin)*m.
+ *          Q5_K and Q6_K (named in the same GgmlType table) follow their
+ *          GGUF layouts the same way (see q5_k_block, q6_k_block).
  *          Parity unpinned against an external GGUF file (none is at hand):
  *          the tests pin these two decoders to blocks built by packers written
  *          separately from this file, field by field.
@@ -64,13 +66,15 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { KQO_Q8_0 = 8, KQO_Q2_K = 10, KQO_Q4_K = 12, KQO_TQ1_G128 = 1001 };
+enum { KQO_Q8_0 = 8, KQO_Q2_K = 10, KQO_Q4_K = 12, KQO_Q5_K = 13, KQO_Q6_K = 14, KQO_TQ1_G128 = 1001 };
 
 int kqo_block_weights(int type) {
     switch (type) {
     case KQO_Q8_0: return 32;
     case KQO_Q2_K: return 256;
     case KQO_Q4_K: return 256;
+    case KQO_Q5_K: return 256;
+    case KQO_Q6_K: return 256;
     case KQO_TQ1_G128: return 128;
     default: return 0;
     }
@@ -81,6 +85,8 @@ int kqo_block_bytes(int type) {
     case KQO_Q8_0: return 34;  /* 2-byte half + 32 int8 */
     case KQO_Q2_K: return 84;  /* 16 + 64 + 2 + 2 */
     case KQO_Q4_K: return 144; /* 2 + 2 + 12 + 128 */
+    case KQO_Q5_K: return 176; /* 2 + 2 + 12 + 32 + 128 */
+    case KQO_Q6_K: return 210; /* 128 + 64 + 16 + 2 */
     case KQO_TQ1_G128: return 28;
     default: return 0;
     }
@@ -174,6 +180,66 @@ static void q2_k_block(const uint8_t *b, float *w32, double *w64) {
     }
 }
 
+/* Q5_K, 176 B / 256 w (GGUF reading): fp16 d @0, fp16 dmin @2, the 12
+ * packed 6-bit scale/min bytes @4 (Q4_K's packing), qh[32] @16, qs[128] @48.
+ * Chunk c (64 weights) takes qs[32c .. 32c+31]: weight 64c+l is the low
+ * nibble of qs[32c+l] plus 16 times bit 2c of qh[l], in sub-block 2c;
+ * weight 64c+32+l the high nibble plus 16 times bit 2c+1 of qh[l], in
+ * sub-block 2c+1.  w = float(d)*sc*q - float(dmin)*m (products exact). */
+static void q5_k_block(const uint8_t *b, float *w32, double *w64) {
+    double d = half_value(b), dmin = half_value(b + 2);
+    float df = (float)d, dminf = (float)dmin;
+    const uint8_t *s = b + 4, *qh = b + 16, *qs = b + 48;
+    for (int c = 0; c < 4; ++c) {
+        for (int half = 0; half < 2; ++half) {
+            int j = 2 * c + half, sc, m;
+            q4_k_scale_min(s, j, &sc, &m);
+            for (int l = 0; l < 32; ++l) {
+                int byte = qs[32 * c + l];
+                int q = (half ? (byte >> 4) : (byte & 15)) + 16 * ((qh[l] >> j) & 1);
+                int idx = 64 * c + 32 * half + l;
+                if (w32) w32[idx] = df * (float)sc * (float)q - dminf * (float)m;
+                if (w64) w64[idx] = d * sc * q - dmin * m;
+            }
+        }
+    }
+}
+
+/* Q6_K, 210 B / 256 w (GGUF reading): ql[128] @0 (low four bits), qh[64]
+ * @128 (high two bits), int8 scales[16] @192, fp16 d @208.  Half h (128
+ * weights) takes ql[64h ..], qh[32h ..], scales[8h ..]; for l in 0..31:
+ *   weight 128h+l    : low nibble of ql[64h+l]    | bits 0-1 of qh[32h+l] << 4
+ *   weight 128h+32+l : low nibble of ql[64h+32+l] | bits 2-3 << 4
+ *   weight 128h+64+l : high nibble of ql[64h+l]   | bits 4-5 << 4
+ *   weight 128h+96+l : high nibble of ql[64h+32+l]| bits 6-7 << 4
+ * each minus 32, in sub-blocks of 16 (scale index 8h + position / 16).
+ * w = (float(d) * sc) * q: d*sc is exact, the product with q rounds once. */
+static void q6_k_block(const uint8_t *b, float *w32, double *w64) {
+    const uint8_t *ql = b, *qh = b + 128;
+    const int8_t *sc = (const int8_t *)(b + 192);
+    double d = half_value(b + 208);
+    float df = (float)d;
+    for (int h = 0; h < 2; ++h) {
+        for (int l = 0; l < 32; ++l) {
+            int hb = qh[32 * h + l];
+            int q[4];
+            q[0] = ((ql[64 * h + l] & 15) | (((hb >> 0) & 3) << 4)) - 32;
+            q[1] = ((ql[64 * h + 32 + l] & 15) | (((hb >> 2) & 3) << 4)) - 32;
+            q[2] = ((ql[64 * h + l] >> 4) | (((hb >> 4) & 3) << 4)) - 32;
+            q[3] = ((ql[64 * h + 32 + l] >> 4) | (((hb >> 6) & 3) << 4)) - 32;
+            for (int r = 0; r < 4; ++r) {
+                int idx = 128 * h + 32 * r + l;
+                int s = sc[8 * h + idx % 128 / 16];
+                if (w32) {
+                    float ds = df * (float)s;
+                    w32[idx] = ds * (float)q[r];
+                }
+                if (w64) w64[idx] = d * s * q[r];
+            }
+        }
+    }
+}
+
 /* Base-3 digit i of a code byte; bytes above the largest legal value decode
  * to the "zero weight" digit 1 for every position. */
 static int tq1_digit(int code, int i, int max_legal) {
@@ -210,9 +276,29 @@ int kqo_decode(int type, const uint8_t *w, int64_t rows, int64_t k, int64_t row_
             case KQO_Q8_0: q8_0_block(b, o32, o64); break;
             case KQO_Q4_K: q4_k_block(b, o32, o64); break;
             case KQO_Q2_K: q2_k_block(b, o32, o64); break;
+            case KQO_Q5_K: q5_k_block(b, o32, o64); break;
+            case KQO_Q6_K: q6_k_block(b, o32, o64); break;
             case KQO_TQ1_G128: tq1_block(b, o32, o64); break;
             }
         }
+    }
+    return 0;
+}
+
+/* Row gather (Ternary Bonsai ternel_packed_model.py, `_GET_ROWS_SOURCE`:
+ * decode exactly the requested rows; an id outside the table reads as an
+ * all-zero row): out[t][:] = fp32 decode of row ids[t] of w. */
+int kqo_get_rows(int type, const uint8_t *w, int64_t rows, int64_t k, int64_t row_stride,
+                 const int32_t *ids, int64_t n_ids, float *out) {
+    int qk = kqo_block_weights(type);
+    if (qk == 0 || k % qk) return -1;
+    for (int64_t t = 0; t < n_ids; ++t) {
+        float *o = out + t * k;
+        if (ids[t] < 0 || ids[t] >= rows) {
+            for (int64_t c = 0; c < k; ++c) o[c] = 0.0f;
+            continue;
+        }
+        kqo_decode(type, w + (int64_t)ids[t] * row_stride, 1, k, row_stride, o, NULL);
     }
     return 0;
 }

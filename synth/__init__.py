@@ -24,6 +24,9 @@ Value distributions (the workloads' own):
   bytes uniform (both nibbles uniform in 0..15).
 * Q2_K: fp16 ``d`` and ``dmin`` as Q4_K; the 16 scale/min bytes and the 64
   quant bytes uniform in 0..255.
+* Q5_K: as Q4_K, plus the 32 high-bit bytes uniform (every fifth bit uniform).
+* Q6_K: fp16 ``d`` as Q4_K; the 128 low-bit bytes, the 64 high-bit bytes and
+  the 16 int8 scales uniform over their byte values.
 * TQ1_G128 (Ternary Bonsai ``ternel_packed_model.py``): 25 full code bytes
   uniform in 0..242 (five i.i.d. uniform trits), one tail byte uniform in
   0..26 (three trits), fp16 scale uniform in [2^-6, 2^-2].
@@ -38,13 +41,16 @@ import numpy as np
 Q8_0 = 8
 Q2_K = 10
 Q4_K = 12
+Q5_K = 13
+Q6_K = 14
 TQ1_G128 = 1001
 
-CODEC_NAMES = {Q8_0: "q8_0", Q2_K: "q2_k", Q4_K: "q4_k", TQ1_G128: "tq1_g128"}
+CODEC_NAMES = {Q8_0: "q8_0", Q2_K: "q2_k", Q4_K: "q4_k", Q5_K: "q5_k", Q6_K: "q6_k", TQ1_G128: "tq1_g128"}
 CODECS_BY_NAME = {v: k for k, v in CODEC_NAMES.items()}
 
 # (weights per block, bytes per block) -- only used to size the byte arrays.
-_GEOMETRY = {Q8_0: (32, 34), Q2_K: (256, 84), Q4_K: (256, 144), TQ1_G128: (128, 28)}
+_GEOMETRY = {Q8_0: (32, 34), Q2_K: (256, 84), Q4_K: (256, 144), Q5_K: (256, 176), Q6_K: (256, 210),
+             TQ1_G128: (128, 28)}
 
 
 def geometry(codec: int) -> tuple[int, int]:
@@ -72,6 +78,8 @@ def gen_weights(codec: int, rows: int, k: int, rng: np.random.Generator) -> np.n
       Q8_0:  d, qs
       Q4_K:  d, dmin, scales[12], qs[128]
       Q2_K:  d, dmin, scales[16], qs[64]
+      Q5_K:  d, dmin, scales[12], qh[32], qs[128]
+      Q6_K:  d, ql[128], qh[64], scales[16]
       TQ1:   full codes[25], tail, scale
     """
     qk, bb = _GEOMETRY[codec]
@@ -102,6 +110,26 @@ def gen_weights(codec: int, rows: int, k: int, rng: np.random.Generator) -> np.n
         out[:, 16:80] = qs
         out[:, 80:82] = _fp16_bytes(d)
         out[:, 82:84] = _fp16_bytes(dmin)
+    elif codec == Q5_K:
+        d = rng.uniform(2.0 ** -10, 2.0 ** -6, size=nb)
+        dmin = rng.uniform(2.0 ** -10, 2.0 ** -6, size=nb)
+        sc = rng.integers(0, 256, size=(nb, 12), dtype=np.int64).astype(np.uint8)
+        qh = rng.integers(0, 256, size=(nb, 32), dtype=np.int64).astype(np.uint8)
+        qs = rng.integers(0, 256, size=(nb, 128), dtype=np.int64).astype(np.uint8)
+        out[:, 0:2] = _fp16_bytes(d)
+        out[:, 2:4] = _fp16_bytes(dmin)
+        out[:, 4:16] = sc
+        out[:, 16:48] = qh
+        out[:, 48:176] = qs
+    elif codec == Q6_K:
+        d = rng.uniform(2.0 ** -10, 2.0 ** -6, size=nb)
+        ql = rng.integers(0, 256, size=(nb, 128), dtype=np.int64).astype(np.uint8)
+        qh = rng.integers(0, 256, size=(nb, 64), dtype=np.int64).astype(np.uint8)
+        sc = rng.integers(0, 256, size=(nb, 16), dtype=np.int64).astype(np.uint8)
+        out[:, 0:128] = ql
+        out[:, 128:192] = qh
+        out[:, 192:208] = sc
+        out[:, 208:210] = _fp16_bytes(d)
     elif codec == TQ1_G128:
         full = rng.integers(0, 243, size=(nb, 25), dtype=np.int64).astype(np.uint8)
         tail = rng.integers(0, 27, size=nb, dtype=np.int64).astype(np.uint8)

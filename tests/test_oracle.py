@@ -17,7 +17,7 @@ import oracle
 import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
-CODECS = {"q8_0": 8, "q2_k": 10, "q4_k": 12, "tq1_g128": 1001}
+CODECS = {"q8_0": 8, "q2_k": 10, "q4_k": 12, "q5_k": 13, "q6_k": 14, "tq1_g128": 1001}
 
 
 def _golden_rows(name):
@@ -155,6 +155,112 @@ def test_q4_k_random_blocks():
         _check_block(12, pack_q4_k(d, dmin, sc, mn, q), q4_k_expected(d, dmin, sc, mn, q))
 
 
+# ---------------------------------------------------------------- Q5_K
+
+def pack_q5_k(d, dmin, sc, mn, q):
+    """Encoder for one GGUF Q5_K block: Q4_K's header and scale packing
+    (pack_q4_k), then 32 high-bit bytes and 128 nibble bytes; weight 64c+l
+    keeps its low four bits in the low nibble of quant byte 32c+l and its
+    fifth bit in bit 2c of high-bit byte l; weight 64c+32+l the high nibble
+    and bit 2c+1."""
+    assert len(q) == 256 and all(0 <= v < 32 for v in q)
+    q4 = [v & 15 for v in q]
+    head = pack_q4_k(d, dmin, sc, mn, q4)   # 16-byte header + 128 nibble bytes
+    qh = [0] * 32
+    for c in range(4):
+        for l in range(32):
+            qh[l] |= (q[64 * c + l] >> 4) << (2 * c)
+            qh[l] |= (q[64 * c + 32 + l] >> 4) << (2 * c + 1)
+    return bytes(head[:16]) + bytes(qh) + bytes(head[16:])
+
+
+def test_q5_k_unit_scales_give_quants():
+    q = [(11 * i + 5) % 32 for i in range(256)]
+    blob = pack_q5_k(1.0, 0.0, [1] * 8, [0] * 8, q)
+    assert oracle.block_bytes(13) == len(blob) == 176
+    w = oracle.decode_f32(13, np.frombuffer(blob, np.uint8), 256)[0]
+    assert w.tolist() == [float(v) for v in q]
+
+
+def test_q5_k_random_blocks_and_fields():
+    rng = np.random.default_rng(5)
+    for it in range(24):
+        sc = rng.integers(0, 64, 8).tolist()
+        mn = rng.integers(0, 64, 8).tolist()
+        if it < 8:                       # each field at its extremes once
+            sc[it], mn[it] = 63, 63
+        q = rng.integers(0, 32, 256).tolist()
+        d = float(np.float16(rng.uniform(-1, 1)))
+        dmin = float(np.float16(rng.uniform(-1, 1)))
+        exp = [Fraction(d) * sc[i // 32] * q[i] - Fraction(dmin) * mn[i // 32] for i in range(256)]
+        _check_block(13, pack_q5_k(d, dmin, sc, mn, q), exp)
+
+
+# ---------------------------------------------------------------- Q6_K
+
+def pack_q6_k(d, sc, q):
+    """Encoder for one GGUF Q6_K block: 128 low-bit bytes, 64 high-bit bytes,
+    16 int8 scales, fp16 d.  Half h, position l: weights 128h+l and
+    128h+64+l share low-bit byte 64h+l (low and high nibble), weights
+    128h+32+l and 128h+96+l share byte 64h+32+l; the four weights' top two
+    bits fill high-bit byte 32h+l from bit 0 up.  Stored quants are q + 32."""
+    assert len(sc) == 16 and len(q) == 256 and all(-32 <= v < 32 for v in q)
+    u = [v + 32 for v in q]
+    ql, qh = [0] * 128, [0] * 64
+    for h in range(2):
+        for l in range(32):
+            a, b, c, e = (u[128 * h + l], u[128 * h + 32 + l], u[128 * h + 64 + l], u[128 * h + 96 + l])
+            ql[64 * h + l] = (a & 15) | ((c & 15) << 4)
+            ql[64 * h + 32 + l] = (b & 15) | ((e & 15) << 4)
+            qh[32 * h + l] = (a >> 4) | ((b >> 4) << 2) | ((c >> 4) << 4) | ((e >> 4) << 6)
+    return bytes(ql + qh + [s & 0xFF for s in sc] + f16(d))
+
+
+def test_q6_k_unit_scales_give_quants():
+    q = [(13 * i + 7) % 64 - 32 for i in range(256)]
+    blob = pack_q6_k(1.0, [1] * 16, q)
+    assert oracle.block_bytes(14) == len(blob) == 210
+    w = oracle.decode_f32(14, np.frombuffer(blob, np.uint8), 256)[0]
+    assert w.tolist() == [float(v) for v in q]
+
+
+def test_q6_k_random_blocks_and_signed_scales():
+    rng = np.random.default_rng(6)
+    for it in range(24):
+        sc = rng.integers(-128, 128, 16).tolist()
+        if it < 16:
+            sc[it] = -128 if it % 2 else 127
+        q = rng.integers(-32, 32, 256).tolist()
+        d = float(np.float16(rng.uniform(-1, 1)))
+        blob = pack_q6_k(d, sc, q)
+        w64 = oracle.decode_f64(14, np.frombuffer(blob, np.uint8), 256)[0]
+        w32 = oracle.decode_f32(14, np.frombuffer(blob, np.uint8), 256)[0]
+        for i in range(256):
+            e = Fraction(d) * sc[i // 16] * q[i]
+            assert Fraction(float(w64[i])) == e
+            # fp32: (d * sc) is exact, the product with q rounds once
+            assert w32[i] == np.float32(float(e))
+
+
+# ---------------------------------------------------------------- row gather
+
+@pytest.mark.parametrize("name", list(CODECS))
+def test_get_rows_is_decode_of_the_rows(name):
+    c = CODECS[name]
+    qk = oracle.block_weights(c)
+    k = qk * (3 if qk == 256 else 5)
+    rng = np.random.Generator(np.random.PCG64(9))
+    w = synth.gen_weights(c, 40, k, rng)
+    ids = np.array([0, 39, 7, 7, 40, -1, 2 ** 31 - 1, 13], dtype=np.int32)
+    got = oracle.get_rows(c, w, k, ids)
+    dec = oracle.decode_f32(c, w, k)
+    for t, i in enumerate(ids):
+        if 0 <= i < 40:
+            assert np.array_equal(got[t].view(np.uint32), dec[i].view(np.uint32))
+        else:
+            assert np.all(got[t] == 0.0)      # outside the table: an all-zero row
+
+
 # ---------------------------------------------------------------- Q2_K
 
 def pack_q2_k(d, dmin, sc, mn, q):
@@ -276,7 +382,7 @@ def test_tq1_illegal_scan():
 
 # ---------------------------------------------------------------- fp32 decode = one rounding
 
-@pytest.mark.parametrize("codec", [8, 10, 12, 1001])
+@pytest.mark.parametrize("codec", [8, 10, 12, 13, 14, 1001])
 def test_f32_decode_is_rounded_exact_value(codec):
     rng = np.random.default_rng(4)
     k = 512
@@ -300,7 +406,7 @@ def _brute(codec, w, k, x):
     return y
 
 
-@pytest.mark.parametrize("codec", [8, 10, 12, 1001])
+@pytest.mark.parametrize("codec", [8, 10, 12, 13, 14, 1001])
 @pytest.mark.parametrize("blocks", [1, 2])
 def test_matmul_tiny_brute_force(codec, blocks):
     rng = np.random.default_rng(5)
