@@ -16,8 +16,8 @@ import torch
 
 from . import _build
 
-Q8_0, Q2_K, Q4_K, TQ1_G128 = 8, 10, 12, 1001
-CODECS = {"q8_0": Q8_0, "q2_k": Q2_K, "q4_k": Q4_K, "tq1_g128": TQ1_G128}
+Q8_0, Q2_K, Q4_K, Q5_K, Q6_K, TQ1_G128 = 8, 10, 12, 13, 14, 1001
+CODECS = {"q8_0": Q8_0, "q2_k": Q2_K, "q4_k": Q4_K, "q5_k": Q5_K, "q6_k": Q6_K, "tq1_g128": TQ1_G128}
 F32, BF16, F16 = 0, 1, 2
 PATH_AUTO, PATH_SIMPLE, PATH_GEMV, PATH_GEMM = 0, 1, 2, 3
 FLAG_CONST_WEIGHTS = 0x100
@@ -67,12 +67,13 @@ def lib():
                                       vp, sz, i32, vp]
         L.kq_moe_group.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.kq_validate.argtypes = [i32, vp, i64, i64, ctypes.POINTER(i64), vp]
+        L.kq_get_rows.argtypes = [i32, vp, i64, i64, vp, i64, vp, i32, vp]
         L.kq_device_status.argtypes = [vp]
         L.kq_status_string.argtypes = [i32]
         L.kq_status_string.restype = ctypes.c_char_p
         for f in ("kq_block_weights", "kq_block_bytes", "kq_dequantize", "kq_matmul",
                   "kq_matmul_ex", "kq_matmul_id", "kq_matmul_id_ex", "kq_moe_group", "kq_validate",
-                  "kq_device_status"):
+                  "kq_device_status", "kq_get_rows"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -154,6 +155,23 @@ def dequantize(w: torch.Tensor, codec, k: int, dtype=torch.float32, out=None) ->
     _check_tensor("out", out, (rows, k), tuple(_DT), w.device)
     _check(lib().kq_dequantize(c, _ptr(w), rows, k, _ptr(out), _DT[out.dtype], _stream()),
            "kq_dequantize")
+    return out
+
+
+def get_rows(w: torch.Tensor, codec, k: int, ids: torch.Tensor, dtype=torch.float32,
+             out=None) -> torch.Tensor:
+    """out[t] = decode of row ids[t] of w ([rows, row_bytes] wire blocks); an id
+    outside the table gives a zero row and sets the device error word."""
+    c = _codec(codec)
+    rows = _weights(w, c, k)
+    if ids.dim() != 1:
+        raise ValueError("ids must be a 1-D int32 tensor")
+    _check_tensor("ids", ids, (ids.shape[0],), (torch.int32,), w.device)
+    if out is None:
+        out = torch.empty((ids.shape[0], k), dtype=dtype, device=w.device)
+    _check_tensor("out", out, (ids.shape[0], k), tuple(_DT), w.device)
+    _check(lib().kq_get_rows(c, _ptr(w), rows, k, _ptr(ids), ids.shape[0], _ptr(out), _DT[out.dtype],
+                             _stream()), "kq_get_rows")
     return out
 
 

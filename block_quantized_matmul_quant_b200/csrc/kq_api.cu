@@ -52,6 +52,8 @@ static int block_weights(int type) {
     case KQ_Q8_0: return Geom<KQ_Q8_0>::QK;
     case KQ_Q2_K: return Geom<KQ_Q2_K>::QK;
     case KQ_Q4_K: return Geom<KQ_Q4_K>::QK;
+    case KQ_Q5_K: return Geom<KQ_Q5_K>::QK;
+    case KQ_Q6_K: return Geom<KQ_Q6_K>::QK;
     case KQ_TQ1_G128: return Geom<KQ_TQ1_G128>::QK;
     default: return 0;
     }
@@ -61,8 +63,21 @@ static int block_bytes(int type) {
     case KQ_Q8_0: return Geom<KQ_Q8_0>::BB;
     case KQ_Q2_K: return Geom<KQ_Q2_K>::BB;
     case KQ_Q4_K: return Geom<KQ_Q4_K>::BB;
+    case KQ_Q5_K: return Geom<KQ_Q5_K>::BB;
+    case KQ_Q6_K: return Geom<KQ_Q6_K>::BB;
     case KQ_TQ1_G128: return Geom<KQ_TQ1_G128>::BB;
     default: return 0;
+    }
+}
+
+// Alignment an expert stride must keep for the codec's loads: 16 bytes for
+// Q4_K and Q5_K (bulk copies, tensor maps and 8-byte loads of the block),
+// 4 for Q2_K's word loads, 2 for the codecs read as bytes and half words.
+static int64_t stride_align(int type) {
+    switch (type) {
+    case KQ_Q4_K: case KQ_Q5_K: return 16;
+    case KQ_Q2_K: return 4;
+    default: return 2;
     }
 }
 
@@ -228,7 +243,7 @@ int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64
     if (top_k <= 0 || top_k > n_experts) return KQ_ERR_ARG;
     int64_t per_expert, last, pairs, ypairs;
     if (!mul_ok(n, rb, &per_expert)) return KQ_ERR_OVERFLOW;
-    if (expert_stride < per_expert || (expert_stride & 15)) return KQ_ERR_SHAPE;
+    if (expert_stride < per_expert || expert_stride % stride_align(type)) return KQ_ERR_SHAPE;
     if (!mul_ok(n_experts - 1, expert_stride, &last) ||
         __builtin_add_overflow(last, per_expert, &last))
         return KQ_ERR_OVERFLOW;
@@ -300,6 +315,19 @@ int kq_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_experts, int32_t
                                       KQ_F32, 0, (cudaStream_t)stream));
 }
 
+int kq_get_rows(int type, const void *w, int64_t rows, int64_t k, const int32_t *ids, int64_t n_ids,
+                void *out, int out_dtype, void *stream) {
+    int64_t rb;
+    int st = check_weights(type, w, rows, k, &rb);
+    if (st) return st;
+    if (ids == nullptr || n_ids <= 0) return KQ_ERR_ARG;
+    if (rows > INT32_MAX) return KQ_ERR_OVERFLOW;
+    if (!aligned16(ids)) return KQ_ERR_ALIGN;
+    if ((st = check_act(out, out_dtype, n_ids, k, true))) return st;
+    if ((st = check_device())) return st;
+    return to_status(launch_get_rows(type, w, rows, k, ids, n_ids, out, out_dtype, (cudaStream_t)stream));
+}
+
 int kq_validate(int type, const void *w, int64_t rows, int64_t k, int64_t *first_bad_block,
                 void *stream) {
     int64_t rb;
@@ -357,7 +385,7 @@ const char *kq_status_string(int status) {
     case KQ_ERR_OVERFLOW: return "size overflow";
     case KQ_ERR_WORKSPACE: return "workspace missing or too small";
     case KQ_ERR_CUDA: return "CUDA runtime error";
-    case KQ_ERR_DEVICE: return "device reported an out-of-range expert id";
+    case KQ_ERR_DEVICE: return "device reported an out-of-range expert or row id";
     case KQ_ERR_DEVICE_TIMEOUT: return "a bounded device wait timed out";
     case KQ_ERR_UNSUPPORTED: return "unsupported device or path for these arguments";
     default: return "unknown status";

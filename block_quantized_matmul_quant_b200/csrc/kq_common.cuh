@@ -15,6 +15,8 @@ template <int TYPE> struct Geom;
 template <> struct Geom<KQ_Q8_0>     { static constexpr int QK = 32;  static constexpr int BB = 34; };
 template <> struct Geom<KQ_Q2_K>     { static constexpr int QK = 256; static constexpr int BB = 84; };
 template <> struct Geom<KQ_Q4_K>     { static constexpr int QK = 256; static constexpr int BB = 144; };
+template <> struct Geom<KQ_Q5_K>     { static constexpr int QK = 256; static constexpr int BB = 176; };
+template <> struct Geom<KQ_Q6_K>     { static constexpr int QK = 256; static constexpr int BB = 210; };
 template <> struct Geom<KQ_TQ1_G128> { static constexpr int QK = 128; static constexpr int BB = 28; };
 
 // Sticky per-device error word (bit 0: bad expert id, bit 1: wait timeout).

@@ -14,8 +14,8 @@
 //    `_GET_ROWS_SOURCE` (weight j: slot j/5, digit j%5; tail slot 25 holds
 //    weights 125..127).  Byte order in the 28-byte block: 25 full code bytes,
 //    the tail byte, then the raw little-endian fp16 scale.
-//  * Q4_K / Q2_K: the GGUF block layouts (named but not printed on the pages:
-//    mlx-native quantized_matmul_id_ggml.rs type table).
+//  * Q4_K / Q2_K / Q5_K / Q6_K: the GGUF block layouts (named but not printed
+//    on the pages: mlx-native quantized_matmul_id_ggml.rs type table).
 #pragma once
 
 #include "kq_common.cuh"
@@ -93,6 +93,56 @@ template <> struct Unit<KQ_Q2_K> {
         for (int i = 0; i < 4; ++i) {
             w[i] = fmaf(a, (float)((q0 >> (8 * i + 2 * j)) & 3u), -bm);
             w[4 + i] = fmaf(a, (float)((q1 >> (8 * i + 2 * j)) & 3u), -bm);
+        }
+    }
+};
+
+// Q5_K (GGUF layout): Q4_K's header and 6-bit scale/min packing, then 32
+// high-bit bytes at 16 and 128 nibble bytes at 48.  Unit u: chunk c = u/8,
+// nibble half hi = (u/4)&1, positions l0..l0+7 (l0 = 8*(u&3)) of the chunk;
+// the fifth bit of position l is bit 2c+hi of high-bit byte l.
+template <> struct Unit<KQ_Q5_K> {
+    static constexpr int PER_BLOCK = 32;
+    __device__ static void decode(const uint8_t *b, int u, float w[8]) {
+        const int c = u >> 3, hi = (u >> 2) & 1, l0 = (u & 3) * 8;
+        const uint32_t dd = ld_u32(b);
+        const float d = half_bits_to_float(dd), dmin = half_bits_to_float(dd >> 16);
+        uint32_t sc, m;
+        q4k_scale_min(ld_u32(b + 4), ld_u32(b + 8), ld_u32(b + 12), 2 * c + hi, sc, m);
+        const float a = d * (float)sc, bm = dmin * (float)m;
+        const uint2 q = *reinterpret_cast<const uint2 *>(b + 48 + 32 * c + l0);
+        const uint2 h = *reinterpret_cast<const uint2 *>(b + 16 + l0);
+        const int sh = hi ? 4 : 0, hb = 2 * c + hi;
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t q0 = ((q.x >> (8 * i + sh)) & 15u) | (((h.x >> (8 * i + hb)) & 1u) << 4);
+            const uint32_t q1 = ((q.y >> (8 * i + sh)) & 15u) | (((h.y >> (8 * i + hb)) & 1u) << 4);
+            w[i] = fmaf(a, (float)q0, -bm);
+            w[4 + i] = fmaf(a, (float)q1, -bm);
+        }
+    }
+};
+
+// Q6_K (GGUF layout): ql[128] low bits, qh[64] high bits, int8 scales[16],
+// fp16 d at 208.  Unit u covers weights 8u..8u+7 of half h = u/16, quarter
+// r = (u/4)&3, positions l0..l0+7 (l0 = 8*(u&3)); quarters 0/1 take the low
+// nibbles of ql[64h + l] / ql[64h + 32 + l], quarters 2/3 the high nibbles,
+// with bits 2r, 2r+1 of qh[32h + l] on top; minus 32.  w = (d*sc)*q: the
+// first product is exact, the second rounds once.
+template <> struct Unit<KQ_Q6_K> {
+    static constexpr int PER_BLOCK = 32;
+    __device__ static void decode(const uint8_t *b, int u, float w[8]) {
+        const int h = u >> 4, r = (u >> 2) & 3, l0 = (u & 3) * 8;
+        const float d = half_bits_to_float(ld_u16(b + 208));
+        const int sidx = 8 * h + (32 * r + l0) / 16;
+        const float ds = d * (float)(int8_t)b[192 + sidx];
+        const uint8_t *lq = b + 64 * h + ((r & 1) ? 32 : 0) + l0;
+        const uint8_t *hq = b + 128 + 32 * h + l0;
+        const int sh = (r & 2) ? 4 : 0;
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int q = (int)(((uint32_t)lq[i] >> sh) & 15u) | (int)((((uint32_t)hq[i] >> (2 * r)) & 3u) << 4);
+            w[i] = ds * (float)(q - 32);
         }
     }
 };

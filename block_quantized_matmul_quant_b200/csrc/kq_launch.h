@@ -26,6 +26,8 @@ cudaError_t launch_simple_matmul(int type, const void *w, int64_t n, int64_t k, 
                                  int xdt, int64_t m, void *y, int ydt, cudaStream_t s);
 cudaError_t launch_tq1_scan(const void *w, int64_t blocks, unsigned long long *first_bad,
                             cudaStream_t s);
+cudaError_t launch_get_rows(int type, const void *w, int64_t rows, int64_t k, const int32_t *ids,
+                            int64_t n_ids, void *out, int dt, cudaStream_t s);
 cudaError_t launch_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_experts,
                              int32_t *counts, int32_t *offsets, int32_t *perm, void *y,
                              int y_dtype, int64_t n, cudaStream_t s);

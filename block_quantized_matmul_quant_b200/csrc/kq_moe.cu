@@ -231,7 +231,10 @@ cudaError_t launch_simple_id(const IdArgs &a, cudaStream_t s) {
     case KQ_Q8_0: return simple_id_xy<KQ_Q8_0>(a, s);
     case KQ_Q4_K: return simple_id_xy<KQ_Q4_K>(a, s);
     case KQ_Q2_K: return simple_id_xy<KQ_Q2_K>(a, s);
-    default: return simple_id_xy<KQ_TQ1_G128>(a, s);
+    case KQ_Q5_K: return simple_id_xy<KQ_Q5_K>(a, s);
+    case KQ_Q6_K: return simple_id_xy<KQ_Q6_K>(a, s);
+    case KQ_TQ1_G128: return simple_id_xy<KQ_TQ1_G128>(a, s);
+    default: return cudaErrorInvalidValue;
     }
 }
 

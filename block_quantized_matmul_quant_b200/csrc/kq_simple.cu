@@ -1,5 +1,6 @@
-// kq_simple.cu -- decode-to-fp32 kernels: dequantize, the plain CUDA-core
-// product (any codec, any m, fp32 or bf16 x) and the TQ1 legality scan.
+// kq_simple.cu -- decode-to-fp32 kernels: dequantize, the row gather, the
+// plain CUDA-core product (any codec, any m, fp32 or bf16 x) and the TQ1
+// legality scan.
 //
 // These kernels decode each weight exactly (kq_decode.cuh) and accumulate in
 // fp32.  The plain product is the general-purpose path; the shape-specialised
@@ -85,6 +86,45 @@ __global__ void __launch_bounds__(256) simple_matmul_kernel(
     }
 }
 
+// ---------------------------------------------------------------- row gather
+// One thread per 8-weight unit of an output row: out[t] = decode of row
+// ids[t]; an id outside [0, rows) gives a zero row and flags the error word.
+template <int TYPE, typename OT>
+__global__ void __launch_bounds__(256) get_rows_kernel(const uint8_t *__restrict__ w, int64_t rows, int64_t k,
+                                                       const int32_t *__restrict__ ids, int64_t n_ids,
+                                                       OT *__restrict__ out, unsigned int *err) {
+    using G = Geom<TYPE>;
+    using U = Unit<TYPE>;
+    const int64_t nb = k / G::QK;
+    const int64_t per_row = nb * U::PER_BLOCK;
+    const int64_t units = n_ids * per_row;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < units;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / per_row, r = i - t * per_row;
+        const int64_t bi = r / U::PER_BLOCK;
+        const int u = (int)(r - bi * U::PER_BLOCK);
+        const int32_t id = __ldg(ids + t);
+        float v[8];
+        if (id < 0 || (int64_t)id >= rows) {
+            #pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = 0.f;
+            if (r == 0) atomicOr(err, ERR_BAD_ID);
+        } else {
+            U::decode(w + (int64_t)id * nb * G::BB + bi * G::BB, u, v);
+        }
+        OT *o = out + t * k + bi * G::QK + 8 * u;
+        if constexpr (sizeof(OT) == 4) {
+            reinterpret_cast<float4 *>(o)[0] = make_float4(v[0], v[1], v[2], v[3]);
+            reinterpret_cast<float4 *>(o)[1] = make_float4(v[4], v[5], v[6], v[7]);
+        } else {
+            OT tt[8];
+            #pragma unroll
+            for (int j = 0; j < 8; ++j) store_out(&tt[j], v[j]);
+            *reinterpret_cast<uint4 *>(o) = *reinterpret_cast<const uint4 *>(tt);
+        }
+    }
+}
+
 // ---------------------------------------------------------------- TQ1 scan
 __global__ void tq1_scan_kernel(const uint8_t *__restrict__ w, int64_t blocks,
                                 unsigned long long *first_bad) {
@@ -129,7 +169,10 @@ cudaError_t launch_dequant(int type, const void *w, int64_t rows, int64_t k, voi
     case KQ_Q8_0: return dequant_t<KQ_Q8_0>(w, rows, k, out, dt, s);
     case KQ_Q4_K: return dequant_t<KQ_Q4_K>(w, rows, k, out, dt, s);
     case KQ_Q2_K: return dequant_t<KQ_Q2_K>(w, rows, k, out, dt, s);
-    default: return dequant_t<KQ_TQ1_G128>(w, rows, k, out, dt, s);
+    case KQ_Q5_K: return dequant_t<KQ_Q5_K>(w, rows, k, out, dt, s);
+    case KQ_Q6_K: return dequant_t<KQ_Q6_K>(w, rows, k, out, dt, s);
+    case KQ_TQ1_G128: return dequant_t<KQ_TQ1_G128>(w, rows, k, out, dt, s);
+    default: return cudaErrorInvalidValue;
     }
 }
 
@@ -160,7 +203,40 @@ cudaError_t launch_simple_matmul(int type, const void *w, int64_t n, int64_t k, 
     case KQ_Q8_0: return simple_xy<KQ_Q8_0>(w, n, k, x, xdt, m, y, ydt, s);
     case KQ_Q4_K: return simple_xy<KQ_Q4_K>(w, n, k, x, xdt, m, y, ydt, s);
     case KQ_Q2_K: return simple_xy<KQ_Q2_K>(w, n, k, x, xdt, m, y, ydt, s);
-    default: return simple_xy<KQ_TQ1_G128>(w, n, k, x, xdt, m, y, ydt, s);
+    case KQ_Q5_K: return simple_xy<KQ_Q5_K>(w, n, k, x, xdt, m, y, ydt, s);
+    case KQ_Q6_K: return simple_xy<KQ_Q6_K>(w, n, k, x, xdt, m, y, ydt, s);
+    case KQ_TQ1_G128: return simple_xy<KQ_TQ1_G128>(w, n, k, x, xdt, m, y, ydt, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int TYPE>
+static cudaError_t get_rows_t(const void *w, int64_t rows, int64_t k, const int32_t *ids, int64_t n_ids,
+                              void *out, int dt, cudaStream_t s) {
+    const int64_t units = n_ids * (k / Geom<TYPE>::QK) * Unit<TYPE>::PER_BLOCK;
+    const int g = grid_for(units, 256);
+    const uint8_t *wp = static_cast<const uint8_t *>(w);
+    unsigned int *err = error_word();
+    if (dt == KQ_F32)
+        get_rows_kernel<TYPE, float><<<g, 256, 0, s>>>(wp, rows, k, ids, n_ids, static_cast<float *>(out), err);
+    else if (dt == KQ_BF16)
+        get_rows_kernel<TYPE, __nv_bfloat16><<<g, 256, 0, s>>>(wp, rows, k, ids, n_ids,
+                                                               static_cast<__nv_bfloat16 *>(out), err);
+    else
+        get_rows_kernel<TYPE, __half><<<g, 256, 0, s>>>(wp, rows, k, ids, n_ids, static_cast<__half *>(out), err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_get_rows(int type, const void *w, int64_t rows, int64_t k, const int32_t *ids,
+                            int64_t n_ids, void *out, int dt, cudaStream_t s) {
+    switch (type) {
+    case KQ_Q8_0: return get_rows_t<KQ_Q8_0>(w, rows, k, ids, n_ids, out, dt, s);
+    case KQ_Q4_K: return get_rows_t<KQ_Q4_K>(w, rows, k, ids, n_ids, out, dt, s);
+    case KQ_Q2_K: return get_rows_t<KQ_Q2_K>(w, rows, k, ids, n_ids, out, dt, s);
+    case KQ_Q5_K: return get_rows_t<KQ_Q5_K>(w, rows, k, ids, n_ids, out, dt, s);
+    case KQ_Q6_K: return get_rows_t<KQ_Q6_K>(w, rows, k, ids, n_ids, out, dt, s);
+    case KQ_TQ1_G128: return get_rows_t<KQ_TQ1_G128>(w, rows, k, ids, n_ids, out, dt, s);
+    default: return cudaErrorInvalidValue;
     }
 }
 

@@ -3,8 +3,8 @@
  *         (GGUF-style) weights on NVIDIA B200 (sm_100a).
  *
  * The library decodes the weight blocks on the fly inside its CUDA kernels.
- * Codecs: Q8_0, Q4_K, Q2_K (GGML block formats) and TQ1_G128 (28-byte,
- * 128-weight ternary blocks).
+ * Codecs: Q8_0, Q2_K, Q4_K, Q5_K, Q6_K (GGML block formats) and TQ1_G128
+ * (28-byte, 128-weight ternary blocks).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -51,6 +51,8 @@ extern "C" {
 #define KQ_Q8_0     8     /* 34 B / 32 w:  fp16 d, int8 q[32]; w = d*q            */
 #define KQ_Q2_K     10    /* 84 B / 256 w: scales[16], qs[64], fp16 d, fp16 dmin   */
 #define KQ_Q4_K     12    /* 144 B / 256 w: fp16 d, fp16 dmin, scales[12], qs[128] */
+#define KQ_Q5_K     13    /* 176 B / 256 w: fp16 d, fp16 dmin, scales[12], qh[32], qs[128] */
+#define KQ_Q6_K     14    /* 210 B / 256 w: ql[128], qh[64], int8 scales[16], fp16 d */
 #define KQ_TQ1_G128 1001  /* 28 B / 128 w: 25 full trit bytes, tail byte, fp16 scale */
 
 /* ---- dtypes ---- */
@@ -68,7 +70,7 @@ extern "C" {
 #define KQ_ERR_OVERFLOW        -6   /* a byte or element count overflows int64 / int32 */
 #define KQ_ERR_WORKSPACE       -7   /* workspace null or smaller than required         */
 #define KQ_ERR_CUDA            -8   /* a CUDA runtime call failed                      */
-#define KQ_ERR_DEVICE          -9   /* device-side error word was set (bad expert id)  */
+#define KQ_ERR_DEVICE          -9   /* device-side error word was set (bad expert/row id) */
 #define KQ_ERR_DEVICE_TIMEOUT  -10  /* a bounded device-side wait gave up              */
 #define KQ_ERR_UNSUPPORTED     -11  /* current device is not sm_100 / path unavailable */
 
@@ -142,8 +144,9 @@ KQ_API int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k,
  *   e = ids[t][s];  y[t][s][j] = sum_k dequant(w_e)[j][k] * x[t][k].
  * Same operation as mlx-kquant `gather_qmm` with rhs_indices = ids.
  *   w    expert stack; expert e's [n, kq_row_bytes(type, k)] rows start at
- *        w + e * expert_stride bytes (expert_stride >= n * row bytes,
- *        a multiple of 16) (device)
+ *        w + e * expert_stride bytes (expert_stride >= n * row bytes, a
+ *        multiple of 16 for Q4_K and Q5_K, of 4 for Q2_K, of 2 for the
+ *        others) (device)
  *   x    [n_tokens, k] of x_dtype (KQ_F32 or KQ_BF16) (device)
  *   ids  [n_tokens, top_k] int32 (device; may be produced by earlier work
  *        on the same stream -- the host never reads it)
@@ -221,6 +224,23 @@ KQ_API int kq_matmul_id_noalloc(int type, const void *w, int64_t n_experts, int6
  */
 KQ_API int kq_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_experts,
                  int32_t *counts, int32_t *offsets, int32_t *perm, void *stream);
+
+/*
+ * kq_get_rows -- decode selected weight rows (an embedding lookup).
+ * Defines: Ternary Bonsai ternel_packed_model.py `_GET_ROWS_SOURCE` /
+ * `tq1_get_rows`: decode exactly the requested rows of a packed table, with
+ * no intermediate row buffer; a row id outside the table reads as an
+ * all-zero row.
+ *   w     [rows, kq_row_bytes(type, k)] u8 wire blocks (device)
+ *   ids   [n_ids] int32 row ids (device; may come from earlier work)
+ *   out   [n_ids, k] of out_dtype (KQ_F32, KQ_BF16 or KQ_F16) (device)
+ * Row t of out is the fp32 decode of row ids[t] (bit-exact, as
+ * kq_dequantize), rounded to nearest even for bf16/f16.  An id outside
+ * [0, rows) writes zeros to its row and sets the device error word
+ * (kq_device_status returns KQ_ERR_DEVICE).  All codecs.
+ */
+KQ_API int kq_get_rows(int type, const void *w, int64_t rows, int64_t k, const int32_t *ids,
+                       int64_t n_ids, void *out, int out_dtype, void *stream);
 
 /*
  * kq_validate -- scan TQ1_G128 weights for bytes above the legal maximum

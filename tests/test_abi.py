@@ -39,6 +39,9 @@ def test_block_geometry_and_row_bytes(L):
     assert (L.kq_block_weights(12), L.kq_block_bytes(12)) == (256, 144)
     assert (L.kq_block_weights(10), L.kq_block_bytes(10)) == (256, 84)
     assert (L.kq_block_weights(1001), L.kq_block_bytes(1001)) == (128, 28)
+    assert (L.kq_block_weights(13), L.kq_block_bytes(13)) == (256, 176)
+    assert (L.kq_block_weights(14), L.kq_block_bytes(14)) == (256, 210)
+    assert L.kq_row_bytes(14, 1024) == 840
     assert L.kq_block_weights(3) == 0
     assert L.kq_row_bytes(12, 4096) == 2304
     assert L.kq_row_bytes(1001, 17408) == 3808
@@ -117,3 +120,14 @@ def test_moe_group_argument_errors(L):
     assert L.kq_moe_group(fake, 8, 70000, fake, fake, fake, None) == -1
     assert L.kq_moe_group(vp((1 << 20) + 4), 8, 4, fake, fake, fake, None) == -5   # ids alignment
     assert L.kq_moe_group(fake, 8, 4, vp((1 << 20) + 2), fake, fake, None) == -5   # counts alignment
+
+
+def test_get_rows_argument_errors(L):
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)
+    assert L.kq_get_rows(12, fake, 8, 256, None, 4, fake, 0, None) == -1             # null ids
+    assert L.kq_get_rows(12, fake, 8, 256, fake, 0, fake, 0, None) == -1             # no ids
+    assert L.kq_get_rows(12, fake, 8, 100, fake, 4, fake, 0, None) == -3             # K % 256
+    assert L.kq_get_rows(12, fake, 8, 256, vp((1 << 20) + 4), 4, fake, 0, None) == -5   # ids alignment
+    assert L.kq_get_rows(12, fake, 8, 256, fake, 4, fake, 7, None) == -4             # out dtype
+    assert L.kq_get_rows(99, fake, 8, 256, fake, 4, fake, 0, None) == -2             # codec

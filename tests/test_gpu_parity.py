@@ -15,7 +15,7 @@ from kqtest import BF16_OUT, FP32_PATH_TOL, GEMV_TOL, TOL, row_rel_err, to_devic
 
 pytestmark = pytest.mark.gpu
 
-CODECS = [synth.Q8_0, synth.Q2_K, synth.Q4_K, synth.TQ1_G128]
+CODECS = [synth.Q8_0, synth.Q2_K, synth.Q4_K, synth.Q5_K, synth.Q6_K, synth.TQ1_G128]
 
 
 def rng(seed):
@@ -61,6 +61,37 @@ def test_dequantize_full_workload_weights(kq, name):
     ref = oracle.decode_f32(wl.codec, w, wl.k)
     got = kq.dequantize(to_device_w(w), wl.codec, wl.k).cpu().numpy()
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+# ---------------------------------------------------------------- row gather
+
+@pytest.mark.parametrize("codec", CODECS)
+def test_get_rows_bit_exact(kq, codec):
+    """Rows picked by id decode exactly as the oracle's fp32 decode (bf16 and
+    f16 outputs: that value rounded to nearest even); ids outside the table
+    give zero rows and the device error word."""
+    import torch
+
+    qk = synth.geometry(codec)[0]
+    k = qk * (6 if qk == 256 else 20)
+    rows = 257
+    w = synth.gen_weights(codec, rows, k, rng(400 + codec))
+    ids = np.array([0, 256, 13, 13, 100, 255, 1, 77, 200, 3, 5, 8], dtype=np.int32)
+    wd = to_device_w(w)
+    ref = oracle.get_rows(codec, w, k, ids)
+    got = kq.get_rows(wd, codec, k, torch.from_numpy(ids).cuda()).cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    for dt in (torch.bfloat16, torch.float16):
+        g = kq.get_rows(wd, codec, k, torch.from_numpy(ids).cuda(), dtype=dt).cpu()
+        assert torch.equal(g.view(torch.int16), torch.from_numpy(ref).to(dt).view(torch.int16))
+    assert kq.device_status() == 0
+    bad = np.array([4, -1, rows, 2 ** 31 - 1, 9, 0, 0, 0], dtype=np.int32)
+    got = kq.get_rows(wd, codec, k, torch.from_numpy(bad).cuda()).cpu().numpy()
+    ref = oracle.get_rows(codec, w, k, bad)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    assert np.all(got[1:4] == 0.0)
+    assert kq.device_status() == -9    # KQ_ERR_DEVICE, then cleared
+    assert kq.device_status() == 0
 
 
 # ---------------------------------------------------------------- matmul
