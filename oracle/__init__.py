@@ -149,3 +149,27 @@ def get_rows(codec: int, w: np.ndarray, k: int, ids: np.ndarray) -> np.ndarray:
     if st:
         raise ValueError(f"oracle get_rows failed ({st})")
     return out
+
+
+def act_f64(g: np.ndarray, act: str) -> np.ndarray:
+    """The GLU activations of mlx-kquant `moe_glu_gather_kq`, in fp64:
+    'silu': g * sigmoid(g) = g / (1 + exp(-g));
+    'gelu': the tanh approximation 0.5 * g * (1 + tanh(sqrt(2/pi) * (g + 0.044715 g^3)))."""
+    g = np.asarray(g, dtype=np.float64)
+    with np.errstate(over="ignore", invalid="ignore"):
+        if act == "silu":
+            return g / (1.0 + np.exp(-g))
+        if act == "gelu":
+            return 0.5 * g * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (g + 0.044715 * g ** 3)))
+    raise ValueError(act)
+
+
+def glu_id(codec: int, w_gate: np.ndarray, w_up: np.ndarray, k: int, x: np.ndarray, ids: np.ndarray,
+           act: str = "silu") -> np.ndarray:
+    """Fused MoE GLU (mlx-kquant bindings.cpp `moe_glu_gather_kq`): for every
+    token t and slot s with e = ids[t][s],
+        y[t][s] = act(x[t] @ dequant(w_gate[e])^T) * (x[t] @ dequant(w_up[e])^T),
+    in fp64; an id outside [0, E) gives a NaN row.  w_*: [E, N, row_bytes]."""
+    g = matmul_id(codec, w_gate, k, x, ids)
+    u = matmul_id(codec, w_up, k, x, ids)
+    return act_f64(g, act) * u

@@ -497,3 +497,46 @@ def test_ids_are_distinct_and_in_range():
     ids = synth.gen_ids(32, 6, 64, np.random.default_rng(0))
     assert ids.min() >= 0 and ids.max() < 64
     assert all(len(set(r)) == 6 for r in ids.tolist())
+
+
+# ---------------------------------------------------------------- fused GLU
+
+def test_glu_activations_match_torch_fp64():
+    import torch
+    import torch.nn.functional as F
+
+    g = np.concatenate([np.linspace(-30, 30, 601), [0.0, -0.5, 1.0, 1e-8, -1e-8]])
+    gt = torch.from_numpy(g)
+    assert np.allclose(oracle.act_f64(g, "silu"), F.silu(gt).numpy(), rtol=1e-14, atol=1e-300)
+    assert np.allclose(oracle.act_f64(g, "gelu"), F.gelu(gt, approximate="tanh").numpy(), rtol=1e-14, atol=1e-300)
+    assert oracle.act_f64(np.array([0.0]), "silu")[0] == 0.0
+    # large positive g: silu(g) -> g; large negative: -> 0
+    assert oracle.act_f64(np.array([50.0]), "silu")[0] == 50.0
+    assert abs(oracle.act_f64(np.array([-50.0]), "silu")[0]) < 1e-19
+
+
+def test_glu_id_brute_force_and_bad_ids():
+    import math
+
+    rng = np.random.default_rng(11)
+    e, n, k, t, top_k = 3, 4, 256, 3, 2
+    wg = synth.gen_weights(12, e * n, k, rng).reshape(e, n, -1)
+    wu = synth.gen_weights(12, e * n, k, rng).reshape(e, n, -1)
+    x = synth.gen_x(t, k, "f32", rng).astype(np.float64)
+    ids = np.array([[0, 2], [1, 1], [2, 3]], dtype=np.int32)   # a duplicate, an id outside [0, E)
+    dg = oracle.decode_f64(12, wg.reshape(e * n, -1), k).reshape(e, n, k)
+    du = oracle.decode_f64(12, wu.reshape(e * n, -1), k).reshape(e, n, k)
+    for act in ("silu", "gelu"):
+        y = oracle.glu_id(12, wg, wu, k, x, ids, act)
+        for tt in range(t):
+            for s in range(top_k):
+                ee = ids[tt, s]
+                if ee >= e:
+                    assert np.all(np.isnan(y[tt, s]))
+                    continue
+                for j in range(n):
+                    gv = sum(dg[ee, j, kk] * x[tt, kk] for kk in range(k))
+                    uv = sum(du[ee, j, kk] * x[tt, kk] for kk in range(k))
+                    a = gv / (1 + math.exp(-gv)) if act == "silu" else \
+                        0.5 * gv * (1 + math.tanh(math.sqrt(2 / math.pi) * (gv + 0.044715 * gv ** 3)))
+                    assert abs(y[tt, s, j] - a * uv) <= 1e-9 * max(1.0, abs(a * uv))
