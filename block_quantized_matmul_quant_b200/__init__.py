@@ -68,12 +68,14 @@ def lib():
         L.kq_moe_group.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.kq_validate.argtypes = [i32, vp, i64, i64, ctypes.POINTER(i64), vp]
         L.kq_get_rows.argtypes = [i32, vp, i64, i64, vp, i64, vp, i32, vp]
+        L.kq_matmul_id_glu.argtypes = [i32, vp, vp, i64, i64, i64, i64, vp, i32, i64, vp, i64, vp, i32,
+                                       i32, vp, sz, vp]
         L.kq_device_status.argtypes = [vp]
         L.kq_status_string.argtypes = [i32]
         L.kq_status_string.restype = ctypes.c_char_p
         for f in ("kq_block_weights", "kq_block_bytes", "kq_dequantize", "kq_matmul",
                   "kq_matmul_ex", "kq_matmul_id", "kq_matmul_id_ex", "kq_moe_group", "kq_validate",
-                  "kq_device_status", "kq_get_rows"):
+                  "kq_device_status", "kq_get_rows", "kq_matmul_id_glu"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -235,6 +237,49 @@ def matmul_id(w: torch.Tensor, codec, x: torch.Tensor, ids: torch.Tensor, out=No
     _check(lib().kq_matmul_id_ex(c, _ptr(w), e, n, k, w.stride(0), _ptr(x), _DT[x.dtype], t,
                                  _ptr(ids), top_k, _ptr(out), _DT[out.dtype], _ptr(workspace),
                                  workspace.numel(), path, _stream()), "kq_matmul_id")
+    return out
+
+
+ACTS = {"silu": 0, "gelu": 1}
+
+
+def matmul_id_glu(w_gate: torch.Tensor, w_up: torch.Tensor, codec, x: torch.Tensor, ids: torch.Tensor,
+                  act: str = "silu", out=None, out_dtype=torch.float32, workspace=None) -> torch.Tensor:
+    """y[t, s, n] = act(x[t] @ dequant(w_gate[e])^T)[n] * (x[t] @ dequant(w_up[e])^T)[n],
+    e = ids[t, s]; act 'silu' or 'gelu' (tanh approximation).  Stacks as matmul_id."""
+    c = _codec(codec)
+    for nm, w in (("w_gate", w_gate), ("w_up", w_up)):
+        if w.dim() != 3 or w.dtype != torch.uint8:
+            raise ValueError(f"{nm} must be uint8 [n_experts, n, row_bytes]")
+        _on_current_device(nm, w)
+    if w_up.shape != w_gate.shape or w_up.stride() != w_gate.stride():
+        raise ValueError("w_gate and w_up must have the same shape and layout")
+    e, n, rb = w_gate.shape
+    if x.dim() != 2:
+        raise ValueError("x must be [n_tokens, k]")
+    t, k = x.shape
+    if rb != row_bytes(c, k):
+        raise ValueError("the stacks' last dimension does not match k")
+    if w_gate.stride(2) != 1 or w_gate.stride(1) != rb:
+        raise ValueError("each expert's rows must be packed back to back")
+    _check_tensor("x", x, (t, k), _ACT, w_gate.device)
+    if ids.dim() != 2:
+        raise ValueError("ids must be int32 [n_tokens, top_k]")
+    top_k = ids.shape[1]
+    _check_tensor("ids", ids, (t, top_k), (torch.int32,), w_gate.device)
+    if act not in ACTS:
+        raise ValueError(f"act must be one of {sorted(ACTS)}")
+    if out is None:
+        out = torch.empty((t, top_k, n), dtype=out_dtype, device=x.device)
+    _check_tensor("out", out, (t, top_k, n), _ACT, w_gate.device)
+    need = matmul_id_workspace_bytes(t, top_k, e)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or workspace.device != w_gate.device:
+        raise ValueError("workspace must be a contiguous uint8 tensor on the weights' device")
+    _check(lib().kq_matmul_id_glu(c, _ptr(w_gate), _ptr(w_up), e, n, k, w_gate.stride(0), _ptr(x),
+                                  _DT[x.dtype], t, _ptr(ids), top_k, _ptr(out), _DT[out.dtype], ACTS[act],
+                                  _ptr(workspace), workspace.numel(), _stream()), "kq_matmul_id_glu")
     return out
 
 

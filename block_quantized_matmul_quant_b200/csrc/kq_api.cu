@@ -232,10 +232,15 @@ size_t kq_matmul_id_workspace_bytes(int64_t n_tokens, int64_t top_k, int64_t n_e
     return l.total;
 }
 
-int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
+}  // extern "C"
+
+namespace kq {
+// Host validation shared by the expert-indexed calls; fills the kernel
+// arguments (workspace sections included).  Nothing is launched.
+static int id_setup(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
                     int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
                     const int32_t *ids, int64_t top_k, void *y, int y_dtype, void *workspace,
-                    size_t workspace_bytes, int path, void *stream) {
+                    size_t workspace_bytes, IdArgs *a, int64_t *pairs_out) {
     int64_t rb;
     int st = check_weights(type, w, n, k, &rb);
     if (st) return st;
@@ -257,19 +262,34 @@ int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64
     if (!id_workspace_layout(n_tokens, top_k, n_experts, &l)) return KQ_ERR_OVERFLOW;
     if (workspace == nullptr || workspace_bytes < l.total) return KQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return KQ_ERR_ALIGN;
+    char *ws = static_cast<char *>(workspace);
+    a->type = type; a->w = w; a->n_experts = n_experts; a->n = n; a->k = k;
+    a->expert_stride = expert_stride; a->x = x; a->x_dtype = x_dtype; a->n_tokens = n_tokens;
+    a->top_k = top_k; a->y = y; a->y_dtype = y_dtype;
+    a->counts = reinterpret_cast<int32_t *>(ws + l.counts);
+    a->offsets = reinterpret_cast<int32_t *>(ws + l.offsets);
+    a->perm = reinterpret_cast<int32_t *>(ws + l.perm);
+    a->tiles = reinterpret_cast<int32_t *>(ws + l.tiles);
+    a->n_tiles = reinterpret_cast<int32_t *>(ws + l.n_tiles);
+    *pairs_out = pairs;
+    return KQ_OK;
+}
+}  // namespace kq
+
+extern "C" {
+
+int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
+                    int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
+                    const int32_t *ids, int64_t top_k, void *y, int y_dtype, void *workspace,
+                    size_t workspace_bytes, int path, void *stream) {
+    IdArgs a;
+    int64_t pairs;
+    int st = id_setup(type, w, n_experts, n, k, expert_stride, x, x_dtype, n_tokens, ids, top_k, y,
+                      y_dtype, workspace, workspace_bytes, &a, &pairs);
+    if (st) return st;
     if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMM) return KQ_ERR_ARG;
     if ((st = check_device())) return st;
     cudaStream_t s = (cudaStream_t)stream;
-    char *ws = static_cast<char *>(workspace);
-    IdArgs a;
-    a.type = type; a.w = w; a.n_experts = n_experts; a.n = n; a.k = k;
-    a.expert_stride = expert_stride; a.x = x; a.x_dtype = x_dtype; a.n_tokens = n_tokens;
-    a.top_k = top_k; a.y = y; a.y_dtype = y_dtype;
-    a.counts = reinterpret_cast<int32_t *>(ws + l.counts);
-    a.offsets = reinterpret_cast<int32_t *>(ws + l.offsets);
-    a.perm = reinterpret_cast<int32_t *>(ws + l.perm);
-    a.tiles = reinterpret_cast<int32_t *>(ws + l.tiles);
-    a.n_tiles = reinterpret_cast<int32_t *>(ws + l.n_tiles);
     const bool can_gemv = moe_gemv_supported(type, n, k, n_experts);
     const bool can_gemm = gemm_supported(type, n, k, x_dtype, y_dtype);
     if (path == KQ_PATH_AUTO) {
@@ -291,6 +311,29 @@ int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64
     }
     if (path == KQ_PATH_GEMV) return to_status(launch_moe_gemv(a, s));
     return to_status(launch_simple_id(a, s));
+}
+
+int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_experts, int64_t n,
+                     int64_t k, int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
+                     const int32_t *ids, int64_t top_k, void *y, int y_dtype, int act, void *workspace,
+                     size_t workspace_bytes, void *stream) {
+    IdArgs a;
+    int64_t pairs, rb_unused;
+    int st = id_setup(type, w_gate, n_experts, n, k, expert_stride, x, x_dtype, n_tokens, ids, top_k,
+                      y, y_dtype, workspace, workspace_bytes, &a, &pairs);
+    if (st) return st;
+    if ((st = check_weights(type, w_up, n, k, &rb_unused))) return st;
+    if (act != KQ_ACT_SILU && act != KQ_ACT_GELU_TANH) return KQ_ERR_ARG;
+    if ((st = check_device())) return st;
+    a.w2 = w_up;
+    a.act = act;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = launch_moe_group(ids, pairs, n_experts, const_cast<int32_t *>(a.counts),
+                                     const_cast<int32_t *>(a.offsets),
+                                     const_cast<int32_t *>(a.perm), y, y_dtype, n, s);
+    if (e != cudaSuccess) return KQ_ERR_CUDA;
+    if (moe_gemv_supported(type, n, k, n_experts)) return to_status(launch_moe_gemv(a, s));
+    return to_status(launch_simple_glu(a, s));
 }
 
 int kq_matmul_id(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,

@@ -18,6 +18,8 @@ struct IdArgs {
     const int32_t *counts, *offsets, *perm;  // grouping (device)
     const int32_t *tiles;                    // tensor-core tile list (device)
     const int32_t *n_tiles;                  // its length (device)
+    const void *w2 = nullptr;                // fused GLU: up stack (w: gate stack)
+    int act = 0;                             // fused GLU activation (KQ_ACT_*)
 };
 
 cudaError_t launch_dequant(int type, const void *w, int64_t rows, int64_t k, void *out, int dt,
@@ -32,6 +34,8 @@ cudaError_t launch_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_expe
                              int32_t *counts, int32_t *offsets, int32_t *perm, void *y,
                              int y_dtype, int64_t n, cudaStream_t s);
 cudaError_t launch_simple_id(const IdArgs &a, cudaStream_t s);
+// Plain fused GLU over the grouping (any codec): y = act(x W_gate^T) * (x W_up^T).
+cudaError_t launch_simple_glu(const IdArgs &a, cudaStream_t s);
 // Token tiles of at most bn pairs per expert segment, (expert, first
 // position in perm) each, and their number -- from the grouping's offsets.
 cudaError_t launch_moe_tiles(const int32_t *offsets, int64_t n_experts, int bn, int32_t *tiles,

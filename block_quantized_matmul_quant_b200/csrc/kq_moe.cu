@@ -206,6 +206,101 @@ __global__ void __launch_bounds__(256) simple_id_kernel(
     }
 }
 
+// Plain fused GLU: the same walk with a gate and an up row per warp;
+// y = act(gate) * up (mlx-kquant `moe_glu_gather_kq`).
+__device__ __forceinline__ float glu_act_plain(float g, int act) {
+    if (act == KQ_ACT_GELU_TANH)
+        return 0.5f * g * (1.0f + tanhf(0.7978845608028654f * fmaf(0.044715f * g, g * g, g)));
+    return g / (1.0f + expf(-g));
+}
+
+template <int TYPE, typename XT, typename YT>
+__global__ void __launch_bounds__(256) simple_glu_kernel(
+    const uint8_t *__restrict__ wg, const uint8_t *__restrict__ wu, int64_t n, int64_t k,
+    int64_t expert_stride, const XT *__restrict__ x, int top_k, const int32_t *__restrict__ counts,
+    const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm, YT *__restrict__ y, int act) {
+    using G = Geom<TYPE>;
+    using U = Unit<TYPE>;
+    constexpr int TB = 4;
+    const int e = blockIdx.y;
+    const int cnt = counts[e];
+    if (cnt == 0) return;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = blockIdx.x * 8LL + (threadIdx.x >> 5);
+    if (row >= n) return;
+    const int64_t nb = k / G::QK;
+    const int64_t off = e * expert_stride + row * nb * G::BB;
+    const int32_t *plist = perm + offsets[e];
+    const int64_t units = nb * U::PER_BLOCK;
+    for (int c0 = 0; c0 < cnt; c0 += TB) {
+        int pr[TB];
+        #pragma unroll
+        for (int t = 0; t < TB; ++t) pr[t] = (c0 + t < cnt) ? plist[c0 + t] : -1;
+        float ag[TB] = {0.f, 0.f, 0.f, 0.f}, au[TB] = {0.f, 0.f, 0.f, 0.f};
+        for (int64_t i = lane; i < units; i += 32) {
+            const int64_t bi = i / U::PER_BLOCK;
+            const int u = (int)(i % U::PER_BLOCK);
+            float vg[8], vu[8];
+            U::decode(wg + off + bi * G::BB, u, vg);
+            U::decode(wu + off + bi * G::BB, u, vu);
+            const int64_t col = bi * G::QK + 8 * u;
+            #pragma unroll
+            for (int t = 0; t < TB; ++t) {
+                if (pr[t] >= 0) {
+                    float xv[8];
+                    load_x8(x + (int64_t)(pr[t] / top_k) * k + col, xv);
+                    #pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        ag[t] = fmaf(vg[j], xv[j], ag[t]);
+                        au[t] = fmaf(vu[j], xv[j], au[t]);
+                    }
+                }
+            }
+        }
+        #pragma unroll
+        for (int t = 0; t < TB; ++t) {
+            float g = ag[t], uu = au[t];
+            #pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                g += __shfl_xor_sync(0xffffffffu, g, o);
+                uu += __shfl_xor_sync(0xffffffffu, uu, o);
+            }
+            if (lane == 0 && pr[t] >= 0) store_out(y + (int64_t)pr[t] * n + row, glu_act_plain(g, act) * uu);
+        }
+    }
+}
+
+template <int TYPE, typename XT, typename YT>
+static cudaError_t simple_glu_t(const IdArgs &a, cudaStream_t s) {
+    dim3 grid((unsigned)((a.n + 7) / 8), (unsigned)a.n_experts);
+    simple_glu_kernel<TYPE, XT, YT><<<grid, 256, 0, s>>>(
+        static_cast<const uint8_t *>(a.w), static_cast<const uint8_t *>(a.w2), a.n, a.k, a.expert_stride,
+        static_cast<const XT *>(a.x), (int)a.top_k, a.counts, a.offsets, a.perm, static_cast<YT *>(a.y), a.act);
+    return cudaGetLastError();
+}
+
+template <int TYPE>
+static cudaError_t simple_glu_xy(const IdArgs &a, cudaStream_t s) {
+    if (a.x_dtype == KQ_F32) {
+        if (a.y_dtype == KQ_F32) return simple_glu_t<TYPE, float, float>(a, s);
+        return simple_glu_t<TYPE, float, __nv_bfloat16>(a, s);
+    }
+    if (a.y_dtype == KQ_F32) return simple_glu_t<TYPE, __nv_bfloat16, float>(a, s);
+    return simple_glu_t<TYPE, __nv_bfloat16, __nv_bfloat16>(a, s);
+}
+
+cudaError_t launch_simple_glu(const IdArgs &a, cudaStream_t s) {
+    switch (a.type) {
+    case KQ_Q8_0: return simple_glu_xy<KQ_Q8_0>(a, s);
+    case KQ_Q4_K: return simple_glu_xy<KQ_Q4_K>(a, s);
+    case KQ_Q2_K: return simple_glu_xy<KQ_Q2_K>(a, s);
+    case KQ_Q5_K: return simple_glu_xy<KQ_Q5_K>(a, s);
+    case KQ_Q6_K: return simple_glu_xy<KQ_Q6_K>(a, s);
+    case KQ_TQ1_G128: return simple_glu_xy<KQ_TQ1_G128>(a, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 template <int TYPE, typename XT, typename YT>
 static cudaError_t simple_id_t(const IdArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)((a.n + 7) / 8), (unsigned)a.n_experts);

@@ -5,6 +5,10 @@
 // quantized_matmul_id_ggml.rs (the mv_id route: every routed pair of an
 // expert shares one pass over that expert's rows), after the device-side
 // grouping of kq_moe.cu (per-expert counts, offsets, ascending pair list).
+// Fused GLU mode (mlx-kquant `moe_glu_gather_kq`): a tile carries each
+// output row's gate and up weights as a group's two rows, both products
+// share the activations in registers, and the finishing step writes
+// act(gate) * up.
 //
 // B200 design
 //  * Work items: (expert, round, tile).  A round is up to four of the
@@ -50,6 +54,8 @@ constexpr int MG_SHIFT = MG_PART == 8 ? 2 : MG_PART == 16 ? 1 : 0;   // 32 = MG_
 
 struct MoeGemvParams {
     const uint8_t *w;
+    const uint8_t *w2;         // fused GLU: the up stack (w is the gate stack)
+    int glu, act;              // fused GLU mode; activation (KQ_ACT_*)
     int64_t expert_stride;
     int n, k, nb, nsub;        // rows per expert, K, super-blocks and sub-blocks per row
     int n_experts, top_k;
@@ -57,7 +63,7 @@ struct MoeGemvParams {
     void *y;
     const int32_t *counts, *offsets, *perm;
     int wg, groups;            // warps per row group, row groups
-    int tile_rows, tiles;      // rows per tile, tiles per expert
+    int tile_rows, tiles;      // output rows per tile, tiles per expert
     int slots, slot_bytes, part_off;
     unsigned int *err;
 };
@@ -72,6 +78,15 @@ __device__ __forceinline__ int dp2a_hi(int a, uint32_t b, int c) {
     asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
 }
+// The GLU activations (mlx-kquant `moe_glu_gather_kq`): silu(g) = g / (1 +
+// exp(-g)); gelu: the tanh approximation 0.5 g (1 + tanh(sqrt(2/pi) (g +
+// 0.044715 g^3))).
+__device__ __forceinline__ float glu_act(float g, int act) {
+    if (act == KQ_ACT_GELU_TANH)
+        return 0.5f * g * (1.0f + tanhf(0.7978845608028654f * fmaf(0.044715f * g, g * g, g)));
+    return g / (1.0f + expf(-g));
+}
+
 __device__ __forceinline__ float byte_f(uint32_t w, int i) {   // byte i of w, exactly
     return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | (uint32_t)i)) - 8388608.0f;
 }
@@ -164,9 +179,12 @@ __global__ void __launch_bounds__(MG_THREADS, 1) moe_gemv_kernel(const MoeGemvPa
             const int row0 = t * p.tile_rows;
             const int rows = min(p.tile_rows, p.n - row0);
             const uint32_t bytes = (uint32_t)(rows * row_bytes);
-            mbar_arrive_expect_tx(&full[s], bytes);
-            bulk_g2s(smem + lay.slots + s * p.slot_bytes,
-                     p.w + (int64_t)e_iss * p.expert_stride + (int64_t)row0 * row_bytes, bytes, &full[s]);
+            const int64_t src = (int64_t)e_iss * p.expert_stride + (int64_t)row0 * row_bytes;
+            uint8_t *dst = smem + lay.slots + s * p.slot_bytes;
+            mbar_arrive_expect_tx(&full[s], p.glu ? 2 * bytes : bytes);
+            bulk_g2s(dst, p.w + src, bytes, &full[s]);
+            // fused GLU: the up rows follow the gate rows, p.groups rows on
+            if (p.glu) bulk_g2s(dst + p.groups * row_bytes, p.w2 + src, bytes, &full[s]);
         };
         if (lane == 0)
             for (int i = i0; i < min(i1, i0 + S); ++i) issue(i);
@@ -185,17 +203,37 @@ __global__ void __launch_bounds__(MG_THREADS, 1) moe_gemv_kernel(const MoeGemvPa
             }
             if (!__all_sync(0xffffffffu, mbar_wait_poll(&empty[s], (uint32_t)((i - i0) / S) & 1u, p.err))) break;
             const float *part = reinterpret_cast<const float *>(smem + lay.slots + s * p.slot_bytes + p.part_off);
-            // output (group g, row r, token t): sum of the group's warps
-            const int outs = p.groups * MG_PART;
-            for (int o0 = 0; o0 < outs; o0 += 32) {
-                const int o = o0 + lane;
-                const int g = o / MG_PART, v = o - g * MG_PART, r = v / MG_TB, t = v - r * MG_TB;
-                const int pr = __shfl_sync(0xffffffffu, my_pair, t & (MG_TB - 1));
-                const int row = tile * p.tile_rows + g * MG_R + r;
-                if (o < outs && t < nt && row < p.n) {
-                    float acc = 0.f;
-                    for (int w = 0; w < p.wg; ++w) acc += part[(g * p.wg + w) * MG_PART + v];
-                    store_out(y + (int64_t)pr * p.n + row, acc);
+            if (p.glu) {
+                // output (group g, token t): act(gate sum) * up sum, each the
+                // sum of the group's warps
+                const int outs = p.groups * MG_TB;
+                for (int o0 = 0; o0 < outs; o0 += 32) {
+                    const int o = o0 + lane;
+                    const int g = o / MG_TB, t = o - g * MG_TB;
+                    const int pr = __shfl_sync(0xffffffffu, my_pair, t);
+                    const int row = tile * p.tile_rows + g;
+                    if (o < outs && t < nt && row < p.n) {
+                        float gs = 0.f, us = 0.f;
+                        for (int w = 0; w < p.wg; ++w) {
+                            gs += part[(g * p.wg + w) * MG_PART + t];
+                            us += part[(g * p.wg + w) * MG_PART + MG_TB + t];
+                        }
+                        store_out(y + (int64_t)pr * p.n + row, glu_act(gs, p.act) * us);
+                    }
+                }
+            } else {
+                // output (group g, row r, token t): sum of the group's warps
+                const int outs = p.groups * MG_PART;
+                for (int o0 = 0; o0 < outs; o0 += 32) {
+                    const int o = o0 + lane;
+                    const int g = o / MG_PART, v = o - g * MG_PART, r = v / MG_TB, t = v - r * MG_TB;
+                    const int pr = __shfl_sync(0xffffffffu, my_pair, t & (MG_TB - 1));
+                    const int row = tile * p.tile_rows + g * MG_R + r;
+                    if (o < outs && t < nt && row < p.n) {
+                        float acc = 0.f;
+                        for (int w = 0; w < p.wg; ++w) acc += part[(g * p.wg + w) * MG_PART + v];
+                        store_out(y + (int64_t)pr * p.n + row, acc);
+                    }
                 }
             }
             __syncwarp();
@@ -323,9 +361,11 @@ __global__ void __launch_bounds__(MG_THREADS, 1) moe_gemv_kernel(const MoeGemvPa
         if (active) {
             #pragma unroll
             for (int r = 0; r < MG_R; ++r) {
-                const int row = tile * p.tile_rows + g * MG_R + r;
+                // plain: rows g*R + r of the tile; fused GLU: row g, gate (r = 0)
+                // and up (r = 1) weights
+                const int row = tile * p.tile_rows + (p.glu ? g : g * MG_R + r);
                 if (row >= p.n) break;
-                const uint8_t *rp = slot + (int64_t)(g * MG_R + r) * row_bytes;
+                const uint8_t *rp = slot + (int64_t)(p.glu ? r * p.groups + g : g * MG_R + r) * row_bytes;
                 const uint4 hd = *reinterpret_cast<const uint4 *>(rp + sb * 144);
                 const float d = half_bits_to_float(hd.x), dmin = half_bits_to_float(hd.x >> 16);
                 // 6-bit scale and min of sub-block sj (GGUF Q4_K packing)
@@ -398,15 +438,16 @@ __global__ void __launch_bounds__(MG_THREADS, 1) moe_gemv_kernel(const MoeGemvPa
     }
 }
 
-bool plan_moe_gemv(int64_t n, int64_t k, int64_t n_experts, MoeGemvParams *p) {
+bool plan_moe_gemv(int64_t n, int64_t k, int64_t n_experts, bool glu, MoeGemvParams *p) {
     if (k % 256 || k > 32 * 32 * MG_CWARPS || n < 1 || n > INT32_MAX / 2 || n_experts < 1) return false;
     const int nb = (int)(k / 256), nsub = (int)(k / 32);
     const int wg = (nsub + 31) / 32;
     const int groups = MG_CWARPS / wg;
     if (groups < 1) return false;
-    const int tile_rows = groups * MG_R;
+    static_assert(MG_R == 2, "the fused GLU takes a group's two rows as gate and up");
+    const int tile_rows = glu ? groups : groups * MG_R;   // output rows per tile
     const int64_t row_bytes = (int64_t)nb * 144;
-    const int part_off = (int)(tile_rows * row_bytes);
+    const int part_off = (int)(groups * MG_R * row_bytes);   // weight rows per slot
     const int slot_bytes = (int)((part_off + MG_CWARPS * MG_PART * 4 + 127) / 128 * 128);
     int slots = 8;
     for (; slots >= 2; --slots)
@@ -433,13 +474,17 @@ cudaError_t launch_mg(const MoeGemvParams &p, cudaStream_t s) {
 
 bool moe_gemv_supported(int type, int64_t n, int64_t k, int64_t n_experts) {
     MoeGemvParams p;
-    return type == KQ_Q4_K && plan_moe_gemv(n, k, n_experts, &p);
+    return type == KQ_Q4_K && plan_moe_gemv(n, k, n_experts, false, &p);
 }
 
 cudaError_t launch_moe_gemv(const IdArgs &a, cudaStream_t s) {
     MoeGemvParams p = {};
-    if (a.type != KQ_Q4_K || !plan_moe_gemv(a.n, a.k, a.n_experts, &p)) return cudaErrorNotSupported;
+    const bool glu = a.w2 != nullptr;
+    if (a.type != KQ_Q4_K || !plan_moe_gemv(a.n, a.k, a.n_experts, glu, &p)) return cudaErrorNotSupported;
     p.w = static_cast<const uint8_t *>(a.w);
+    p.w2 = static_cast<const uint8_t *>(a.w2);
+    p.glu = glu ? 1 : 0;
+    p.act = a.act;
     p.expert_stride = a.expert_stride;
     p.top_k = (int)a.top_k;
     p.x = a.x;

@@ -206,6 +206,32 @@ KQ_API int kq_matmul_id_noalloc(int type, const void *w, int64_t n_experts, int6
                                 const int32_t *ids, int64_t top_k, void *y, int y_dtype,
                                 void *stream);
 
+/* ---- fused GLU activations (kq_matmul_id_glu) ---- */
+#define KQ_ACT_SILU       0   /* g / (1 + exp(-g))                                   */
+#define KQ_ACT_GELU_TANH  1   /* 0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3)))      */
+
+/*
+ * kq_matmul_id_glu -- fused mixture-of-experts GLU: gate and up expert
+ * products share the grouping and each activation load, and the epilogue
+ * writes act(gate) * up.
+ * Defines: mlx-kquant bindings.cpp `moe_glu_gather_kq(x, gate_w, up_w,
+ * kquant_type, indices, act)`: for every token t and slot s, e = ids[t][s],
+ *   y[t][s][j] = act(sum_k dequant(w_gate_e)[j][k] x[t][k]) *
+ *                sum_k dequant(w_up_e)[j][k] x[t][k].
+ *   w_gate, w_up  two expert stacks of the same shape and expert_stride, laid
+ *                 out as kq_matmul_id's w (device)
+ *   act           KQ_ACT_SILU or KQ_ACT_GELU_TANH
+ * Other arguments, the workspace (kq_matmul_id_workspace_bytes), invalid
+ * ids (NaN rows, device error word) and errors as kq_matmul_id.  Q4_K runs
+ * the grouped bandwidth kernel (16-bit activation codes, a tile holding each
+ * output row's gate and up weights); other codecs the plain grouped kernel.
+ */
+KQ_API int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_experts,
+                            int64_t n, int64_t k, int64_t expert_stride, const void *x, int x_dtype,
+                            int64_t n_tokens, const int32_t *ids, int64_t top_k, void *y,
+                            int y_dtype, int act, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
 /*
  * kq_moe_group -- the grouping step of kq_matmul_id, exposed for testing.
  * Defines: mlx-kquant bindings.cpp `expert_tile_map` and mlx-native's map0

@@ -501,6 +501,39 @@ def test_matmul_id_grouped_gemv_skewed_and_nonfinite(kq):
     assert kq.device_status() == 0
 
 
+@pytest.mark.parametrize("codec,t,top_k,e,n,k", [
+    (synth.Q4_K, 32, 6, 64, 1408, 2048),   # the MoE workload's shape, gate and up stacks
+    (synth.Q4_K, 20, 4, 5, 300, 1024),     # several rounds per expert
+    (synth.Q4_K, 7, 3, 4, 129, 1280),      # ragged tiles, a group with idle lanes
+    (synth.Q8_0, 9, 2, 3, 70, 256),        # other codecs: the plain fused kernel
+    (synth.Q6_K, 9, 2, 3, 70, 512),
+    (synth.TQ1_G128, 9, 2, 3, 70, 384),
+])
+@pytest.mark.parametrize("act", ["silu", "gelu"])
+@pytest.mark.parametrize("xdt", ["f32", "bf16"])
+def test_matmul_id_glu(kq, codec, t, top_k, e, n, k, act, xdt):
+    """Fused MoE GLU: act(gate) * up per routed pair against the fp64
+    oracle, with an out-of-range id giving a NaN row."""
+    import torch
+
+    r = rng(t + n + k + codec)
+    wg = synth.gen_weights(codec, e * n, k, r).reshape(e, n, -1)
+    wu = synth.gen_weights(codec, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, xdt, r)
+    ids = synth.gen_ids(t, top_k, e, r)
+    ids[t // 2, 0] = e                        # outside the stack: a NaN row
+    ref = oracle.glu_id(codec, wg, wu, k, x, ids, act)
+    y = kq.matmul_id_glu(to_device_w(wg), to_device_w(wu), codec, to_device_x(x, xdt),
+                         torch.from_numpy(ids).cuda(), act=act).cpu().numpy()
+    assert np.all(np.isnan(y[t // 2, 0]))
+    good = ~np.isnan(ref[..., 0])
+    # the product of two results each within its path's bound
+    tol = 2 * (GEMV_TOL if codec == synth.Q4_K else FP32_PATH_TOL)
+    assert row_rel_err(y[good], ref[good]) <= tol
+    assert kq.device_status() == -9
+    assert kq.device_status() == 0
+
+
 def _bf16_weight_reference_id(w, k, x, ids):
     """y[t, s] = x[t] @ bf16(decode_f32(w[ids[t, s]]))^T in fp64 (NaN rows for
     ids outside [0, E)): the tensor-core expert product up to fp32 accumulation."""
