@@ -173,3 +173,28 @@ def glu_id(codec: int, w_gate: np.ndarray, w_up: np.ndarray, k: int, x: np.ndarr
     g = matmul_id(codec, w_gate, k, x, ids)
     u = matmul_id(codec, w_up, k, x, ids)
     return act_f64(g, act) * u
+
+
+def mix_id(codec: int, w: np.ndarray, k: int, x_slotted: np.ndarray, ids: np.ndarray,
+           scores: np.ndarray) -> np.ndarray:
+    """MoE down projection with the routing mix folded in (mlx-kquant
+    `gather_qmv_mix_kq`; slotted input of mlx-native's pooled slotted mm_id):
+    every (token, slot) pair has its own activation row x[t][s] and
+        y[t] = sum_s scores[t][s] * (x[t][s] @ dequant(w[ids[t][s]])^T),
+    in fp64, slots summed in order; a token with an id outside [0, E) gets a
+    NaN row.  w: [E, N, row_bytes]; x: [T, top_k, K]; ids, scores: [T, top_k]."""
+    w = np.ascontiguousarray(w, dtype=np.uint8)
+    e, n, rb = w.shape
+    x = np.asarray(x_slotted, dtype=np.float64)
+    t, top_k, kk = x.shape
+    assert kk == k and ids.shape == (t, top_k) and scores.shape == (t, top_k)
+    dec = decode_f64(codec, w.reshape(e * n, rb), k).reshape(e, n, k)
+    y = np.zeros((t, n))
+    for tt in range(t):
+        for s in range(top_k):
+            ee = int(ids[tt, s])
+            if ee < 0 or ee >= e:
+                y[tt, :] = np.nan
+                break
+            y[tt] += float(scores[tt, s]) * (dec[ee] @ x[tt, s])
+    return y

@@ -542,3 +542,38 @@ def test_glu_id_brute_force_and_bad_ids():
                     a = gv / (1 + math.exp(-gv)) if act == "silu" else \
                         0.5 * gv * (1 + math.tanh(math.sqrt(2 / math.pi) * (gv + 0.044715 * gv ** 3)))
                     assert abs(y[tt, s, j] - a * uv) <= 1e-9 * max(1.0, abs(a * uv))
+
+
+# ---------------------------------------------------------------- down projection with the mix
+
+def test_mix_id_reduces_to_matmul_id_and_brute_force():
+    rng = np.random.default_rng(12)
+    e, n, k, t, top_k = 4, 6, 256, 5, 3
+    w = synth.gen_weights(12, e * n, k, rng).reshape(e, n, -1)
+    ids = synth.gen_ids(t, top_k, e, rng)
+    scores = rng.uniform(0, 1, (t, top_k)).astype(np.float32)
+    # every slot carries its token's row: the mix of matmul_id's rows
+    x = synth.gen_x(t, k, "f32", rng).astype(np.float64)
+    xs = np.repeat(x[:, None, :], top_k, axis=1)
+    y = oracle.mix_id(12, w, k, xs, ids, scores)
+    yid = oracle.matmul_id(12, w, k, x, ids)
+    assert np.allclose(y, (scores[..., None].astype(np.float64) * yid).sum(axis=1), rtol=1e-12, atol=1e-12)
+    # distinct slot rows: brute force
+    xs = synth.gen_x(t * top_k, k, "f32", rng).astype(np.float64).reshape(t, top_k, k)
+    y = oracle.mix_id(12, w, k, xs, ids, scores)
+    dec = oracle.decode_f64(12, w.reshape(e * n, -1), k).reshape(e, n, k)
+    for tt in range(t):
+        for j in range(n):
+            v = sum(float(scores[tt, s]) * sum(dec[ids[tt, s], j, q] * xs[tt, s, q] for q in range(k))
+                    for s in range(top_k))
+            assert abs(y[tt, j] - v) <= 1e-9 * max(1.0, abs(v))
+    # one-hot scores pick a slot's product; a bad id poisons its token
+    sc = np.zeros((t, top_k), np.float32)
+    sc[:, 1] = 1
+    y = oracle.mix_id(12, w, k, xs, ids, sc)
+    for tt in range(t):
+        assert np.allclose(y[tt], dec[ids[tt, 1]] @ xs[tt, 1], rtol=1e-12, atol=1e-12)
+    bad = ids.copy()
+    bad[2, 0] = e
+    y = oracle.mix_id(12, w, k, xs, bad, scores)
+    assert np.all(np.isnan(y[2])) and np.isfinite(y[[0, 1, 3, 4]]).all()
