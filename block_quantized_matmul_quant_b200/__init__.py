@@ -70,12 +70,16 @@ def lib():
         L.kq_get_rows.argtypes = [i32, vp, i64, i64, vp, i64, vp, i32, vp]
         L.kq_matmul_id_glu.argtypes = [i32, vp, vp, i64, i64, i64, i64, vp, i32, i64, vp, i64, vp, i32,
                                        i32, vp, sz, vp]
+        L.kq_matmul_id_mix_workspace_bytes.argtypes = [i64, i64, i64, i64]
+        L.kq_matmul_id_mix_workspace_bytes.restype = sz
+        L.kq_matmul_id_mix.argtypes = [i32, vp, i64, i64, i64, i64, vp, i32, i64, vp, vp, i64, vp, i32,
+                                       vp, sz, i32, vp]
         L.kq_device_status.argtypes = [vp]
         L.kq_status_string.argtypes = [i32]
         L.kq_status_string.restype = ctypes.c_char_p
         for f in ("kq_block_weights", "kq_block_bytes", "kq_dequantize", "kq_matmul",
                   "kq_matmul_ex", "kq_matmul_id", "kq_matmul_id_ex", "kq_moe_group", "kq_validate",
-                  "kq_device_status", "kq_get_rows", "kq_matmul_id_glu"):
+                  "kq_device_status", "kq_get_rows", "kq_matmul_id_glu", "kq_matmul_id_mix"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -280,6 +284,54 @@ def matmul_id_glu(w_gate: torch.Tensor, w_up: torch.Tensor, codec, x: torch.Tens
     _check(lib().kq_matmul_id_glu(c, _ptr(w_gate), _ptr(w_up), e, n, k, w_gate.stride(0), _ptr(x),
                                   _DT[x.dtype], t, _ptr(ids), top_k, _ptr(out), _DT[out.dtype], ACTS[act],
                                   _ptr(workspace), workspace.numel(), _stream()), "kq_matmul_id_glu")
+    return out
+
+
+FLAG_REUSE_GROUPING = 0x400
+
+
+def matmul_id_mix_workspace_bytes(n_tokens: int, top_k: int, n_experts: int, n: int) -> int:
+    return int(lib().kq_matmul_id_mix_workspace_bytes(n_tokens, top_k, n_experts, n))
+
+
+def matmul_id_mix(w: torch.Tensor, codec, x: torch.Tensor, ids: torch.Tensor, scores: torch.Tensor,
+                  out=None, out_dtype=torch.float32, workspace=None, path: int = PATH_AUTO,
+                  reuse_grouping: bool = False) -> torch.Tensor:
+    """y[t, n] = sum_s scores[t, s] * (x[t, s] @ dequant(w[ids[t, s]])^T)[n].
+    w: [E, n, row_bytes] uint8; x: [T, top_k, k] (one row per routed slot);
+    ids: [T, top_k] int32; scores: [T, top_k] float32.  reuse_grouping: the
+    workspace already holds the grouping of these ids from an earlier
+    expert-indexed call on this stream (see kq.h)."""
+    c = _codec(codec)
+    if w.dim() != 3 or w.dtype != torch.uint8:
+        raise ValueError("w must be uint8 [n_experts, n, row_bytes]")
+    e, n, rb = w.shape
+    if x.dim() != 3:
+        raise ValueError("x must be [n_tokens, top_k, k]")
+    t, top_k, k = x.shape
+    if rb != row_bytes(c, k):
+        raise ValueError("w's last dimension does not match k")
+    if w.stride(2) != 1 or w.stride(1) != rb:
+        raise ValueError("each expert's rows must be packed back to back")
+    _on_current_device("w", w)
+    _check_tensor("x", x, (t, top_k, k), _ACT, w.device)
+    _check_tensor("ids", ids, (t, top_k), (torch.int32,), w.device)
+    _check_tensor("scores", scores, (t, top_k), (torch.float32,), w.device)
+    if out is None:
+        out = torch.empty((t, n), dtype=out_dtype, device=x.device)
+    _check_tensor("out", out, (t, n), _ACT, w.device)
+    need = matmul_id_mix_workspace_bytes(t, top_k, e, n)
+    if workspace is None:
+        if reuse_grouping:
+            raise ValueError("reuse_grouping needs the workspace that holds the grouping")
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or workspace.device != w.device:
+        raise ValueError("workspace must be a contiguous uint8 tensor on the weights' device")
+    flags = path | (FLAG_REUSE_GROUPING if reuse_grouping else 0)
+    _check(lib().kq_matmul_id_mix(c, _ptr(w), e, n, k, w.stride(0), _ptr(x), _DT[x.dtype], t,
+                                  _ptr(ids), _ptr(scores), top_k, _ptr(out), _DT[out.dtype],
+                                  _ptr(workspace), workspace.numel(), flags, _stream()),
+           "kq_matmul_id_mix")
     return out
 
 

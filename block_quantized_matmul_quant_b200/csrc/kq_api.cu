@@ -132,6 +132,14 @@ struct IdWorkspace {
     size_t counts, offsets, perm, tiles, n_tiles, total;
 };
 static size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
+// The routing-mix call adds one section after the grouping: the fp32
+// per-pair products [pairs, n].
+static bool mix_workspace_bytes(const struct IdWorkspace &l, int64_t pairs, int64_t n, size_t *total) {
+    int64_t e, b;
+    if (n <= 0 || !mul_ok(pairs, n, &e) || !mul_ok(e, 4, &b) || b > INT64_MAX - 512) return false;
+    *total = l.total + up256((size_t)b);
+    return true;
+}
 static bool id_workspace_layout(int64_t n_tokens, int64_t top_k, int64_t n_experts, IdWorkspace *l) {
     int64_t pairs;
     if (n_tokens <= 0 || top_k <= 0 || n_experts <= 0) return false;
@@ -232,15 +240,26 @@ size_t kq_matmul_id_workspace_bytes(int64_t n_tokens, int64_t top_k, int64_t n_e
     return l.total;
 }
 
+size_t kq_matmul_id_mix_workspace_bytes(int64_t n_tokens, int64_t top_k, int64_t n_experts, int64_t n) {
+    IdWorkspace l;
+    size_t total;
+    if (!id_workspace_layout(n_tokens, top_k, n_experts, &l)) return 0;
+    if (!mix_workspace_bytes(l, n_tokens * top_k, n, &total)) return 0;
+    return total;
+}
+
 }  // extern "C"
 
 namespace kq {
 // Host validation shared by the expert-indexed calls; fills the kernel
-// arguments (workspace sections included).  Nothing is launched.
+// arguments (workspace sections included).  Nothing is launched.  With
+// `slotted` (the routing-mix call) x has one row per pair, y one row per
+// token, and the per-pair products go to an fp32 section of the workspace
+// after the grouping's sections.
 static int id_setup(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
                     int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
                     const int32_t *ids, int64_t top_k, void *y, int y_dtype, void *workspace,
-                    size_t workspace_bytes, IdArgs *a, int64_t *pairs_out) {
+                    size_t workspace_bytes, IdArgs *a, int64_t *pairs_out, bool slotted = false) {
     int64_t rb;
     int st = check_weights(type, w, n, k, &rb);
     if (st) return st;
@@ -254,13 +273,15 @@ static int id_setup(int type, const void *w, int64_t n_experts, int64_t n, int64
         return KQ_ERR_OVERFLOW;
     if (!mul_ok(n_tokens, top_k, &pairs) || pairs > INT32_MAX) return KQ_ERR_OVERFLOW;
     if (!mul_ok(pairs, n, &ypairs)) return KQ_ERR_OVERFLOW;
-    if ((st = check_act(x, x_dtype, n_tokens, k, false))) return st;
-    if ((st = check_act(y, y_dtype, pairs, n, false))) return st;
+    if ((st = check_act(x, x_dtype, slotted ? pairs : n_tokens, k, false))) return st;
+    if ((st = check_act(y, y_dtype, slotted ? n_tokens : pairs, n, false))) return st;
     if (ids == nullptr) return KQ_ERR_ARG;
     if (!aligned16(ids)) return KQ_ERR_ALIGN;
     IdWorkspace l;
     if (!id_workspace_layout(n_tokens, top_k, n_experts, &l)) return KQ_ERR_OVERFLOW;
-    if (workspace == nullptr || workspace_bytes < l.total) return KQ_ERR_WORKSPACE;
+    size_t need = l.total;
+    if (slotted && !mix_workspace_bytes(l, pairs, n, &need)) return KQ_ERR_OVERFLOW;
+    if (workspace == nullptr || workspace_bytes < need) return KQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return KQ_ERR_ALIGN;
     char *ws = static_cast<char *>(workspace);
     a->type = type; a->w = w; a->n_experts = n_experts; a->n = n; a->k = k;
@@ -271,6 +292,11 @@ static int id_setup(int type, const void *w, int64_t n_experts, int64_t n, int64
     a->perm = reinterpret_cast<int32_t *>(ws + l.perm);
     a->tiles = reinterpret_cast<int32_t *>(ws + l.tiles);
     a->n_tiles = reinterpret_cast<int32_t *>(ws + l.n_tiles);
+    if (slotted) {
+        a->x_slotted = true;
+        a->y = ws + l.total;
+        a->y_dtype = KQ_F32;
+    }
     *pairs_out = pairs;
     return KQ_OK;
 }
@@ -334,6 +360,51 @@ int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_e
     if (e != cudaSuccess) return KQ_ERR_CUDA;
     if (moe_gemv_supported(type, n, k, n_experts)) return to_status(launch_moe_gemv(a, s));
     return to_status(launch_simple_glu(a, s));
+}
+
+int kq_matmul_id_mix(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
+                     int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
+                     const int32_t *ids, const float *scores, int64_t top_k, void *y, int y_dtype,
+                     void *workspace, size_t workspace_bytes, int path, void *stream) {
+    IdArgs a;
+    int64_t pairs;
+    int st = id_setup(type, w, n_experts, n, k, expert_stride, x, x_dtype, n_tokens, ids, top_k, y,
+                      y_dtype, workspace, workspace_bytes, &a, &pairs, true);
+    if (st) return st;
+    if (scores == nullptr) return KQ_ERR_ARG;
+    if (!aligned16(scores)) return KQ_ERR_ALIGN;
+    const bool reuse = (path & KQ_FLAG_REUSE_GROUPING) != 0;
+    path &= ~KQ_FLAG_REUSE_GROUPING;
+    if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMM) return KQ_ERR_ARG;
+    if ((st = check_device())) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool can_gemv = moe_gemv_supported(type, n, k, n_experts);
+    const bool can_gemm = gemm_supported(type, n, k, x_dtype, KQ_F32);
+    if (path == KQ_PATH_AUTO) {
+        if (can_gemm && (!can_gemv || pairs > ID_GEMV_MAX_PAIRS_PER_EXPERT * n_experts)) path = KQ_PATH_GEMM;
+        else path = can_gemv ? KQ_PATH_GEMV : KQ_PATH_SIMPLE;
+    }
+    if (path == KQ_PATH_GEMM && !can_gemm) return KQ_ERR_UNSUPPORTED;
+    if (path == KQ_PATH_GEMV && !can_gemv) return KQ_ERR_UNSUPPORTED;
+    cudaError_t e = cudaSuccess;
+    if (!reuse)
+        e = launch_moe_group(ids, pairs, n_experts, const_cast<int32_t *>(a.counts),
+                             const_cast<int32_t *>(a.offsets), const_cast<int32_t *>(a.perm), nullptr,
+                             KQ_F32, n, s);
+    if (e != cudaSuccess) return KQ_ERR_CUDA;
+    if (path == KQ_PATH_GEMM) {
+        const int bn = gemm_id_bn(n_tokens, top_k, n_experts);
+        e = launch_moe_tiles(a.offsets, n_experts, bn, const_cast<int32_t *>(a.tiles),
+                             const_cast<int32_t *>(a.n_tiles), s);
+        if (e == cudaSuccess) e = launch_gemm_id(a, bn, s);
+    } else if (path == KQ_PATH_GEMV) {
+        e = launch_moe_gemv(a, s);
+    } else {
+        e = launch_simple_id(a, s);
+    }
+    if (e != cudaSuccess) return KQ_ERR_CUDA;
+    return to_status(launch_moe_mix(static_cast<const float *>(a.y), ids, scores, n_tokens, top_k,
+                                    n_experts, n, y, y_dtype, s));
 }
 
 int kq_matmul_id(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,

@@ -797,9 +797,9 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     p.offsets = a.offsets;
     p.id_tiles = reinterpret_cast<const int2 *>(a.tiles);
     p.id_n_tiles = a.n_tiles;
-    p.top_k = (int)a.top_k;
+    p.top_k = a.x_div();
     CUtensorMap tx, tw;
-    if (!encode_x_map(&tx, a.x, a.n_tokens, a.k, 1) ||
+    if (!encode_x_map(&tx, a.x, a.x_rows(), a.k, 1) ||
         !encode_w_map(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride))
         return cudaErrorInvalidValue;
     // persistent grid: the number of token tiles is only known on the device

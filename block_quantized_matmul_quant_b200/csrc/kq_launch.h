@@ -20,6 +20,10 @@ struct IdArgs {
     const int32_t *n_tiles;                  // its length (device)
     const void *w2 = nullptr;                // fused GLU: up stack (w: gate stack)
     int act = 0;                             // fused GLU activation (KQ_ACT_*)
+    bool x_slotted = false;                  // x holds one row per pair [n_tokens * top_k, k]
+    // Pair index p = t * top_k + s reads x row p / x_div().
+    int x_div() const { return x_slotted ? 1 : (int)top_k; }
+    int64_t x_rows() const { return x_slotted ? n_tokens * top_k : n_tokens; }
 };
 
 cudaError_t launch_dequant(int type, const void *w, int64_t rows, int64_t k, void *out, int dt,
@@ -36,6 +40,12 @@ cudaError_t launch_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_expe
 cudaError_t launch_simple_id(const IdArgs &a, cudaStream_t s);
 // Plain fused GLU over the grouping (any codec): y = act(x W_gate^T) * (x W_up^T).
 cudaError_t launch_simple_glu(const IdArgs &a, cudaStream_t s);
+// Routing mix: y[t] = sum over s of scores[t][s] * pair_out[t * top_k + s]
+// (fp32 rows of n), slots in order; a token with an id outside [0, E) gets a
+// NaN row.
+cudaError_t launch_moe_mix(const float *pair_out, const int32_t *ids, const float *scores,
+                           int64_t n_tokens, int64_t top_k, int64_t n_experts, int64_t n, void *y,
+                           int y_dtype, cudaStream_t s);
 // Token tiles of at most bn pairs per expert segment, (expert, first
 // position in perm) each, and their number -- from the grouping's offsets.
 cudaError_t launch_moe_tiles(const int32_t *offsets, int64_t n_experts, int bn, int32_t *tiles,

@@ -270,12 +270,81 @@ __global__ void __launch_bounds__(256) simple_glu_kernel(
     }
 }
 
+// ---------------------------------------------------------------- routing mix
+// mlx-kquant `gather_qmv_mix_kq`: the slots' products are summed in fp32,
+// each weighted by its routing score.  Grid (column chunks, tokens); a
+// thread owns VW adjacent columns of one token and reads the token's top_k
+// pair rows in slot order, so the sum is the same on every run.
+constexpr int MIX_THREADS = 256;
+
+template <int VW, typename YT>
+__global__ void __launch_bounds__(MIX_THREADS) moe_mix_kernel(
+    const float *__restrict__ pair_out, const int32_t *__restrict__ ids,
+    const float *__restrict__ scores, int n_tokens, int top_k, int n_experts, int64_t n,
+    YT *__restrict__ y) {
+    const int64_t j0 = ((int64_t)blockIdx.x * MIX_THREADS + threadIdx.x) * VW;
+    if (j0 >= n) return;
+    for (int t = blockIdx.y; t < n_tokens; t += gridDim.y) {
+        float acc[VW];
+        #pragma unroll
+        for (int v = 0; v < VW; ++v) acc[v] = 0.f;
+        bool bad = false;
+        for (int sl = 0; sl < top_k; ++sl) {
+            const int64_t pr = (int64_t)t * top_k + sl;
+            const int e = ids[pr];
+            bad |= e < 0 || e >= n_experts;
+            const float sc = scores[pr];
+            const float *row = pair_out + pr * n + j0;
+            float q[VW];
+            if constexpr (VW == 4) {
+                const float4 f = *reinterpret_cast<const float4 *>(row);
+                q[0] = f.x; q[1] = f.y; q[2] = f.z; q[3] = f.w;
+            } else {
+                q[0] = row[0];
+            }
+            #pragma unroll
+            for (int v = 0; v < VW; ++v) acc[v] = fmaf(sc, q[v], acc[v]);
+        }
+        YT *yr = y + (int64_t)t * n + j0;
+        #pragma unroll
+        for (int v = 0; v < VW; ++v) store_out(yr + v, bad ? __int_as_float(0x7fc00000) : acc[v]);
+    }
+}
+
+template <typename YT>
+static cudaError_t moe_mix_t(const float *pair_out, const int32_t *ids, const float *scores,
+                             int64_t n_tokens, int64_t top_k, int64_t n_experts, int64_t n, YT *y,
+                             cudaStream_t s) {
+    const int vw = n % 4 == 0 ? 4 : 1;
+    const int64_t chunks = (n / vw + MIX_THREADS - 1) / MIX_THREADS;
+    if (chunks > INT32_MAX) return cudaErrorInvalidValue;
+    dim3 grid((unsigned)chunks, (unsigned)(n_tokens < 65535 ? n_tokens : 65535));
+    if (vw == 4)
+        moe_mix_kernel<4, YT><<<grid, MIX_THREADS, 0, s>>>(pair_out, ids, scores, (int)n_tokens,
+                                                          (int)top_k, (int)n_experts, n, y);
+    else
+        moe_mix_kernel<1, YT><<<grid, MIX_THREADS, 0, s>>>(pair_out, ids, scores, (int)n_tokens,
+                                                          (int)top_k, (int)n_experts, n, y);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_moe_mix(const float *pair_out, const int32_t *ids, const float *scores,
+                           int64_t n_tokens, int64_t top_k, int64_t n_experts, int64_t n, void *y,
+                           int y_dtype, cudaStream_t s) {
+    if (y_dtype == KQ_F32)
+        return moe_mix_t(pair_out, ids, scores, n_tokens, top_k, n_experts, n, static_cast<float *>(y), s);
+    if (y_dtype == KQ_BF16)
+        return moe_mix_t(pair_out, ids, scores, n_tokens, top_k, n_experts, n,
+                         static_cast<__nv_bfloat16 *>(y), s);
+    return cudaErrorInvalidValue;
+}
+
 template <int TYPE, typename XT, typename YT>
 static cudaError_t simple_glu_t(const IdArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)((a.n + 7) / 8), (unsigned)a.n_experts);
     simple_glu_kernel<TYPE, XT, YT><<<grid, 256, 0, s>>>(
         static_cast<const uint8_t *>(a.w), static_cast<const uint8_t *>(a.w2), a.n, a.k, a.expert_stride,
-        static_cast<const XT *>(a.x), (int)a.top_k, a.counts, a.offsets, a.perm, static_cast<YT *>(a.y), a.act);
+        static_cast<const XT *>(a.x), a.x_div(), a.counts, a.offsets, a.perm, static_cast<YT *>(a.y), a.act);
     return cudaGetLastError();
 }
 
@@ -306,7 +375,7 @@ static cudaError_t simple_id_t(const IdArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)((a.n + 7) / 8), (unsigned)a.n_experts);
     simple_id_kernel<TYPE, XT, YT><<<grid, 256, 0, s>>>(
         static_cast<const uint8_t *>(a.w), a.n, a.k, a.expert_stride,
-        static_cast<const XT *>(a.x), (int)a.top_k, a.counts, a.offsets, a.perm,
+        static_cast<const XT *>(a.x), a.x_div(), a.counts, a.offsets, a.perm,
         static_cast<YT *>(a.y));
     return cudaGetLastError();
 }

@@ -486,7 +486,7 @@ cudaError_t launch_moe_gemv(const IdArgs &a, cudaStream_t s) {
     p.glu = glu ? 1 : 0;
     p.act = a.act;
     p.expert_stride = a.expert_stride;
-    p.top_k = (int)a.top_k;
+    p.top_k = a.x_div();
     p.x = a.x;
     p.y = a.y;
     p.counts = a.counts;

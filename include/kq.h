@@ -233,6 +233,51 @@ KQ_API int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int6
                             void *stream);
 
 /*
+ * kq_matmul_id_mix -- mixture-of-experts down projection with the routing
+ * mix folded in.
+ * Defines: mlx-kquant bindings.cpp `gather_qmv_mix_kq(x, w, shexp_w,
+ * kquant_type, indices, scores)` (every slot's product accumulated in f32,
+ * weighted by its score, in place of a gather followed by a weighted sum),
+ * with the slotted input of mlx-native's `quantized_matmul_id_ggml_pooled_
+ * slotted` (one activation row per routed slot).  For every token t:
+ *   y[t][j] = sum over s = 0 .. top_k-1 of
+ *             scores[t][s] * sum_k dequant(w_{ids[t][s]})[j][k] x[t][s][k].
+ *   x        [n_tokens, top_k, k] f32 or bf16 (device), e.g. the output of
+ *            kq_matmul_id_glu for the same ids
+ *   ids      [n_tokens, top_k] int32 (device)
+ *   scores   [n_tokens, top_k] f32 (device)
+ *   y        [n_tokens, n] f32 or bf16 (device)
+ *   w, n_experts, n, k, expert_stride  as kq_matmul_id
+ *   workspace  device scratch of at least
+ *        kq_matmul_id_mix_workspace_bytes(n_tokens, top_k, n_experts, n) bytes:
+ *        kq_matmul_id's sections at the same offsets, then the fp32
+ *        per-pair products [n_tokens * top_k, n].
+ *   path     KQ_PATH_AUTO / SIMPLE / GEMV / GEMM as kq_matmul_id_ex,
+ *            optionally OR KQ_FLAG_REUSE_GROUPING.
+ * The slots are summed in order in fp32, so equal inputs give equal bits.
+ * A shared expert of the routed experts' shape is one more slot: store it in
+ * the stack as one more expert and give each token a slot with its id and
+ * weight.  A token with any id outside [0, n_experts) gets a NaN row and the
+ * device error word is set (KQ_ERR_DEVICE from kq_device_status).
+ * KQ_FLAG_REUSE_GROUPING skips the grouping step and uses the one the
+ * workspace already holds.  Use it only when an earlier kq_matmul_id,
+ * kq_matmul_id_ex, kq_matmul_id_glu or kq_matmul_id_mix call on the same
+ * stream grouped these same ids (same n_tokens, top_k, n_experts) into this
+ * workspace and nothing has written the workspace's first
+ * kq_matmul_id_workspace_bytes(n_tokens, top_k, n_experts) bytes since: a
+ * stale grouping makes the kernels read and write outside the buffers.
+ * Errors as kq_matmul_id; scores null gives KQ_ERR_ARG.
+ */
+#define KQ_FLAG_REUSE_GROUPING 0x400
+KQ_API size_t kq_matmul_id_mix_workspace_bytes(int64_t n_tokens, int64_t top_k, int64_t n_experts,
+                                               int64_t n);
+KQ_API int kq_matmul_id_mix(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
+                            int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
+                            const int32_t *ids, const float *scores, int64_t top_k, void *y,
+                            int y_dtype, void *workspace, size_t workspace_bytes, int path,
+                            void *stream);
+
+/*
  * kq_moe_group -- the grouping step of kq_matmul_id, exposed for testing.
  * Defines: mlx-kquant bindings.cpp `expert_tile_map` and mlx-native's map0
  * schedule (per-expert routed counts and routed-token lists, built on the

@@ -131,3 +131,29 @@ def test_get_rows_argument_errors(L):
     assert L.kq_get_rows(12, fake, 8, 256, vp((1 << 20) + 4), 4, fake, 0, None) == -5   # ids alignment
     assert L.kq_get_rows(12, fake, 8, 256, fake, 4, fake, 7, None) == -4             # out dtype
     assert L.kq_get_rows(99, fake, 8, 256, fake, 4, fake, 0, None) == -2             # codec
+
+
+def test_mix_workspace_and_argument_errors(L):
+    vp = ctypes.c_void_p
+    idb = L.kq_matmul_id_workspace_bytes(4, 2, 3)
+    mb = L.kq_matmul_id_mix_workspace_bytes(4, 2, 3, 100)
+    # the grouping's sections, then the fp32 per-pair products (8 pairs x 100), 256-byte steps
+    assert mb == idb + (8 * 100 * 4 + 255) // 256 * 256
+    assert L.kq_matmul_id_mix_workspace_bytes(4, 2, 3, 0) == 0
+    assert L.kq_matmul_id_mix_workspace_bytes(0, 2, 3, 100) == 0
+    fake = vp(1 << 20)
+    args = lambda **kw: dict(dict(t=12, w=fake, e=3, n=100, k=256, es=100 * 144, x=fake, xdt=0, nt=4,
+                                  ids=fake, sc=fake, tk=2, y=fake, ydt=0, ws=fake, wsb=mb, path=0), **kw)
+
+    def call(a):
+        return L.kq_matmul_id_mix(a["t"], a["w"], a["e"], a["n"], a["k"], a["es"], a["x"], a["xdt"],
+                                  a["nt"], a["ids"], a["sc"], a["tk"], a["y"], a["ydt"], a["ws"],
+                                  a["wsb"], a["path"], None)
+
+    assert call(args(sc=None)) == -1                         # null scores
+    assert call(args(sc=vp((1 << 20) + 4))) == -5            # scores alignment
+    assert call(args(wsb=idb)) == -7                         # no room for the per-pair products
+    assert call(args(path=9)) == -1                          # unknown path
+    assert call(args(ydt=2)) == -4                           # f16 output
+    assert call(args(tk=4)) == -1                            # top_k > n_experts
+    assert call(args(k=100)) == -3                           # K % 256

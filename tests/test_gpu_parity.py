@@ -534,6 +534,135 @@ def test_matmul_id_glu(kq, codec, t, top_k, e, n, k, act, xdt):
     assert kq.device_status() == 0
 
 
+def _pair_refs(codec, w, k, xs, ids):
+    """Per-pair fp64 oracle products [T, top_k, n] of a slotted input."""
+    t, top_k, _ = xs.shape
+    flat = oracle.matmul_id(codec, w, k, xs.reshape(t * top_k, k), ids.reshape(-1, 1))
+    return flat.reshape(t, top_k, -1)
+
+
+def _mix_err_ok(y, ref, pair_ref, scores, tol):
+    """|y - ref| per token within tol times the mix of its slots' row maxima:
+    each slot's product is within tol of its row maximum and the mix weights
+    it by |score|."""
+    bound = tol * (np.abs(scores.astype(np.float64)) * np.abs(pair_ref).max(axis=2)).sum(axis=1)
+    err = np.abs(np.asarray(y, np.float64) - ref).max(axis=1)
+    return bool(np.all(err <= bound + 1e-30)), float((err / np.maximum(bound, 1e-30)).max())
+
+
+@pytest.mark.parametrize("codec,path,xdt,t,top_k,e,n,k", [
+    (synth.Q4_K, 2, "bf16", 32, 6, 64, 512, 1536),    # decode routing, a down projection's shape
+    (synth.Q4_K, 2, "f32", 5, 3, 6, 130, 512),        # ragged rows
+    (synth.Q4_K, 3, "bf16", 200, 4, 8, 300, 1024),    # tensor-core path, slotted rows by TMA
+    (synth.Q4_K, 0, "bf16", 64, 6, 16, 256, 768),     # auto
+    (synth.Q4_K, 1, "f32", 9, 2, 5, 129, 256),
+    (synth.Q8_0, 0, "bf16", 11, 3, 6, 96, 1408),      # K = 1408: 44 blocks of 32
+    (synth.Q2_K, 0, "f32", 6, 2, 4, 70, 512),
+    (synth.Q5_K, 0, "bf16", 6, 2, 4, 70, 512),
+    (synth.Q6_K, 0, "f32", 6, 2, 4, 70, 512),
+    (synth.TQ1_G128, 0, "bf16", 7, 2, 4, 64, 1408),
+])
+def test_matmul_id_mix(kq, codec, path, xdt, t, top_k, e, n, k):
+    """Down projection with the routing mix: per token, the score-weighted sum
+    of its slots' products against the fp64 oracle; deterministic; bf16 out."""
+    import torch
+
+    r = rng(3 * t + n + k + codec + path)
+    w = synth.gen_weights(codec, e * n, k, r).reshape(e, n, -1)
+    xs = synth.gen_x(t * top_k, k, xdt, r).reshape(t, top_k, k)
+    ids = synth.gen_ids(t, top_k, e, r)
+    scores = r.uniform(0.0, 1.0, (t, top_k)).astype(np.float32)
+    ref = oracle.mix_id(codec, w, k, xs, ids, scores)
+    pref = _pair_refs(codec, w, k, xs, ids)
+    wd, xd = to_device_w(w), to_device_x(xs, xdt)
+    idd, sd = torch.from_numpy(ids).cuda(), torch.from_numpy(scores).cuda()
+    y = kq.matmul_id_mix(wd, codec, xd, idd, sd, path=path).cpu().numpy()
+    if path == 3 or (path == 0 and codec == synth.Q4_K and xdt == "bf16" and t * top_k > e):
+        tol = TOL["bf16"]
+    elif codec == synth.Q4_K and path in (0, 2):
+        tol = GEMV_TOL
+    else:
+        tol = FP32_PATH_TOL
+    ok, worst = _mix_err_ok(y, ref, pref, scores, tol)
+    assert ok, worst
+    y2 = kq.matmul_id_mix(wd, codec, xd, idd, sd, path=path).cpu().numpy()
+    assert np.array_equal(y.view(np.uint32), y2.view(np.uint32))
+    yb = kq.matmul_id_mix(wd, codec, xd, idd, sd, path=path, out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert np.all(np.abs(yb - y) <= BF16_OUT * np.abs(y) + 1e-30)
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_matmul_id_mix_scores_and_bad_ids(kq, path):
+    """One-hot scores give one slot's product; zero scores give zero rows;
+    a token with an id outside the stack gets a NaN row and the error word."""
+    import torch
+
+    t, top_k, e, n, k = 10, 3, 5, 200, 512
+    r = rng(91 + path)
+    w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
+    xs = synth.gen_x(t * top_k, k, "f32", r).reshape(t, top_k, k)
+    ids = synth.gen_ids(t, top_k, e, r)
+    wd, xd, idd = to_device_w(w), to_device_x(xs, "f32"), torch.from_numpy(ids).cuda()
+    one = np.zeros((t, top_k), np.float32)
+    one[:, 2] = 1.0
+    y = kq.matmul_id_mix(wd, synth.Q4_K, xd, idd, torch.from_numpy(one).cuda(), path=path).cpu().numpy()
+    y1 = kq.matmul_id(wd, synth.Q4_K, xd.reshape(t * top_k, k),
+                      idd.reshape(-1, 1).contiguous(), path=path).cpu().numpy()[:, 0].reshape(t, top_k, n)
+    assert np.array_equal(y.view(np.uint32), y1[:, 2].copy().view(np.uint32))
+    z = kq.matmul_id_mix(wd, synth.Q4_K, xd, idd, torch.zeros(t, top_k).cuda(), path=path).cpu().numpy()
+    assert np.all(z == 0)
+    assert kq.device_status() == 0
+    bad = ids.copy()
+    bad[4, 1] = e
+    bad[7, 0] = -3
+    scores = r.uniform(0, 1, (t, top_k)).astype(np.float32)
+    y = kq.matmul_id_mix(wd, synth.Q4_K, xd, torch.from_numpy(bad).cuda(), torch.from_numpy(scores).cuda(),
+                         path=path).cpu().numpy()
+    assert np.all(np.isnan(y[[4, 7]]))
+    good = [i for i in range(t) if i not in (4, 7)]
+    ref = oracle.mix_id(synth.Q4_K, w, k, xs, bad, scores)
+    pref = _pair_refs(synth.Q4_K, w, k, xs[good], ids[good])
+    ok, worst = _mix_err_ok(y[good], ref[good], pref, scores[good], GEMV_TOL if path == 2 else FP32_PATH_TOL)
+    assert ok, worst
+    assert kq.device_status() == -9
+    assert kq.device_status() == 0
+
+
+@pytest.mark.parametrize("xdt", ["bf16", "f32"])
+def test_moe_ffn_chain_reuses_the_grouping(kq, xdt):
+    """GLU over the gate/up stacks, then the down projection with the mix on
+    the GLU's slotted output, the second call reusing the first call's
+    grouping from the shared workspace: the same bits as grouping again, and
+    the oracle's mix of the GPU's GLU output within the path's bound."""
+    import torch
+
+    t, top_k, e, hdim, fdim = 12, 4, 16, 512, 768
+    r = rng(1234 + len(xdt))
+    wg = synth.gen_weights(synth.Q4_K, e * fdim, hdim, r).reshape(e, fdim, -1)
+    wu = synth.gen_weights(synth.Q4_K, e * fdim, hdim, r).reshape(e, fdim, -1)
+    wdn = synth.gen_weights(synth.Q4_K, e * hdim, fdim, r).reshape(e, hdim, -1)
+    x = synth.gen_x(t, hdim, xdt, r)
+    ids = synth.gen_ids(t, top_k, e, r)
+    scores = r.uniform(0, 1, (t, top_k)).astype(np.float32)
+    idd, sd = torch.from_numpy(ids).cuda(), torch.from_numpy(scores).cuda()
+    ws = torch.empty(kq.matmul_id_mix_workspace_bytes(t, top_k, e, hdim), dtype=torch.uint8, device="cuda")
+    h = kq.matmul_id_glu(to_device_w(wg), to_device_w(wu), synth.Q4_K, to_device_x(x, xdt), idd,
+                         workspace=ws)
+    y = kq.matmul_id_mix(to_device_w(wdn), synth.Q4_K, h, idd, sd, workspace=ws, reuse_grouping=True,
+                         path=2).cpu().numpy()
+    y_fresh = kq.matmul_id_mix(to_device_w(wdn), synth.Q4_K, h, idd, sd, path=2).cpu().numpy()
+    assert np.array_equal(y.view(np.uint32), y_fresh.view(np.uint32))
+    hn = h.cpu().numpy().astype(np.float64)
+    ref = oracle.mix_id(synth.Q4_K, wdn, fdim, hn, ids, scores)
+    ok, worst = _mix_err_ok(y, ref, _pair_refs(synth.Q4_K, wdn, fdim, hn, ids), scores, GEMV_TOL)
+    assert ok, worst
+    # and the whole block against the oracle's chain
+    full = oracle.mix_id(synth.Q4_K, wdn, fdim, oracle.glu_id(synth.Q4_K, wg, wu, hdim, x, ids, "silu"),
+                         ids, scores)
+    assert row_rel_err(y, full) <= 4 * GEMV_TOL
+    assert kq.device_status() == 0
+
+
 def _bf16_weight_reference_id(w, k, x, ids):
     """y[t, s] = x[t] @ bf16(decode_f32(w[ids[t, s]]))^T in fp64 (NaN rows for
     ids outside [0, E)): the tensor-core expert product up to fp32 accumulation."""
