@@ -25,7 +25,10 @@ FLAG_INDEPENDENT = 0x200
 
 _DT = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}
 
-LIB_PATH = _build.LIB
+# KQ_DEBUG_LIBRARY=1 in the environment loads the KQ_DEBUG build instead
+# (device bounds checks, short bounded waits; include/kq_debug.h).
+DEBUG_LIBRARY = os.environ.get("KQ_DEBUG_LIBRARY", "") == "1"
+LIB_PATH = _build.LIB_DEBUG if DEBUG_LIBRARY else _build.LIB
 
 
 class KQError(RuntimeError):
@@ -74,6 +77,11 @@ def lib():
         L.kq_matmul_id_mix_workspace_bytes.restype = sz
         L.kq_matmul_id_mix.argtypes = [i32, vp, i64, i64, i64, i64, vp, i32, i64, vp, vp, i64, vp, i32,
                                        vp, sz, i32, vp]
+        if DEBUG_LIBRARY:
+            L.kq_debug_wait_timeout.argtypes = [i32, vp]
+            L.kq_debug_wait_timeout.restype = i32
+            L.kq_debug_spin_limit.argtypes = []
+            L.kq_debug_spin_limit.restype = i32
         L.kq_device_status.argtypes = [vp]
         L.kq_status_string.argtypes = [i32]
         L.kq_status_string.restype = ctypes.c_char_p
@@ -362,3 +370,12 @@ def validate(w: torch.Tensor, codec, k: int) -> int:
 def device_status() -> int:
     """Synchronize and return (and clear) the device error word as a status code."""
     return int(lib().kq_device_status(_stream()))
+
+
+def debug_wait_timeout(mode: int = 0) -> None:
+    """KQ_DEBUG build only: launch one warp whose bounded wait runs out (mode 0
+    the suspending wait loop, 1 the test-and-sleep loop); the next
+    device_status() returns -10 (KQ_ERR_DEVICE_TIMEOUT)."""
+    if not DEBUG_LIBRARY:
+        raise RuntimeError("debug_wait_timeout needs the KQ_DEBUG build (KQ_DEBUG_LIBRARY=1)")
+    _check(lib().kq_debug_wait_timeout(int(mode), _stream()), "kq_debug_wait_timeout")

@@ -132,6 +132,9 @@ struct IdWorkspace {
     size_t counts, offsets, perm, tiles, n_tiles, total;
 };
 static size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
+// Entries of the tensor-core tile list: tiles of at least 16 pairs, one
+// ragged tile per expert at most.
+static int64_t id_max_tiles(int64_t pairs, int64_t n_experts) { return pairs / 16 + n_experts + 1; }
 // The routing-mix call adds one section after the grouping: the fp32
 // per-pair products [pairs, n].
 static bool mix_workspace_bytes(const struct IdWorkspace &l, int64_t pairs, int64_t n, size_t *total) {
@@ -148,7 +151,7 @@ static bool id_workspace_layout(int64_t n_tokens, int64_t top_k, int64_t n_exper
     l->counts = off;  off += up256(4 * (size_t)n_experts);
     l->offsets = off; off += up256(4 * (size_t)(n_experts + 1));
     l->perm = off;    off += up256(4 * (size_t)pairs);
-    l->tiles = off;   off += up256(8 * (size_t)(pairs / 16 + n_experts + 1));
+    l->tiles = off;   off += up256(8 * (size_t)id_max_tiles(pairs, n_experts));
     l->n_tiles = off; off += 256;
     l->total = off;
     return true;
@@ -331,7 +334,7 @@ int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64
     if (path == KQ_PATH_GEMM) {
         const int bn = gemm_id_bn(n_tokens, top_k, n_experts);
         e = launch_moe_tiles(a.offsets, n_experts, bn, const_cast<int32_t *>(a.tiles),
-                             const_cast<int32_t *>(a.n_tiles), s);
+                             const_cast<int32_t *>(a.n_tiles), id_max_tiles(pairs, n_experts), s);
         if (e != cudaSuccess) return KQ_ERR_CUDA;
         return to_status(launch_gemm_id(a, bn, s));
     }
@@ -395,7 +398,7 @@ int kq_matmul_id_mix(int type, const void *w, int64_t n_experts, int64_t n, int6
     if (path == KQ_PATH_GEMM) {
         const int bn = gemm_id_bn(n_tokens, top_k, n_experts);
         e = launch_moe_tiles(a.offsets, n_experts, bn, const_cast<int32_t *>(a.tiles),
-                             const_cast<int32_t *>(a.n_tiles), s);
+                             const_cast<int32_t *>(a.n_tiles), id_max_tiles(pairs, n_experts), s);
         if (e == cudaSuccess) e = launch_gemm_id(a, bn, s);
     } else if (path == KQ_PATH_GEMV) {
         e = launch_moe_gemv(a, s);
@@ -484,6 +487,7 @@ int kq_device_status(void *stream) {
         cudaStreamSynchronize(s) != cudaSuccess)
         return KQ_ERR_CUDA;
     if (word & ERR_TIMEOUT) return KQ_ERR_DEVICE_TIMEOUT;
+    if (word & ERR_BOUNDS) return KQ_ERR_DEVICE_BOUNDS;
     if (word & ERR_BAD_ID) return KQ_ERR_DEVICE;
     return KQ_OK;
 }
@@ -502,6 +506,7 @@ const char *kq_status_string(int status) {
     case KQ_ERR_DEVICE: return "device reported an out-of-range expert or row id";
     case KQ_ERR_DEVICE_TIMEOUT: return "a bounded device wait timed out";
     case KQ_ERR_UNSUPPORTED: return "unsupported device or path for these arguments";
+    case KQ_ERR_DEVICE_BOUNDS: return "a device bounds check (debug build) found an index out of range";
     default: return "unknown status";
     }
 }

@@ -19,7 +19,8 @@ template <> struct Geom<KQ_Q5_K>     { static constexpr int QK = 256; static con
 template <> struct Geom<KQ_Q6_K>     { static constexpr int QK = 256; static constexpr int BB = 210; };
 template <> struct Geom<KQ_TQ1_G128> { static constexpr int QK = 128; static constexpr int BB = 28; };
 
-// Sticky per-device error word (bit 0: bad expert id, bit 1: wait timeout).
+// Sticky per-device error word (bit 0: bad expert id, bit 1: wait timeout,
+// bit 2: a KQ_DEBUG build's bounds check failed).
 // It lives in kq_api.cu; kernels receive its device address as a parameter
 // (error_word() on the host), since each translation unit is compiled
 // without relocatable device code.
@@ -28,6 +29,31 @@ unsigned int *error_word();
 int sm_count();
 constexpr unsigned ERR_BAD_ID = 1u;
 constexpr unsigned ERR_TIMEOUT = 2u;
+constexpr unsigned ERR_BOUNDS = 4u;
+
+// Device bounds checks of the KQ_DEBUG build.  KQ_DCHECK(cond, err) checks
+// an index that comes from data (a grouping entry, a tile list, a shared-
+// memory layout) before it is used: when cond is false it sets ERR_BOUNDS in
+// the error word and yields false, and the caller skips or clamps the
+// access instead of touching memory outside its buffer.  In the release
+// build it is the constant true and cond is not evaluated.
+#ifdef KQ_DEBUG
+constexpr bool kDebug = true;
+#else
+constexpr bool kDebug = false;
+#endif
+__device__ __forceinline__ bool dcheck_record(bool ok, unsigned int *err) {
+    if (!ok) atomicOr(err, ERR_BOUNDS);
+    return ok;
+}
+#define KQ_DCHECK(cond, err) (!::kq::kDebug || ::kq::dcheck_record((cond), (err)))
+
+// Bytes of dynamic shared memory this launch was given.
+__device__ __forceinline__ uint32_t dynamic_smem_size() {
+    uint32_t v;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(v));
+    return v;
+}
 
 __device__ __forceinline__ float half_bits_to_float(uint32_t bits16) {
     return __half2float(__ushort_as_half((unsigned short)(bits16 & 0xFFFFu)));

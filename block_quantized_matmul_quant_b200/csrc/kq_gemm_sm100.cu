@@ -88,6 +88,7 @@ struct GemmParams {
     const int2 *id_tiles;     // (expert, first position in perm) per token tile
     const int32_t *id_n_tiles;
     int top_k;
+    int n_pairs, n_experts;   // entries of perm; experts of the stack
 };
 
 // One output tile: weight rows n0.. of expert e times BN activation rows.
@@ -101,11 +102,16 @@ template <bool ID>
 __device__ __forceinline__ Tile tile_at(const GemmParams &p, int u) {
     Tile t;
     if constexpr (ID) {
-        const int2 tt = p.id_tiles[u / p.n_tiles];
+        int2 tt = p.id_tiles[u / p.n_tiles];
+        // KQ_DEBUG: a tile outside the grouping becomes an empty tile of
+        // expert 0 at position 0 (its loads stay in bounds, nothing is stored)
+        const bool ok = KQ_DCHECK(tt.x >= 0 && tt.x < p.n_experts && tt.y >= 0 && tt.y < p.n_pairs &&
+                                      p.offsets[tt.x + 1] <= p.n_pairs, p.err);
+        if (!ok) tt = make_int2(0, 0);
         t.n0 = (u % p.n_tiles) * BM;
         t.e = tt.x;
         t.m0 = tt.y;
-        t.rows = min(p.bn, p.offsets[tt.x + 1] - tt.y);
+        t.rows = ok ? min(p.bn, p.offsets[tt.x + 1] - tt.y) : 0;
     } else {
         t.n0 = (u / p.m_tiles) * BM;
         t.e = 0;
@@ -307,6 +313,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t *acc_empty = acc_full + 2;           // [2] epilogue -> MMA
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
     int *s_rows = reinterpret_cast<int *>(bars + 128);  // expert-indexed: activation row per tile row
+    if ((uint32_t)(reinterpret_cast<uint8_t *>(s_rows + MAX_BN) - smem_raw) > dynamic_smem_size()) {
+        if (threadIdx.x == 0) atomicOr(p.err, ERR_BOUNDS);   // the host planned another layout: no work
+        return;
+    }
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int SPS = 4 / CPS;           // stages per raw super-block (256 K)
@@ -380,8 +390,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const Tile t = tile_at<ID>(p, u);
             if constexpr (ID) {
                 __syncwarp();  // lane 0 has issued every load of the previous tile
-                for (int i = lane; i < p.bn; i += 32)
-                    s_rows[i] = p.perm[t.m0 + (i < t.rows ? i : 0)] / p.top_k;
+                for (int i = lane; i < p.bn; i += 32) {
+                    int pr = p.perm[t.m0 + (i < t.rows ? i : 0)];
+                    if (!KQ_DCHECK(pr >= 0 && pr < p.n_pairs, p.err)) pr = 0;
+                    s_rows[i] = pr / p.top_k;
+                }
                 __syncwarp();
             }
             if (lane == 0) {
@@ -495,7 +508,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         if (c0 + j < t.rows) {
                             // output row: the activation row, or the (token, slot) pair
                             const int64_t m = ID ? (int64_t)__ldg(p.perm + t.m0 + c0 + j) : (int64_t)(t.m0 + c0 + j);
-                            store_out(y + m * p.n + n, __uint_as_float(r[j]));
+                            if (!ID || KQ_DCHECK(m >= 0 && m < p.n_pairs, p.err))
+                                store_out(y + m * p.n + n, __uint_as_float(r[j]));
                         }
                     }
                 }
@@ -798,6 +812,8 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     p.id_tiles = reinterpret_cast<const int2 *>(a.tiles);
     p.id_n_tiles = a.n_tiles;
     p.top_k = a.x_div();
+    p.n_pairs = (int)(a.n_tokens * a.top_k);
+    p.n_experts = (int)a.n_experts;
     CUtensorMap tx, tw;
     if (!encode_x_map(&tx, a.x, a.x_rows(), a.k, 1) ||
         !encode_w_map(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride))

@@ -206,8 +206,8 @@ __global__ void __launch_bounds__(T1_THREADS, 1) gemv_tq1_split_kernel(const Tq1
 
     const uint32_t base = smem_addr(smem);
     const T1Layout lay = t1_layout(base, nb, S, p.slot_bytes);
-    if (lay.end - base > (uint32_t)p.smem_bytes) {   // the host planned another layout: no work
-        if (tid == 0) atomicOr(p.err, ERR_TIMEOUT);
+    if (lay.end - base > dynamic_smem_size()) {   // the host planned another layout: no work
+        if (tid == 0) atomicOr(p.err, ERR_BOUNDS);
         return;
     }
     // Pointers into shared memory are formed as smem + offset, so that the

@@ -47,9 +47,10 @@ cudaError_t launch_moe_mix(const float *pair_out, const int32_t *ids, const floa
                            int64_t n_tokens, int64_t top_k, int64_t n_experts, int64_t n, void *y,
                            int y_dtype, cudaStream_t s);
 // Token tiles of at most bn pairs per expert segment, (expert, first
-// position in perm) each, and their number -- from the grouping's offsets.
+// position in perm) each, and their number -- from the grouping's offsets;
+// the tile list holds max_tiles entries.
 cudaError_t launch_moe_tiles(const int32_t *offsets, int64_t n_experts, int bn, int32_t *tiles,
-                             int32_t *n_tiles, cudaStream_t s);
+                             int32_t *n_tiles, int64_t max_tiles, cudaStream_t s);
 
 // Bandwidth kernels (kq_gemv.cu).  Return cudaErrorNotSupported when the
 // shape is outside what the kernel serves.

@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(GROUP_THREADS) moe_group_kernel(
             const int p = base + lane;
             const bool hit = p < n_pairs && ids[p] == e;
             const unsigned mask = __ballot_sync(0xffffffffu, hit);
-            if (hit) perm[pos + __popc(mask & lt)] = p;
+            if (hit && KQ_DCHECK(pos + __popc(mask & lt) < n_pairs, err)) perm[pos + __popc(mask & lt)] = p;
             pos += __popc(mask);
         }
     }
@@ -114,7 +114,8 @@ constexpr int TILE_THREADS = 256;
 __global__ void __launch_bounds__(TILE_THREADS) moe_tiles_kernel(const int32_t *__restrict__ offsets,
                                                                  int n_experts, int bn,
                                                                  int2 *__restrict__ tiles,
-                                                                 int32_t *__restrict__ n_tiles) {
+                                                                 int32_t *__restrict__ n_tiles,
+                                                                 int max_tiles, unsigned int *err) {
     extern __shared__ int s_first[];  // n_experts: first tile index of each expert
     const int lane = threadIdx.x & 31;
     if (threadIdx.x < 32) {
@@ -131,18 +132,19 @@ __global__ void __launch_bounds__(TILE_THREADS) moe_tiles_kernel(const int32_t *
             if (e < n_experts) s_first[e] = carry + incl - c;
             carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) *n_tiles = carry;
+        if (lane == 0) *n_tiles = KQ_DCHECK(carry <= max_tiles, err) ? carry : max_tiles;
     }
     __syncthreads();
     for (int e = threadIdx.x; e < n_experts; e += blockDim.x) {
         const int p0 = offsets[e], p1 = offsets[e + 1];
         int i = s_first[e];
-        for (int q = p0; q < p1; q += bn) tiles[i++] = make_int2(e, q);
+        for (int q = p0; q < p1; q += bn, ++i)
+            if (KQ_DCHECK(i < max_tiles, err)) tiles[i] = make_int2(e, q);
     }
 }
 
 cudaError_t launch_moe_tiles(const int32_t *offsets, int64_t n_experts, int bn, int32_t *tiles,
-                             int32_t *n_tiles, cudaStream_t s) {
+                             int32_t *n_tiles, int64_t max_tiles, cudaStream_t s) {
     const size_t smem = sizeof(int) * (size_t)n_experts;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(moe_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -150,7 +152,8 @@ cudaError_t launch_moe_tiles(const int32_t *offsets, int64_t n_experts, int bn, 
         if (e != cudaSuccess) return e;
     }
     moe_tiles_kernel<<<1, TILE_THREADS, smem, s>>>(offsets, (int)n_experts, bn,
-                                                   reinterpret_cast<int2 *>(tiles), n_tiles);
+                                                   reinterpret_cast<int2 *>(tiles), n_tiles,
+                                                   (int)max_tiles, error_word());
     return cudaGetLastError();
 }
 
@@ -161,7 +164,8 @@ template <int TYPE, typename XT, typename YT>
 __global__ void __launch_bounds__(256) simple_id_kernel(
     const uint8_t *__restrict__ w, int64_t n, int64_t k, int64_t expert_stride,
     const XT *__restrict__ x, int top_k, const int32_t *__restrict__ counts,
-    const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm, YT *__restrict__ y) {
+    const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm, YT *__restrict__ y, int n_pairs,
+    unsigned int *err) {
     using G = Geom<TYPE>;
     using U = Unit<TYPE>;
     constexpr int TB = 4;
@@ -173,12 +177,16 @@ __global__ void __launch_bounds__(256) simple_id_kernel(
     if (row >= n) return;
     const int64_t nb = k / G::QK;
     const uint8_t *wr = w + e * expert_stride + row * nb * G::BB;
+    if (!KQ_DCHECK(offsets[e] >= 0 && offsets[e] + cnt <= n_pairs, err)) return;
     const int32_t *plist = perm + offsets[e];
     const int64_t units = nb * U::PER_BLOCK;
     for (int c0 = 0; c0 < cnt; c0 += TB) {
         int pr[TB];
         #pragma unroll
-        for (int t = 0; t < TB; ++t) pr[t] = (c0 + t < cnt) ? plist[c0 + t] : -1;
+        for (int t = 0; t < TB; ++t) {
+            pr[t] = (c0 + t < cnt) ? plist[c0 + t] : -1;
+            if (pr[t] >= 0 && !KQ_DCHECK(pr[t] < n_pairs, err)) pr[t] = -1;
+        }
         float acc[TB] = {0.f, 0.f, 0.f, 0.f};
         for (int64_t i = lane; i < units; i += 32) {
             const int64_t bi = i / U::PER_BLOCK;
@@ -218,7 +226,8 @@ template <int TYPE, typename XT, typename YT>
 __global__ void __launch_bounds__(256) simple_glu_kernel(
     const uint8_t *__restrict__ wg, const uint8_t *__restrict__ wu, int64_t n, int64_t k,
     int64_t expert_stride, const XT *__restrict__ x, int top_k, const int32_t *__restrict__ counts,
-    const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm, YT *__restrict__ y, int act) {
+    const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm, YT *__restrict__ y, int act,
+    int n_pairs, unsigned int *err) {
     using G = Geom<TYPE>;
     using U = Unit<TYPE>;
     constexpr int TB = 4;
@@ -230,12 +239,16 @@ __global__ void __launch_bounds__(256) simple_glu_kernel(
     if (row >= n) return;
     const int64_t nb = k / G::QK;
     const int64_t off = e * expert_stride + row * nb * G::BB;
+    if (!KQ_DCHECK(offsets[e] >= 0 && offsets[e] + cnt <= n_pairs, err)) return;
     const int32_t *plist = perm + offsets[e];
     const int64_t units = nb * U::PER_BLOCK;
     for (int c0 = 0; c0 < cnt; c0 += TB) {
         int pr[TB];
         #pragma unroll
-        for (int t = 0; t < TB; ++t) pr[t] = (c0 + t < cnt) ? plist[c0 + t] : -1;
+        for (int t = 0; t < TB; ++t) {
+            pr[t] = (c0 + t < cnt) ? plist[c0 + t] : -1;
+            if (pr[t] >= 0 && !KQ_DCHECK(pr[t] < n_pairs, err)) pr[t] = -1;
+        }
         float ag[TB] = {0.f, 0.f, 0.f, 0.f}, au[TB] = {0.f, 0.f, 0.f, 0.f};
         for (int64_t i = lane; i < units; i += 32) {
             const int64_t bi = i / U::PER_BLOCK;
@@ -344,7 +357,8 @@ static cudaError_t simple_glu_t(const IdArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)((a.n + 7) / 8), (unsigned)a.n_experts);
     simple_glu_kernel<TYPE, XT, YT><<<grid, 256, 0, s>>>(
         static_cast<const uint8_t *>(a.w), static_cast<const uint8_t *>(a.w2), a.n, a.k, a.expert_stride,
-        static_cast<const XT *>(a.x), a.x_div(), a.counts, a.offsets, a.perm, static_cast<YT *>(a.y), a.act);
+        static_cast<const XT *>(a.x), a.x_div(), a.counts, a.offsets, a.perm, static_cast<YT *>(a.y), a.act,
+        (int)(a.n_tokens * a.top_k), error_word());
     return cudaGetLastError();
 }
 
@@ -376,7 +390,7 @@ static cudaError_t simple_id_t(const IdArgs &a, cudaStream_t s) {
     simple_id_kernel<TYPE, XT, YT><<<grid, 256, 0, s>>>(
         static_cast<const uint8_t *>(a.w), a.n, a.k, a.expert_stride,
         static_cast<const XT *>(a.x), a.x_div(), a.counts, a.offsets, a.perm,
-        static_cast<YT *>(a.y));
+        static_cast<YT *>(a.y), (int)(a.n_tokens * a.top_k), error_word());
     return cudaGetLastError();
 }
 

@@ -62,6 +62,7 @@ struct MoeGemvParams {
     const void *x;
     void *y;
     const int32_t *counts, *offsets, *perm;
+    int n_pairs;                    // entries of perm; pair ids are below it
     int wg, groups;            // warps per row group, row groups
     int tile_rows, tiles;      // output rows per tile, tiles per expert
     int slots, slot_bytes, part_off;
@@ -129,6 +130,17 @@ __global__ void __launch_bounds__(MG_THREADS, 1) moe_gemv_kernel(const MoeGemvPa
     float2 *xs = reinterpret_cast<float2 *>(smem + lay.xs);        // [TB][nsub]: (scale, exact sum)
     const int64_t row_bytes = (int64_t)p.nb * 144;
     const int E = p.n_experts;
+    if ((uint32_t)lay.total > dynamic_smem_size()) {   // the host planned another layout: no work
+        if (tid == 0) atomicOr(p.err, ERR_BOUNDS);
+        return;
+    }
+    // A pair id of the grouping at position idx of perm (checked in KQ_DEBUG
+    // builds: a bad position or id reads pair 0's activations instead).
+    auto pair_at = [&](int idx) -> int {
+        int v = 0;
+        if (KQ_DCHECK(idx >= 0 && idx < p.n_pairs, p.err)) v = p.perm[idx];
+        return KQ_DCHECK(v >= 0 && v < p.n_pairs, p.err) ? v : 0;
+    };
 
     // ---- items: expert e has ceil(count / 4) rounds of p.tiles tiles
     if (warp == 0) {
@@ -199,7 +211,13 @@ __global__ void __launch_bounds__(MG_THREADS, 1) moe_gemv_kernel(const MoeGemvPa
                 f_e = e_fin;
                 f_round = round;
                 nt = min(MG_TB, p.counts[e_fin] - MG_TB * round);
-                my_pair = lane < nt ? p.perm[p.offsets[e_fin] + MG_TB * round + lane] : 0;
+                // a pair id that fails a KQ_DEBUG check becomes -1: no store
+                const int idx = p.offsets[e_fin] + MG_TB * round + lane;
+                my_pair = -1;
+                if (lane < nt && KQ_DCHECK(idx >= 0 && idx < p.n_pairs, p.err)) {
+                    my_pair = p.perm[idx];
+                    if (!KQ_DCHECK(my_pair >= 0 && my_pair < p.n_pairs, p.err)) my_pair = -1;
+                }
             }
             if (!__all_sync(0xffffffffu, mbar_wait_poll(&empty[s], (uint32_t)((i - i0) / S) & 1u, p.err))) break;
             const float *part = reinterpret_cast<const float *>(smem + lay.slots + s * p.slot_bytes + p.part_off);
@@ -212,7 +230,7 @@ __global__ void __launch_bounds__(MG_THREADS, 1) moe_gemv_kernel(const MoeGemvPa
                     const int g = o / MG_TB, t = o - g * MG_TB;
                     const int pr = __shfl_sync(0xffffffffu, my_pair, t);
                     const int row = tile * p.tile_rows + g;
-                    if (o < outs && t < nt && row < p.n) {
+                    if (o < outs && t < nt && row < p.n && pr >= 0) {
                         float gs = 0.f, us = 0.f;
                         for (int w = 0; w < p.wg; ++w) {
                             gs += part[(g * p.wg + w) * MG_PART + t];
@@ -229,7 +247,7 @@ __global__ void __launch_bounds__(MG_THREADS, 1) moe_gemv_kernel(const MoeGemvPa
                     const int g = o / MG_PART, v = o - g * MG_PART, r = v / MG_TB, t = v - r * MG_TB;
                     const int pr = __shfl_sync(0xffffffffu, my_pair, t & (MG_TB - 1));
                     const int row = tile * p.tile_rows + g * MG_R + r;
-                    if (o < outs && t < nt && row < p.n) {
+                    if (o < outs && t < nt && row < p.n && pr >= 0) {
                         float acc = 0.f;
                         for (int w = 0; w < p.wg; ++w) acc += part[(g * p.wg + w) * MG_PART + v];
                         store_out(y + (int64_t)pr * p.n + row, acc);
@@ -280,7 +298,7 @@ __global__ void __launch_bounds__(MG_THREADS, 1) moe_gemv_kernel(const MoeGemvPa
             ++stage_no;
             for (int it = tid; it < nt * p.nsub; it += MG_CWARPS * 32) {
                 const int t = it / p.nsub, sjj = it - t * p.nsub;
-                const int tok = p.perm[pbase + t] / p.top_k;
+                const int tok = pair_at(pbase + t) / p.top_k;
                 const XT *src = x + (int64_t)tok * p.k + 32 * sjj;
                 float v[32];
                 if (sizeof(XT) == 2) {
@@ -379,7 +397,7 @@ __global__ void __launch_bounds__(MG_THREADS, 1) moe_gemv_kernel(const MoeGemvPa
                     #pragma unroll
                     for (int t = 0; t < MG_TB; ++t) {
                         if (t < nt) {
-                            const int tok = p.perm[p.offsets[e_cur] + MG_TB * round + t] / p.top_k;
+                            const int tok = pair_at(p.offsets[e_cur] + MG_TB * round + t) / p.top_k;
                             const XT *xt = x + (int64_t)tok * p.k + 32 * j;
                             float v = 0.f;
                             for (int l = 0; l < 32; ++l) {
@@ -492,6 +510,7 @@ cudaError_t launch_moe_gemv(const IdArgs &a, cudaStream_t s) {
     p.counts = a.counts;
     p.offsets = a.offsets;
     p.perm = a.perm;
+    p.n_pairs = (int)(a.n_tokens * a.top_k);
     p.err = error_word();
     if (a.x_dtype == KQ_F32)
         return a.y_dtype == KQ_F32 ? launch_mg<float, float>(p, s) : launch_mg<float, __nv_bfloat16>(p, s);

@@ -73,6 +73,7 @@ extern "C" {
 #define KQ_ERR_DEVICE          -9   /* device-side error word was set (bad expert/row id) */
 #define KQ_ERR_DEVICE_TIMEOUT  -10  /* a bounded device-side wait gave up              */
 #define KQ_ERR_UNSUPPORTED     -11  /* current device is not sm_100 / path unavailable */
+#define KQ_ERR_DEVICE_BOUNDS   -12  /* a KQ_DEBUG build's device bounds check failed  */
 
 /* ---- matmul paths (kq_matmul_ex / kq_matmul_id_ex) ---- */
 #define KQ_PATH_AUTO     0  /* dispatch by shape (the default of kq_matmul)          */
@@ -326,7 +327,11 @@ KQ_API int kq_validate(int type, const void *w, int64_t rows, int64_t k,
 /*
  * kq_device_status -- SYNCHRONIZES `stream`, then returns and clears the
  * current device's sticky error word: KQ_OK, KQ_ERR_DEVICE (an expert id was
- * out of range in some call since the last check) or KQ_ERR_DEVICE_TIMEOUT.
+ * out of range in some call since the last check), KQ_ERR_DEVICE_TIMEOUT (a
+ * kernel gave up a bounded wait and left its outputs incomplete) or, from
+ * the KQ_DEBUG build only, KQ_ERR_DEVICE_BOUNDS (a device bounds check found
+ * an index out of range and skipped the access).  When more than one is set
+ * it reports the timeout before the bounds check and that before the ids.
  */
 KQ_API int kq_device_status(void *stream);
 

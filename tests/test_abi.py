@@ -157,3 +157,22 @@ def test_mix_workspace_and_argument_errors(L):
     assert call(args(ydt=2)) == -4                           # f16 output
     assert call(args(tk=4)) == -1                            # top_k > n_experts
     assert call(args(k=100)) == -3                           # K % 256
+
+
+def test_debug_build_exports_its_entry_points(L):
+    """libkq_debug.so exports kq.h's calls and kq_debug.h's; the release
+    library has no debug entry points."""
+    from block_quantized_matmul_quant_b200 import _build
+
+    D = ctypes.CDLL(_build.LIB_DEBUG)
+    src = open(os.path.join(ROOT, "include", "kq_debug.h")).read()
+    debug_names = re.findall(r"KQ_API\s+[\w\s\*]+?\b(kq_\w+)\s*\(", src)
+    assert set(debug_names) == {"kq_debug_wait_timeout", "kq_debug_spin_limit"}
+    for name in declared_functions() + debug_names:
+        assert hasattr(D, name), name
+    for name in debug_names:
+        assert not hasattr(L, name), name
+    D.kq_debug_spin_limit.restype = ctypes.c_int
+    assert D.kq_debug_spin_limit() == _build.DEBUG_SPIN_LIMIT
+    D.kq_debug_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_void_p]
+    assert D.kq_debug_wait_timeout(5, None) == -1     # unknown mode, before any device call
