@@ -263,9 +263,9 @@ class GemvStep:
 class PoolStep:
     """A workload's calls over a pool of weight copies larger than 4x L2."""
 
-    def __init__(self, torch, kq, wl, l2_bytes):
+    def __init__(self, torch, kq, wl, l2_bytes, glu=False):
         w, x, ids = synth.make_inputs(wl)
-        self.wl, self.kq = wl, kq
+        self.wl, self.kq, self.glu = wl, kq, glu
         self.wbytes = w.nbytes
         self.pool = max(4, -(-4 * l2_bytes // w.nbytes))
         base = torch.from_numpy(w).cuda()
@@ -285,7 +285,11 @@ class PoolStep:
 
     def run(self):
         for i in range(self.pool):
-            if self.wl.kind == "moe":
+            if self.wl.kind == "moe" and self.glu:
+                # fused gate and up projections: two stacks of the pool per call
+                self.kq.matmul_id_glu(self.ws[i], self.ws[(i + 1) % self.pool], self.wl.codec, self.x,
+                                      self.ids, out=self.y, workspace=self.scratch)
+            elif self.wl.kind == "moe":
                 self.kq.matmul_id(self.ws[i], self.wl.codec, self.x, self.ids, out=self.y,
                                   workspace=self.scratch)
             elif self.wl.kind == "gemv":
@@ -307,7 +311,26 @@ def secondary_metrics(torch, kq, l2, peaks):
         out[name] = secondary_entry(wl, us, st.wbytes, getattr(st, "hit_experts", 0), peaks)
         del st
         torch.cuda.empty_cache()
+    # the fused GLU (gate and up in one call) on the MoE workload's routing
+    name = "moe_q4_k_e64_1408x2048_t32_top6"
+    wl = synth.WORKLOADS[name]
+    st = PoolStep(torch, kq, wl, l2, glu=True)
+    ms = time_graph(torch, st.run, 5, 3, None)
+    us = ms * 1e3 / (5 * st.pool)
+    out[name + "_glu"] = glu_entry(wl, us, st.wbytes, st.hit_experts, out[name]["gate_up_pair_us"], peaks)
+    del st
+    torch.cuda.empty_cache()
     return out
+
+
+def glu_entry(wl, us, wbytes, hit_experts, gate_up_pair_us, peaks):
+    """The fused GLU's figures: both stacks' hit experts stream once per call."""
+    per_expert = wbytes // wl.n_experts
+    moved = 2 * hit_experts * per_expert + wl.m * wl.k * 2 + wl.m * wl.top_k * wl.n * 4
+    return {"us_per_call": round(us, 2), "vs_gate_up_pair_us": gate_up_pair_us,
+            "GB/s": round(moved / (us * 1e-6) / 1e9, 1),
+            "frac_hbm": round(moved / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+            "kernel": "moe_group + fused GLU (kq_matmul_id_glu)"}
 
 
 def secondary_entry(wl, us, wbytes, hit_experts, peaks):
@@ -620,6 +643,59 @@ def run_profile(args):
     print(json.dumps({"profiled": wl.name, "calls": args.profile_calls}))
 
 
+def run_sweep(args):
+    """Dispatch evidence: per-call time of the bandwidth kernel against the
+    tensor-core kernel over the activation-row count (dense Q4_K product,
+    11008 x 4096) and the token count (MoE, 64 experts of 1408 x 2048,
+    top-6), bf16 activations, each call on its own weight copy of a pool
+    larger than 4x L2.  One JSON line per point."""
+    import torch
+
+    import block_quantized_matmul_quant_b200 as kq
+
+    kq.lib()
+    l2 = l2_bytes(0)
+    dense = synth.Workload("sweep_dense", "gemm", synth.Q4_K, 11008, 4096, 1, "bf16", "f32")
+    w, _, _ = synth.make_inputs(dense)
+    wd = torch.from_numpy(w).cuda()
+    pool = [wd.clone() for _ in range(pool_size(w.nbytes, l2))]
+    r = np.random.Generator(np.random.PCG64(1))
+    for m in (1, 2, 4, 8, 9, 12, 16, 24, 32, 48, 64):
+        x = torch.from_numpy(synth.gen_x(m, dense.k, "bf16", r)).to(torch.bfloat16).cuda()
+        y = torch.empty((m, dense.n), device="cuda")
+        line = {"sweep": "dense_q4_k_11008x4096", "m": m, "pool": len(pool)}
+        for name, path in (("gemv", kq.PATH_GEMV), ("gemm", kq.PATH_GEMM)):
+            def fn():
+                for wi in pool:
+                    kq.matmul(wi, synth.Q4_K, x, out=y, path=path, const_weights=True)
+            line[name + "_us"] = round(time_graph(torch, fn, 5, 3, None) * 1e3 / (5 * len(pool)), 2)
+        print(json.dumps(line), flush=True)
+    del pool, wd
+    torch.cuda.empty_cache()
+    for t in (8, 16, 32, 64, 128, 256, 512):
+        wl = synth.Workload("sweep_moe", "moe", synth.Q4_K, 1408, 2048, t, "bf16", "f32", n_experts=64, top_k=6)
+        w, x, ids = synth.make_inputs(wl)
+        wd = torch.from_numpy(w).cuda()
+        pool = [wd.clone() for _ in range(pool_size(w.nbytes, l2))]
+        xd = torch.from_numpy(x).to(torch.bfloat16).cuda()
+        idd = torch.from_numpy(ids).cuda()
+        y = torch.empty((t, 6, 1408), device="cuda")
+        ws = torch.empty(kq.matmul_id_workspace_bytes(t, 6, 64), dtype=torch.uint8, device="cuda")
+        line = {"sweep": "moe_q4_k_e64_1408x2048_top6", "tokens": t, "pairs_per_expert": round(6 * t / 64, 2),
+                "pool": len(pool)}
+        for name, path in (("gemv", kq.PATH_GEMV), ("gemm", kq.PATH_GEMM)):
+            def fn():
+                for wi in pool:
+                    kq.matmul_id(wi, synth.Q4_K, xd, idd, out=y, workspace=ws, path=path)
+            line[name + "_us"] = round(time_graph(torch, fn, 5, 3, None) * 1e3 / (5 * len(pool)), 2)
+        print(json.dumps(line), flush=True)
+        del pool, wd
+        torch.cuda.empty_cache()
+    status = kq.device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status} after the sweep")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -635,10 +711,14 @@ def main():
                     help="GEMV call ordering in --profile (the headline step uses independent calls)")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the other workloads' numbers (prefill GEMM, MoE, TQ1, Q8_0)")
+    ap.add_argument("--sweep", default=None, choices=["dispatch"],
+                    help="print the dispatch sweep (bandwidth vs tensor-core kernel) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.profile:
+    if args.sweep:
+        run_sweep(args)
+    elif args.profile:
         run_profile(args)
     elif args.impl == "reference":
         run_reference(args)

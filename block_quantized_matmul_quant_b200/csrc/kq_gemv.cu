@@ -33,6 +33,7 @@
 //    row copies are issued before it, overlapping the previous kernel; an
 //    independent call never waits before its work and waits once at its end,
 //    so that it completes after the work before it.
+#include "kq_decode.cuh"
 #include "kq_ptx.cuh"
 #include "kq_launch.h"
 
@@ -138,7 +139,8 @@ __device__ __forceinline__ void load_x8v(const __nv_bfloat16 *p, float v[8]) {
 // adjacent lanes.  All loads of up to XIT rounds are issued before use.
 template <int C, int TB, typename XT, typename F>
 __device__ __forceinline__ void stage_activations(const GemvParams &p, const int *tok, int4 *xq,
-                                                  float *xsc, float *xsum, F &&after_first_loads) {
+                                                  float *xsc, float *xsum, int *nonfinite,
+                                                  F &&after_first_loads) {
     constexpr int XIT = 4;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nthr = blockDim.x;
     const int per_row = p.k / 8, nitems = TB * per_row;
@@ -163,16 +165,19 @@ __device__ __forceinline__ void stage_activations(const GemvParams &p, const int
             if (r0 + it >= nrounds || (r0 + it) * nthr + warp * 32 >= nitems) break;  // warp-uniform
             const int idx = (r0 + it) * nthr + (int)threadIdx.x;
             float amax = 0.f, sum = 0.f;
+            bool nf = false;   // an infinity or NaN: the call takes the exact path
             #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 amax = fmaxf(amax, fabsf(v[it][e]));
                 sum += v[it][e];
+                nf |= !(fabsf(v[it][e]) <= 3.402823466e38f);
             }
             #pragma unroll
             for (int o = 1; o < 4; o <<= 1) {
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                 sum += __shfl_xor_sync(0xffffffffu, sum, o);
             }
+            if (__any_sync(0xffffffffu, nf) && lane == 0) *nonfinite = 1;
             if (idx >= nitems) continue;
             int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;  // floor(log2 amax)
             e = max(e, -100);
@@ -232,7 +237,7 @@ template <> struct Vec<4> {
 template <int C, int TB, int R, bool XREG, typename XT, typename YT>
 __device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w, int row_begin,
                                           int row_end, const int *tok, const int64_t *yrow,
-                                          uint8_t *smem, int pass) {
+                                          uint8_t *smem, int *nonfinite, int pass) {
     int4 *xq = reinterpret_cast<int4 *>(smem);
     float *xsc = reinterpret_cast<float *>(smem + p.xq_bytes);
     float *xsum = reinterpret_cast<float *>(smem + p.xq_bytes + p.xs_bytes);
@@ -291,13 +296,58 @@ __device__ __forceinline__ bool gemv_pass(const GemvParams &p, const uint8_t *w,
     // behind them.  An independent call asks L2 for nothing more: its ring
     // keeps enough bytes in flight (an L2 prefetch of its rows, before or
     // after staging, measured slower).
-    stage_activations<C, TB, XT>(p, tok, xq, xsc, xsum, [&]() {
+    stage_activations<C, TB, XT>(p, tok, xq, xsc, xsum, nonfinite, [&]() {
         if (!copies_first && lane == 0) {
             fence_proxy_async_smem();  // generic reads of the slots in an earlier pass
             for (int i = 0; i < first; ++i) issue(i);
         }
     });
     __syncthreads();
+    // Non-finite activations (block-uniform): every weight is decoded to fp32
+    // and multiplied by the activation itself, so that infinities and NaNs
+    // combine with the weights' signs and zeros as IEEE arithmetic does (the
+    // 16-bit codes cannot hold them).  The ring is consumed as usual.
+    if (*nonfinite) {
+        const XT *x = static_cast<const XT *>(p.x);
+        YT *y = static_cast<YT *>(p.y);
+        for (int i = 0; i < my_rows; ++i) {
+            const int ii = base + i, slot = ii % p.slots;
+            const uint32_t par = (uint32_t)(ii / p.slots) & 1u;
+            if (!__all_sync(0xffffffffu, mbar_wait(&my_full[slot], par, p.err))) return false;
+            const uint8_t *rp = my_ring + slot * row_bytes;
+            float acc[TB];
+            #pragma unroll
+            for (int t = 0; t < TB; ++t) acc[t] = 0.f;
+            for (int u8 = lane; u8 < p.nb * Unit<KQ_Q4_K>::PER_BLOCK; u8 += 32) {   // weights 8 u8 ..
+                const int b = u8 / Unit<KQ_Q4_K>::PER_BLOCK;
+                float wv[8];
+                Unit<KQ_Q4_K>::decode(rp + b * 144, u8 - b * Unit<KQ_Q4_K>::PER_BLOCK, wv);
+                #pragma unroll
+                for (int t = 0; t < TB; ++t) {
+                    if (tok[t] < 0) continue;
+                    float xv[8];
+                    load_x8v(x + (int64_t)tok[t] * p.k + 8 * u8, xv);
+                    #pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[t] = fmaf(wv[j], xv[j], acc[t]);
+                }
+            }
+            #pragma unroll
+            for (int t = 0; t < TB; ++t) {
+                #pragma unroll
+                for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+            }
+            const int64_t row = row_begin + warp + (int64_t)i * p.warps;
+            #pragma unroll
+            for (int t = 0; t < TB; ++t)
+                if (lane == 0 && tok[t] >= 0) store_out(y + yrow[t] * p.n + row, acc[t]);
+            __syncwarp();
+            if (lane == 0 && i + p.slots < my_rows) {
+                fence_proxy_async_smem();
+                issue(i + p.slots);
+            }
+        }
+        return true;
+    }
 
     // Lane constants: which chunks of a block this lane's units cover, which
     // form of the packed scale bytes they use, and which byte of that word.
@@ -470,6 +520,7 @@ __global__ void __launch_bounds__(MINB == 1 ? 32 * GEMV_MAX_WARPS : 32 * GEMV_HA
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_tok[TB];
     __shared__ int64_t s_yrow[TB];
+    __shared__ int s_nonfinite;
     const int row_begin = blockIdx.x * p.rows_per_cta;
     const int row_end = min(p.n, row_begin + p.rows_per_cta);
     if (row_begin >= row_end) return;
@@ -477,8 +528,9 @@ __global__ void __launch_bounds__(MINB == 1 ? 32 * GEMV_MAX_WARPS : 32 * GEMV_HA
         s_tok[threadIdx.x] = (int)threadIdx.x < p.m ? (int)threadIdx.x : -1;
         s_yrow[threadIdx.x] = threadIdx.x;
     }
+    if (threadIdx.x == 0) s_nonfinite = 0;
     __syncthreads();
-    gemv_pass<C, TB, R, XREG, XT, YT>(p, p.w, row_begin, row_end, s_tok, s_yrow, smem, 0);
+    gemv_pass<C, TB, R, XREG, XT, YT>(p, p.w, row_begin, row_end, s_tok, s_yrow, smem, &s_nonfinite, 0);
     // An independent call still completes after the work before it, so that
     // stream order holds for whatever follows.
     if (p.indep) griddep_wait();

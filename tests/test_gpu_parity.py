@@ -192,11 +192,14 @@ def test_matmul_gemv_tq1(kq, n, k, m, xdt):
     assert kq.device_status() == 0
 
 
-@pytest.mark.parametrize("codec,n,k", [(synth.TQ1_G128, 300, 2048), (synth.TQ1_G128, 200, 1280)])
+@pytest.mark.parametrize("codec,n,k", [(synth.TQ1_G128, 300, 2048), (synth.TQ1_G128, 200, 1280),
+                                       (synth.Q4_K, 300, 2048), (synth.Q4_K, 130, 4096)])
 def test_matmul_gemv_nonfinite_activations(kq, codec, n, k):
     """An infinite and a NaN activation: the fixed-point kernels compute such
     a call exactly in fp32, so each output is NaN, +-inf or finite as in the
-    IEEE product (the fp64 oracle), and the finite outputs stay in tolerance."""
+    IEEE product (the fp64 oracle), and the finite outputs stay in tolerance.
+    One activation row (Q4_K: codes held in registers) and three rows; Q4_K
+    also as an independent call (the shared-SM build)."""
     r = rng(41 + n)
     w = synth.gen_weights(codec, n, k, r)
     x = synth.gen_x(3, k, "f32", r)
@@ -204,14 +207,23 @@ def test_matmul_gemv_nonfinite_activations(kq, codec, n, k):
     x[1, k - 3] = -np.inf      # row 1: one -inf and one NaN
     x[1, 11] = np.nan
     ref = oracle.matmul(codec, w, k, x, threads=8)
-    y = kq.matmul(to_device_w(w), codec, to_device_x(x, "f32"), path=kq.PATH_GEMV).cpu().numpy()
-    assert np.array_equal(np.isnan(y), np.isnan(ref))
-    assert np.array_equal(np.isposinf(y), np.isposinf(ref))
-    assert np.array_equal(np.isneginf(y), np.isneginf(ref))
     assert np.isnan(ref[1]).all() and np.isinf(ref[0]).any()
-    fin = np.isfinite(ref)
-    assert row_rel_err(y[2:], ref[2:]) <= GEMV_TOL      # the finite row
-    assert np.allclose(y[fin], ref[fin], rtol=1e-3, atol=1e-3 * np.abs(ref[2]).max())
+    wd = to_device_w(w)
+
+    def same_classes(y, ref):
+        return (np.array_equal(np.isnan(y), np.isnan(ref)) and np.array_equal(np.isposinf(y), np.isposinf(ref))
+                and np.array_equal(np.isneginf(y), np.isneginf(ref)))
+
+    for indep in ((False, True) if codec == synth.Q4_K else (False,)):
+        y = kq.matmul(wd, codec, to_device_x(x, "f32"), path=kq.PATH_GEMV, independent=indep).cpu().numpy()
+        assert same_classes(y, ref)
+        fin = np.isfinite(ref)
+        assert row_rel_err(y[2:], ref[2:]) <= GEMV_TOL      # the finite row
+        assert np.allclose(y[fin], ref[fin], rtol=1e-3, atol=1e-3 * np.abs(ref[2]).max())
+        y1 = kq.matmul(wd, codec, to_device_x(x[:1], "f32"), path=kq.PATH_GEMV, independent=indep).cpu().numpy()
+        assert same_classes(y1, ref[:1])
+        assert np.allclose(y1[np.isfinite(ref[:1])], ref[:1][np.isfinite(ref[:1])], rtol=1e-3,
+                           atol=1e-3 * np.abs(ref[2]).max())
     assert kq.device_status() == 0
 
 
