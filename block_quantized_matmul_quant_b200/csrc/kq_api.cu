@@ -157,9 +157,11 @@ static bool id_workspace_layout(int64_t n_tokens, int64_t top_k, int64_t n_exper
     return true;
 }
 
-// Activation rows from which the tensor-core kernel serves bf16 inputs; the
-// bandwidth kernel handles up to eight rows per launch.
-constexpr int64_t GEMM_MIN_M = 9;
+// Activation rows from which the tensor-core kernel serves bf16 inputs.
+// Measured on B200 (Q4_K 11008 x 4096, us per call, bandwidth vs tensor-core
+// kernel): 4 rows 20.3 vs 26.9, 8 rows 34.4 vs 26.9; the bandwidth kernel
+// takes 5..8 rows in one pass of eight, so five rows already cost 34.
+constexpr int64_t GEMM_MIN_M = 5;
 // Mean (token, slot) pairs per expert above which the expert-indexed
 // product runs on the tensor cores (each hit expert's weights are then
 // decoded once per token tile of up to 176 pairs); at or below it the
