@@ -683,7 +683,7 @@ def run_sweep(args):
         ws = torch.empty(kq.matmul_id_workspace_bytes(t, 6, 64), dtype=torch.uint8, device="cuda")
         line = {"sweep": "moe_q4_k_e64_1408x2048_top6", "tokens": t, "pairs_per_expert": round(6 * t / 64, 2),
                 "pool": len(pool)}
-        for name, path in (("gemv", kq.PATH_GEMV), ("gemm", kq.PATH_GEMM)):
+        for name, path in (("gemv", kq.PATH_GEMV), ("gemm", kq.PATH_GEMM), ("gemv_tc", kq.PATH_GEMV_TC)):
             def fn():
                 for wi in pool:
                     kq.matmul_id(wi, synth.Q4_K, xd, idd, out=y, workspace=ws, path=path)

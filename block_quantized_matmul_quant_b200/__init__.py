@@ -19,7 +19,7 @@ from . import _build
 Q8_0, Q2_K, Q4_K, Q5_K, Q6_K, TQ1_G128 = 8, 10, 12, 13, 14, 1001
 CODECS = {"q8_0": Q8_0, "q2_k": Q2_K, "q4_k": Q4_K, "q5_k": Q5_K, "q6_k": Q6_K, "tq1_g128": TQ1_G128}
 F32, BF16, F16 = 0, 1, 2
-PATH_AUTO, PATH_SIMPLE, PATH_GEMV, PATH_GEMM = 0, 1, 2, 3
+PATH_AUTO, PATH_SIMPLE, PATH_GEMV, PATH_GEMM, PATH_GEMV_TC = 0, 1, 2, 3, 4
 FLAG_CONST_WEIGHTS = 0x100
 FLAG_INDEPENDENT = 0x200
 

@@ -170,6 +170,9 @@ constexpr int64_t GEMM_MIN_M = 5;
 // bandwidth vs tensor-core kernel): 8 tokens 47 vs 55, 32 tokens 96 vs 84,
 // 64 tokens 147 vs 85, 128 tokens 259 vs 113.
 constexpr int64_t ID_GEMV_MAX_PAIRS_PER_EXPERT = 1;
+// Mean pairs per expert up to which the few-pairs tensor-core kernel runs
+// (one token tile of 16 pairs per expert covers them).
+constexpr int64_t ID_TC_MAX_PAIRS_PER_EXPERT = 12;
 // The TQ1 bandwidth kernel takes two activation rows per pass over the
 // weights; beyond this many rows the plain kernel is used.
 constexpr int64_t TQ1_GEMV_MAX_M = 8;
@@ -307,6 +310,35 @@ static int id_setup(int type, const void *w, int64_t n_experts, int64_t n, int64
 }
 }  // namespace kq
 
+// The expert product over a grouping already in the workspace (a.y: its
+// output, a.y_dtype), by `path` (KQ_PATH_AUTO resolved here).
+static int id_product(const IdArgs &a, int path, int64_t pairs, cudaStream_t s) {
+    const bool can_gemv = moe_gemv_supported(a.type, a.n, a.k, a.n_experts);
+    const bool can_gemm = gemm_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
+    const bool can_tc = moe_mma_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
+    if (path == KQ_PATH_AUTO) {
+        if (can_tc && pairs <= ID_TC_MAX_PAIRS_PER_EXPERT * a.n_experts) path = KQ_PATH_GEMV_TC;
+        else if (can_gemm && (!can_gemv || pairs > ID_GEMV_MAX_PAIRS_PER_EXPERT * a.n_experts)) path = KQ_PATH_GEMM;
+        else path = can_gemv ? KQ_PATH_GEMV : KQ_PATH_SIMPLE;
+    }
+    if (path == KQ_PATH_GEMM && !can_gemm) return KQ_ERR_UNSUPPORTED;
+    if (path == KQ_PATH_GEMV && !can_gemv) return KQ_ERR_UNSUPPORTED;
+    if (path == KQ_PATH_GEMV_TC && !can_tc) return KQ_ERR_UNSUPPORTED;
+    const int64_t max_tiles = id_max_tiles(pairs, a.n_experts);
+    cudaError_t e;
+    if (path == KQ_PATH_GEMM || path == KQ_PATH_GEMV_TC) {
+        const int bn = path == KQ_PATH_GEMM ? gemm_id_bn(a.n_tokens, a.top_k, a.n_experts) : moe_mma_bn();
+        e = launch_moe_tiles(a.offsets, a.n_experts, bn, const_cast<int32_t *>(a.tiles),
+                             const_cast<int32_t *>(a.n_tiles), max_tiles, s);
+        if (e == cudaSuccess) e = path == KQ_PATH_GEMM ? launch_gemm_id(a, bn, s) : launch_moe_mma(a, s);
+    } else if (path == KQ_PATH_GEMV) {
+        e = launch_moe_gemv(a, s);
+    } else {
+        e = launch_simple_id(a, s);
+    }
+    return to_status(e);
+}
+
 extern "C" {
 
 int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
@@ -318,30 +350,14 @@ int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64
     int st = id_setup(type, w, n_experts, n, k, expert_stride, x, x_dtype, n_tokens, ids, top_k, y,
                       y_dtype, workspace, workspace_bytes, &a, &pairs);
     if (st) return st;
-    if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMM) return KQ_ERR_ARG;
+    if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMV_TC) return KQ_ERR_ARG;
     if ((st = check_device())) return st;
     cudaStream_t s = (cudaStream_t)stream;
-    const bool can_gemv = moe_gemv_supported(type, n, k, n_experts);
-    const bool can_gemm = gemm_supported(type, n, k, x_dtype, y_dtype);
-    if (path == KQ_PATH_AUTO) {
-        if (can_gemm && (!can_gemv || pairs > ID_GEMV_MAX_PAIRS_PER_EXPERT * n_experts)) path = KQ_PATH_GEMM;
-        else path = can_gemv ? KQ_PATH_GEMV : KQ_PATH_SIMPLE;
-    }
-    if (path == KQ_PATH_GEMM && !can_gemm) return KQ_ERR_UNSUPPORTED;
-    if (path == KQ_PATH_GEMV && !can_gemv) return KQ_ERR_UNSUPPORTED;
     cudaError_t e = launch_moe_group(ids, pairs, n_experts, const_cast<int32_t *>(a.counts),
                                      const_cast<int32_t *>(a.offsets),
                                      const_cast<int32_t *>(a.perm), y, y_dtype, n, s);
     if (e != cudaSuccess) return KQ_ERR_CUDA;
-    if (path == KQ_PATH_GEMM) {
-        const int bn = gemm_id_bn(n_tokens, top_k, n_experts);
-        e = launch_moe_tiles(a.offsets, n_experts, bn, const_cast<int32_t *>(a.tiles),
-                             const_cast<int32_t *>(a.n_tiles), id_max_tiles(pairs, n_experts), s);
-        if (e != cudaSuccess) return KQ_ERR_CUDA;
-        return to_status(launch_gemm_id(a, bn, s));
-    }
-    if (path == KQ_PATH_GEMV) return to_status(launch_moe_gemv(a, s));
-    return to_status(launch_simple_id(a, s));
+    return id_product(a, path, pairs, s);
 }
 
 int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_experts, int64_t n,
@@ -380,34 +396,14 @@ int kq_matmul_id_mix(int type, const void *w, int64_t n_experts, int64_t n, int6
     if (!aligned16(scores)) return KQ_ERR_ALIGN;
     const bool reuse = (path & KQ_FLAG_REUSE_GROUPING) != 0;
     path &= ~KQ_FLAG_REUSE_GROUPING;
-    if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMM) return KQ_ERR_ARG;
+    if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMV_TC) return KQ_ERR_ARG;
     if ((st = check_device())) return st;
     cudaStream_t s = (cudaStream_t)stream;
-    const bool can_gemv = moe_gemv_supported(type, n, k, n_experts);
-    const bool can_gemm = gemm_supported(type, n, k, x_dtype, KQ_F32);
-    if (path == KQ_PATH_AUTO) {
-        if (can_gemm && (!can_gemv || pairs > ID_GEMV_MAX_PAIRS_PER_EXPERT * n_experts)) path = KQ_PATH_GEMM;
-        else path = can_gemv ? KQ_PATH_GEMV : KQ_PATH_SIMPLE;
-    }
-    if (path == KQ_PATH_GEMM && !can_gemm) return KQ_ERR_UNSUPPORTED;
-    if (path == KQ_PATH_GEMV && !can_gemv) return KQ_ERR_UNSUPPORTED;
-    cudaError_t e = cudaSuccess;
-    if (!reuse)
-        e = launch_moe_group(ids, pairs, n_experts, const_cast<int32_t *>(a.counts),
-                             const_cast<int32_t *>(a.offsets), const_cast<int32_t *>(a.perm), nullptr,
-                             KQ_F32, n, s);
-    if (e != cudaSuccess) return KQ_ERR_CUDA;
-    if (path == KQ_PATH_GEMM) {
-        const int bn = gemm_id_bn(n_tokens, top_k, n_experts);
-        e = launch_moe_tiles(a.offsets, n_experts, bn, const_cast<int32_t *>(a.tiles),
-                             const_cast<int32_t *>(a.n_tiles), id_max_tiles(pairs, n_experts), s);
-        if (e == cudaSuccess) e = launch_gemm_id(a, bn, s);
-    } else if (path == KQ_PATH_GEMV) {
-        e = launch_moe_gemv(a, s);
-    } else {
-        e = launch_simple_id(a, s);
-    }
-    if (e != cudaSuccess) return KQ_ERR_CUDA;
+    if (!reuse &&
+        launch_moe_group(ids, pairs, n_experts, const_cast<int32_t *>(a.counts), const_cast<int32_t *>(a.offsets),
+                         const_cast<int32_t *>(a.perm), nullptr, KQ_F32, n, s) != cudaSuccess)
+        return KQ_ERR_CUDA;
+    if ((st = id_product(a, path, pairs, s))) return st;
     return to_status(launch_moe_mix(static_cast<const float *>(a.y), ids, scores, n_tokens, top_k,
                                     n_experts, n, y, y_dtype, s));
 }

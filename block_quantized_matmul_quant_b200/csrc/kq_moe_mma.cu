@@ -1,0 +1,506 @@
+// kq_moe_mma.cu -- expert-indexed Q4_K product for few routed pairs per
+// expert, on the tensor cores (bf16 activations).
+//
+// The product of mlx-native `quantized_matmul_id_ggml` / mlx-kquant
+// `gather_qmm` (y[t][s] = x[t] @ dequant(W_e)^T, e = ids[t][s]) when every
+// expert has only a handful of routed pairs, the decode step of a
+// mixture-of-experts layer.  There the weights dominate the bytes, each
+// expert's rows are read once, and the work is to decode them fast enough
+// to keep up with HBM.  A Q4_K weight is d*sc_j*q - dmin*m_j with q a 4-bit
+// code and (sc_j, m_j) the scale and min of its 32-weight sub-block j, so
+//
+//   sum_k w_k x_k = d*sc_j * sum_k q_k x_k - dmin*m_j * sum_k x_k   (per sub-block)
+//
+// and the codes alone can go through the tensor core, the scales being
+// applied once per (row, sub-block, token) afterwards:
+//
+//  * A decoder thread per weight row (lane = TMEM lane = row) writes the
+//    codes of one 256-weight super-block as bf16 (128 + q: the nibble ORed
+//    into the mantissa of 128.0, exact) straight into tensor memory; no
+//    scale arithmetic per weight.
+//  * The MMA (tcgen05 kind::f16, M = 128 rows, N = 16 pairs, A from TMEM, B
+//    = the pairs' activations in shared memory) runs each 32-weight
+//    sub-block into an accumulator of its own: D_j = sum (128 + q) x.
+//  * The same threads, one stage later, read the eight accumulators and add
+//    d*sc_j * D_j - (128*d*sc_j + dmin*m_j) * S_j to the row's outputs, S_j
+//    the activations' sum over the sub-block (computed once per token tile).
+//
+// Work units are (token tile of <= 16 pairs of one expert, 128-row tile); a
+// CTA per SM takes a contiguous range of units, so consecutive units share
+// a token tile, whose activations (16 rows x K, 128-byte swizzle, gathered
+// four rows at a time by TMA) stay in shared memory until the tile changes.
+// Raw super-blocks stream through a ring by TMA (3-D map: row bytes, rows,
+// expert).  Warp roles: 0 raw producer, 1 MMA issuer (and TMEM owner), 2
+// activation loader, 4..7 the row warps (warp 4+q owns TMEM lanes 32q..).
+// TMEM: accumulators at columns 0 and 128 (8 sub-blocks x 16 pairs, two
+// stages in flight), A slots at 256 and 384 (256 codes of 128 rows each).
+// Every wait is bounded (kq_ptx.cuh); activations that are not finite make
+// the row warps compute that token tile exactly in fp32 instead.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "kq_decode.cuh"
+#include "kq_ptx.cuh"
+#include "kq_tc.cuh"
+#include "kq_launch.h"
+
+namespace kq {
+
+namespace {
+
+constexpr int MM_BM = 128;                        // weight rows per unit (MMA M)
+constexpr int MM_BN = 16;                         // pairs per token tile (MMA N)
+constexpr int MM_SB = 144;                        // Q4_K super-block bytes
+constexpr int MM_RAW_BYTES = MM_BM * MM_SB;       // one raw stage: 128 rows x one super-block
+constexpr int MM_THREADS = 256;
+constexpr int MM_RAW_WARP = 0, MM_MMA_WARP = 1, MM_X_WARP = 2, MM_ROW_WARP0 = 4;
+constexpr int MM_MAX_K = 4096;
+constexpr int MM_MAX_RAW = 8, MM_MIN_RAW = 3;
+constexpr int MM_SMEM_LIMIT = 232448;             // dynamic shared memory of one CTA
+constexpr uint32_t MM_ACC_COL = 0, MM_A_COL = 256;  // TMEM columns: accumulators, A slots
+
+struct MoeMmaParams {
+    int n, k, nk;                 // weight rows, K, super-blocks per row
+    int n_row_tiles;              // ceil(n / 128)
+    int raw_slots;
+    int x_div;                    // pair p reads activation row p / x_div
+    int n_pairs, n_experts;
+    const int32_t *perm, *offsets;
+    const int2 *tiles;            // (expert, first position in perm) per token tile
+    const int32_t *n_tiles;
+    void *y;
+    unsigned int *err;
+};
+
+// Shared-memory layout, bytes from the 1024-aligned base.
+struct MmLayout {
+    int x, raw, s, pairs, bars, total;
+};
+__host__ __device__ inline MmLayout mm_layout(int k, int raw_slots) {
+    MmLayout l;
+    int off = 0;
+    l.x = off;     off += 32 * k;                           // 16 rows x K bf16, 64-K atoms of 2 KB
+    l.raw = off;   off += raw_slots * MM_RAW_BYTES;
+    l.s = off;     off += 2 * (k / 32) * MM_BN * 4;         // two tiles' sub-block sums [K/32][16]
+    l.pairs = off; off += 2 * MM_BN * 4 + 2 * 4 + 2 * 4;    // pair ids [2][16], counts [2], flags [2]
+    off = (off + 7) / 8 * 8;
+    l.bars = off;  off += (2 * raw_slots + 7) * 8 + 8;      // barriers and the TMEM address
+    l.total = off + 1024;                                   // alignment slack
+    return l;
+}
+
+// Four codes (bytes 0..3 of v, each < 16) -> two bf16x2 words of 128 + q.
+__device__ __forceinline__ void codes4(uint32_t v, uint32_t &w01, uint32_t &w23) {
+    w01 = __byte_perm(v, 0x43434343u, 0x4140);
+    w23 = __byte_perm(v, 0x43434343u, 0x4342);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// Byte i of w as an exact float.
+__device__ __forceinline__ float mm_byte_f(uint32_t w, int i) {
+    return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | (uint32_t)i)) - 8388608.0f;
+}
+
+// Activation (row t, column k) of the swizzled tile: 64-column atoms of 16
+// rows x 128 bytes; 16-byte chunk c of row t sits at chunk c ^ (t & 7).
+__device__ __forceinline__ const uint8_t *x_chunk(const uint8_t *xt, int t, int k) {
+    return xt + (k >> 6) * 2048 + t * 128 + ((((k & 63) >> 3) ^ (t & 7)) << 4);
+}
+
+}  // namespace
+
+template <typename YT>
+__global__ void __launch_bounds__(MM_THREADS, 1)
+    moe_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                   const MoeMmaParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+    const MmLayout lay = mm_layout(p.k, p.raw_slots);
+    const int R = p.raw_slots;
+    uint8_t *x_tile = smem + lay.x;
+    uint8_t *raw = smem + lay.raw;
+    float *s_sum = reinterpret_cast<float *>(smem + lay.s);          // [2][K/32][16]
+    int *s_pair = reinterpret_cast<int *>(smem + lay.pairs);         // [2][16]
+    int *s_ntok = s_pair + 2 * MM_BN;                                // [2]
+    int *s_nf = s_ntok + 2;                                          // [2] non-finite activations
+    uint64_t *raw_full = reinterpret_cast<uint64_t *>(smem + lay.bars);
+    uint64_t *raw_empty = raw_full + R;
+    uint64_t *a_full = raw_empty + R;      // [2] row warps -> MMA: codes in the A slot
+    uint64_t *mma_done = a_full + 2;       // [2] MMA -> row warps: accumulators ready, A slot free
+    uint64_t *x_full = mma_done + 2;       // loader -> all: the token tile's activations
+    uint64_t *x_empty = x_full + 1;        // MMA -> loader: the tile's MMAs are done
+    uint64_t *s_ready = x_empty + 1;       // row warps: the tile's sub-block sums written
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(s_ready + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if ((uint32_t)(smem - smem_raw) + (uint32_t)lay.total - 1024u > dynamic_smem_size()) {
+        if (threadIdx.x == 0) atomicOr(p.err, ERR_BOUNDS);   // the host planned another layout: no work
+        return;
+    }
+    if (threadIdx.x == 0) {
+        for (int r = 0; r < R; ++r) {
+            mbar_init(&raw_full[r], 1);
+            mbar_init(&raw_empty[r], 4);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&a_full[b], 4);
+            mbar_init(&mma_done[b], 1);
+        }
+        mbar_init(x_full, 1);
+        mbar_init(x_empty, 1);
+        mbar_init(s_ready, 4);
+        fence_mbar_init();
+    }
+    if (warp == MM_MMA_WARP) tmem_alloc(tmem_slot, 512);
+    if (warp == MM_RAW_WARP && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    griddep_wait();   // the grouping and the tile list come from the preceding kernels
+
+    const int nrt = p.n_row_tiles, nk = p.nk;
+    const int total = *p.n_tiles * nrt;
+    const int u0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
+    const int u1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
+    // Token tile -> (expert, first position in perm, pairs); KQ_DEBUG: a tile
+    // outside the grouping becomes an empty tile of expert 0.
+    auto tile_info = [&](int tile, int &e, int &m0, int &rows) {
+        const int2 tt = p.tiles[tile];
+        const bool ok = KQ_DCHECK(tt.x >= 0 && tt.x < p.n_experts && tt.y >= 0 && tt.y < p.n_pairs &&
+                                      p.offsets[tt.x + 1] <= p.n_pairs, p.err);
+        e = ok ? tt.x : 0;
+        m0 = ok ? tt.y : 0;
+        rows = ok ? min(MM_BN, p.offsets[tt.x + 1] - tt.y) : 0;
+    };
+
+    if (warp == MM_RAW_WARP) {
+        // ---------------- raw super-block producer ----------------
+        if (lane == 0) {
+            uint32_t g = 0;
+            bool ok = true;
+            for (int u = u0; u < u1 && ok; ++u) {
+                int e, m0, rows;
+                tile_info(u / nrt, e, m0, rows);
+                const int n0 = (u % nrt) * MM_BM;
+                for (int s = 0; s < nk; ++s, ++g) {
+                    const uint32_t slot = g % (uint32_t)R, ph = (g / (uint32_t)R) & 1u;
+                    ok = mbar_wait(&raw_empty[slot], ph ^ 1u, p.err);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&raw_full[slot], MM_RAW_BYTES);
+                    tma_load_3d(raw + slot * MM_RAW_BYTES, &tmap_w, s * MM_SB, n0, e, &raw_full[slot]);
+                }
+            }
+        }
+    } else if (warp == MM_X_WARP) {
+        // ---------------- activation loader ----------------
+        // When the token tile changes: wait until the previous tile's MMAs
+        // are done, publish the tile's pair ids, gather its 16 activation
+        // rows (rows past the segment repeat its first row; their outputs
+        // are dropped).
+        if (lane == 0) {
+            int xt = 0, prev = -1;
+            bool ok = true;
+            for (int u = u0; u < u1 && ok; ++u) {
+                const int tile = u / nrt;
+                if (tile == prev) continue;
+                prev = tile;
+                if (xt > 0) {
+                    ok = mbar_wait(x_empty, (uint32_t)(xt - 1) & 1u, p.err);
+                    if (!ok) break;
+                }
+                int e, m0, rows;
+                tile_info(tile, e, m0, rows);
+                const int buf = xt & 1;
+                int xr[MM_BN];
+                int first = 0;
+                #pragma unroll
+                for (int i = 0; i < MM_BN; ++i) {
+                    int pr = -1;
+                    if (i < rows) {
+                        pr = p.perm[m0 + i];
+                        if (!KQ_DCHECK(pr >= 0 && pr < p.n_pairs, p.err)) pr = -1;
+                    }
+                    if (i == 0 && pr >= 0) first = pr;
+                    s_pair[buf * MM_BN + i] = pr;
+                    xr[i] = (pr >= 0 ? pr : first) / p.x_div;
+                }
+                s_ntok[buf] = rows;
+                s_nf[buf] = 0;
+                mbar_arrive_expect_tx(x_full, (uint32_t)(MM_BN * p.k * 2));
+                for (int a = 0; a < p.k / 64; ++a)
+                    #pragma unroll
+                    for (int i = 0; i < MM_BN; i += 4)
+                        tma_gather4(x_tile + a * 2048 + i * 128, &tmap_x, a * 64, xr[i], xr[i + 1], xr[i + 2],
+                                    xr[i + 3], x_full);
+                ++xt;
+            }
+        }
+    } else if (warp == MM_MMA_WARP) {
+        // ---------------- MMA issuer ----------------
+        // Per stage (one super-block): eight sub-blocks, each two MMAs of
+        // K = 16 into its own 16-column accumulator; one commit frees the A
+        // slot and publishes the accumulators.
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(MM_BM, MM_BN);
+            const uint64_t xdesc0 = sw128_desc(smem_addr(x_tile));
+            uint32_t g = 0;
+            int xt = 0, prev = -1;
+            bool ok = true;
+            for (int u = u0; u < u1 && ok; ++u) {
+                const int tile = u / nrt;
+                if (tile != prev) {
+                    if (xt > 0) mma_commit(x_empty);   // once the previous tile's MMAs are done
+                    ok = mbar_wait(x_full, (uint32_t)xt & 1u, p.err);
+                    if (!ok) break;
+                    prev = tile;
+                    ++xt;
+                }
+                for (int s = 0; s < nk; ++s, ++g) {
+                    const uint32_t b = g & 1u;
+                    ok = mbar_wait(&a_full[b], (g >> 1) & 1u, p.err);
+                    if (!ok) break;
+                    tc_fence_after();
+                    #pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int kidx = 256 * s + 32 * j;     // first K of the sub-block
+                        const uint64_t bd = xdesc0 + (uint64_t)((kidx >> 6) * (2048 >> 4) + ((kidx & 63) >> 3));
+                        const uint32_t d = tmem_base + MM_ACC_COL + b * 128u + 16u * j;
+                        const uint32_t a = tmem_base + MM_A_COL + b * 128u + 16u * j;
+                        mma_bf16_ts(d, a, bd, idesc, 0u);
+                        mma_bf16_ts(d, a + 8, bd + 2, idesc, 1u);
+                    }
+                    mma_commit(&mma_done[b]);
+                }
+            }
+        }
+    } else if (warp >= MM_ROW_WARP0) {
+        // ---------------- row warps ----------------
+        // Lane l of warp 4+q owns weight row 32q + l of the unit (TMEM lane
+        // 32q + l).  Per stage: codes of the row's super-block into the A
+        // slot, then the scales applied to the previous stage's
+        // accumulators.  Per token tile: the sub-block sums S of its
+        // activations (thread i of the 128 takes sums i, i + 128, ...).
+        const int q = warp & 3, r = 32 * q + lane, ti = threadIdx.x - 32 * MM_ROW_WARP0;
+        const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16);
+        const int nsub = p.k / 32;
+        YT *y = static_cast<YT *>(p.y);
+        uint32_t g = 0;
+        int xt = 0, prev = -1, buf = 0, ntok = 0;
+        bool nf = false;
+        bool ok = true;
+        float acc[MM_BN];
+        float ap[8], cp[8];   // the previous stage's d*sc and 128*d*sc + dmin*m
+        // Scales of the previous stage applied to its accumulators (stage
+        // index sp within the unit, global stage gp).
+        auto epilogue = [&](uint32_t gp, int sp) -> bool {
+            const uint32_t b = gp & 1u;
+            if (!__all_sync(0xffffffffu, mbar_wait(&mma_done[b], (gp >> 1) & 1u, p.err))) return false;
+            tc_fence_after();
+            if (nf) return true;   // the exact path has added this stage already
+            const float *sb = s_sum + (buf * nsub + 8 * sp) * MM_BN;
+            #pragma unroll
+            for (int tg = 0; tg < MM_BN / 4; ++tg) {
+                if (4 * tg >= ntok) break;   // warp-uniform
+                uint32_t dv[32];
+                tmem_ld4x8(t_lane + MM_ACC_COL + b * 128u + 4u * tg, dv);
+                #pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 sv = *reinterpret_cast<const float4 *>(sb + j * MM_BN + 4 * tg);
+                    acc[4 * tg + 0] = fmaf(ap[j], __uint_as_float(dv[4 * j + 0]), fmaf(-cp[j], sv.x, acc[4 * tg + 0]));
+                    acc[4 * tg + 1] = fmaf(ap[j], __uint_as_float(dv[4 * j + 1]), fmaf(-cp[j], sv.y, acc[4 * tg + 1]));
+                    acc[4 * tg + 2] = fmaf(ap[j], __uint_as_float(dv[4 * j + 2]), fmaf(-cp[j], sv.z, acc[4 * tg + 2]));
+                    acc[4 * tg + 3] = fmaf(ap[j], __uint_as_float(dv[4 * j + 3]), fmaf(-cp[j], sv.w, acc[4 * tg + 3]));
+                }
+            }
+            return true;
+        };
+        for (int u = u0; u < u1 && ok; ++u) {
+            const int tile = u / nrt;
+            if (tile != prev) {
+                ok = __all_sync(0xffffffffu, mbar_wait(x_full, (uint32_t)xt & 1u, p.err));
+                if (!ok) break;
+                buf = xt & 1;
+                float *sb = s_sum + buf * nsub * MM_BN;
+                bool bad = false;
+                for (int v = ti; v < nsub * MM_BN; v += 128) {
+                    const int jg = v >> 4, t = v & 15;
+                    float sum = 0.f;
+                    #pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(x_chunk(x_tile, t, 32 * jg + 8 * c));
+                        sum += ((bf16_lo(w.x) + bf16_hi(w.x)) + (bf16_lo(w.y) + bf16_hi(w.y))) +
+                               ((bf16_lo(w.z) + bf16_hi(w.z)) + (bf16_lo(w.w) + bf16_hi(w.w)));
+                    }
+                    sb[v] = sum;
+                    bad |= !(fabsf(sum) <= 3.402823466e38f);   // an infinity or NaN in the sub-block
+                }
+                if (__any_sync(0xffffffffu, bad) && lane == 0) s_nf[buf] = 1;
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(s_ready);
+                ok = __all_sync(0xffffffffu, mbar_wait(s_ready, (uint32_t)xt & 1u, p.err));
+                if (!ok) break;
+                ntok = s_ntok[buf];
+                nf = s_nf[buf] != 0;
+                prev = tile;
+                ++xt;
+            }
+            const int row = (u % nrt) * MM_BM + r;
+            #pragma unroll
+            for (int t = 0; t < MM_BN; ++t) acc[t] = 0.f;
+            for (int s = 0; s < nk; ++s, ++g) {
+                const uint32_t rs = g % (uint32_t)R, rph = (g / (uint32_t)R) & 1u;
+                ok = __all_sync(0xffffffffu, mbar_wait(&raw_full[rs], rph, p.err));
+                if (!ok) break;
+                const uint8_t *blk = raw + rs * MM_RAW_BYTES + r * MM_SB;
+                const uint4 hd = *reinterpret_cast<const uint4 *>(blk);
+                const float d = half_bits_to_float(hd.x), dmin = half_bits_to_float(hd.x >> 16);
+                const uint32_t sc_lo = hd.y & 0x3F3F3F3Fu, m_lo = hd.z & 0x3F3F3F3Fu;
+                const uint32_t sc_hi = (hd.w & 0x0F0F0F0Fu) | ((hd.y >> 2) & 0x30303030u);
+                const uint32_t m_hi = ((hd.w >> 4) & 0x0F0F0F0Fu) | ((hd.z >> 2) & 0x30303030u);
+                float a[8], dm[8];
+                #pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    a[j] = d * mm_byte_f(j < 4 ? sc_lo : sc_hi, j & 3);      // exact
+                    dm[j] = dmin * mm_byte_f(j < 4 ? m_lo : m_hi, j & 3);    // exact
+                }
+                // codes of the stage into A slot g & 1 (free: the MMA of stage
+                // g - 2 is done, waited in its epilogue)
+                const uint32_t acol = MM_A_COL + (g & 1u) * 128u;
+                #pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const uint4 v0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * cc);
+                    const uint4 v1 = *reinterpret_cast<const uint4 *>(blk + 32 + 32 * cc);
+                    const uint32_t qw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                    uint32_t out[32];
+                    #pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        codes4(qw[i] & 0x0F0F0F0Fu, out[2 * i], out[2 * i + 1]);
+                        codes4((qw[i] >> 4) & 0x0F0F0F0Fu, out[16 + 2 * i], out[17 + 2 * i]);
+                    }
+                    tmem_st32(t_lane + acol + 32u * cc, out);
+                }
+                if (nf) {
+                    // exact fp32: each decoded weight times the activation
+                    // itself, so infinities and NaNs combine as IEEE does
+                    #pragma unroll 1
+                    for (int t = 0; t < MM_BN; ++t) {
+                        if (t >= ntok) break;
+                        float v = 0.f;
+                        #pragma unroll 1
+                        for (int kk = 0; kk < 256; ++kk) {
+                            const int j = kk >> 5, cc = kk >> 6, l = kk & 31;
+                            const uint32_t byte = blk[16 + 32 * cc + l];
+                            const float qv = (float)((j & 1) ? (byte >> 4) : (byte & 15u));
+                            const int k = 256 * s + kk;
+                            const uint16_t xb = *reinterpret_cast<const uint16_t *>(x_chunk(x_tile, t, k) + 2 * (k & 7));
+                            v = fmaf(fmaf(a[j], qv, -dm[j]), __uint_as_float((uint32_t)xb << 16), v);
+                        }
+                        #pragma unroll
+                        for (int tt = 0; tt < MM_BN; ++tt)
+                            if (tt == t) acc[tt] += v;
+                    }
+                }
+                tc_fence_before();
+                fence_proxy_async_smem();   // generic reads of the raw slot and the tile before TMA refills
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&a_full[g & 1u]);
+                    mbar_arrive(&raw_empty[rs]);
+                }
+                if (s > 0) {
+                    ok = epilogue(g - 1, s - 1);
+                    if (!ok) break;
+                }
+                #pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    ap[j] = a[j];
+                    cp[j] = fmaf(128.0f, a[j], dm[j]);
+                }
+            }
+            if (!ok) break;
+            ok = epilogue(g - 1, nk - 1);
+            if (!ok) break;
+            if (row < p.n) {
+                #pragma unroll
+                for (int t = 0; t < MM_BN; ++t) {
+                    const int pr = s_pair[buf * MM_BN + t];
+                    if (t < ntok && pr >= 0) store_out(y + (int64_t)pr * p.n + row, acc[t]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    griddep_launch_dependents();
+    if (warp == MM_MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+namespace {
+
+// Raw ring depth that fits next to the activation tile and the sums.
+int mm_raw_slots(int64_t k) {
+    int r = MM_MAX_RAW;
+    while (r >= MM_MIN_RAW && mm_layout((int)k, r).total > MM_SMEM_LIMIT) --r;
+    return r;
+}
+
+}  // namespace
+
+bool moe_mma_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype) {
+    if (type != KQ_Q4_K || x_dtype != KQ_BF16) return false;
+    if (y_dtype != KQ_F32 && y_dtype != KQ_BF16) return false;
+    if (k % 256 || k > MM_MAX_K || n < 1 || n > (1 << 30)) return false;
+    return mm_raw_slots(k) >= MM_MIN_RAW && encode_fn() != nullptr;
+}
+
+int moe_mma_bn() { return MM_BN; }
+
+cudaError_t launch_moe_mma(const IdArgs &a, cudaStream_t s) {
+    if (!moe_mma_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype)) return cudaErrorNotSupported;
+    MoeMmaParams p = {};
+    p.n = (int)a.n;
+    p.k = (int)a.k;
+    p.nk = (int)(a.k / 256);
+    p.n_row_tiles = (int)((a.n + MM_BM - 1) / MM_BM);
+    p.raw_slots = mm_raw_slots(a.k);
+    p.x_div = a.x_div();
+    p.n_pairs = (int)(a.n_tokens * a.top_k);
+    p.n_experts = (int)a.n_experts;
+    p.perm = a.perm;
+    p.offsets = a.offsets;
+    p.tiles = reinterpret_cast<const int2 *>(a.tiles);
+    p.n_tiles = a.n_tiles;
+    p.y = a.y;
+    p.err = error_word();
+    CUtensorMap tx, tw;
+    if (!encode_x_map(&tx, a.x, a.x_rows(), a.k, 1) ||
+        !encode_w_map(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride))
+        return cudaErrorInvalidValue;
+    const int smem = mm_layout(p.k, p.raw_slots).total;
+    auto kern = a.y_dtype == KQ_F32 ? moe_mma_kernel<float> : moe_mma_kernel<__nv_bfloat16>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)sm_count());
+    cfg.blockDim = dim3(MM_THREADS);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+}
+
+}  // namespace kq

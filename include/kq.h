@@ -80,6 +80,10 @@ extern "C" {
 #define KQ_PATH_SIMPLE   1  /* plain CUDA-core kernel, any codec/shape               */
 #define KQ_PATH_GEMV     2  /* bandwidth kernel: weights decoded in registers         */
 #define KQ_PATH_GEMM     3  /* TMA + tcgen05 tensor-core kernel (bf16 x only)         */
+/* Expert-indexed calls only: the tensor-core kernel for few pairs per expert
+ * (4-bit codes through the MMA, one accumulator per 32-weight sub-block, the
+ * scales applied after it; Q4_K, bf16 x, K <= 4096, token tiles of 16). */
+#define KQ_PATH_GEMV_TC  4
 /* Flag OR-ed into `path`: the caller guarantees that no work enqueued earlier
  * on the stream writes the weight bytes (they are constant, as model weights
  * are).  The kernel may then start streaming weights before the preceding
@@ -172,7 +176,8 @@ KQ_API int kq_matmul_id(int type, const void *w, int64_t n_experts, int64_t n, i
                  const int32_t *ids, int64_t top_k, void *y, int y_dtype,
                  void *workspace, size_t workspace_bytes, void *stream);
 /* kq_matmul_id with an explicit path: KQ_PATH_SIMPLE, KQ_PATH_GEMV (grouped
- * mat-vec) or KQ_PATH_GEMM (grouped tensor-core GEMM, bf16 x only). */
+ * mat-vec), KQ_PATH_GEMM (grouped tensor-core GEMM, bf16 x only) or
+ * KQ_PATH_GEMV_TC (tensor-core kernel for few pairs per expert). */
 KQ_API int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
                     int64_t expert_stride, const void *x, int x_dtype, int64_t n_tokens,
                     const int32_t *ids, int64_t top_k, void *y, int y_dtype,

@@ -442,12 +442,12 @@ def test_matmul_id_small(kq, codec, path):
     y = kq.matmul_id(to_device_w(w), codec, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
                      path=p).cpu().numpy()
     if path == "auto" and codec == synth.Q4_K:
-        # bf16 Q4_K: the dispatch picks the grouped bandwidth kernel or the
-        # grouped tensor-core kernel by pairs per expert; the result is one
-        # of the two, bit for bit, within the bf16 contract
+        # bf16 Q4_K: the dispatch picks one of the grouped kernels by pairs
+        # per expert; the result is one of theirs, bit for bit, within the
+        # bf16 contract
         assert row_rel_err(y, ref) <= TOL["bf16"]
         outs = [kq.matmul_id(to_device_w(w), codec, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
-                             path=pp).cpu().numpy() for pp in (kq.PATH_GEMV, kq.PATH_GEMM)]
+                             path=pp).cpu().numpy() for pp in (kq.PATH_GEMV, kq.PATH_GEMM, kq.PATH_GEMV_TC)]
         assert any(np.array_equal(y.view(np.uint32), o.view(np.uint32)) for o in outs)
     else:
         assert row_rel_err(y, ref) <= FP32_PATH_TOL
@@ -672,6 +672,77 @@ def test_moe_ffn_chain_reuses_the_grouping(kq, xdt):
     full = oracle.mix_id(synth.Q4_K, wdn, fdim, oracle.glu_id(synth.Q4_K, wg, wu, hdim, x, ids, "silu"),
                          ids, scores)
     assert row_rel_err(y, full) <= 4 * GEMV_TOL
+    assert kq.device_status() == 0
+
+
+@pytest.mark.parametrize("t,top_k,e,n,k,skew", [
+    (32, 6, 64, 1408, 2048, False),    # the MoE workload: ~3 pairs per expert, one token tile each
+    (5, 3, 6, 130, 512, False),        # ragged weight rows, one tile of rows and a partial one
+    (100, 2, 3, 300, 1024, False),     # ~66 pairs per expert: five token tiles each
+    (7, 3, 4, 129, 4096, False),       # the largest K the kernel takes
+    (64, 4, 8, 256, 768, True),        # one expert takes most pairs: many tiles, other experts one
+])
+def test_matmul_id_tensor_core_few_pairs(kq, t, top_k, e, n, k, skew):
+    """The few-pairs tensor-core kernel: codes through the MMA, a sub-block
+    accumulator each, scales applied after it -- against the fp64 oracle
+    (bf16 activations exact in the MMA), f32 and bf16 outputs, bit-stable,
+    and a NaN row for an id outside the stack."""
+    import torch
+
+    r = rng(11 * t + e + n + k)
+    w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, "bf16", r)
+    ids = synth.gen_ids(t, top_k, e, r)
+    if skew:
+        ids[:, 0] = np.where(np.arange(t) % 9 == 0, 1, 2)
+    ids[t // 2, top_k - 1] = e                 # outside the stack: a NaN row
+    ref = oracle.matmul_id(synth.Q4_K, w, k, x, ids)
+    wd, xd, idd = to_device_w(w), to_device_x(x, "bf16"), torch.from_numpy(ids).cuda()
+    y = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMV_TC).cpu().numpy()
+    assert np.all(np.isnan(y[t // 2, top_k - 1]))
+    good = ~np.isnan(ref[..., 0])
+    err = row_rel_err(y[good], ref[good])
+    assert err <= GEMV_TOL, err
+    assert kq.device_status() == -9
+    y2 = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMV_TC).cpu().numpy()
+    assert np.array_equal(y.view(np.uint32), y2.view(np.uint32))
+    yb = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMV_TC,
+                      out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert row_rel_err(yb[good], ref[good]) <= GEMV_TOL + BF16_OUT
+    assert kq.device_status() == -9
+    assert kq.device_status() == 0
+
+
+def test_matmul_id_tensor_core_nonfinite_and_slotted(kq):
+    """Non-finite activations send their token tile through the exact fp32
+    path (IEEE classes as the oracle's); the slotted input of the down
+    projection (one activation row per pair) through the same kernel."""
+    import torch
+
+    t, top_k, e, n, k = 12, 2, 5, 160, 512
+    r = rng(77)
+    w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, "bf16", r)
+    ids = synth.gen_ids(t, top_k, e, r)
+    x[3, 10] = np.inf
+    x[5, 100] = np.nan
+    ref = oracle.matmul_id(synth.Q4_K, w, k, x, ids)
+    y = kq.matmul_id(to_device_w(w), synth.Q4_K, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
+                     path=kq.PATH_GEMV_TC).cpu().numpy()
+    assert np.array_equal(np.isnan(y), np.isnan(ref))
+    assert np.array_equal(np.isposinf(y), np.isposinf(ref)) and np.array_equal(np.isneginf(y), np.isneginf(ref))
+    assert np.isinf(ref[3]).any() and np.isnan(ref[5]).all()
+    fin = np.isfinite(ref)
+    scale = np.abs(ref[fin]).max()
+    assert np.all(np.abs(y[fin] - ref[fin]) <= GEMV_TOL * scale)
+    assert kq.device_status() == 0
+    xs = synth.gen_x(t * top_k, k, "bf16", r).reshape(t, top_k, k)
+    scores = r.uniform(0, 1, (t, top_k)).astype(np.float32)
+    ym = kq.matmul_id_mix(to_device_w(w), synth.Q4_K, to_device_x(xs, "bf16"), torch.from_numpy(ids).cuda(),
+                          torch.from_numpy(scores).cuda(), path=kq.PATH_GEMV_TC).cpu().numpy()
+    refm = oracle.mix_id(synth.Q4_K, w, k, xs, ids, scores)
+    ok, worst = _mix_err_ok(ym, refm, _pair_refs(synth.Q4_K, w, k, xs, ids), scores, GEMV_TOL)
+    assert ok, worst
     assert kq.device_status() == 0
 
 
