@@ -664,7 +664,7 @@ def run_sweep(args):
         x = torch.from_numpy(synth.gen_x(m, dense.k, "bf16", r)).to(torch.bfloat16).cuda()
         y = torch.empty((m, dense.n), device="cuda")
         line = {"sweep": "dense_q4_k_11008x4096", "m": m, "pool": len(pool)}
-        for name, path in (("gemv", kq.PATH_GEMV), ("gemm", kq.PATH_GEMM)):
+        for name, path in (("gemv", kq.PATH_GEMV), ("gemm", kq.PATH_GEMM), ("gemv_tc", kq.PATH_GEMV_TC)):
             def fn():
                 for wi in pool:
                     kq.matmul(wi, synth.Q4_K, x, out=y, path=path, const_weights=True)

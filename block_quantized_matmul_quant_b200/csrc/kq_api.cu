@@ -212,9 +212,10 @@ int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, i
     const bool indep = (path & KQ_FLAG_INDEPENDENT) != 0;
     const bool const_w = indep || (path & KQ_FLAG_CONST_WEIGHTS) != 0;
     path &= ~(KQ_FLAG_CONST_WEIGHTS | KQ_FLAG_INDEPENDENT);
-    if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMM) return KQ_ERR_ARG;
+    if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMV_TC) return KQ_ERR_ARG;
     if ((st = check_device())) return st;
     cudaStream_t s = (cudaStream_t)stream;
+    const bool can_tc = moe_mma_supported(type, n, k, x_dtype, y_dtype);
     const bool can_gemm = gemm_supported(type, n, k, x_dtype, y_dtype);
     const bool can_gemv = gemv_supported(type, n, k, x_dtype, m);
     if (path == KQ_PATH_AUTO) {
@@ -223,6 +224,9 @@ int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, i
         else path = KQ_PATH_SIMPLE;
     }
     switch (path) {
+    case KQ_PATH_GEMV_TC:
+        if (!can_tc) return KQ_ERR_UNSUPPORTED;
+        return to_status(launch_gemv_tc(w, n, k, x, m, y, y_dtype, s));
     case KQ_PATH_GEMM:
         if (!can_gemm) return KQ_ERR_UNSUPPORTED;
         return to_status(launch_gemm(type, w, n, k, x, m, y, y_dtype, s));
@@ -379,6 +383,13 @@ int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_e
                                      const_cast<int32_t *>(a.offsets),
                                      const_cast<int32_t *>(a.perm), y, y_dtype, n, s);
     if (e != cudaSuccess) return KQ_ERR_CUDA;
+    // bf16 activations: the tensor-core kernel (gate and up passes per unit);
+    // otherwise the bandwidth kernel, or the plain one for other codecs
+    if (moe_mma_supported(type, n, k, x_dtype, y_dtype)) {
+        e = launch_moe_tiles(a.offsets, n_experts, moe_mma_bn(), const_cast<int32_t *>(a.tiles),
+                             const_cast<int32_t *>(a.n_tiles), id_max_tiles(pairs, n_experts), s);
+        return to_status(e == cudaSuccess ? launch_moe_mma(a, s) : e);
+    }
     if (moe_gemv_supported(type, n, k, n_experts)) return to_status(launch_moe_gemv(a, s));
     return to_status(launch_simple_glu(a, s));
 }

@@ -55,6 +55,15 @@ __device__ __forceinline__ uint32_t dynamic_smem_size() {
     return v;
 }
 
+// GLU activation (KQ_ACT_*, mlx-kquant `moe_glu_gather_kq`): SiLU
+// g / (1 + e^-g), or the tanh form of GELU 0.5 g (1 + tanh(sqrt(2/pi) (g +
+// 0.044715 g^3))).
+__device__ __forceinline__ float glu_activation(float g, int act) {
+    if (act == KQ_ACT_GELU_TANH)
+        return 0.5f * g * (1.0f + tanhf(0.7978845608028654f * fmaf(0.044715f * g, g * g, g)));
+    return g / (1.0f + expf(-g));
+}
+
 __device__ __forceinline__ float half_bits_to_float(uint32_t bits16) {
     return __half2float(__ushort_as_half((unsigned short)(bits16 & 0xFFFFu)));
 }

@@ -85,6 +85,9 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s);
 // (kq_moe_mma.cu), over token tiles of moe_mma_bn() pairs.
 bool moe_mma_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype);
 int moe_mma_bn();
-cudaError_t launch_moe_mma(const IdArgs &a, cudaStream_t s);
+cudaError_t launch_moe_mma(const IdArgs &a, cudaStream_t s);   // a.w2 set: fused GLU
+// The same kernel on one matrix and m activation rows (tiles of 16 rows).
+cudaError_t launch_gemv_tc(const void *w, int64_t n, int64_t k, const void *x, int64_t m, void *y, int y_dtype,
+                           cudaStream_t s);
 
 }  // namespace kq

@@ -216,12 +216,6 @@ __global__ void __launch_bounds__(256) simple_id_kernel(
 
 // Plain fused GLU: the same walk with a gate and an up row per warp;
 // y = act(gate) * up (mlx-kquant `moe_glu_gather_kq`).
-__device__ __forceinline__ float glu_act_plain(float g, int act) {
-    if (act == KQ_ACT_GELU_TANH)
-        return 0.5f * g * (1.0f + tanhf(0.7978845608028654f * fmaf(0.044715f * g, g * g, g)));
-    return g / (1.0f + expf(-g));
-}
-
 template <int TYPE, typename XT, typename YT>
 __global__ void __launch_bounds__(256) simple_glu_kernel(
     const uint8_t *__restrict__ wg, const uint8_t *__restrict__ wu, int64_t n, int64_t k,
@@ -278,7 +272,7 @@ __global__ void __launch_bounds__(256) simple_glu_kernel(
                 g += __shfl_xor_sync(0xffffffffu, g, o);
                 uu += __shfl_xor_sync(0xffffffffu, uu, o);
             }
-            if (lane == 0 && pr[t] >= 0) store_out(y + (int64_t)pr[t] * n + row, glu_act_plain(g, act) * uu);
+            if (lane == 0 && pr[t] >= 0) store_out(y + (int64_t)pr[t] * n + row, glu_activation(g, act) * uu);
         }
     }
 }

@@ -79,15 +79,6 @@ __device__ __forceinline__ int dp2a_hi(int a, uint32_t b, int c) {
     asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
 }
-// The GLU activations (mlx-kquant `moe_glu_gather_kq`): silu(g) = g / (1 +
-// exp(-g)); gelu: the tanh approximation 0.5 g (1 + tanh(sqrt(2/pi) (g +
-// 0.044715 g^3))).
-__device__ __forceinline__ float glu_act(float g, int act) {
-    if (act == KQ_ACT_GELU_TANH)
-        return 0.5f * g * (1.0f + tanhf(0.7978845608028654f * fmaf(0.044715f * g, g * g, g)));
-    return g / (1.0f + expf(-g));
-}
-
 __device__ __forceinline__ float byte_f(uint32_t w, int i) {   // byte i of w, exactly
     return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | (uint32_t)i)) - 8388608.0f;
 }
@@ -236,7 +227,7 @@ __global__ void __launch_bounds__(MG_THREADS, 1) moe_gemv_kernel(const MoeGemvPa
                             gs += part[(g * p.wg + w) * MG_PART + t];
                             us += part[(g * p.wg + w) * MG_PART + MG_TB + t];
                         }
-                        store_out(y + (int64_t)pr * p.n + row, glu_act(gs, p.act) * us);
+                        store_out(y + (int64_t)pr * p.n + row, glu_activation(gs, p.act) * us);
                     }
                 }
             } else {

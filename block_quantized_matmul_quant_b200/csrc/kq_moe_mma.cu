@@ -14,14 +14,14 @@
 // and the codes alone can go through the tensor core, the scales being
 // applied once per (row, sub-block, token) afterwards:
 //
-//  * A decoder thread per weight row (lane = TMEM lane = row) writes the
-//    codes of one 256-weight super-block as bf16 (128 + q: the nibble ORed
-//    into the mantissa of 128.0, exact) straight into tensor memory; no
-//    scale arithmetic per weight.
+//  * Decoder threads (lane = TMEM lane = weight row) write the codes of one
+//    256-weight super-block as bf16 (128 + q: the nibble ORed into the
+//    mantissa of 128.0, exact) straight into tensor memory; no scale
+//    arithmetic per weight.
 //  * The MMA (tcgen05 kind::f16, M = 128 rows, N = 16 pairs, A from TMEM, B
 //    = the pairs' activations in shared memory) runs each 32-weight
 //    sub-block into an accumulator of its own: D_j = sum (128 + q) x.
-//  * The same threads, one stage later, read the eight accumulators and add
+//  * Epilogue threads (lane = row again) read the eight accumulators and add
 //    d*sc_j * D_j - (128*d*sc_j + dmin*m_j) * S_j to the row's outputs, S_j
 //    the activations' sum over the sub-block (computed once per token tile).
 //
@@ -31,11 +31,17 @@
 // four rows at a time by TMA) stay in shared memory until the tile changes.
 // Raw super-blocks stream through a ring by TMA (3-D map: row bytes, rows,
 // expert).  Warp roles: 0 raw producer, 1 MMA issuer (and TMEM owner), 2
-// activation loader, 4..7 the row warps (warp 4+q owns TMEM lanes 32q..).
-// TMEM: accumulators at columns 0 and 128 (8 sub-blocks x 16 pairs, two
-// stages in flight), A slots at 256 and 384 (256 codes of 128 rows each).
-// Every wait is bounded (kq_ptx.cuh); activations that are not finite make
-// the row warps compute that token tile exactly in fp32 instead.
+// activation loader, 4..7 epilogue (warp 4+q reads TMEM lanes 32q..), 8..15
+// decoders (two per lane quadrant, half a super-block each).  Splitting the
+// decode from the epilogue, and the decode over two warps, keeps several
+// warps per scheduler: with one thread doing both per row the stage was
+// latency-bound (about 2 us).  TMEM: accumulators at columns 0 and 128 (8
+// sub-blocks x 16 pairs, two stages in flight), A slots at 256 and 384 (256
+// codes of 128 rows each).  Fused GLU: each unit runs the gate stack's
+// stages, then the up stack's, into two sets of row sums.  Dense mode: one
+// matrix, activation rows in tiles of 16, no grouping.  Every wait is
+// bounded (kq_ptx.cuh); activations that are not finite make the epilogue
+// compute that token tile exactly in fp32 instead.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -52,17 +58,17 @@ constexpr int MM_BM = 128;                        // weight rows per unit (MMA M
 constexpr int MM_BN = 16;                         // pairs per token tile (MMA N)
 constexpr int MM_SB = 144;                        // Q4_K super-block bytes
 constexpr int MM_RAW_BYTES = MM_BM * MM_SB;       // one raw stage: 128 rows x one super-block
-constexpr int MM_THREADS = 256;
-constexpr int MM_RAW_WARP = 0, MM_MMA_WARP = 1, MM_X_WARP = 2, MM_ROW_WARP0 = 4;
+constexpr int MM_THREADS = 512;
+constexpr int MM_RAW_WARP = 0, MM_MMA_WARP = 1, MM_X_WARP = 2, MM_EPI_WARP0 = 4, MM_DEC_WARP0 = 8;
 constexpr int MM_MAX_K = 4096;
-constexpr int MM_MAX_RAW = 8, MM_MIN_RAW = 3;
 constexpr int MM_SMEM_LIMIT = 232448;             // dynamic shared memory of one CTA
 constexpr uint32_t MM_ACC_COL = 0, MM_A_COL = 256;  // TMEM columns: accumulators, A slots
 
 struct MoeMmaParams {
     int n, k, nk;                 // weight rows, K, super-blocks per row
     int n_row_tiles;              // ceil(n / 128)
-    int raw_slots;
+    int raw_slots;                // ring slots, each spb super-blocks of the unit's 128 rows
+    int spb;
     int x_div;                    // pair p reads activation row p / x_div
     int n_pairs, n_experts;
     const int32_t *perm, *offsets;
@@ -70,21 +76,23 @@ struct MoeMmaParams {
     const int32_t *n_tiles;
     void *y;
     unsigned int *err;
+    int glu, act;                 // fused GLU: each unit runs the gate stack, then the up stack
+    int dense_m;                  // > 0: no grouping, activation rows 0..dense_m-1 of one matrix
 };
 
 // Shared-memory layout, bytes from the 1024-aligned base.
 struct MmLayout {
     int x, raw, s, pairs, bars, total;
 };
-__host__ __device__ inline MmLayout mm_layout(int k, int raw_slots) {
+__host__ __device__ inline MmLayout mm_layout(int k, int raw_slots, int spb) {
     MmLayout l;
     int off = 0;
     l.x = off;     off += 32 * k;                           // 16 rows x K bf16, 64-K atoms of 2 KB
-    l.raw = off;   off += raw_slots * MM_RAW_BYTES;
+    l.raw = off;   off += raw_slots * spb * MM_RAW_BYTES;
     l.s = off;     off += 2 * (k / 32) * MM_BN * 4;         // two tiles' sub-block sums [K/32][16]
     l.pairs = off; off += 2 * MM_BN * 4 + 2 * 4 + 2 * 4;    // pair ids [2][16], counts [2], flags [2]
     off = (off + 7) / 8 * 8;
-    l.bars = off;  off += (2 * raw_slots + 7) * 8 + 8;      // barriers and the TMEM address
+    l.bars = off;  off += (2 * raw_slots + 9) * 8 + 8;      // barriers and the TMEM address
     l.total = off + 1024;                                   // alignment slack
     return l;
 }
@@ -114,11 +122,12 @@ __device__ __forceinline__ const uint8_t *x_chunk(const uint8_t *xt, int t, int 
 template <typename YT>
 __global__ void __launch_bounds__(MM_THREADS, 1)
     moe_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                   const MoeMmaParams p) {
+                   const __grid_constant__ CUtensorMap tmap_w2, const MoeMmaParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
-    const MmLayout lay = mm_layout(p.k, p.raw_slots);
-    const int R = p.raw_slots;
+    const MmLayout lay = mm_layout(p.k, p.raw_slots, p.spb);
+    const int R = p.raw_slots, SPB = p.spb;
+    const int slot_bytes = SPB * MM_RAW_BYTES;
     uint8_t *x_tile = smem + lay.x;
     uint8_t *raw = smem + lay.raw;
     float *s_sum = reinterpret_cast<float *>(smem + lay.s);          // [2][K/32][16]
@@ -127,11 +136,12 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
     int *s_nf = s_ntok + 2;                                          // [2] non-finite activations
     uint64_t *raw_full = reinterpret_cast<uint64_t *>(smem + lay.bars);
     uint64_t *raw_empty = raw_full + R;
-    uint64_t *a_full = raw_empty + R;      // [2] row warps -> MMA: codes in the A slot
-    uint64_t *mma_done = a_full + 2;       // [2] MMA -> row warps: accumulators ready, A slot free
-    uint64_t *x_full = mma_done + 2;       // loader -> all: the token tile's activations
-    uint64_t *x_empty = x_full + 1;        // MMA -> loader: the tile's MMAs are done
-    uint64_t *s_ready = x_empty + 1;       // row warps: the tile's sub-block sums written
+    uint64_t *a_full = raw_empty + R;      // [2] decoders -> MMA: codes in the A slot
+    uint64_t *mma_done = a_full + 2;       // [2] MMA -> epilogue and decoders: accumulators ready, A slot free
+    uint64_t *acc_empty = mma_done + 2;    // [2] epilogue -> MMA: the accumulators are read
+    uint64_t *x_full = acc_empty + 2;      // loader -> all: the token tile's activations
+    uint64_t *x_empty = x_full + 1;        // MMA and epilogue -> loader: done with the tile
+    uint64_t *s_ready = x_empty + 1;       // epilogue warps: the tile's sub-block sums written
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(s_ready + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if ((uint32_t)(smem - smem_raw) + (uint32_t)lay.total - 1024u > dynamic_smem_size()) {
@@ -141,14 +151,15 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int r = 0; r < R; ++r) {
             mbar_init(&raw_full[r], 1);
-            mbar_init(&raw_empty[r], 4);
+            mbar_init(&raw_empty[r], 12);   // 8 decode warps, 4 epilogue warps
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&a_full[b], 4);
+            mbar_init(&a_full[b], 8);
             mbar_init(&mma_done[b], 1);
+            mbar_init(&acc_empty[b], 4);
         }
         mbar_init(x_full, 1);
-        mbar_init(x_empty, 1);
+        mbar_init(x_empty, 5);              // the MMA commit and the 4 epilogue warps
         mbar_init(s_ready, 4);
         fence_mbar_init();
     }
@@ -156,6 +167,7 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
     if (warp == MM_RAW_WARP && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+        if (p.glu) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w2)) : "memory");
     }
     tc_fence_before();
     __syncthreads();
@@ -164,12 +176,20 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
     griddep_wait();   // the grouping and the tile list come from the preceding kernels
 
     const int nrt = p.n_row_tiles, nk = p.nk;
-    const int total = *p.n_tiles * nrt;
+    const int ns = p.glu ? 2 * nk : nk;   // stages per unit (GLU: gate stages, then up stages)
+    const int n_tok_tiles = p.dense_m > 0 ? (p.dense_m + MM_BN - 1) / MM_BN : *p.n_tiles;
+    const int total = n_tok_tiles * nrt;
     const int u0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
     const int u1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
     // Token tile -> (expert, first position in perm, pairs); KQ_DEBUG: a tile
     // outside the grouping becomes an empty tile of expert 0.
     auto tile_info = [&](int tile, int &e, int &m0, int &rows) {
+        if (p.dense_m > 0) {
+            e = 0;
+            m0 = tile * MM_BN;
+            rows = min(MM_BN, p.dense_m - m0);
+            return;
+        }
         const int2 tt = p.tiles[tile];
         const bool ok = KQ_DCHECK(tt.x >= 0 && tt.x < p.n_experts && tt.y >= 0 && tt.y < p.n_pairs &&
                                       p.offsets[tt.x + 1] <= p.n_pairs, p.err);
@@ -187,12 +207,17 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                 int e, m0, rows;
                 tile_info(u / nrt, e, m0, rows);
                 const int n0 = (u % nrt) * MM_BM;
-                for (int s = 0; s < nk; ++s, ++g) {
-                    const uint32_t slot = g % (uint32_t)R, ph = (g / (uint32_t)R) & 1u;
-                    ok = mbar_wait(&raw_empty[slot], ph ^ 1u, p.err);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&raw_full[slot], MM_RAW_BYTES);
-                    tma_load_3d(raw + slot * MM_RAW_BYTES, &tmap_w, s * MM_SB, n0, e, &raw_full[slot]);
+                // one ring slot per spb super-blocks of a matrix (the GLU's
+                // gate and up stacks fill separate slots)
+                for (int mat = 0; mat < ns / nk && ok; ++mat) {
+                    for (int sb0 = 0; sb0 < nk; sb0 += SPB, ++g) {
+                        const uint32_t slot = g % (uint32_t)R, ph = (g / (uint32_t)R) & 1u;
+                        ok = mbar_wait(&raw_empty[slot], ph ^ 1u, p.err);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(&raw_full[slot], (uint32_t)slot_bytes);
+                        tma_load_4d(raw + slot * slot_bytes, mat == 0 ? &tmap_w : &tmap_w2, 0, sb0, n0, e,
+                                    &raw_full[slot]);
+                    }
                 }
             }
         }
@@ -222,7 +247,7 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                 for (int i = 0; i < MM_BN; ++i) {
                     int pr = -1;
                     if (i < rows) {
-                        pr = p.perm[m0 + i];
+                        pr = p.dense_m > 0 ? m0 + i : p.perm[m0 + i];
                         if (!KQ_DCHECK(pr >= 0 && pr < p.n_pairs, p.err)) pr = -1;
                     }
                     if (i == 0 && pr >= 0) first = pr;
@@ -260,14 +285,15 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                     prev = tile;
                     ++xt;
                 }
-                for (int s = 0; s < nk; ++s, ++g) {
+                for (int s = 0; s < ns; ++s, ++g) {
                     const uint32_t b = g & 1u;
-                    ok = mbar_wait(&a_full[b], (g >> 1) & 1u, p.err);
+                    ok = mbar_wait(&acc_empty[b], ((g >> 1) & 1u) ^ 1u, p.err) &&
+                         mbar_wait(&a_full[b], (g >> 1) & 1u, p.err);
                     if (!ok) break;
                     tc_fence_after();
                     #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const int kidx = 256 * s + 32 * j;     // first K of the sub-block
+                        const int kidx = 256 * (s % nk) + 32 * j;     // first K of the sub-block
                         const uint64_t bd = xdesc0 + (uint64_t)((kidx >> 6) * (2048 >> 4) + ((kidx & 63) >> 3));
                         const uint32_t d = tmem_base + MM_ACC_COL + b * 128u + 16u * j;
                         const uint32_t a = tmem_base + MM_A_COL + b * 128u + 16u * j;
@@ -278,31 +304,27 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                 }
             }
         }
-    } else if (warp >= MM_ROW_WARP0) {
-        // ---------------- row warps ----------------
+    } else if (warp >= MM_EPI_WARP0 && warp < MM_EPI_WARP0 + 4) {
+        // ---------------- epilogue warps ----------------
         // Lane l of warp 4+q owns weight row 32q + l of the unit (TMEM lane
-        // 32q + l).  Per stage: codes of the row's super-block into the A
-        // slot, then the scales applied to the previous stage's
-        // accumulators.  Per token tile: the sub-block sums S of its
-        // activations (thread i of the 128 takes sums i, i + 128, ...).
-        const int q = warp & 3, r = 32 * q + lane, ti = threadIdx.x - 32 * MM_ROW_WARP0;
+        // 32q + l).  Per token tile: the sub-block sums S of its activations
+        // (thread i of the 128 takes sums i, i + 128, ...).  Per stage: the
+        // row's scales from the raw slot, applied to the eight sub-block
+        // accumulators once the stage's MMAs are done; then the accumulator
+        // and the raw slot are released.
+        const int q = warp & 3, r = 32 * q + lane, ti = threadIdx.x - 32 * MM_EPI_WARP0;
         const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16);
         const int nsub = p.k / 32;
         YT *y = static_cast<YT *>(p.y);
-        uint32_t g = 0;
+        uint32_t g = 0, L = 0;   // stages and raw ring slots consumed
         int xt = 0, prev = -1, buf = 0, ntok = 0;
         bool nf = false;
         bool ok = true;
-        float acc[MM_BN];
-        float ap[8], cp[8];   // the previous stage's d*sc and 128*d*sc + dmin*m
-        // Scales of the previous stage applied to its accumulators (stage
-        // index sp within the unit, global stage gp).
-        auto epilogue = [&](uint32_t gp, int sp) -> bool {
-            const uint32_t b = gp & 1u;
-            if (!__all_sync(0xffffffffu, mbar_wait(&mma_done[b], (gp >> 1) & 1u, p.err))) return false;
-            tc_fence_after();
-            if (nf) return true;   // the exact path has added this stage already
-            const float *sb = s_sum + (buf * nsub + 8 * sp) * MM_BN;
+        float acc[MM_BN];     // the row's outputs (GLU: the up projection)
+        float accg[MM_BN];    // GLU: the gate projection
+        float a[8], c[8];     // the stage's d*sc_j and 128*d*sc_j + dmin*m_j
+        auto apply = [&](float (&A)[MM_BN], uint32_t b, int sp) {
+            const float *sb = s_sum + (buf * nsub + 8 * (sp % nk)) * MM_BN;
             #pragma unroll
             for (int tg = 0; tg < MM_BN / 4; ++tg) {
                 if (4 * tg >= ntok) break;   // warp-uniform
@@ -311,17 +333,43 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const float4 sv = *reinterpret_cast<const float4 *>(sb + j * MM_BN + 4 * tg);
-                    acc[4 * tg + 0] = fmaf(ap[j], __uint_as_float(dv[4 * j + 0]), fmaf(-cp[j], sv.x, acc[4 * tg + 0]));
-                    acc[4 * tg + 1] = fmaf(ap[j], __uint_as_float(dv[4 * j + 1]), fmaf(-cp[j], sv.y, acc[4 * tg + 1]));
-                    acc[4 * tg + 2] = fmaf(ap[j], __uint_as_float(dv[4 * j + 2]), fmaf(-cp[j], sv.z, acc[4 * tg + 2]));
-                    acc[4 * tg + 3] = fmaf(ap[j], __uint_as_float(dv[4 * j + 3]), fmaf(-cp[j], sv.w, acc[4 * tg + 3]));
+                    A[4 * tg + 0] = fmaf(a[j], __uint_as_float(dv[4 * j + 0]), fmaf(-c[j], sv.x, A[4 * tg + 0]));
+                    A[4 * tg + 1] = fmaf(a[j], __uint_as_float(dv[4 * j + 1]), fmaf(-c[j], sv.y, A[4 * tg + 1]));
+                    A[4 * tg + 2] = fmaf(a[j], __uint_as_float(dv[4 * j + 2]), fmaf(-c[j], sv.z, A[4 * tg + 2]));
+                    A[4 * tg + 3] = fmaf(a[j], __uint_as_float(dv[4 * j + 3]), fmaf(-c[j], sv.w, A[4 * tg + 3]));
                 }
             }
-            return true;
+        };
+        // Exact fp32 (non-finite activations): each decoded weight of the
+        // stage times the activation itself, so infinities and NaNs combine
+        // as IEEE arithmetic does.
+        auto exact = [&](float (&A)[MM_BN], const uint8_t *blk, const float *dm, int sp) {
+            #pragma unroll 1
+            for (int t = 0; t < MM_BN; ++t) {
+                if (t >= ntok) break;
+                float v = 0.f;
+                #pragma unroll 1
+                for (int kk = 0; kk < 256; ++kk) {
+                    const int j = kk >> 5, cc = kk >> 6, l = kk & 31;
+                    const uint32_t byte = blk[16 + 32 * cc + l];
+                    const float qv = (float)((j & 1) ? (byte >> 4) : (byte & 15u));
+                    const int k = 256 * (sp % nk) + kk;
+                    const uint16_t xb = *reinterpret_cast<const uint16_t *>(x_chunk(x_tile, t, k) + 2 * (k & 7));
+                    v = fmaf(fmaf(a[j], qv, -dm[j]), __uint_as_float((uint32_t)xb << 16), v);
+                }
+                #pragma unroll
+                for (int tt = 0; tt < MM_BN; ++tt)
+                    if (tt == t) A[tt] += v;
+            }
         };
         for (int u = u0; u < u1 && ok; ++u) {
             const int tile = u / nrt;
             if (tile != prev) {
+                if (xt > 0) {   // done with the previous tile's activations and pair ids
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(x_empty);
+                }
                 ok = __all_sync(0xffffffffu, mbar_wait(x_full, (uint32_t)xt & 1u, p.err));
                 if (!ok) break;
                 buf = xt & 1;
@@ -331,8 +379,8 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                     const int jg = v >> 4, t = v & 15;
                     float sum = 0.f;
                     #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 w = *reinterpret_cast<const uint4 *>(x_chunk(x_tile, t, 32 * jg + 8 * c));
+                    for (int cq = 0; cq < 4; ++cq) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(x_chunk(x_tile, t, 32 * jg + 8 * cq));
                         sum += ((bf16_lo(w.x) + bf16_hi(w.x)) + (bf16_lo(w.y) + bf16_hi(w.y))) +
                                ((bf16_lo(w.z) + bf16_hi(w.z)) + (bf16_lo(w.w) + bf16_hi(w.w)));
                     }
@@ -340,7 +388,6 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                     bad |= !(fabsf(sum) <= 3.402823466e38f);   // an infinity or NaN in the sub-block
                 }
                 if (__any_sync(0xffffffffu, bad) && lane == 0) s_nf[buf] = 1;
-                fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_ready);
                 ok = __all_sync(0xffffffffu, mbar_wait(s_ready, (uint32_t)xt & 1u, p.err));
@@ -352,28 +399,79 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
             }
             const int row = (u % nrt) * MM_BM + r;
             #pragma unroll
-            for (int t = 0; t < MM_BN; ++t) acc[t] = 0.f;
-            for (int s = 0; s < nk; ++s, ++g) {
-                const uint32_t rs = g % (uint32_t)R, rph = (g / (uint32_t)R) & 1u;
-                ok = __all_sync(0xffffffffu, mbar_wait(&raw_full[rs], rph, p.err));
+            for (int t = 0; t < MM_BN; ++t) acc[t] = accg[t] = 0.f;
+            for (int s = 0; s < ns && ok; ++s, ++g) {
+                const uint32_t rs = L % (uint32_t)R, rph = (L / (uint32_t)R) & 1u, b = g & 1u;
+                const int sb = s % nk;
+                const bool slot_end = (sb % SPB) == SPB - 1 || sb == nk - 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(&raw_full[rs], rph, p.err) &&
+                                                 mbar_wait(&mma_done[b], (g >> 1) & 1u, p.err));
                 if (!ok) break;
-                const uint8_t *blk = raw + rs * MM_RAW_BYTES + r * MM_SB;
+                tc_fence_after();
+                const uint8_t *blk = raw + rs * slot_bytes + (r * SPB + sb % SPB) * MM_SB;
                 const uint4 hd = *reinterpret_cast<const uint4 *>(blk);
                 const float d = half_bits_to_float(hd.x), dmin = half_bits_to_float(hd.x >> 16);
                 const uint32_t sc_lo = hd.y & 0x3F3F3F3Fu, m_lo = hd.z & 0x3F3F3F3Fu;
                 const uint32_t sc_hi = (hd.w & 0x0F0F0F0Fu) | ((hd.y >> 2) & 0x30303030u);
                 const uint32_t m_hi = ((hd.w >> 4) & 0x0F0F0F0Fu) | ((hd.z >> 2) & 0x30303030u);
-                float a[8], dm[8];
+                float dm[8];
                 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     a[j] = d * mm_byte_f(j < 4 ? sc_lo : sc_hi, j & 3);      // exact
                     dm[j] = dmin * mm_byte_f(j < 4 ? m_lo : m_hi, j & 3);    // exact
+                    c[j] = fmaf(128.0f, a[j], dm[j]);
                 }
-                // codes of the stage into A slot g & 1 (free: the MMA of stage
-                // g - 2 is done, waited in its epilogue)
-                const uint32_t acol = MM_A_COL + (g & 1u) * 128u;
+                const bool gate = p.glu && s < nk;
+                if (nf) {
+                    if (gate) exact(accg, blk, dm, s);
+                    else exact(acc, blk, dm, s);
+                } else if (gate) {
+                    apply(accg, b, s);
+                } else {
+                    apply(acc, b, s);
+                }
+                tc_fence_before();
+                fence_proxy_async_smem();   // generic reads of the raw slot before TMA refills it
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&acc_empty[b]);
+                    if (slot_end) mbar_arrive(&raw_empty[rs]);
+                }
+                if (slot_end) ++L;
+            }
+            if (!ok) break;
+            if (row < p.n) {
                 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                for (int t = 0; t < MM_BN; ++t) {
+                    const int pr = s_pair[buf * MM_BN + t];
+                    const float v = p.glu ? glu_activation(accg[t], p.act) * acc[t] : acc[t];
+                    if (t < ntok && pr >= 0) store_out(y + (int64_t)pr * p.n + row, v);
+                }
+            }
+        }
+    } else if (warp >= MM_DEC_WARP0) {
+        // ---------------- decode warps ----------------
+        // Two warps per TMEM lane quadrant: warp 8 + 4h + q writes the codes
+        // of chunks 2h and 2h+1 (128 weights) of row 32q + lane's
+        // super-block into the stage's A slot, once the MMAs that read the
+        // slot two stages ago are done.
+        const int q = warp & 3, r = 32 * q + lane, half = (warp - MM_DEC_WARP0) >> 2;
+        const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16);
+        uint32_t g = 0, L = 0;   // stages and raw ring slots consumed
+        bool ok = true;
+        for (int u = u0; u < u1 && ok; ++u) {
+            for (int s = 0; s < ns; ++s, ++g) {
+                const uint32_t rs = L % (uint32_t)R, rph = (L / (uint32_t)R) & 1u, b = g & 1u;
+                const int sb = s % nk;
+                const bool slot_end = (sb % SPB) == SPB - 1 || sb == nk - 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(&raw_full[rs], rph, p.err) &&
+                                                 (g < 2 || mbar_wait(&mma_done[b], ((g - 2) >> 1) & 1u, p.err)));
+                if (!ok) break;
+                tc_fence_after();
+                const uint8_t *blk = raw + rs * slot_bytes + (r * SPB + sb % SPB) * MM_SB;
+                #pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int cc = 2 * half + c2;
                     const uint4 v0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * cc);
                     const uint4 v1 = *reinterpret_cast<const uint4 *>(blk + 32 + 32 * cc);
                     const uint32_t qw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
@@ -383,55 +481,16 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                         codes4(qw[i] & 0x0F0F0F0Fu, out[2 * i], out[2 * i + 1]);
                         codes4((qw[i] >> 4) & 0x0F0F0F0Fu, out[16 + 2 * i], out[17 + 2 * i]);
                     }
-                    tmem_st32(t_lane + acol + 32u * cc, out);
-                }
-                if (nf) {
-                    // exact fp32: each decoded weight times the activation
-                    // itself, so infinities and NaNs combine as IEEE does
-                    #pragma unroll 1
-                    for (int t = 0; t < MM_BN; ++t) {
-                        if (t >= ntok) break;
-                        float v = 0.f;
-                        #pragma unroll 1
-                        for (int kk = 0; kk < 256; ++kk) {
-                            const int j = kk >> 5, cc = kk >> 6, l = kk & 31;
-                            const uint32_t byte = blk[16 + 32 * cc + l];
-                            const float qv = (float)((j & 1) ? (byte >> 4) : (byte & 15u));
-                            const int k = 256 * s + kk;
-                            const uint16_t xb = *reinterpret_cast<const uint16_t *>(x_chunk(x_tile, t, k) + 2 * (k & 7));
-                            v = fmaf(fmaf(a[j], qv, -dm[j]), __uint_as_float((uint32_t)xb << 16), v);
-                        }
-                        #pragma unroll
-                        for (int tt = 0; tt < MM_BN; ++tt)
-                            if (tt == t) acc[tt] += v;
-                    }
+                    tmem_st32(t_lane + MM_A_COL + b * 128u + 32u * cc, out);
                 }
                 tc_fence_before();
-                fence_proxy_async_smem();   // generic reads of the raw slot and the tile before TMA refills
+                fence_proxy_async_smem();   // generic reads of the raw slot before TMA refills it
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&a_full[g & 1u]);
-                    mbar_arrive(&raw_empty[rs]);
+                    mbar_arrive(&a_full[b]);
+                    if (slot_end) mbar_arrive(&raw_empty[rs]);
                 }
-                if (s > 0) {
-                    ok = epilogue(g - 1, s - 1);
-                    if (!ok) break;
-                }
-                #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    ap[j] = a[j];
-                    cp[j] = fmaf(128.0f, a[j], dm[j]);
-                }
-            }
-            if (!ok) break;
-            ok = epilogue(g - 1, nk - 1);
-            if (!ok) break;
-            if (row < p.n) {
-                #pragma unroll
-                for (int t = 0; t < MM_BN; ++t) {
-                    const int pr = s_pair[buf * MM_BN + t];
-                    if (t < ntok && pr >= 0) store_out(y + (int64_t)pr * p.n + row, acc[t]);
-                }
+                if (slot_end) ++L;
             }
         }
     }
@@ -447,11 +506,35 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
 
 namespace {
 
-// Raw ring depth that fits next to the activation tile and the sums.
-int mm_raw_slots(int64_t k) {
-    int r = MM_MAX_RAW;
-    while (r >= MM_MIN_RAW && mm_layout((int)k, r).total > MM_SMEM_LIMIT) --r;
-    return r;
+// Raw ring: slots of spb super-blocks (the longest contiguous run of each
+// row that still leaves two slots next to the activation tile and the
+// sums; 4, 2 or 1), as many slots as fit, at most four.
+bool mm_ring(int64_t k, int *slots, int *spb) {
+    for (int b = 4; b >= 1; b >>= 1) {
+        if (b > 1 && b > k / 256) continue;
+        int r = 4;
+        while (r >= 2 && mm_layout((int)k, r, b).total > MM_SMEM_LIMIT) --r;
+        if (r >= 2) {
+            *slots = r;
+            *spb = b;
+            return true;
+        }
+    }
+    return false;
+}
+
+// Raw Q4_K rows as (bytes of a super-block, super-blocks, rows, experts):
+// a box of spb super-blocks of 128 rows reads spb * 144 contiguous bytes a row.
+bool encode_w_map4(CUtensorMap *m, const void *w, int64_t n, int64_t k, int64_t n_experts, int64_t expert_stride,
+                   int spb) {
+    const int64_t nk = k / 256;
+    cuuint64_t dims[4] = {(cuuint64_t)MM_SB, (cuuint64_t)nk, (cuuint64_t)n, (cuuint64_t)n_experts};
+    cuuint64_t strides[3] = {(cuuint64_t)MM_SB, (cuuint64_t)(nk * MM_SB), (cuuint64_t)expert_stride};
+    cuuint32_t box[4] = {MM_SB, (cuuint32_t)spb, MM_BM, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(w), dims, strides, box, es,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -460,34 +543,21 @@ bool moe_mma_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype)
     if (type != KQ_Q4_K || x_dtype != KQ_BF16) return false;
     if (y_dtype != KQ_F32 && y_dtype != KQ_BF16) return false;
     if (k % 256 || k > MM_MAX_K || n < 1 || n > (1 << 30)) return false;
-    return mm_raw_slots(k) >= MM_MIN_RAW && encode_fn() != nullptr;
+    int slots, spb;
+    return mm_ring(k, &slots, &spb) && encode_fn() != nullptr;
 }
 
 int moe_mma_bn() { return MM_BN; }
 
-cudaError_t launch_moe_mma(const IdArgs &a, cudaStream_t s) {
-    if (!moe_mma_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype)) return cudaErrorNotSupported;
-    MoeMmaParams p = {};
-    p.n = (int)a.n;
-    p.k = (int)a.k;
-    p.nk = (int)(a.k / 256);
-    p.n_row_tiles = (int)((a.n + MM_BM - 1) / MM_BM);
-    p.raw_slots = mm_raw_slots(a.k);
-    p.x_div = a.x_div();
-    p.n_pairs = (int)(a.n_tokens * a.top_k);
-    p.n_experts = (int)a.n_experts;
-    p.perm = a.perm;
-    p.offsets = a.offsets;
-    p.tiles = reinterpret_cast<const int2 *>(a.tiles);
-    p.n_tiles = a.n_tiles;
-    p.y = a.y;
+namespace {
+
+cudaError_t launch_mm(MoeMmaParams p, const CUtensorMap &tx, const CUtensorMap &tw, const CUtensorMap &tw2,
+                      int y_dtype, cudaStream_t s) {
+    p.nk = p.k / 256;
+    p.n_row_tiles = (p.n + MM_BM - 1) / MM_BM;
     p.err = error_word();
-    CUtensorMap tx, tw;
-    if (!encode_x_map(&tx, a.x, a.x_rows(), a.k, 1) ||
-        !encode_w_map(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride))
-        return cudaErrorInvalidValue;
-    const int smem = mm_layout(p.k, p.raw_slots).total;
-    auto kern = a.y_dtype == KQ_F32 ? moe_mma_kernel<float> : moe_mma_kernel<__nv_bfloat16>;
+    const int smem = mm_layout(p.k, p.raw_slots, p.spb).total;
+    auto kern = y_dtype == KQ_F32 ? moe_mma_kernel<float> : moe_mma_kernel<__nv_bfloat16>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -500,7 +570,52 @@ cudaError_t launch_moe_mma(const IdArgs &a, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+    return cudaLaunchKernelEx(&cfg, kern, tx, tw, tw2, p);
+}
+
+}  // namespace
+
+cudaError_t launch_moe_mma(const IdArgs &a, cudaStream_t s) {
+    if (!moe_mma_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype)) return cudaErrorNotSupported;
+    MoeMmaParams p = {};
+    p.n = (int)a.n;
+    p.k = (int)a.k;
+    p.x_div = a.x_div();
+    p.n_pairs = (int)(a.n_tokens * a.top_k);
+    p.n_experts = (int)a.n_experts;
+    p.perm = a.perm;
+    p.offsets = a.offsets;
+    p.tiles = reinterpret_cast<const int2 *>(a.tiles);
+    p.n_tiles = a.n_tiles;
+    p.y = a.y;
+    p.glu = a.w2 != nullptr;
+    p.act = a.act;
+    mm_ring(a.k, &p.raw_slots, &p.spb);
+    CUtensorMap tx, tw, tw2;
+    if (!encode_x_map(&tx, a.x, a.x_rows(), a.k, 1) ||
+        !encode_w_map4(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride, p.spb) ||
+        !encode_w_map4(&tw2, p.glu ? a.w2 : a.w, a.n, a.k, a.n_experts, a.expert_stride, p.spb))
+        return cudaErrorInvalidValue;
+    return launch_mm(p, tx, tw, tw2, a.y_dtype, s);
+}
+
+cudaError_t launch_gemv_tc(const void *w, int64_t n, int64_t k, const void *x, int64_t m, void *y, int y_dtype,
+                           cudaStream_t s) {
+    if (!moe_mma_supported(KQ_Q4_K, n, k, KQ_BF16, y_dtype) || m < 1 || m > INT32_MAX / 2)
+        return cudaErrorNotSupported;
+    MoeMmaParams p = {};
+    p.n = (int)n;
+    p.k = (int)k;
+    p.x_div = 1;
+    p.n_pairs = (int)m;
+    p.n_experts = 1;
+    p.dense_m = (int)m;
+    p.y = y;
+    mm_ring(k, &p.raw_slots, &p.spb);
+    CUtensorMap tx, tw;
+    if (!encode_x_map(&tx, x, m, k, 1) || !encode_w_map4(&tw, w, n, k, 1, n * (k / 256) * MM_SB, p.spb))
+        return cudaErrorInvalidValue;
+    return launch_mm(p, tx, tw, tw, y_dtype, s);
 }
 
 }  // namespace kq

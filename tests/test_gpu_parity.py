@@ -746,6 +746,25 @@ def test_matmul_id_tensor_core_nonfinite_and_slotted(kq):
     assert kq.device_status() == 0
 
 
+@pytest.mark.parametrize("n,k,m", [(4096, 4096, 1), (1000, 2048, 3), (300, 512, 16), (777, 4096, 21),
+                                   (11008 // 8, 4096, 8)])
+def test_matmul_dense_tensor_core_few_rows(kq, n, k, m):
+    """The few-rows tensor-core kernel on one matrix (tiles of 16 activation
+    rows, a ragged last tile past 16) against the fp64 oracle."""
+    import torch
+
+    r = rng(5 * n + k + m)
+    w = synth.gen_weights(synth.Q4_K, n, k, r)
+    x = synth.gen_x(m, k, "bf16", r)
+    ref = oracle.matmul(synth.Q4_K, w, k, x, threads=8)
+    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    y = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV_TC).cpu().numpy()
+    assert row_rel_err(y, ref) <= GEMV_TOL
+    yb = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV_TC, out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert row_rel_err(yb, ref) <= GEMV_TOL + BF16_OUT
+    assert kq.device_status() == 0
+
+
 def _bf16_weight_reference_id(w, k, x, ids):
     """y[t, s] = x[t] @ bf16(decode_f32(w[ids[t, s]]))^T in fp64 (NaN rows for
     ids outside [0, E)): the tensor-core expert product up to fp32 accumulation."""
