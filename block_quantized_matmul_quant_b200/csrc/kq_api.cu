@@ -162,16 +162,14 @@ static bool id_workspace_layout(int64_t n_tokens, int64_t top_k, int64_t n_exper
 // kernel): 4 rows 20.3 vs 26.9, 8 rows 34.4 vs 26.9; the bandwidth kernel
 // takes 5..8 rows in one pass of eight, so five rows already cost 34.
 constexpr int64_t GEMM_MIN_M = 5;
-// Mean (token, slot) pairs per expert above which the expert-indexed
-// product runs on the tensor cores (each hit expert's weights are then
-// decoded once per token tile of up to 176 pairs); at or below it the
-// bandwidth kernel streams each hit expert's rows once per four pairs.
-// Measured on B200, 64 experts of 1408 x 2048, top-6, bf16 (us per call,
-// bandwidth vs tensor-core kernel): 8 tokens 47 vs 55, 32 tokens 96 vs 84,
-// 64 tokens 147 vs 85, 128 tokens 259 vs 113.
+// Expert-indexed dispatch by mean (token, slot) pairs per expert, from the
+// sweep on B200 (64 experts of 1408 x 2048, top-6, bf16; us per call,
+// bandwidth kernel / few-pairs tensor-core kernel / GEMM): 8 tokens 48.7 /
+// 55.4 / 54.4, 16 tokens 73.8 / 66.9 / 79.0, 32 tokens 98.9 / 81.4 / 84.5,
+// 128 tokens 264.5 / 103.2 / 115.2, 256 tokens 494.2 / 168.5 / 154.7.  Up
+// to one pair per expert the bandwidth kernel, up to twelve the few-pairs
+// kernel (one token tile of 16 per expert), beyond that the GEMM.
 constexpr int64_t ID_GEMV_MAX_PAIRS_PER_EXPERT = 1;
-// Mean pairs per expert up to which the few-pairs tensor-core kernel runs
-// (one token tile of 16 pairs per expert covers them).
 constexpr int64_t ID_TC_MAX_PAIRS_PER_EXPERT = 12;
 // The TQ1 bandwidth kernel takes two activation rows per pass over the
 // weights; beyond this many rows the plain kernel is used.
@@ -321,8 +319,10 @@ static int id_product(const IdArgs &a, int path, int64_t pairs, cudaStream_t s) 
     const bool can_gemm = gemm_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
     const bool can_tc = moe_mma_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
     if (path == KQ_PATH_AUTO) {
-        if (can_tc && pairs <= ID_TC_MAX_PAIRS_PER_EXPERT * a.n_experts) path = KQ_PATH_GEMV_TC;
-        else if (can_gemm && (!can_gemv || pairs > ID_GEMV_MAX_PAIRS_PER_EXPERT * a.n_experts)) path = KQ_PATH_GEMM;
+        if (can_gemv && (pairs <= ID_GEMV_MAX_PAIRS_PER_EXPERT * a.n_experts || !(can_tc || can_gemm)))
+            path = KQ_PATH_GEMV;
+        else if (can_tc && pairs <= ID_TC_MAX_PAIRS_PER_EXPERT * a.n_experts) path = KQ_PATH_GEMV_TC;
+        else if (can_gemm) path = KQ_PATH_GEMM;
         else path = can_gemv ? KQ_PATH_GEMV : KQ_PATH_SIMPLE;
     }
     if (path == KQ_PATH_GEMM && !can_gemm) return KQ_ERR_UNSUPPORTED;

@@ -256,12 +256,16 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                 }
                 s_ntok[buf] = rows;
                 s_nf[buf] = 0;
-                mbar_arrive_expect_tx(x_full, (uint32_t)(MM_BN * p.k * 2));
+                // only the four-row groups that hold pairs: the MMA columns of
+                // the other rows are never read
+                const int groups = rows > 0 ? (rows + 3) / 4 : 1;
+                mbar_arrive_expect_tx(x_full, (uint32_t)(groups * 4 * 128 * (p.k / 64)));
                 for (int a = 0; a < p.k / 64; ++a)
                     #pragma unroll
                     for (int i = 0; i < MM_BN; i += 4)
-                        tma_gather4(x_tile + a * 2048 + i * 128, &tmap_x, a * 64, xr[i], xr[i + 1], xr[i + 2],
-                                    xr[i + 3], x_full);
+                        if (i < 4 * groups)
+                            tma_gather4(x_tile + a * 2048 + i * 128, &tmap_x, a * 64, xr[i], xr[i + 1], xr[i + 2],
+                                        xr[i + 3], x_full);
                 ++xt;
             }
         }
@@ -373,10 +377,12 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                 ok = __all_sync(0xffffffffu, mbar_wait(x_full, (uint32_t)xt & 1u, p.err));
                 if (!ok) break;
                 buf = xt & 1;
+                ntok = s_ntok[buf];
                 float *sb = s_sum + buf * nsub * MM_BN;
                 bool bad = false;
                 for (int v = ti; v < nsub * MM_BN; v += 128) {
                     const int jg = v >> 4, t = v & 15;
+                    if (t >= ntok) continue;   // rows not loaded
                     float sum = 0.f;
                     #pragma unroll
                     for (int cq = 0; cq < 4; ++cq) {
@@ -392,7 +398,6 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                 if (lane == 0) mbar_arrive(s_ready);
                 ok = __all_sync(0xffffffffu, mbar_wait(s_ready, (uint32_t)xt & 1u, p.err));
                 if (!ok) break;
-                ntok = s_ntok[buf];
                 nf = s_nf[buf] != 0;
                 prev = tile;
                 ++xt;
