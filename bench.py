@@ -518,7 +518,7 @@ def run_gpu(args):
     value = job_throughput(step.step_units(), args.steps, world, ms) / 1e9
     launch_us = ms * 1e3 / (args.steps * step.launches)
     achieved = step.algo_bytes_per_launch / (launch_us * 1e-6) / 1e9
-    traffic = measured_traffic("gemv_q4k_4096x4096", ["kq_gemv.cu", "kq_ptx.cuh", "kq_common.cuh"])
+    traffic = measured_traffic("gemv_q4k_4096x4096", ["kq_gemv.cu", "kq_ptx.cuh", "kq_common.cuh", "kq_decode.cuh"])
     out = {
         "metric": "Q4_K GEMV weight GB/s",
         "value": round(value, 2),

@@ -218,13 +218,17 @@ int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, i
     const bool can_gemv = gemv_supported(type, n, k, x_dtype, m);
     if (path == KQ_PATH_AUTO) {
         if (can_gemm && m >= GEMM_MIN_M) path = KQ_PATH_GEMM;
+        // fp32 activations past one pass of the bandwidth kernel: the
+        // few-rows tensor-core kernel reads the weights once per 8 rows of a
+        // tile instead of once per 8-row launch
+        else if (can_tc && x_dtype == KQ_F32 && m > 8) path = KQ_PATH_GEMV_TC;
         else if (can_gemv && (type != KQ_TQ1_G128 || m <= TQ1_GEMV_MAX_M)) path = KQ_PATH_GEMV;
         else path = KQ_PATH_SIMPLE;
     }
     switch (path) {
     case KQ_PATH_GEMV_TC:
         if (!can_tc) return KQ_ERR_UNSUPPORTED;
-        return to_status(launch_gemv_tc(w, n, k, x, m, y, y_dtype, s));
+        return to_status(launch_gemv_tc(w, n, k, x, x_dtype, m, y, y_dtype, s));
     case KQ_PATH_GEMM:
         if (!can_gemm) return KQ_ERR_UNSUPPORTED;
         return to_status(launch_gemm(type, w, n, k, x, m, y, y_dtype, s));
@@ -321,7 +325,7 @@ static int id_product(const IdArgs &a, int path, int64_t pairs, cudaStream_t s) 
     if (path == KQ_PATH_AUTO) {
         if (can_gemv && (pairs <= ID_GEMV_MAX_PAIRS_PER_EXPERT * a.n_experts || !(can_tc || can_gemm)))
             path = KQ_PATH_GEMV;
-        else if (can_tc && pairs <= ID_TC_MAX_PAIRS_PER_EXPERT * a.n_experts) path = KQ_PATH_GEMV_TC;
+        else if (can_tc && (pairs <= ID_TC_MAX_PAIRS_PER_EXPERT * a.n_experts || !can_gemm)) path = KQ_PATH_GEMV_TC;
         else if (can_gemm) path = KQ_PATH_GEMM;
         else path = can_gemv ? KQ_PATH_GEMV : KQ_PATH_SIMPLE;
     }
@@ -331,7 +335,7 @@ static int id_product(const IdArgs &a, int path, int64_t pairs, cudaStream_t s) 
     const int64_t max_tiles = id_max_tiles(pairs, a.n_experts);
     cudaError_t e;
     if (path == KQ_PATH_GEMM || path == KQ_PATH_GEMV_TC) {
-        const int bn = path == KQ_PATH_GEMM ? gemm_id_bn(a.n_tokens, a.top_k, a.n_experts) : moe_mma_bn();
+        const int bn = path == KQ_PATH_GEMM ? gemm_id_bn(a.n_tokens, a.top_k, a.n_experts) : moe_mma_bn(a.x_dtype);
         e = launch_moe_tiles(a.offsets, a.n_experts, bn, const_cast<int32_t *>(a.tiles),
                              const_cast<int32_t *>(a.n_tiles), max_tiles, s);
         if (e == cudaSuccess) e = path == KQ_PATH_GEMM ? launch_gemm_id(a, bn, s) : launch_moe_mma(a, s);
@@ -383,10 +387,12 @@ int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_e
                                      const_cast<int32_t *>(a.offsets),
                                      const_cast<int32_t *>(a.perm), y, y_dtype, n, s);
     if (e != cudaSuccess) return KQ_ERR_CUDA;
-    // bf16 activations: the tensor-core kernel (gate and up passes per unit);
-    // otherwise the bandwidth kernel, or the plain one for other codecs
-    if (moe_mma_supported(type, n, k, x_dtype, y_dtype)) {
-        e = launch_moe_tiles(a.offsets, n_experts, moe_mma_bn(), const_cast<int32_t *>(a.tiles),
+    // Q4_K: up to one pair per expert the bandwidth kernel, beyond it the
+    // tensor-core kernel (a gate pass and an up pass per unit); other codecs
+    // the plain kernel
+    const bool few = pairs <= ID_GEMV_MAX_PAIRS_PER_EXPERT * n_experts;
+    if (moe_mma_supported(type, n, k, x_dtype, y_dtype) && !(few && moe_gemv_supported(type, n, k, n_experts))) {
+        e = launch_moe_tiles(a.offsets, n_experts, moe_mma_bn(x_dtype), const_cast<int32_t *>(a.tiles),
                              const_cast<int32_t *>(a.n_tiles), id_max_tiles(pairs, n_experts), s);
         return to_status(e == cudaSuccess ? launch_moe_mma(a, s) : e);
     }

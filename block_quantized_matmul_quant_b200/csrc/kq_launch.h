@@ -82,12 +82,13 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
 int gemm_id_bn(int64_t n_tokens, int64_t top_k, int64_t n_experts);
 cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s);
 // Expert-indexed tensor-core kernel for few pairs per expert
-// (kq_moe_mma.cu), over token tiles of moe_mma_bn() pairs.
+// (kq_moe_mma.cu), over token tiles of moe_mma_bn(x_dtype) pairs.
 bool moe_mma_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype);
-int moe_mma_bn();
+int moe_mma_bn(int x_dtype);
 cudaError_t launch_moe_mma(const IdArgs &a, cudaStream_t s);   // a.w2 set: fused GLU
-// The same kernel on one matrix and m activation rows (tiles of 16 rows).
-cudaError_t launch_gemv_tc(const void *w, int64_t n, int64_t k, const void *x, int64_t m, void *y, int y_dtype,
-                           cudaStream_t s);
+// The same kernel on one matrix and m activation rows (tiles of
+// moe_mma_bn(x_dtype) rows).
+cudaError_t launch_gemv_tc(const void *w, int64_t n, int64_t k, const void *x, int x_dtype, int64_t m, void *y,
+                           int y_dtype, cudaStream_t s);
 
 }  // namespace kq

@@ -78,6 +78,9 @@ struct MoeMmaParams {
     unsigned int *err;
     int glu, act;                 // fused GLU: each unit runs the gate stack, then the up stack
     int dense_m;                  // > 0: no grouping, activation rows 0..dense_m-1 of one matrix
+    const void *x;                // activations [rows][k], bf16 or (x32) fp32
+    int x32;                      // fp32 activations: two MMA rows per token (bf16 high and low parts)
+    int tpt;                      // tokens per tile: 16, or 8 with fp32 activations
 };
 
 // Shared-memory layout, bytes from the 1024-aligned base.
@@ -90,7 +93,7 @@ __host__ __device__ inline MmLayout mm_layout(int k, int raw_slots, int spb) {
     l.x = off;     off += 32 * k;                           // 16 rows x K bf16, 64-K atoms of 2 KB
     l.raw = off;   off += raw_slots * spb * MM_RAW_BYTES;
     l.s = off;     off += 2 * (k / 32) * MM_BN * 4;         // two tiles' sub-block sums [K/32][16]
-    l.pairs = off; off += 2 * MM_BN * 4 + 2 * 4 + 2 * 4;    // pair ids [2][16], counts [2], flags [2]
+    l.pairs = off; off += 4 * MM_BN * 4 + 2 * 4 + 2 * 4;    // pair ids and x rows [2][16] each, counts [2], flags [2]
     off = (off + 7) / 8 * 8;
     l.bars = off;  off += (2 * raw_slots + 9) * 8 + 8;      // barriers and the TMEM address
     l.total = off + 1024;                                   // alignment slack
@@ -112,8 +115,9 @@ __device__ __forceinline__ float mm_byte_f(uint32_t w, int i) {
 }
 
 // Activation (row t, column k) of the swizzled tile: 64-column atoms of 16
-// rows x 128 bytes; 16-byte chunk c of row t sits at chunk c ^ (t & 7).
-__device__ __forceinline__ const uint8_t *x_chunk(const uint8_t *xt, int t, int k) {
+// rows x 128 bytes; 16-byte chunk c of row t sits at chunk c ^ (t & 7) (the
+// layout the MMA's 128-byte-swizzle descriptor reads).
+__device__ __forceinline__ uint8_t *x_tile_w(uint8_t *xt, int t, int k) {
     return xt + (k >> 6) * 2048 + t * 128 + ((((k & 63) >> 3) ^ (t & 7)) << 4);
 }
 
@@ -121,8 +125,8 @@ __device__ __forceinline__ const uint8_t *x_chunk(const uint8_t *xt, int t, int 
 
 template <typename YT>
 __global__ void __launch_bounds__(MM_THREADS, 1)
-    moe_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                   const __grid_constant__ CUtensorMap tmap_w2, const MoeMmaParams p) {
+    moe_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_w2,
+                   const MoeMmaParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     const MmLayout lay = mm_layout(p.k, p.raw_slots, p.spb);
@@ -131,18 +135,19 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
     uint8_t *x_tile = smem + lay.x;
     uint8_t *raw = smem + lay.raw;
     float *s_sum = reinterpret_cast<float *>(smem + lay.s);          // [2][K/32][16]
-    int *s_pair = reinterpret_cast<int *>(smem + lay.pairs);         // [2][16]
-    int *s_ntok = s_pair + 2 * MM_BN;                                // [2]
+    int *s_pair = reinterpret_cast<int *>(smem + lay.pairs);         // [2][16] output row (pair) per token
+    int *s_xrow = s_pair + 2 * MM_BN;                                // [2][16] activation row per token
+    int *s_ntok = s_xrow + 2 * MM_BN;                                // [2]
     int *s_nf = s_ntok + 2;                                          // [2] non-finite activations
     uint64_t *raw_full = reinterpret_cast<uint64_t *>(smem + lay.bars);
     uint64_t *raw_empty = raw_full + R;
     uint64_t *a_full = raw_empty + R;      // [2] decoders -> MMA: codes in the A slot
     uint64_t *mma_done = a_full + 2;       // [2] MMA -> epilogue and decoders: accumulators ready, A slot free
     uint64_t *acc_empty = mma_done + 2;    // [2] epilogue -> MMA: the accumulators are read
-    uint64_t *x_full = acc_empty + 2;      // loader -> all: the token tile's activations
+    uint64_t *x_full = acc_empty + 2;      // epilogue warps -> MMA, themselves: tile and sums written
     uint64_t *x_empty = x_full + 1;        // MMA and epilogue -> loader: done with the tile
-    uint64_t *s_ready = x_empty + 1;       // epilogue warps: the tile's sub-block sums written
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(s_ready + 1);
+    uint64_t *x_meta = x_empty + 1;        // loader -> epilogue warps: the tile's pair list
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(x_meta + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if ((uint32_t)(smem - smem_raw) + (uint32_t)lay.total - 1024u > dynamic_smem_size()) {
         if (threadIdx.x == 0) atomicOr(p.err, ERR_BOUNDS);   // the host planned another layout: no work
@@ -158,14 +163,13 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
             mbar_init(&mma_done[b], 1);
             mbar_init(&acc_empty[b], 4);
         }
-        mbar_init(x_full, 1);
+        mbar_init(x_full, 4);               // the 4 epilogue warps
         mbar_init(x_empty, 5);              // the MMA commit and the 4 epilogue warps
-        mbar_init(s_ready, 4);
+        mbar_init(x_meta, 1);
         fence_mbar_init();
     }
     if (warp == MM_MMA_WARP) tmem_alloc(tmem_slot, 512);
     if (warp == MM_RAW_WARP && lane == 0) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
         if (p.glu) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w2)) : "memory");
     }
@@ -177,7 +181,8 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
 
     const int nrt = p.n_row_tiles, nk = p.nk;
     const int ns = p.glu ? 2 * nk : nk;   // stages per unit (GLU: gate stages, then up stages)
-    const int n_tok_tiles = p.dense_m > 0 ? (p.dense_m + MM_BN - 1) / MM_BN : *p.n_tiles;
+    const int tpt = p.tpt;
+    const int n_tok_tiles = p.dense_m > 0 ? (p.dense_m + tpt - 1) / tpt : *p.n_tiles;
     const int total = n_tok_tiles * nrt;
     const int u0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
     const int u1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
@@ -186,8 +191,8 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
     auto tile_info = [&](int tile, int &e, int &m0, int &rows) {
         if (p.dense_m > 0) {
             e = 0;
-            m0 = tile * MM_BN;
-            rows = min(MM_BN, p.dense_m - m0);
+            m0 = tile * tpt;
+            rows = min(tpt, p.dense_m - m0);
             return;
         }
         const int2 tt = p.tiles[tile];
@@ -195,7 +200,7 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                                       p.offsets[tt.x + 1] <= p.n_pairs, p.err);
         e = ok ? tt.x : 0;
         m0 = ok ? tt.y : 0;
-        rows = ok ? min(MM_BN, p.offsets[tt.x + 1] - tt.y) : 0;
+        rows = ok ? min(tpt, p.offsets[tt.x + 1] - tt.y) : 0;
     };
 
     if (warp == MM_RAW_WARP) {
@@ -222,11 +227,10 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
             }
         }
     } else if (warp == MM_X_WARP) {
-        // ---------------- activation loader ----------------
+        // ---------------- pair list ----------------
         // When the token tile changes: wait until the previous tile's MMAs
-        // are done, publish the tile's pair ids, gather its 16 activation
-        // rows (rows past the segment repeat its first row; their outputs
-        // are dropped).
+        // and epilogues are done with the tile, then publish its pair ids
+        // and activation rows for the epilogue warps, which load the tile.
         if (lane == 0) {
             int xt = 0, prev = -1;
             bool ok = true;
@@ -241,31 +245,18 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                 int e, m0, rows;
                 tile_info(tile, e, m0, rows);
                 const int buf = xt & 1;
-                int xr[MM_BN];
-                int first = 0;
-                #pragma unroll
-                for (int i = 0; i < MM_BN; ++i) {
+                for (int i = 0; i < tpt; ++i) {
                     int pr = -1;
                     if (i < rows) {
                         pr = p.dense_m > 0 ? m0 + i : p.perm[m0 + i];
                         if (!KQ_DCHECK(pr >= 0 && pr < p.n_pairs, p.err)) pr = -1;
                     }
-                    if (i == 0 && pr >= 0) first = pr;
                     s_pair[buf * MM_BN + i] = pr;
-                    xr[i] = (pr >= 0 ? pr : first) / p.x_div;
+                    s_xrow[buf * MM_BN + i] = pr >= 0 ? pr / p.x_div : -1;
                 }
                 s_ntok[buf] = rows;
                 s_nf[buf] = 0;
-                // only the four-row groups that hold pairs: the MMA columns of
-                // the other rows are never read
-                const int groups = rows > 0 ? (rows + 3) / 4 : 1;
-                mbar_arrive_expect_tx(x_full, (uint32_t)(groups * 4 * 128 * (p.k / 64)));
-                for (int a = 0; a < p.k / 64; ++a)
-                    #pragma unroll
-                    for (int i = 0; i < MM_BN; i += 4)
-                        if (i < 4 * groups)
-                            tma_gather4(x_tile + a * 2048 + i * 128, &tmap_x, a * 64, xr[i], xr[i + 1], xr[i + 2],
-                                        xr[i + 3], x_full);
+                mbar_arrive(x_meta);
                 ++xt;
             }
         }
@@ -311,8 +302,10 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
     } else if (warp >= MM_EPI_WARP0 && warp < MM_EPI_WARP0 + 4) {
         // ---------------- epilogue warps ----------------
         // Lane l of warp 4+q owns weight row 32q + l of the unit (TMEM lane
-        // 32q + l).  Per token tile: the sub-block sums S of its activations
-        // (thread i of the 128 takes sums i, i + 128, ...).  Per stage: the
+        // 32q + l).  Per token tile: the activations into the swizzled tile
+        // (bf16 as they are; fp32 as a bf16 high row and a bf16 low row per
+        // token) and their exact sub-block sums S (thread i of the 128 takes
+        // (token, sub-block) items i, i + 128, ...).  Per stage: the
         // row's scales from the raw slot, applied to the eight sub-block
         // accumulators once the stage's MMAs are done; then the accumulator
         // and the raw slot are released.
@@ -329,6 +322,24 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
         float a[8], c[8];     // the stage's d*sc_j and 128*d*sc_j + dmin*m_j
         auto apply = [&](float (&A)[MM_BN], uint32_t b, int sp) {
             const float *sb = s_sum + (buf * nsub + 8 * (sp % nk)) * MM_BN;
+            if (p.x32) {
+                // columns 2t and 2t+1: token t's high and low parts
+                #pragma unroll
+                for (int tg = 0; tg < MM_BN / 4; ++tg) {
+                    if (2 * tg >= ntok) break;   // warp-uniform
+                    uint32_t dv[32];
+                    tmem_ld4x8(t_lane + MM_ACC_COL + b * 128u + 4u * tg, dv);
+                    #pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float2 sv = *reinterpret_cast<const float2 *>(sb + j * MM_BN + 2 * tg);
+                        const float d0 = __uint_as_float(dv[4 * j + 0]) + __uint_as_float(dv[4 * j + 1]);
+                        const float d1 = __uint_as_float(dv[4 * j + 2]) + __uint_as_float(dv[4 * j + 3]);
+                        A[2 * tg + 0] = fmaf(a[j], d0, fmaf(-c[j], sv.x, A[2 * tg + 0]));
+                        A[2 * tg + 1] = fmaf(a[j], d1, fmaf(-c[j], sv.y, A[2 * tg + 1]));
+                    }
+                }
+                return;
+            }
             #pragma unroll
             for (int tg = 0; tg < MM_BN / 4; ++tg) {
                 if (4 * tg >= ntok) break;   // warp-uniform
@@ -357,9 +368,12 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                     const int j = kk >> 5, cc = kk >> 6, l = kk & 31;
                     const uint32_t byte = blk[16 + 32 * cc + l];
                     const float qv = (float)((j & 1) ? (byte >> 4) : (byte & 15u));
-                    const int k = 256 * (sp % nk) + kk;
-                    const uint16_t xb = *reinterpret_cast<const uint16_t *>(x_chunk(x_tile, t, k) + 2 * (k & 7));
-                    v = fmaf(fmaf(a[j], qv, -dm[j]), __uint_as_float((uint32_t)xb << 16), v);
+                    const int64_t k = 256 * (sp % nk) + kk;
+                    const int xr = s_xrow[buf * MM_BN + t];
+                    const int64_t xi = (int64_t)(xr < 0 ? 0 : xr) * p.k + k;
+                    const float xv = p.x32 ? static_cast<const float *>(p.x)[xi]
+                                           : __bfloat162float(static_cast<const __nv_bfloat16 *>(p.x)[xi]);
+                    v = fmaf(fmaf(a[j], qv, -dm[j]), xv, v);
                 }
                 #pragma unroll
                 for (int tt = 0; tt < MM_BN; ++tt)
@@ -374,29 +388,64 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(x_empty);
                 }
-                ok = __all_sync(0xffffffffu, mbar_wait(x_full, (uint32_t)xt & 1u, p.err));
+                ok = __all_sync(0xffffffffu, mbar_wait(x_meta, (uint32_t)xt & 1u, p.err));
                 if (!ok) break;
                 buf = xt & 1;
                 ntok = s_ntok[buf];
                 float *sb = s_sum + buf * nsub * MM_BN;
                 bool bad = false;
-                for (int v = ti; v < nsub * MM_BN; v += 128) {
-                    const int jg = v >> 4, t = v & 15;
-                    if (t >= ntok) continue;   // rows not loaded
+                for (int v = ti; v < ntok * nsub; v += 128) {
+                    const int t = v / nsub, jg = v - t * nsub;
+                    const int xr = s_xrow[buf * MM_BN + t];   // -1 only for a pair a KQ_DEBUG check dropped
+                    const int64_t xi = (int64_t)(xr < 0 ? 0 : xr) * p.k + 32 * jg;
+                    float xf[32];
+                    if (p.x32) {
+                        const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(p.x) + xi);
+                        #pragma unroll
+                        for (int c4 = 0; c4 < 8; ++c4) {
+                            const float4 f = src[c4];
+                            xf[4 * c4] = f.x; xf[4 * c4 + 1] = f.y; xf[4 * c4 + 2] = f.z; xf[4 * c4 + 3] = f.w;
+                        }
+                        // rows 2t (bf16 high part) and 2t+1 (bf16 low part)
+                        #pragma unroll
+                        for (int cq = 0; cq < 4; ++cq) {
+                            uint32_t hw[4], lw[4];
+                            #pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                const float x0 = xf[8 * cq + 2 * h], x1 = xf[8 * cq + 2 * h + 1];
+                                const __nv_bfloat162 hi = __floats2bfloat162_rn(x0, x1);
+                                const __nv_bfloat162 lo = __floats2bfloat162_rn(x0 - __low2float(hi), x1 - __high2float(hi));
+                                hw[h] = *reinterpret_cast<const uint32_t *>(&hi);
+                                lw[h] = *reinterpret_cast<const uint32_t *>(&lo);
+                            }
+                            *reinterpret_cast<uint4 *>(x_tile_w(x_tile, 2 * t, 32 * jg + 8 * cq)) =
+                                make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                            *reinterpret_cast<uint4 *>(x_tile_w(x_tile, 2 * t + 1, 32 * jg + 8 * cq)) =
+                                make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                        }
+                    } else {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + xi);
+                        #pragma unroll
+                        for (int cq = 0; cq < 4; ++cq) {
+                            const uint4 w = src[cq];
+                            xf[8 * cq] = bf16_lo(w.x); xf[8 * cq + 1] = bf16_hi(w.x);
+                            xf[8 * cq + 2] = bf16_lo(w.y); xf[8 * cq + 3] = bf16_hi(w.y);
+                            xf[8 * cq + 4] = bf16_lo(w.z); xf[8 * cq + 5] = bf16_hi(w.z);
+                            xf[8 * cq + 6] = bf16_lo(w.w); xf[8 * cq + 7] = bf16_hi(w.w);
+                            *reinterpret_cast<uint4 *>(x_tile_w(x_tile, t, 32 * jg + 8 * cq)) = w;
+                        }
+                    }
                     float sum = 0.f;
                     #pragma unroll
-                    for (int cq = 0; cq < 4; ++cq) {
-                        const uint4 w = *reinterpret_cast<const uint4 *>(x_chunk(x_tile, t, 32 * jg + 8 * cq));
-                        sum += ((bf16_lo(w.x) + bf16_hi(w.x)) + (bf16_lo(w.y) + bf16_hi(w.y))) +
-                               ((bf16_lo(w.z) + bf16_hi(w.z)) + (bf16_lo(w.w) + bf16_hi(w.w)));
-                    }
-                    sb[v] = sum;
+                    for (int i = 0; i < 32; i += 4) sum += (xf[i] + xf[i + 1]) + (xf[i + 2] + xf[i + 3]);
+                    sb[jg * MM_BN + t] = sum;
                     bad |= !(fabsf(sum) <= 3.402823466e38f);   // an infinity or NaN in the sub-block
                 }
                 if (__any_sync(0xffffffffu, bad) && lane == 0) s_nf[buf] = 1;
+                fence_proxy_async_smem();   // the tile's generic writes before the MMA reads them
                 __syncwarp();
-                if (lane == 0) mbar_arrive(s_ready);
-                ok = __all_sync(0xffffffffu, mbar_wait(s_ready, (uint32_t)xt & 1u, p.err));
+                if (lane == 0) mbar_arrive(x_full);
+                ok = __all_sync(0xffffffffu, mbar_wait(x_full, (uint32_t)xt & 1u, p.err));
                 if (!ok) break;
                 nf = s_nf[buf] != 0;
                 prev = tile;
@@ -545,21 +594,24 @@ bool encode_w_map4(CUtensorMap *m, const void *w, int64_t n, int64_t k, int64_t 
 }  // namespace
 
 bool moe_mma_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype) {
-    if (type != KQ_Q4_K || x_dtype != KQ_BF16) return false;
+    if (type != KQ_Q4_K || (x_dtype != KQ_BF16 && x_dtype != KQ_F32)) return false;
     if (y_dtype != KQ_F32 && y_dtype != KQ_BF16) return false;
     if (k % 256 || k > MM_MAX_K || n < 1 || n > (1 << 30)) return false;
     int slots, spb;
     return mm_ring(k, &slots, &spb) && encode_fn() != nullptr;
 }
 
-int moe_mma_bn() { return MM_BN; }
+// Tokens per tile: 16 bf16 activation rows, or 8 fp32 ones (two MMA rows each).
+int moe_mma_bn(int x_dtype) { return x_dtype == KQ_F32 ? MM_BN / 2 : MM_BN; }
 
 namespace {
 
-cudaError_t launch_mm(MoeMmaParams p, const CUtensorMap &tx, const CUtensorMap &tw, const CUtensorMap &tw2,
-                      int y_dtype, cudaStream_t s) {
+cudaError_t launch_mm(MoeMmaParams p, const CUtensorMap &tw, const CUtensorMap &tw2, int x_dtype, int y_dtype,
+                      cudaStream_t s) {
     p.nk = p.k / 256;
     p.n_row_tiles = (p.n + MM_BM - 1) / MM_BM;
+    p.x32 = x_dtype == KQ_F32 ? 1 : 0;
+    p.tpt = moe_mma_bn(x_dtype);
     p.err = error_word();
     const int smem = mm_layout(p.k, p.raw_slots, p.spb).total;
     auto kern = y_dtype == KQ_F32 ? moe_mma_kernel<float> : moe_mma_kernel<__nv_bfloat16>;
@@ -575,7 +627,7 @@ cudaError_t launch_mm(MoeMmaParams p, const CUtensorMap &tx, const CUtensorMap &
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tx, tw, tw2, p);
+    return cudaLaunchKernelEx(&cfg, kern, tw, tw2, p);
 }
 
 }  // namespace
@@ -593,20 +645,20 @@ cudaError_t launch_moe_mma(const IdArgs &a, cudaStream_t s) {
     p.tiles = reinterpret_cast<const int2 *>(a.tiles);
     p.n_tiles = a.n_tiles;
     p.y = a.y;
+    p.x = a.x;
     p.glu = a.w2 != nullptr;
     p.act = a.act;
     mm_ring(a.k, &p.raw_slots, &p.spb);
-    CUtensorMap tx, tw, tw2;
-    if (!encode_x_map(&tx, a.x, a.x_rows(), a.k, 1) ||
-        !encode_w_map4(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride, p.spb) ||
+    CUtensorMap tw, tw2;
+    if (!encode_w_map4(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride, p.spb) ||
         !encode_w_map4(&tw2, p.glu ? a.w2 : a.w, a.n, a.k, a.n_experts, a.expert_stride, p.spb))
         return cudaErrorInvalidValue;
-    return launch_mm(p, tx, tw, tw2, a.y_dtype, s);
+    return launch_mm(p, tw, tw2, a.x_dtype, a.y_dtype, s);
 }
 
-cudaError_t launch_gemv_tc(const void *w, int64_t n, int64_t k, const void *x, int64_t m, void *y, int y_dtype,
-                           cudaStream_t s) {
-    if (!moe_mma_supported(KQ_Q4_K, n, k, KQ_BF16, y_dtype) || m < 1 || m > INT32_MAX / 2)
+cudaError_t launch_gemv_tc(const void *w, int64_t n, int64_t k, const void *x, int x_dtype, int64_t m, void *y,
+                           int y_dtype, cudaStream_t s) {
+    if (!moe_mma_supported(KQ_Q4_K, n, k, x_dtype, y_dtype) || m < 1 || m > INT32_MAX / 2)
         return cudaErrorNotSupported;
     MoeMmaParams p = {};
     p.n = (int)n;
@@ -616,11 +668,11 @@ cudaError_t launch_gemv_tc(const void *w, int64_t n, int64_t k, const void *x, i
     p.n_experts = 1;
     p.dense_m = (int)m;
     p.y = y;
+    p.x = x;
     mm_ring(k, &p.raw_slots, &p.spb);
-    CUtensorMap tx, tw;
-    if (!encode_x_map(&tx, x, m, k, 1) || !encode_w_map4(&tw, w, n, k, 1, n * (k / 256) * MM_SB, p.spb))
-        return cudaErrorInvalidValue;
-    return launch_mm(p, tx, tw, tw, y_dtype, s);
+    CUtensorMap tw;
+    if (!encode_w_map4(&tw, w, n, k, 1, n * (k / 256) * MM_SB, p.spb)) return cudaErrorInvalidValue;
+    return launch_mm(p, tw, tw, x_dtype, y_dtype, s);
 }
 
 }  // namespace kq

@@ -82,7 +82,8 @@ extern "C" {
 #define KQ_PATH_GEMM     3  /* TMA + tcgen05 tensor-core kernel (bf16 x only)         */
 /* Tensor-core kernel for few activation rows / pairs per expert: 4-bit codes
  * through the MMA, one accumulator per 32-weight sub-block, the scales
- * applied after it (Q4_K, bf16 x, K <= 4096, tiles of 16 rows). */
+ * applied after it (Q4_K, K <= 4096; tiles of 16 bf16 activation rows, or 8
+ * fp32 rows each split into a bf16 high and low part). */
 #define KQ_PATH_GEMV_TC  4
 /* Flag OR-ed into `path`: the caller guarantees that no work enqueued earlier
  * on the stream writes the weight bytes (they are constant, as model weights
@@ -228,11 +229,11 @@ KQ_API int kq_matmul_id_noalloc(int type, const void *w, int64_t n_experts, int6
  *                 out as kq_matmul_id's w (device)
  *   act           KQ_ACT_SILU or KQ_ACT_GELU_TANH
  * Other arguments, the workspace (kq_matmul_id_workspace_bytes), invalid
- * ids (NaN rows, device error word) and errors as kq_matmul_id.  Q4_K with
- * bf16 activations runs the few-pairs tensor-core kernel (a gate pass and an
- * up pass per unit over the same activation tile); Q4_K with fp32
- * activations the grouped bandwidth kernel (a tile holding each output row's
- * gate and up weights); other codecs the plain grouped kernel.
+ * ids (NaN rows, device error word) and errors as kq_matmul_id.  Q4_K up to
+ * one routed pair per expert runs the grouped bandwidth kernel (a tile
+ * holding each output row's gate and up weights), beyond it the few-pairs
+ * tensor-core kernel (a gate pass and an up pass per unit over the same
+ * activation tile); other codecs the plain grouped kernel.
  */
 KQ_API int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_experts,
                             int64_t n, int64_t k, int64_t expert_stride, const void *x, int x_dtype,

@@ -682,7 +682,8 @@ def test_moe_ffn_chain_reuses_the_grouping(kq, xdt):
     (7, 3, 4, 129, 4096, False),       # the largest K the kernel takes
     (64, 4, 8, 256, 768, True),        # one expert takes most pairs: many tiles, other experts one
 ])
-def test_matmul_id_tensor_core_few_pairs(kq, t, top_k, e, n, k, skew):
+@pytest.mark.parametrize("xdt", ["bf16", "f32"])
+def test_matmul_id_tensor_core_few_pairs(kq, t, top_k, e, n, k, skew, xdt):
     """The few-pairs tensor-core kernel: codes through the MMA, a sub-block
     accumulator each, scales applied after it -- against the fp64 oracle
     (bf16 activations exact in the MMA), f32 and bf16 outputs, bit-stable,
@@ -691,13 +692,13 @@ def test_matmul_id_tensor_core_few_pairs(kq, t, top_k, e, n, k, skew):
 
     r = rng(11 * t + e + n + k)
     w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
-    x = synth.gen_x(t, k, "bf16", r)
+    x = synth.gen_x(t, k, xdt, r)
     ids = synth.gen_ids(t, top_k, e, r)
     if skew:
         ids[:, 0] = np.where(np.arange(t) % 9 == 0, 1, 2)
     ids[t // 2, top_k - 1] = e                 # outside the stack: a NaN row
     ref = oracle.matmul_id(synth.Q4_K, w, k, x, ids)
-    wd, xd, idd = to_device_w(w), to_device_x(x, "bf16"), torch.from_numpy(ids).cuda()
+    wd, xd, idd = to_device_w(w), to_device_x(x, xdt), torch.from_numpy(ids).cuda()
     y = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMV_TC).cpu().numpy()
     assert np.all(np.isnan(y[t // 2, top_k - 1]))
     good = ~np.isnan(ref[..., 0])
@@ -713,7 +714,8 @@ def test_matmul_id_tensor_core_few_pairs(kq, t, top_k, e, n, k, skew):
     assert kq.device_status() == 0
 
 
-def test_matmul_id_tensor_core_nonfinite_and_slotted(kq):
+@pytest.mark.parametrize("xdt", ["bf16", "f32"])
+def test_matmul_id_tensor_core_nonfinite_and_slotted(kq, xdt):
     """Non-finite activations send their token tile through the exact fp32
     path (IEEE classes as the oracle's); the slotted input of the down
     projection (one activation row per pair) through the same kernel."""
@@ -722,12 +724,12 @@ def test_matmul_id_tensor_core_nonfinite_and_slotted(kq):
     t, top_k, e, n, k = 12, 2, 5, 160, 512
     r = rng(77)
     w = synth.gen_weights(synth.Q4_K, e * n, k, r).reshape(e, n, -1)
-    x = synth.gen_x(t, k, "bf16", r)
+    x = synth.gen_x(t, k, xdt, r)
     ids = synth.gen_ids(t, top_k, e, r)
     x[3, 10] = np.inf
     x[5, 100] = np.nan
     ref = oracle.matmul_id(synth.Q4_K, w, k, x, ids)
-    y = kq.matmul_id(to_device_w(w), synth.Q4_K, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
+    y = kq.matmul_id(to_device_w(w), synth.Q4_K, to_device_x(x, xdt), torch.from_numpy(ids).cuda(),
                      path=kq.PATH_GEMV_TC).cpu().numpy()
     assert np.array_equal(np.isnan(y), np.isnan(ref))
     assert np.array_equal(np.isposinf(y), np.isposinf(ref)) and np.array_equal(np.isneginf(y), np.isneginf(ref))
@@ -736,9 +738,9 @@ def test_matmul_id_tensor_core_nonfinite_and_slotted(kq):
     scale = np.abs(ref[fin]).max()
     assert np.all(np.abs(y[fin] - ref[fin]) <= GEMV_TOL * scale)
     assert kq.device_status() == 0
-    xs = synth.gen_x(t * top_k, k, "bf16", r).reshape(t, top_k, k)
+    xs = synth.gen_x(t * top_k, k, xdt, r).reshape(t, top_k, k)
     scores = r.uniform(0, 1, (t, top_k)).astype(np.float32)
-    ym = kq.matmul_id_mix(to_device_w(w), synth.Q4_K, to_device_x(xs, "bf16"), torch.from_numpy(ids).cuda(),
+    ym = kq.matmul_id_mix(to_device_w(w), synth.Q4_K, to_device_x(xs, xdt), torch.from_numpy(ids).cuda(),
                           torch.from_numpy(scores).cuda(), path=kq.PATH_GEMV_TC).cpu().numpy()
     refm = oracle.mix_id(synth.Q4_K, w, k, xs, ids, scores)
     ok, worst = _mix_err_ok(ym, refm, _pair_refs(synth.Q4_K, w, k, xs, ids), scores, GEMV_TOL)
@@ -748,16 +750,17 @@ def test_matmul_id_tensor_core_nonfinite_and_slotted(kq):
 
 @pytest.mark.parametrize("n,k,m", [(4096, 4096, 1), (1000, 2048, 3), (300, 512, 16), (777, 4096, 21),
                                    (11008 // 8, 4096, 8)])
-def test_matmul_dense_tensor_core_few_rows(kq, n, k, m):
-    """The few-rows tensor-core kernel on one matrix (tiles of 16 activation
-    rows, a ragged last tile past 16) against the fp64 oracle."""
+@pytest.mark.parametrize("xdt", ["bf16", "f32"])
+def test_matmul_dense_tensor_core_few_rows(kq, n, k, m, xdt):
+    """The few-rows tensor-core kernel on one matrix (tiles of 16 bf16 or 8
+    fp32 activation rows, ragged last tiles) against the fp64 oracle."""
     import torch
 
     r = rng(5 * n + k + m)
     w = synth.gen_weights(synth.Q4_K, n, k, r)
-    x = synth.gen_x(m, k, "bf16", r)
+    x = synth.gen_x(m, k, xdt, r)
     ref = oracle.matmul(synth.Q4_K, w, k, x, threads=8)
-    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    wd, xd = to_device_w(w), to_device_x(x, xdt)
     y = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV_TC).cpu().numpy()
     assert row_rel_err(y, ref) <= GEMV_TOL
     yb = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV_TC, out_dtype=torch.bfloat16).float().cpu().numpy()
