@@ -132,9 +132,10 @@ struct IdWorkspace {
     size_t counts, offsets, perm, tiles, n_tiles, total;
 };
 static size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
-// Entries of the tensor-core tile list: tiles of at least 16 pairs, one
-// ragged tile per expert at most.
-static int64_t id_max_tiles(int64_t pairs, int64_t n_experts) { return pairs / 16 + n_experts + 1; }
+// Entries of the tensor-core tile list: tiles of at least 8 pairs (the
+// few-pairs kernel with fp32 activations; 16 and more otherwise), one ragged
+// tile per expert at most.
+static int64_t id_max_tiles(int64_t pairs, int64_t n_experts) { return pairs / 8 + n_experts + 1; }
 // The routing-mix call adds one section after the grouping: the fp32
 // per-pair products [pairs, n].
 static bool mix_workspace_bytes(const struct IdWorkspace &l, int64_t pairs, int64_t n, size_t *total) {

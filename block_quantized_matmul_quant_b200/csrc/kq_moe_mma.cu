@@ -25,23 +25,26 @@
 //    d*sc_j * D_j - (128*d*sc_j + dmin*m_j) * S_j to the row's outputs, S_j
 //    the activations' sum over the sub-block (computed once per token tile).
 //
-// Work units are (token tile of <= 16 pairs of one expert, 128-row tile); a
-// CTA per SM takes a contiguous range of units, so consecutive units share
-// a token tile, whose activations (16 rows x K, 128-byte swizzle, gathered
-// four rows at a time by TMA) stay in shared memory until the tile changes.
-// Raw super-blocks stream through a ring by TMA (3-D map: row bytes, rows,
-// expert).  Warp roles: 0 raw producer, 1 MMA issuer (and TMEM owner), 2
-// activation loader, 4..7 epilogue (warp 4+q reads TMEM lanes 32q..), 8..15
-// decoders (two per lane quadrant, half a super-block each).  Splitting the
-// decode from the epilogue, and the decode over two warps, keeps several
-// warps per scheduler: with one thread doing both per row the stage was
-// latency-bound (about 2 us).  TMEM: accumulators at columns 0 and 128 (8
-// sub-blocks x 16 pairs, two stages in flight), A slots at 256 and 384 (256
-// codes of 128 rows each).  Fused GLU: each unit runs the gate stack's
-// stages, then the up stack's, into two sets of row sums.  Dense mode: one
-// matrix, activation rows in tiles of 16, no grouping.  Every wait is
-// bounded (kq_ptx.cuh); activations that are not finite make the epilogue
-// compute that token tile exactly in fp32 instead.
+// Work units are (token tile of one expert's pairs, 128-row tile); a CTA
+// per SM takes a contiguous range of units, so consecutive units share a
+// token tile, whose activations stay in shared memory (16 MMA rows x K,
+// 128-byte swizzle) until the tile changes.  The epilogue warps fill the
+// tile with plain loads and compute its exact sub-block sums in the same
+// pass: bf16 activations as they are (16 tokens a tile), fp32 ones as a
+// bf16 high row and a bf16 low row per token (8 tokens a tile; the MMA sums
+// both, so the product keeps fp32 accuracy).  Raw super-blocks stream
+// through a ring by TMA (several super-blocks of the tile's 128 rows per
+// slot).  Warp roles: 0 raw producer, 1 MMA issuer (and TMEM owner), 2 pair
+// list, 4..7 epilogue (warp 4+q reads TMEM lanes 32q..), 8..15 decoders
+// (two per lane quadrant, half a super-block each).  TMEM: accumulators at
+// columns 0 and 128 (8 sub-blocks x 16 columns, two stages in flight), A
+// slots at 256 and 384 (256 codes of 128 rows each).  Fused GLU: each unit
+// runs the gate stack's stages, then the up stack's, into two sets of row
+// sums.  Dense mode: one matrix, activation rows in tiles, no grouping.
+// What bounds it (measured): a tcgen05.mma of M = 128, K = 16 costs a fixed
+// ~83 cycles whatever N is, so 16 of them per super-block set the pace.
+// Every wait is bounded (kq_ptx.cuh); activations that are not finite make
+// the epilogue compute that token tile exactly in fp32 instead.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
