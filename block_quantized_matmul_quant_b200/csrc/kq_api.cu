@@ -317,9 +317,10 @@ static int id_setup(int type, const void *w, int64_t n_experts, int64_t n, int64
 }
 }  // namespace kq
 
-// The expert product over a grouping already in the workspace (a.y: its
-// output, a.y_dtype), by `path` (KQ_PATH_AUTO resolved here).
-static int id_product(const IdArgs &a, int path, int64_t pairs, cudaStream_t s) {
+// The expert product's kernel for these arguments (KQ_PATH_AUTO resolved),
+// or a negative status; *bn: the token-tile width its tile list needs (0:
+// none).
+static int id_path(const IdArgs &a, int path, int64_t pairs, int *bn) {
     const bool can_gemv = moe_gemv_supported(a.type, a.n, a.k, a.n_experts);
     const bool can_gemm = gemm_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
     const bool can_tc = moe_mma_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
@@ -333,18 +334,28 @@ static int id_product(const IdArgs &a, int path, int64_t pairs, cudaStream_t s) 
     if (path == KQ_PATH_GEMM && !can_gemm) return KQ_ERR_UNSUPPORTED;
     if (path == KQ_PATH_GEMV && !can_gemv) return KQ_ERR_UNSUPPORTED;
     if (path == KQ_PATH_GEMV_TC && !can_tc) return KQ_ERR_UNSUPPORTED;
-    const int64_t max_tiles = id_max_tiles(pairs, a.n_experts);
+    *bn = path == KQ_PATH_GEMM ? gemm_id_bn(a.n_tokens, a.top_k, a.n_experts)
+        : path == KQ_PATH_GEMV_TC ? moe_mma_bn(a.x_dtype) : 0;
+    return path;
+}
+
+// The grouping (and the tile list when bn > 0) into the workspace; y (or
+// nullptr) takes the NaN rows of invalid ids.
+static cudaError_t id_group(const IdArgs &a, const int32_t *ids, int64_t pairs, void *y, int y_dtype, int bn,
+                            cudaStream_t s) {
+    return launch_moe_group(ids, pairs, a.n_experts, const_cast<int32_t *>(a.counts), const_cast<int32_t *>(a.offsets),
+                            const_cast<int32_t *>(a.perm), y, y_dtype, a.n, s, bn, const_cast<int32_t *>(a.tiles),
+                            const_cast<int32_t *>(a.n_tiles), id_max_tiles(pairs, a.n_experts));
+}
+
+// The expert product over a grouping (and tile list) already in the
+// workspace (a.y: its output, a.y_dtype).
+static int id_product(const IdArgs &a, int path, int bn, cudaStream_t s) {
     cudaError_t e;
-    if (path == KQ_PATH_GEMM || path == KQ_PATH_GEMV_TC) {
-        const int bn = path == KQ_PATH_GEMM ? gemm_id_bn(a.n_tokens, a.top_k, a.n_experts) : moe_mma_bn(a.x_dtype);
-        e = launch_moe_tiles(a.offsets, a.n_experts, bn, const_cast<int32_t *>(a.tiles),
-                             const_cast<int32_t *>(a.n_tiles), max_tiles, s);
-        if (e == cudaSuccess) e = path == KQ_PATH_GEMM ? launch_gemm_id(a, bn, s) : launch_moe_mma(a, s);
-    } else if (path == KQ_PATH_GEMV) {
-        e = launch_moe_gemv(a, s);
-    } else {
-        e = launch_simple_id(a, s);
-    }
+    if (path == KQ_PATH_GEMM) e = launch_gemm_id(a, bn, s);
+    else if (path == KQ_PATH_GEMV_TC) e = launch_moe_mma(a, s);
+    else if (path == KQ_PATH_GEMV) e = launch_moe_gemv(a, s);
+    else e = launch_simple_id(a, s);
     return to_status(e);
 }
 
@@ -361,12 +372,11 @@ int kq_matmul_id_ex(int type, const void *w, int64_t n_experts, int64_t n, int64
     if (st) return st;
     if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMV_TC) return KQ_ERR_ARG;
     if ((st = check_device())) return st;
+    int bn = 0;
+    if ((path = id_path(a, path, pairs, &bn)) < 0) return path;
     cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = launch_moe_group(ids, pairs, n_experts, const_cast<int32_t *>(a.counts),
-                                     const_cast<int32_t *>(a.offsets),
-                                     const_cast<int32_t *>(a.perm), y, y_dtype, n, s);
-    if (e != cudaSuccess) return KQ_ERR_CUDA;
-    return id_product(a, path, pairs, s);
+    if (id_group(a, ids, pairs, y, y_dtype, bn, s) != cudaSuccess) return KQ_ERR_CUDA;
+    return id_product(a, path, bn, s);
 }
 
 int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_experts, int64_t n,
@@ -384,19 +394,13 @@ int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_e
     a.w2 = w_up;
     a.act = act;
     cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = launch_moe_group(ids, pairs, n_experts, const_cast<int32_t *>(a.counts),
-                                     const_cast<int32_t *>(a.offsets),
-                                     const_cast<int32_t *>(a.perm), y, y_dtype, n, s);
-    if (e != cudaSuccess) return KQ_ERR_CUDA;
     // Q4_K: up to one pair per expert the bandwidth kernel, beyond it the
     // tensor-core kernel (a gate pass and an up pass per unit); other codecs
     // the plain kernel
     const bool few = pairs <= ID_GEMV_MAX_PAIRS_PER_EXPERT * n_experts;
-    if (moe_mma_supported(type, n, k, x_dtype, y_dtype) && !(few && moe_gemv_supported(type, n, k, n_experts))) {
-        e = launch_moe_tiles(a.offsets, n_experts, moe_mma_bn(x_dtype), const_cast<int32_t *>(a.tiles),
-                             const_cast<int32_t *>(a.n_tiles), id_max_tiles(pairs, n_experts), s);
-        return to_status(e == cudaSuccess ? launch_moe_mma(a, s) : e);
-    }
+    const bool tc = moe_mma_supported(type, n, k, x_dtype, y_dtype) && !(few && moe_gemv_supported(type, n, k, n_experts));
+    if (id_group(a, ids, pairs, y, y_dtype, tc ? moe_mma_bn(x_dtype) : 0, s) != cudaSuccess) return KQ_ERR_CUDA;
+    if (tc) return to_status(launch_moe_mma(a, s));
     if (moe_gemv_supported(type, n, k, n_experts)) return to_status(launch_moe_gemv(a, s));
     return to_status(launch_simple_glu(a, s));
 }
@@ -416,12 +420,17 @@ int kq_matmul_id_mix(int type, const void *w, int64_t n_experts, int64_t n, int6
     path &= ~KQ_FLAG_REUSE_GROUPING;
     if (path < KQ_PATH_AUTO || path > KQ_PATH_GEMV_TC) return KQ_ERR_ARG;
     if ((st = check_device())) return st;
+    int bn = 0;
+    if ((path = id_path(a, path, pairs, &bn)) < 0) return path;
     cudaStream_t s = (cudaStream_t)stream;
-    if (!reuse &&
-        launch_moe_group(ids, pairs, n_experts, const_cast<int32_t *>(a.counts), const_cast<int32_t *>(a.offsets),
-                         const_cast<int32_t *>(a.perm), nullptr, KQ_F32, n, s) != cudaSuccess)
-        return KQ_ERR_CUDA;
-    if ((st = id_product(a, path, pairs, s))) return st;
+    if (!reuse) {
+        if (id_group(a, ids, pairs, nullptr, KQ_F32, bn, s) != cudaSuccess) return KQ_ERR_CUDA;
+    } else if (bn > 0 &&
+               launch_moe_tiles(a.offsets, n_experts, bn, const_cast<int32_t *>(a.tiles),
+                                const_cast<int32_t *>(a.n_tiles), id_max_tiles(pairs, n_experts), s) != cudaSuccess) {
+        return KQ_ERR_CUDA;   // a reused grouping gets the tile list this product needs
+    }
+    if ((st = id_product(a, path, bn, s))) return st;
     return to_status(launch_moe_mix(static_cast<const float *>(a.y), ids, scores, n_tokens, top_k,
                                     n_experts, n, y, y_dtype, s));
 }

@@ -34,9 +34,13 @@ cudaError_t launch_tq1_scan(const void *w, int64_t blocks, unsigned long long *f
                             cudaStream_t s);
 cudaError_t launch_get_rows(int type, const void *w, int64_t rows, int64_t k, const int32_t *ids,
                             int64_t n_ids, void *out, int dt, cudaStream_t s);
+// Grouping of the (token, slot) pairs by expert; with bn > 0 also the token
+// tiles of at most bn pairs (as launch_moe_tiles).  Programmatic dependent
+// launch: it waits for the preceding kernel before touching memory.
 cudaError_t launch_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_experts,
                              int32_t *counts, int32_t *offsets, int32_t *perm, void *y,
-                             int y_dtype, int64_t n, cudaStream_t s);
+                             int y_dtype, int64_t n, cudaStream_t s, int bn = 0, int32_t *tiles = nullptr,
+                             int32_t *n_tiles = nullptr, int64_t max_tiles = 0);
 cudaError_t launch_simple_id(const IdArgs &a, cudaStream_t s);
 // Plain fused GLU over the grouping (any codec): y = act(x W_gate^T) * (x W_up^T).
 cudaError_t launch_simple_glu(const IdArgs &a, cudaStream_t s);

@@ -9,6 +9,7 @@
 // `quantized_matmul_id_ggml`: invalid routing metadata reads no expert
 // weights and writes a non-finite poison sentinel).
 #include "kq_decode.cuh"
+#include "kq_ptx.cuh"
 #include "kq_launch.h"
 
 namespace kq {
@@ -16,14 +17,19 @@ namespace kq {
 constexpr int GROUP_THREADS = 1024;
 
 // One CTA.  Warp w owns experts w, w + 32, ...; it scans the ids in order,
-// so each expert's pair list comes out ascending.
+// so each expert's pair list comes out ascending.  With bn > 0 it also
+// writes the tensor-core kernels' token tiles: each expert's segment in
+// tiles of at most bn pairs, (expert, first position in perm) each, and
+// their number.  Launched as a programmatic dependent of the preceding
+// kernel: nothing is read or written before that kernel has completed.
 __global__ void __launch_bounds__(GROUP_THREADS) moe_group_kernel(
     const int32_t *__restrict__ ids, int n_pairs, int n_experts, int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets, int32_t *__restrict__ perm, void *y, int y_dtype, int64_t n,
-    unsigned int *err) {
-    extern __shared__ int s_off[];  // n_experts + 1
+    int bn, int2 *__restrict__ tiles, int32_t *__restrict__ n_tiles, int max_tiles, unsigned int *err) {
+    extern __shared__ int s_off[];  // n_experts + 1, then (bn > 0) the first tile of each expert
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     __shared__ int s_bad;
+    griddep_wait();
     if (threadIdx.x == 0) s_bad = 0;
     __syncthreads();
     // validation (+ poison rows)
@@ -89,20 +95,58 @@ __global__ void __launch_bounds__(GROUP_THREADS) moe_group_kernel(
     }
     for (int p = s_off[n_experts] + threadIdx.x; p < n_pairs; p += blockDim.x) perm[p] = -1;
     if (threadIdx.x == 0 && s_bad) atomicOr(err, ERR_BAD_ID);
+    if (bn > 0) {
+        int *s_first = s_off + n_experts + 1;
+        if (warp == 0) {
+            int carry = 0;
+            for (int base = 0; base < n_experts; base += 32) {
+                const int e = base + lane;
+                const int c = e < n_experts ? (s_off[e + 1] - s_off[e] + bn - 1) / bn : 0;
+                int incl = c;
+                #pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                if (e < n_experts) s_first[e] = carry + incl - c;
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) *n_tiles = KQ_DCHECK(carry <= max_tiles, err) ? carry : max_tiles;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < n_experts; e += blockDim.x) {
+            const int p0 = s_off[e], p1 = s_off[e + 1];
+            int i = s_first[e];
+            for (int q = p0; q < p1; q += bn, ++i)
+                if (KQ_DCHECK(i < max_tiles, err)) tiles[i] = make_int2(e, q);
+        }
+    }
+    griddep_launch_dependents();
 }
 
 cudaError_t launch_moe_group(const int32_t *ids, int64_t n_pairs, int64_t n_experts,
                              int32_t *counts, int32_t *offsets, int32_t *perm, void *y,
-                             int y_dtype, int64_t n, cudaStream_t s) {
-    const size_t smem = sizeof(int) * (size_t)(n_experts + 1);
+                             int y_dtype, int64_t n, cudaStream_t s, int bn, int32_t *tiles,
+                             int32_t *n_tiles, int64_t max_tiles) {
+    const size_t smem = sizeof(int) * (size_t)(n_experts + 1) * (bn > 0 ? 2 : 1);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(moe_group_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    moe_group_kernel<<<1, GROUP_THREADS, smem, s>>>(ids, (int)n_pairs, (int)n_experts, counts,
-                                                     offsets, perm, y, y_dtype, n, error_word());
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(GROUP_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, moe_group_kernel, ids, (int)n_pairs, (int)n_experts, counts, offsets, perm,
+                              y, y_dtype, n, bn, reinterpret_cast<int2 *>(tiles), n_tiles, (int)max_tiles,
+                              error_word());
 }
 
 // Token tiles for the tensor-core expert product: expert e's segment
