@@ -165,13 +165,15 @@ static bool id_workspace_layout(int64_t n_tokens, int64_t top_k, int64_t n_exper
 constexpr int64_t GEMM_MIN_M = 5;
 // Expert-indexed dispatch by mean (token, slot) pairs per expert, from the
 // sweep on B200 (64 experts of 1408 x 2048, top-6, bf16; us per call,
-// bandwidth kernel / few-pairs tensor-core kernel / GEMM): 8 tokens 48.7 /
-// 55.4 / 54.4, 16 tokens 73.8 / 66.9 / 79.0, 32 tokens 98.9 / 81.4 / 84.5,
-// 128 tokens 264.5 / 103.2 / 115.2, 256 tokens 494.2 / 168.5 / 154.7.  Up
-// to one pair per expert the bandwidth kernel, up to twelve the few-pairs
-// kernel (one token tile of 16 per expert), beyond that the GEMM.
+// bandwidth kernel / few-pairs tensor-core kernel / GEMM): 8 tokens 48.9 /
+// 41.7 / 51.8, 32 tokens 98.6 / 65.5 / 82.0, 128 tokens 265.4 / 93.3 /
+// 112.1, 256 tokens 494.2 / 144.7 / 151.9, 512 tokens 943.4 / 243.4 /
+// 227.9.  With bf16 activations the few-pairs kernel up to 32 pairs per
+// expert, the GEMM beyond; with fp32 ones (no GEMM, tiles of 8 in the
+// few-pairs kernel) the bandwidth kernel up to one pair per expert and the
+// few-pairs kernel beyond.
 constexpr int64_t ID_GEMV_MAX_PAIRS_PER_EXPERT = 1;
-constexpr int64_t ID_TC_MAX_PAIRS_PER_EXPERT = 12;
+constexpr int64_t ID_TC_MAX_PAIRS_PER_EXPERT = 32;
 // The TQ1 bandwidth kernel takes two activation rows per pass over the
 // weights; beyond this many rows the plain kernel is used.
 constexpr int64_t TQ1_GEMV_MAX_M = 8;
@@ -325,7 +327,8 @@ static int id_path(const IdArgs &a, int path, int64_t pairs, int *bn) {
     const bool can_gemm = gemm_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
     const bool can_tc = moe_mma_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
     if (path == KQ_PATH_AUTO) {
-        if (can_gemv && (pairs <= ID_GEMV_MAX_PAIRS_PER_EXPERT * a.n_experts || !(can_tc || can_gemm)))
+        const bool f32x = a.x_dtype == KQ_F32;
+        if (can_gemv && ((f32x && pairs <= ID_GEMV_MAX_PAIRS_PER_EXPERT * a.n_experts) || !(can_tc || can_gemm)))
             path = KQ_PATH_GEMV;
         else if (can_tc && (pairs <= ID_TC_MAX_PAIRS_PER_EXPERT * a.n_experts || !can_gemm)) path = KQ_PATH_GEMV_TC;
         else if (can_gemm) path = KQ_PATH_GEMM;
@@ -394,10 +397,10 @@ int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_e
     a.w2 = w_up;
     a.act = act;
     cudaStream_t s = (cudaStream_t)stream;
-    // Q4_K: up to one pair per expert the bandwidth kernel, beyond it the
-    // tensor-core kernel (a gate pass and an up pass per unit); other codecs
-    // the plain kernel
-    const bool few = pairs <= ID_GEMV_MAX_PAIRS_PER_EXPERT * n_experts;
+    // Q4_K: the few-pairs tensor-core kernel (a gate pass and an up pass per
+    // unit), except fp32 activations up to one pair per expert (the
+    // bandwidth kernel); other codecs the plain kernel
+    const bool few = x_dtype == KQ_F32 && pairs <= ID_GEMV_MAX_PAIRS_PER_EXPERT * n_experts;
     const bool tc = moe_mma_supported(type, n, k, x_dtype, y_dtype) && !(few && moe_gemv_supported(type, n, k, n_experts));
     if (id_group(a, ids, pairs, y, y_dtype, tc ? moe_mma_bn(x_dtype) : 0, s) != cudaSuccess) return KQ_ERR_CUDA;
     if (tc) return to_status(launch_moe_mma(a, s));
