@@ -174,6 +174,10 @@ constexpr int64_t GEMM_MIN_M = 5;
 // few-pairs kernel beyond.
 constexpr int64_t ID_GEMV_MAX_PAIRS_PER_EXPERT = 1;
 constexpr int64_t ID_TC_MAX_PAIRS_PER_EXPERT = 32;
+// The few-pairs kernel's int8 form (one K = 32 MMA per sub-block, 8 pairs a
+// tile) measured faster only at the smallest routings (8 tokens: 40.1 vs
+// 41.7 us; 32 tokens: 69.4 vs 65.5; 64 tokens: 89.8 vs 72.1).
+constexpr int64_t ID_TC_I8_MAX_PAIRS_PER_EXPERT = 1;
 // The TQ1 bandwidth kernel takes two activation rows per pass over the
 // weights; beyond this many rows the plain kernel is used.
 constexpr int64_t TQ1_GEMV_MAX_M = 8;
@@ -231,7 +235,7 @@ int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, i
     switch (path) {
     case KQ_PATH_GEMV_TC:
         if (!can_tc) return KQ_ERR_UNSUPPORTED;
-        return to_status(launch_gemv_tc(w, n, k, x, x_dtype, m, y, y_dtype, s));
+        return to_status(launch_gemv_tc(w, n, k, x, x_dtype, m, y, y_dtype, m <= 4, s));
     case KQ_PATH_GEMM:
         if (!can_gemm) return KQ_ERR_UNSUPPORTED;
         return to_status(launch_gemm(type, w, n, k, x, m, y, y_dtype, s));
@@ -322,7 +326,7 @@ static int id_setup(int type, const void *w, int64_t n_experts, int64_t n, int64
 // The expert product's kernel for these arguments (KQ_PATH_AUTO resolved),
 // or a negative status; *bn: the token-tile width its tile list needs (0:
 // none).
-static int id_path(const IdArgs &a, int path, int64_t pairs, int *bn) {
+static int id_path(IdArgs &a, int path, int64_t pairs, int *bn) {
     const bool can_gemv = moe_gemv_supported(a.type, a.n, a.k, a.n_experts);
     const bool can_gemm = gemm_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
     const bool can_tc = moe_mma_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
@@ -337,8 +341,11 @@ static int id_path(const IdArgs &a, int path, int64_t pairs, int *bn) {
     if (path == KQ_PATH_GEMM && !can_gemm) return KQ_ERR_UNSUPPORTED;
     if (path == KQ_PATH_GEMV && !can_gemv) return KQ_ERR_UNSUPPORTED;
     if (path == KQ_PATH_GEMV_TC && !can_tc) return KQ_ERR_UNSUPPORTED;
+    // the few-pairs kernel's int8 form (8 pairs a tile) while the pairs of
+    // an expert fit one such tile on average
+    a.tc_i8 = path == KQ_PATH_GEMV_TC && pairs <= ID_TC_I8_MAX_PAIRS_PER_EXPERT * a.n_experts;
     *bn = path == KQ_PATH_GEMM ? gemm_id_bn(a.n_tokens, a.top_k, a.n_experts)
-        : path == KQ_PATH_GEMV_TC ? moe_mma_bn(a.x_dtype) : 0;
+        : path == KQ_PATH_GEMV_TC ? moe_mma_bn(a.x_dtype, a.tc_i8) : 0;
     return path;
 }
 
@@ -402,7 +409,9 @@ int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_e
     // bandwidth kernel); other codecs the plain kernel
     const bool few = x_dtype == KQ_F32 && pairs <= ID_GEMV_MAX_PAIRS_PER_EXPERT * n_experts;
     const bool tc = moe_mma_supported(type, n, k, x_dtype, y_dtype) && !(few && moe_gemv_supported(type, n, k, n_experts));
-    if (id_group(a, ids, pairs, y, y_dtype, tc ? moe_mma_bn(x_dtype) : 0, s) != cudaSuccess) return KQ_ERR_CUDA;
+    a.tc_i8 = tc && pairs <= ID_TC_I8_MAX_PAIRS_PER_EXPERT * n_experts;
+    if (id_group(a, ids, pairs, y, y_dtype, tc ? moe_mma_bn(x_dtype, a.tc_i8) : 0, s) != cudaSuccess)
+        return KQ_ERR_CUDA;
     if (tc) return to_status(launch_moe_mma(a, s));
     if (moe_gemv_supported(type, n, k, n_experts)) return to_status(launch_moe_gemv(a, s));
     return to_status(launch_simple_glu(a, s));

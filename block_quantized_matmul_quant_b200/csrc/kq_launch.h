@@ -21,6 +21,7 @@ struct IdArgs {
     const void *w2 = nullptr;                // fused GLU: up stack (w: gate stack)
     int act = 0;                             // fused GLU activation (KQ_ACT_*)
     bool x_slotted = false;                  // x holds one row per pair [n_tokens * top_k, k]
+    bool tc_i8 = false;                      // few-pairs kernel: the int8 form
     // Pair index p = t * top_k + s reads x row p / x_div().
     int x_div() const { return x_slotted ? 1 : (int)top_k; }
     int64_t x_rows() const { return x_slotted ? n_tokens * top_k : n_tokens; }
@@ -88,11 +89,11 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s);
 // Expert-indexed tensor-core kernel for few pairs per expert
 // (kq_moe_mma.cu), over token tiles of moe_mma_bn(x_dtype) pairs.
 bool moe_mma_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype);
-int moe_mma_bn(int x_dtype);
+int moe_mma_bn(int x_dtype, bool i8);
 cudaError_t launch_moe_mma(const IdArgs &a, cudaStream_t s);   // a.w2 set: fused GLU
 // The same kernel on one matrix and m activation rows (tiles of
 // moe_mma_bn(x_dtype) rows).
 cudaError_t launch_gemv_tc(const void *w, int64_t n, int64_t k, const void *x, int x_dtype, int64_t m, void *y,
-                           int y_dtype, cudaStream_t s);
+                           int y_dtype, bool i8, cudaStream_t s);
 
 }  // namespace kq

@@ -83,19 +83,20 @@ struct MoeMmaParams {
     int dense_m;                  // > 0: no grouping, activation rows 0..dense_m-1 of one matrix
     const void *x;                // activations [rows][k], bf16 or (x32) fp32
     int x32;                      // fp32 activations: two MMA rows per token (bf16 high and low parts)
-    int tpt;                      // tokens per tile: 16, or 8 with fp32 activations
+    int tpt;                      // tokens per tile: 16, or 8 (fp32 activations, or the int8 form)
 };
 
 // Shared-memory layout, bytes from the 1024-aligned base.
 struct MmLayout {
-    int x, raw, s, pairs, bars, total;
+    int x, raw, s, sx, pairs, bars, total;
 };
-__host__ __device__ inline MmLayout mm_layout(int k, int raw_slots, int spb) {
+__host__ __device__ inline MmLayout mm_layout(int k, int raw_slots, int spb, bool i8) {
     MmLayout l;
     int off = 0;
-    l.x = off;     off += 32 * k;                           // 16 rows x K bf16, 64-K atoms of 2 KB
+    l.x = off;     off += (i8 ? 16 : 32) * k;               // 16 rows x K (bf16: 64-K atoms; int8: 128-K atoms; 2 KB each)
     l.raw = off;   off += raw_slots * spb * MM_RAW_BYTES;
     l.s = off;     off += 2 * (k / 32) * MM_BN * 4;         // two tiles' sub-block sums [K/32][16]
+    l.sx = off;    off += i8 ? 2 * (k / 32) * MM_BN * 4 : 0;   // int8 form: the codes' scales [K/32][16]
     l.pairs = off; off += 4 * MM_BN * 4 + 2 * 4 + 2 * 4;    // pair ids and x rows [2][16] each, counts [2], flags [2]
     off = (off + 7) / 8 * 8;
     l.bars = off;  off += (2 * raw_slots + 9) * 8 + 8;      // barriers and the TMEM address
@@ -123,21 +124,43 @@ __device__ __forceinline__ float mm_byte_f(uint32_t w, int i) {
 __device__ __forceinline__ uint8_t *x_tile_w(uint8_t *xt, int t, int k) {
     return xt + (k >> 6) * 2048 + t * 128 + ((((k & 63) >> 3) ^ (t & 7)) << 4);
 }
+// The int8 form of the tile: 128-column atoms (one byte an element).
+__device__ __forceinline__ uint8_t *x_tile_w8(uint8_t *xt, int t, int k) {
+    return xt + (k >> 7) * 2048 + t * 128 + ((((k & 127) >> 4) ^ (t & 7)) << 4);
+}
+
+// D (TMEM, s32) += A (TMEM, u8) * B (shared memory, s8), K = 32.
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Instruction descriptor, kind::i8: u8 A, s8 B (K-major), s32 D.
+__host__ __device__ constexpr uint32_t idesc_u8s8(int m, int n) {
+    return (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
 
 }  // namespace
 
-template <typename YT>
+// I8: the int8 form -- 4-bit codes as u8 and 14-bit activation codes as
+// two s8 rows per token (high = c >> 7, low = c & 127, so c = 128 high +
+// low), one K = 32 MMA per sub-block instead of two K = 16 ones.
+template <typename YT, bool I8>
 __global__ void __launch_bounds__(MM_THREADS, 1)
     moe_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_w2,
                    const MoeMmaParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
-    const MmLayout lay = mm_layout(p.k, p.raw_slots, p.spb);
+    const MmLayout lay = mm_layout(p.k, p.raw_slots, p.spb, I8);
     const int R = p.raw_slots, SPB = p.spb;
     const int slot_bytes = SPB * MM_RAW_BYTES;
     uint8_t *x_tile = smem + lay.x;
     uint8_t *raw = smem + lay.raw;
     float *s_sum = reinterpret_cast<float *>(smem + lay.s);          // [2][K/32][16]
+    float *s_xsc = reinterpret_cast<float *>(smem + lay.sx);         // [2][K/32][16] (int8 form)
     int *s_pair = reinterpret_cast<int *>(smem + lay.pairs);         // [2][16] output row (pair) per token
     int *s_xrow = s_pair + 2 * MM_BN;                                // [2][16] activation row per token
     int *s_ntok = s_xrow + 2 * MM_BN;                                // [2]
@@ -269,7 +292,7 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
         // K = 16 into its own 16-column accumulator; one commit frees the A
         // slot and publishes the accumulators.
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(MM_BM, MM_BN);
+            const uint32_t idesc = I8 ? idesc_u8s8(MM_BM, MM_BN) : idesc_bf16(MM_BM, MM_BN);
             const uint64_t xdesc0 = sw128_desc(smem_addr(x_tile));
             uint32_t g = 0;
             int xt = 0, prev = -1;
@@ -292,11 +315,17 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                     #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int kidx = 256 * (s % nk) + 32 * j;     // first K of the sub-block
-                        const uint64_t bd = xdesc0 + (uint64_t)((kidx >> 6) * (2048 >> 4) + ((kidx & 63) >> 3));
                         const uint32_t d = tmem_base + MM_ACC_COL + b * 128u + 16u * j;
-                        const uint32_t a = tmem_base + MM_A_COL + b * 128u + 16u * j;
-                        mma_bf16_ts(d, a, bd, idesc, 0u);
-                        mma_bf16_ts(d, a + 8, bd + 2, idesc, 1u);
+                        if constexpr (I8) {
+                            // one K = 32 MMA: 8 TMEM columns of codes, 32 bytes of the 128-K atom
+                            const uint64_t bd = xdesc0 + (uint64_t)((kidx >> 7) * (2048 >> 4) + ((kidx & 127) >> 4));
+                            mma_i8_ts(d, tmem_base + MM_A_COL + b * 128u + 8u * j, bd, idesc, 0u);
+                        } else {
+                            const uint64_t bd = xdesc0 + (uint64_t)((kidx >> 6) * (2048 >> 4) + ((kidx & 63) >> 3));
+                            const uint32_t a = tmem_base + MM_A_COL + b * 128u + 16u * j;
+                            mma_bf16_ts(d, a, bd, idesc, 0u);
+                            mma_bf16_ts(d, a + 8, bd + 2, idesc, 1u);
+                        }
                     }
                     mma_commit(&mma_done[b]);
                 }
@@ -323,8 +352,29 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
         float acc[MM_BN];     // the row's outputs (GLU: the up projection)
         float accg[MM_BN];    // GLU: the gate projection
         float a[8], c[8];     // the stage's d*sc_j and 128*d*sc_j + dmin*m_j
+        float dm[8];          // and dmin*m_j
         auto apply = [&](float (&A)[MM_BN], uint32_t b, int sp) {
             const float *sb = s_sum + (buf * nsub + 8 * (sp % nk)) * MM_BN;
+            if constexpr (I8) {
+                // columns 2t and 2t+1: token t's high and low code rows (int32)
+                const float *xs = s_xsc + (buf * nsub + 8 * (sp % nk)) * MM_BN;
+                #pragma unroll
+                for (int tg = 0; tg < MM_BN / 4; ++tg) {
+                    if (2 * tg >= ntok) break;   // warp-uniform
+                    uint32_t dv[32];
+                    tmem_ld4x8(t_lane + MM_ACC_COL + b * 128u + 4u * tg, dv);
+                    #pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float2 sv = *reinterpret_cast<const float2 *>(sb + j * MM_BN + 2 * tg);
+                        const float2 xv = *reinterpret_cast<const float2 *>(xs + j * MM_BN + 2 * tg);
+                        const float d0 = (float)(128 * (int)dv[4 * j + 0] + (int)dv[4 * j + 1]);   // exact
+                        const float d1 = (float)(128 * (int)dv[4 * j + 2] + (int)dv[4 * j + 3]);
+                        A[2 * tg + 0] = fmaf(a[j] * xv.x, d0, fmaf(-dm[j], sv.x, A[2 * tg + 0]));
+                        A[2 * tg + 1] = fmaf(a[j] * xv.y, d1, fmaf(-dm[j], sv.y, A[2 * tg + 1]));
+                    }
+                }
+                return;
+            }
             if (p.x32) {
                 // columns 2t and 2t+1: token t's high and low parts
                 #pragma unroll
@@ -409,6 +459,49 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                             const float4 f = src[c4];
                             xf[4 * c4] = f.x; xf[4 * c4 + 1] = f.y; xf[4 * c4 + 2] = f.z; xf[4 * c4 + 3] = f.w;
                         }
+                    } else {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + xi);
+                        #pragma unroll
+                        for (int cq = 0; cq < 4; ++cq) {
+                            const uint4 w = src[cq];
+                            xf[8 * cq] = bf16_lo(w.x); xf[8 * cq + 1] = bf16_hi(w.x);
+                            xf[8 * cq + 2] = bf16_lo(w.y); xf[8 * cq + 3] = bf16_hi(w.y);
+                            xf[8 * cq + 4] = bf16_lo(w.z); xf[8 * cq + 5] = bf16_hi(w.z);
+                            xf[8 * cq + 6] = bf16_lo(w.w); xf[8 * cq + 7] = bf16_hi(w.w);
+                            if (!I8) *reinterpret_cast<uint4 *>(x_tile_w(x_tile, t, 32 * jg + 8 * cq)) = w;
+                        }
+                    }
+                    if constexpr (I8) {
+                        // 14-bit codes c = x / 2^(e-13), e = floor(log2 max |x|): rows 2t
+                        // (c >> 7) and 2t+1 (c & 127) of the int8 tile
+                        float amax = 0.f;
+                        #pragma unroll
+                        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(xf[i]));
+                        int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+                        e = min(max(e, -100), 100);
+                        const float inv = __uint_as_float((uint32_t)(13 - e + 127) << 23);
+                        s_xsc[(buf * nsub + jg) * MM_BN + t] = __uint_as_float((uint32_t)(e - 13 + 127) << 23);
+                        uint32_t hw[8], lw[8];
+                        #pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            uint32_t h = 0, l = 0;
+                            #pragma unroll
+                            for (int bb = 0; bb < 4; ++bb) {
+                                const int cv = min(__float2int_rn(xf[4 * i + bb] * inv), 16383);
+                                h |= (uint32_t)((cv >> 7) & 0xFF) << (8 * bb);
+                                l |= (uint32_t)(cv & 127) << (8 * bb);
+                            }
+                            hw[i] = h;
+                            lw[i] = l;
+                        }
+                        #pragma unroll
+                        for (int c16 = 0; c16 < 2; ++c16) {
+                            *reinterpret_cast<uint4 *>(x_tile_w8(x_tile, 2 * t, 32 * jg + 16 * c16)) =
+                                make_uint4(hw[4 * c16], hw[4 * c16 + 1], hw[4 * c16 + 2], hw[4 * c16 + 3]);
+                            *reinterpret_cast<uint4 *>(x_tile_w8(x_tile, 2 * t + 1, 32 * jg + 16 * c16)) =
+                                make_uint4(lw[4 * c16], lw[4 * c16 + 1], lw[4 * c16 + 2], lw[4 * c16 + 3]);
+                        }
+                    } else if (p.x32) {
                         // rows 2t (bf16 high part) and 2t+1 (bf16 low part)
                         #pragma unroll
                         for (int cq = 0; cq < 4; ++cq) {
@@ -425,17 +518,6 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                                 make_uint4(hw[0], hw[1], hw[2], hw[3]);
                             *reinterpret_cast<uint4 *>(x_tile_w(x_tile, 2 * t + 1, 32 * jg + 8 * cq)) =
                                 make_uint4(lw[0], lw[1], lw[2], lw[3]);
-                        }
-                    } else {
-                        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + xi);
-                        #pragma unroll
-                        for (int cq = 0; cq < 4; ++cq) {
-                            const uint4 w = src[cq];
-                            xf[8 * cq] = bf16_lo(w.x); xf[8 * cq + 1] = bf16_hi(w.x);
-                            xf[8 * cq + 2] = bf16_lo(w.y); xf[8 * cq + 3] = bf16_hi(w.y);
-                            xf[8 * cq + 4] = bf16_lo(w.z); xf[8 * cq + 5] = bf16_hi(w.z);
-                            xf[8 * cq + 6] = bf16_lo(w.w); xf[8 * cq + 7] = bf16_hi(w.w);
-                            *reinterpret_cast<uint4 *>(x_tile_w(x_tile, t, 32 * jg + 8 * cq)) = w;
                         }
                     }
                     float sum = 0.f;
@@ -471,7 +553,6 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                 const uint32_t sc_lo = hd.y & 0x3F3F3F3Fu, m_lo = hd.z & 0x3F3F3F3Fu;
                 const uint32_t sc_hi = (hd.w & 0x0F0F0F0Fu) | ((hd.y >> 2) & 0x30303030u);
                 const uint32_t m_hi = ((hd.w >> 4) & 0x0F0F0F0Fu) | ((hd.z >> 2) & 0x30303030u);
-                float dm[8];
                 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     a[j] = d * mm_byte_f(j < 4 ? sc_lo : sc_hi, j & 3);      // exact
@@ -533,19 +614,38 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const uint8_t *blk = raw + rs * slot_bytes + (r * SPB + sb % SPB) * MM_SB;
-                #pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    const int cc = 2 * half + c2;
-                    const uint4 v0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * cc);
-                    const uint4 v1 = *reinterpret_cast<const uint4 *>(blk + 32 + 32 * cc);
-                    const uint32_t qw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                if constexpr (I8) {
+                    // u8 codes, four a column: chunk cc's low nibbles (sub-block
+                    // 2cc) then its high nibbles (2cc+1), 16 columns a chunk
                     uint32_t out[32];
                     #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        codes4(qw[i] & 0x0F0F0F0Fu, out[2 * i], out[2 * i + 1]);
-                        codes4((qw[i] >> 4) & 0x0F0F0F0Fu, out[16 + 2 * i], out[17 + 2 * i]);
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        const int cc = 2 * half + c2;
+                        const uint4 v0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * cc);
+                        const uint4 v1 = *reinterpret_cast<const uint4 *>(blk + 32 + 32 * cc);
+                        const uint32_t qw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                        #pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            out[16 * c2 + i] = qw[i] & 0x0F0F0F0Fu;
+                            out[16 * c2 + 8 + i] = (qw[i] >> 4) & 0x0F0F0F0Fu;
+                        }
                     }
-                    tmem_st32(t_lane + MM_A_COL + b * 128u + 32u * cc, out);
+                    tmem_st32(t_lane + MM_A_COL + b * 128u + 32u * half, out);
+                } else {
+                    #pragma unroll
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        const int cc = 2 * half + c2;
+                        const uint4 v0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * cc);
+                        const uint4 v1 = *reinterpret_cast<const uint4 *>(blk + 32 + 32 * cc);
+                        const uint32_t qw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                        uint32_t out[32];
+                        #pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            codes4(qw[i] & 0x0F0F0F0Fu, out[2 * i], out[2 * i + 1]);
+                            codes4((qw[i] >> 4) & 0x0F0F0F0Fu, out[16 + 2 * i], out[17 + 2 * i]);
+                        }
+                        tmem_st32(t_lane + MM_A_COL + b * 128u + 32u * cc, out);
+                    }
                 }
                 tc_fence_before();
                 fence_proxy_async_smem();   // generic reads of the raw slot before TMA refills it
@@ -573,11 +673,11 @@ namespace {
 // Raw ring: slots of spb super-blocks (the longest contiguous run of each
 // row that still leaves two slots next to the activation tile and the
 // sums; 4, 2 or 1), as many slots as fit, at most four.
-bool mm_ring(int64_t k, int *slots, int *spb) {
+bool mm_ring(int64_t k, bool i8, int *slots, int *spb) {
     for (int b = 4; b >= 1; b >>= 1) {
         if (b > 1 && b > k / 256) continue;
         int r = 4;
-        while (r >= 2 && mm_layout((int)k, r, b).total > MM_SMEM_LIMIT) --r;
+        while (r >= 2 && mm_layout((int)k, r, b, i8).total > MM_SMEM_LIMIT) --r;
         if (r >= 2) {
             *slots = r;
             *spb = b;
@@ -608,23 +708,25 @@ bool moe_mma_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype)
     if (y_dtype != KQ_F32 && y_dtype != KQ_BF16) return false;
     if (k % 256 || k > MM_MAX_K || n < 1 || n > (1 << 30)) return false;
     int slots, spb;
-    return mm_ring(k, &slots, &spb) && encode_fn() != nullptr;
+    return mm_ring(k, false, &slots, &spb) && mm_ring(k, true, &slots, &spb) && encode_fn() != nullptr;
 }
 
-// Tokens per tile: 16 bf16 activation rows, or 8 fp32 ones (two MMA rows each).
-int moe_mma_bn(int x_dtype) { return x_dtype == KQ_F32 ? MM_BN / 2 : MM_BN; }
+// Tokens per tile: 16 bf16 activation rows, or 8 (fp32 rows, or the int8
+// form): two MMA rows each.
+int moe_mma_bn(int x_dtype, bool i8) { return x_dtype == KQ_F32 || i8 ? MM_BN / 2 : MM_BN; }
 
 namespace {
 
 cudaError_t launch_mm(MoeMmaParams p, const CUtensorMap &tw, const CUtensorMap &tw2, int x_dtype, int y_dtype,
-                      cudaStream_t s) {
+                      bool i8, cudaStream_t s) {
     p.nk = p.k / 256;
     p.n_row_tiles = (p.n + MM_BM - 1) / MM_BM;
     p.x32 = x_dtype == KQ_F32 ? 1 : 0;
-    p.tpt = moe_mma_bn(x_dtype);
+    p.tpt = moe_mma_bn(x_dtype, i8);
     p.err = error_word();
-    const int smem = mm_layout(p.k, p.raw_slots, p.spb).total;
-    auto kern = y_dtype == KQ_F32 ? moe_mma_kernel<float> : moe_mma_kernel<__nv_bfloat16>;
+    const int smem = mm_layout(p.k, p.raw_slots, p.spb, i8).total;
+    auto kern = y_dtype == KQ_F32 ? (i8 ? moe_mma_kernel<float, true> : moe_mma_kernel<float, false>)
+                                  : (i8 ? moe_mma_kernel<__nv_bfloat16, true> : moe_mma_kernel<__nv_bfloat16, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -658,16 +760,16 @@ cudaError_t launch_moe_mma(const IdArgs &a, cudaStream_t s) {
     p.x = a.x;
     p.glu = a.w2 != nullptr;
     p.act = a.act;
-    mm_ring(a.k, &p.raw_slots, &p.spb);
+    mm_ring(a.k, a.tc_i8, &p.raw_slots, &p.spb);
     CUtensorMap tw, tw2;
     if (!encode_w_map4(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride, p.spb) ||
         !encode_w_map4(&tw2, p.glu ? a.w2 : a.w, a.n, a.k, a.n_experts, a.expert_stride, p.spb))
         return cudaErrorInvalidValue;
-    return launch_mm(p, tw, tw2, a.x_dtype, a.y_dtype, s);
+    return launch_mm(p, tw, tw2, a.x_dtype, a.y_dtype, a.tc_i8, s);
 }
 
 cudaError_t launch_gemv_tc(const void *w, int64_t n, int64_t k, const void *x, int x_dtype, int64_t m, void *y,
-                           int y_dtype, cudaStream_t s) {
+                           int y_dtype, bool i8, cudaStream_t s) {
     if (!moe_mma_supported(KQ_Q4_K, n, k, x_dtype, y_dtype) || m < 1 || m > INT32_MAX / 2)
         return cudaErrorNotSupported;
     MoeMmaParams p = {};
@@ -679,10 +781,10 @@ cudaError_t launch_gemv_tc(const void *w, int64_t n, int64_t k, const void *x, i
     p.dense_m = (int)m;
     p.y = y;
     p.x = x;
-    mm_ring(k, &p.raw_slots, &p.spb);
+    mm_ring(k, i8, &p.raw_slots, &p.spb);
     CUtensorMap tw;
     if (!encode_w_map4(&tw, w, n, k, 1, n * (k / 256) * MM_SB, p.spb)) return cudaErrorInvalidValue;
-    return launch_mm(p, tw, tw, x_dtype, y_dtype, s);
+    return launch_mm(p, tw, tw, x_dtype, y_dtype, i8, s);
 }
 
 }  // namespace kq
