@@ -681,6 +681,7 @@ def test_moe_ffn_chain_reuses_the_grouping(kq, xdt):
     (100, 2, 3, 300, 1024, False),     # ~66 pairs per expert: five token tiles each
     (7, 3, 4, 129, 4096, False),       # the largest K the kernel takes
     (64, 4, 8, 256, 768, True),        # one expert takes most pairs: many tiles, other experts one
+    (8, 2, 32, 1408, 2048, False),     # at most one pair per expert: the int8 form
 ])
 @pytest.mark.parametrize("xdt", ["bf16", "f32"])
 def test_matmul_id_tensor_core_few_pairs(kq, t, top_k, e, n, k, skew, xdt):
