@@ -303,7 +303,7 @@ def secondary_metrics(torch, kq, l2, peaks):
     """The other measured workloads, one short timed graph each."""
     out = {}
     for name in ("q4_k_gemm_512x11008x4096", "moe_q4_k_e64_1408x2048_t32_top6",
-                 "tq1_g128_gemv_5120x17408", "q8_0_gemv_256x1024"):
+                 "tq1_g128_gemv_5120x17408", "tq1_g128_gemm_512x5120x17408", "q8_0_gemv_256x1024"):
         wl = synth.WORKLOADS[name]
         st = PoolStep(torch, kq, wl, l2)
         ms = time_graph(torch, st.run, 5, 3, None)
@@ -340,7 +340,7 @@ def secondary_entry(wl, us, wbytes, hit_experts, peaks):
         return {"us_per_call": round(us, 2), "TFLOP/s": round(tf, 1),
                 "frac_burst": round(tf / peaks["bf16_tflops"], 4),
                 "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
-                "kernel": "gemm_q4k_kernel (tcgen05)"}
+                "kernel": ("gemm_tq1_kernel" if wl.codec == synth.TQ1_G128 else "gemm_q4k_kernel") + " (tcgen05)"}
     if wl.kind == "moe":
         per_expert = wbytes // wl.n_experts
         moved = hit_experts * per_expert + wl.m * wl.k * 2 + wl.m * wl.top_k * wl.n * 4
@@ -643,18 +643,50 @@ def run_profile(args):
     print(json.dumps({"profiled": wl.name, "calls": args.profile_calls}))
 
 
+def run_tq1_sweep(torch, kq, l2):
+    """TQ1_G128 5120 x 17408 (bf16 activations): the bandwidth kernel (one
+    launch per two rows, up to 16 rows here) against the tensor-core kernel
+    over the activation-row count."""
+    dense = synth.Workload("sweep_tq1", "gemm", synth.TQ1_G128, 5120, 17408, 1, "bf16", "f32")
+    w, _, _ = synth.make_inputs(dense)
+    wd = torch.from_numpy(w).cuda()
+    pool = [wd.clone() for _ in range(pool_size(w.nbytes, l2))]
+    r = np.random.Generator(np.random.PCG64(2))
+    for m in (1, 2, 4, 5, 6, 8, 12, 16, 32, 64, 128, 256, 512):
+        x = torch.from_numpy(synth.gen_x(m, dense.k, "bf16", r)).to(torch.bfloat16).cuda()
+        y = torch.empty((m, dense.n), device="cuda")
+        line = {"sweep": "dense_tq1_g128_5120x17408", "m": m, "pool": len(pool)}
+        for name, path in (("gemv", kq.PATH_GEMV), ("gemm", kq.PATH_GEMM)):
+            if name == "gemv" and m > 16:
+                continue
+            def fn():
+                for wi in pool:
+                    kq.matmul(wi, synth.TQ1_G128, x, out=y, path=path, const_weights=True)
+            line[name + "_us"] = round(time_graph(torch, fn, 5, 3, None) * 1e3 / (5 * len(pool)), 2)
+        print(json.dumps(line), flush=True)
+    del pool, wd
+    torch.cuda.empty_cache()
+
+
 def run_sweep(args):
     """Dispatch evidence: per-call time of the bandwidth kernel against the
     tensor-core kernel over the activation-row count (dense Q4_K product,
-    11008 x 4096) and the token count (MoE, 64 experts of 1408 x 2048,
-    top-6), bf16 activations, each call on its own weight copy of a pool
-    larger than 4x L2.  One JSON line per point."""
+    11008 x 4096; dense TQ1_G128, 5120 x 17408) and the token count (MoE, 64
+    experts of 1408 x 2048, top-6), bf16 activations, each call on its own
+    weight copy of a pool larger than 4x L2.  One JSON line per point
+    (`--sweep tq1`: the TQ1 points only)."""
     import torch
 
     import block_quantized_matmul_quant_b200 as kq
 
     kq.lib()
     l2 = l2_bytes(0)
+    run_tq1_sweep(torch, kq, l2)
+    if args.sweep == "tq1":
+        status = kq.device_status()
+        if status != 0:
+            raise SystemExit(f"device status {status} after the sweep")
+        return
     dense = synth.Workload("sweep_dense", "gemm", synth.Q4_K, 11008, 4096, 1, "bf16", "f32")
     w, _, _ = synth.make_inputs(dense)
     wd = torch.from_numpy(w).cuda()
@@ -711,7 +743,7 @@ def main():
                     help="GEMV call ordering in --profile (the headline step uses independent calls)")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the other workloads' numbers (prefill GEMM, MoE, TQ1, Q8_0)")
-    ap.add_argument("--sweep", default=None, choices=["dispatch"],
+    ap.add_argument("--sweep", default=None, choices=["dispatch", "tq1"],
                     help="print the dispatch sweep (bandwidth vs tensor-core kernel) and exit")
     args = ap.parse_args()
     if args.warmup < 3:

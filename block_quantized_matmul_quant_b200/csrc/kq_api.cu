@@ -179,8 +179,15 @@ constexpr int64_t ID_TC_MAX_PAIRS_PER_EXPERT = 32;
 // 41.7 us; 32 tokens: 69.4 vs 65.5; 64 tokens: 89.8 vs 72.1).
 constexpr int64_t ID_TC_I8_MAX_PAIRS_PER_EXPERT = 1;
 // The TQ1 bandwidth kernel takes two activation rows per pass over the
-// weights; beyond this many rows the plain kernel is used.
+// weights; beyond this many rows the tensor-core kernel (K % 512 == 0, bf16
+// activations) or else the plain kernel is used.
 constexpr int64_t TQ1_GEMV_MAX_M = 8;
+// Activation rows from which the tensor-core kernel serves TQ1 products.
+// Measured on B200 (TQ1_G128 5120 x 17408, bf16, us per call, bandwidth vs
+// tensor-core kernel): 4 rows 56.4 vs 116.2, 8 rows 111.9 vs 116.2, 12 rows
+// 167.5 vs 116.3 (the tensor-core kernel has only 40 weight-row tiles here,
+// so its time stays flat up to 16 rows; 512 rows 167.9).
+constexpr int64_t TQ1_GEMM_MIN_M = TQ1_GEMV_MAX_M + 1;
 
 }  // namespace kq
 
@@ -224,7 +231,7 @@ int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, i
     const bool can_gemm = gemm_supported(type, n, k, x_dtype, y_dtype);
     const bool can_gemv = gemv_supported(type, n, k, x_dtype, m);
     if (path == KQ_PATH_AUTO) {
-        if (can_gemm && m >= GEMM_MIN_M) path = KQ_PATH_GEMM;
+        if (can_gemm && m >= (type == KQ_TQ1_G128 ? TQ1_GEMM_MIN_M : GEMM_MIN_M)) path = KQ_PATH_GEMM;
         // fp32 activations past one pass of the bandwidth kernel: the
         // few-rows tensor-core kernel reads the weights once per 8 rows of a
         // tile instead of once per 8-row launch
@@ -328,7 +335,7 @@ static int id_setup(int type, const void *w, int64_t n_experts, int64_t n, int64
 // none).
 static int id_path(IdArgs &a, int path, int64_t pairs, int *bn) {
     const bool can_gemv = moe_gemv_supported(a.type, a.n, a.k, a.n_experts);
-    const bool can_gemm = gemm_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
+    const bool can_gemm = gemm_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype, true);
     const bool can_tc = moe_mma_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
     if (path == KQ_PATH_AUTO) {
         const bool f32x = a.x_dtype == KQ_F32;

@@ -17,8 +17,9 @@
 //    tensor core's operand reads do not compete with decoder stores.
 //  * Warp roles:  warp 0  TMA producer of bf16 activation tiles (64 K x BN,
 //                         128-byte swizzle) into a shared-memory ring;
-//                 warp 6  TMA producer of raw Q4_K super-blocks (128 rows x
-//                         144 bytes) into their own ring;
+//                 warp 6  TMA producer of raw weight units (128 rows x one
+//                         Q4_K super-block, 144 bytes, or four TQ1_G128
+//                         blocks, 112 bytes) into their own ring;
 //                 warp 1  MMA issuer -- one thread issues tcgen05.mma
 //                         (kind::f16, bf16 x bf16 -> fp32 in TMEM) and
 //                         tcgen05.commit's to the stage / accumulator barriers;
@@ -26,9 +27,13 @@
 //                 warps 7..  decoders, in groups of four warps (one per TMEM
 //                         lane quadrant, so lane = weight row): group j
 //                         decodes the stages s with s % groups == j, 64 K
-//                         positions of its 32 rows per warp, exact fp32
-//                         (d*sc*q - dmin*m, one rounding) -> bf16 (round to
-//                         nearest even).
+//                         positions of its 32 rows per warp.  Q4_K: exact
+//                         fp32 (d*sc*q - dmin*m, one rounding) -> bf16 (round
+//                         to nearest even).  TQ1_G128 (Ternary Bonsai
+//                         `tq1_gemm`, the prefill form of the ternary
+//                         product): base-3 digits by integer arithmetic, two
+//                         bytes' digits a 32-bit word, then (t - 1) * bf16(scale)
+//                         -- the round-to-nearest-even bf16 of the weight.
 //  * TMEM (512 columns): accumulators at columns 0 and 256 (BN each, so the
 //    epilogue of tile i overlaps the main loop of tile i+1); the stage ring's
 //    A slots (32 columns = 128 rows x 64 bf16) fill the gaps after them.
@@ -51,12 +56,17 @@ namespace {
 
 constexpr int BM = 128;            // weight rows per tile (MMA M)
 constexpr int BK = 64;             // K per swizzle atom (128 bytes of bf16); a stage holds CPS atoms
-constexpr int SB_BYTES = 144;      // Q4_K super-block
-constexpr int RAW_STAGE_BYTES = BM * SB_BYTES;   // 18432
+// Raw weights move in units of one TMA box row: a Q4_K super-block (144
+// bytes, 256 K) or four TQ1_G128 blocks (112 bytes, 512 K; a box row must be
+// a multiple of 16 bytes, so TQ1 rows need K % 512 == 0).
+template <int FMT> struct RawUnit;
+template <> struct RawUnit<KQ_Q4_K> { static constexpr int BYTES = 144, K = 256; };
+template <> struct RawUnit<KQ_TQ1_G128> { static constexpr int BYTES = 112, K = 512; };
+constexpr int raw_stage_bytes(int type) { return BM * (type == KQ_TQ1_G128 ? 112 : 144); }
 #ifndef KQ_GEMM_DEC_WARPS
 #define KQ_GEMM_DEC_WARPS 16
 #endif
-constexpr int RAW_WARP = 6;  // raw super-block producer
+constexpr int RAW_WARP = 6;  // raw weight producer
 constexpr int DEC_WARP0 = 7, DEC_WARPS = KQ_GEMM_DEC_WARPS;  // 8 or 16
 constexpr int DEC_GROUPS = DEC_WARPS / 4;                    // 2 or 4
 static_assert(DEC_GROUPS == 2 || DEC_GROUPS == 4, "decoder warps come in 2 or 4 groups of 4");
@@ -77,7 +87,7 @@ struct GemmParams {
     int bn, m_tiles, n_tiles, tiles;
     int a_stages;  // decoded-weight ring: A slots in TMEM
     int b_stages;  // activation ring: tiles in shared memory (deeper: their loads come from L2)
-    int raw_stages;  // raw super-block ring (each slot: 128 rows x 144 bytes, 4 stages of K)
+    int raw_stages;  // raw weight ring (each slot: 128 rows x one raw unit)
     int a_col0;    // first TMEM column after an accumulator (BN rounded up to 32)
     int b_stage_bytes;
     void *y;
@@ -167,19 +177,103 @@ __device__ __forceinline__ void decode4(uint32_t nib, float2 scale, float2 bias,
     o1 = *reinterpret_cast<const uint32_t *>(&b1);
 }
 
+// Base-3 digits of a TQ1 code byte b (0..242), two to a 32-bit word in
+// 16-bit lanes, the order of the weights: lo = (d1 << 16) | d0,
+// mid = (d3 << 16) | d2, hi = d4.  Division by 3 of both lanes at once is a
+// multiply by 171 and a shift by 9 (exact for 0..255; a lane's product stays
+// below 2^16, so the lanes do not mix).
+__device__ __forceinline__ void tq1_digits(uint32_t b, uint32_t &lo, uint32_t &mid, uint32_t &hi) {
+    const uint32_t x0 = b | (((b * 171u) >> 9) << 16);          // (b, b/3)
+    const uint32_t q0 = ((x0 * 171u) >> 9) & 0x007F007Fu;       // (b/3, b/9)
+    lo = x0 - 3u * q0;                                           // (d0, d1)
+    const uint32_t x1 = ((q0 * 171u) >> 9) & 0x007F007Fu;       // (b/9, b/27)
+    const uint32_t q1 = ((x1 * 171u) >> 9) & 0x007F007Fu;       // (b/27, b/81)
+    mid = x1 - 3u * q1;                                          // (d2, d3)
+    hi = q1 >> 16;                                               // b/81 = d4
+}
+
+// Two digits (16-bit lanes, 0..2) -> bf16x2 of (d - 1) * s: the lanes as
+// bf16 are 128 + d, and 128 + d - 129 and the product with +-1 or 0 are exact.
+__device__ __forceinline__ uint32_t tq1_word(uint32_t dd, __nv_bfloat162 s2) {
+    const uint32_t v = dd | 0x43004300u, c = 0x43014301u;   // bf16x2 (128 + d), (129, 129)
+    const __nv_bfloat162 t = __hmul2(__hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&v),
+                                             *reinterpret_cast<const __nv_bfloat162 *>(&c)),
+                                     s2);
+    return *reinterpret_cast<const uint32_t *>(&t);
+}
+
+// Weights 64 H .. 64 H + 63 of block B of a row's raw TQ1 unit (four
+// 28-byte blocks, 112 bytes from `row`, 16-byte aligned) as 32 bf16x2 words
+// of bf16(scale) * (t - 1), word j holding weights 64 H + 2 j and + 1.
+// Weight i of a block is digit i % 5 of byte i / 5 (the tail byte 25 holds
+// weights 125..127); a full byte above 242 or a tail byte above 26 is not a
+// code and decodes to zeros (as byte 121, all digits 1).
+template <int B, int H>
+__device__ __forceinline__ void tq1_decode64(const uint8_t *row, uint32_t out[32]) {
+    constexpr int LO = 28 * B + 12 * H;         // first byte needed (byte 12 of a block is in both halves)
+    constexpr int C0 = LO / 16, C1 = (28 * B + 27) / 16;   // 16-byte chunks through the scale
+    uint32_t wv[4 * (C1 - C0 + 1)];
+    #pragma unroll
+    for (int c = C0; c <= C1; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(row + 16 * c);
+        wv[4 * (c - C0)] = v.x; wv[4 * (c - C0) + 1] = v.y; wv[4 * (c - C0) + 2] = v.z; wv[4 * (c - C0) + 3] = v.w;
+    }
+    const uint32_t sbits = wv[(28 * B + 26) / 4 - 4 * C0] >> 16;   // bytes 26..27: fp16 scale
+    const __nv_bfloat16 sb = __float2bfloat16_rn(half_bits_to_float(sbits));
+    const __nv_bfloat162 s2 = __halves2bfloat162(sb, sb);
+    // digit words of block bytes J0 .. J0 + 13 (13 used by half 0)
+    constexpr int J0 = H == 0 ? 0 : 12;
+    uint32_t dg[14][3];
+    #pragma unroll
+    for (int jj = 0; jj < 14; ++jj) {
+        const int j = J0 + jj;
+        if (j > 25 || (H == 0 && j > 12)) continue;
+        const int i = 28 * B + j;
+        uint32_t b = (wv[i / 4 - 4 * C0] >> (8 * (i % 4))) & 0xFFu;
+        b = b > (j == 25 ? 26u : 242u) ? 121u : b;
+        tq1_digits(b, dg[jj][0], dg[jj][1], dg[jj][2]);
+    }
+    #pragma unroll
+    for (int w = 0; w < 32; ++w) {
+        const int i0 = 64 * H + 2 * w, i1 = i0 + 1;
+        const int j0 = i0 / 5 - J0, d0 = i0 % 5, j1 = i1 / 5 - J0, d1 = i1 % 5;
+        // lane of digit d in its byte's words: word d / 2, 16-bit half d % 2
+        const uint32_t a = dg[j0][d0 >> 1], c = dg[j1][d1 >> 1];
+        uint32_t dd;
+        if (j0 == j1 && (d0 & 1) == 0) dd = a;                           // (d0, d0 + 1) of one word
+        else dd = __byte_perm(a, c, ((d0 & 1) ? 0x32u : 0x10u) | ((d1 & 1) ? 0x7600u : 0x5400u));
+        out[w] = tq1_word(dd, s2);
+    }
+}
+
+// 64-K chunk cc (0..7) of a row's raw TQ1 unit: half cc % 2 of block cc / 2.
+__device__ __forceinline__ void tq1_decode_chunk(const uint8_t *row, int cc, uint32_t out[32]) {
+    switch (cc) {
+    case 0: tq1_decode64<0, 0>(row, out); break;
+    case 1: tq1_decode64<0, 1>(row, out); break;
+    case 2: tq1_decode64<1, 0>(row, out); break;
+    case 3: tq1_decode64<1, 1>(row, out); break;
+    case 4: tq1_decode64<2, 0>(row, out); break;
+    case 5: tq1_decode64<2, 1>(row, out); break;
+    case 6: tq1_decode64<3, 0>(row, out); break;
+    default: tq1_decode64<3, 1>(row, out); break;
+    }
+}
+
 // CPS: 64-K swizzle atoms per pipeline stage (1, or 2 for narrow token tiles,
-// which halves the per-K barrier traffic of the single MMA thread).
-template <typename YT, bool ID, int CPS>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm_q4k_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                    const __grid_constant__ CUtensorMap tmap_w,
-                    const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+// which halves the per-K barrier traffic of the single MMA thread).  FMT: the
+// weight format (KQ_Q4_K or KQ_TQ1_G128; TQ1 dense only).
+template <typename YT, bool ID, int CPS, int FMT>
+__device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w,
+                                          const CUtensorMap &tmap_y, const GemmParams &p) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     const int SA = p.a_stages, SB = p.b_stages, SR = p.raw_stages;
     uint8_t *b_ring = smem;                                    // SB x bn*128
-    uint8_t *raw_ring = b_ring + SB * p.b_stage_bytes;         // SR x 18 KB
+    constexpr int UNIT_BYTES = RawUnit<FMT>::BYTES, UNIT_K = RawUnit<FMT>::K;
+    constexpr int RAW_STAGE_BYTES = BM * UNIT_BYTES;
+    uint8_t *raw_ring = b_ring + SB * p.b_stage_bytes;         // SR x 18 or 14 KB
     uint8_t *epi_stage = raw_ring + SR * RAW_STAGE_BYTES;      // EPI_STAGE_BYTES
     uint64_t *bars = reinterpret_cast<uint64_t *>(epi_stage + EPI_STAGE_BYTES);
     uint64_t *full_a = bars;                 // [SA] one decoder group (4 warps) -> MMA
@@ -198,7 +292,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int SPS = 4 / CPS;           // stages per raw super-block (256 K)
+    constexpr int SPS = UNIT_K / (BK * CPS);   // stages per raw unit
     const int nk = p.k / (BK * CPS);       // stages per tile
 
     if (threadIdx.x == 0) {
@@ -237,7 +331,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int units = ID ? *p.id_n_tiles * p.n_tiles : p.tiles;
 
     if (warp == RAW_WARP) {
-        // ---------------- raw super-block producer ----------------
+        // ---------------- raw weight producer ----------------
         // Runs ahead of the decoders by the whole raw ring, independently of
         // the activation ring (narrow token tiles stream fresh weights).
         if (lane == 0) {
@@ -245,11 +339,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
                 const Tile t = tile_at<ID>(p, u);
-                for (int sb = 0; sb < p.k / 256; ++sb) {
+                for (int sb = 0; sb < p.k / UNIT_K; ++sb) {
                     ok = mbar_wait(&raw_empty[rslot], rphase ^ 1, p.err);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&raw_full[rslot], RAW_STAGE_BYTES);
-                    tma_load_3d(raw_ring + rslot * RAW_STAGE_BYTES, &tmap_w, sb * SB_BYTES, t.n0, t.e,
+                    tma_load_3d(raw_ring + rslot * RAW_STAGE_BYTES, &tmap_w, sb * UNIT_BYTES, t.n0, t.e,
                                 &raw_full[rslot]);
                     if (++rslot == (uint32_t)SR) { rslot = 0; rphase ^= 1; }
                 }
@@ -415,11 +509,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t g = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-            for (int sb = 0; sb < p.k / 256 && ok; ++sb) {
+            for (int sb = 0; sb < p.k / UNIT_K && ok; ++sb) {
                 ok = warp_wait(&raw_full[rs], rph, p.err);
                 if (!ok) break;
-                const uint8_t *blk = raw_ring + rs * RAW_STAGE_BYTES + r * SB_BYTES;
-                const uint4 hd = *reinterpret_cast<const uint4 *>(blk);
+                const uint8_t *blk = raw_ring + rs * RAW_STAGE_BYTES + r * UNIT_BYTES;
+                // Q4_K super-block header (unused for TQ1)
+                const uint4 hd = FMT == KQ_Q4_K ? *reinterpret_cast<const uint4 *>(blk) : make_uint4(0u, 0u, 0u, 0u);
                 const float d = half_f(hd.x), dmin = half_f(hd.x >> 16);
                 // packed 6-bit scales / mins of sub-blocks 0..3 and 4..7
                 const uint32_t sc_lo = hd.y & 0x3F3F3F3Fu, m_lo = hd.z & 0x3F3F3F3Fu;
@@ -434,24 +529,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         tc_fence_after();
                       #pragma unroll
                       for (int c = 0; c < CPS; ++c) {
-                        const int cc = st * CPS + c;   // 64-K chunk of the super-block
-                        const uint32_t scw = cc < 2 ? sc_lo : sc_hi, mw = cc < 2 ? m_lo : m_hi;
-                        const int b0 = (2 * cc) & 3;
-                        // exact products: d*sc (17 bits), dmin*m (17 bits); high
-                        // nibbles arrive as 16*q, so their scale is divided by 16
-                        const float ds_lo = d * byte_float(scw, b0), dm_lo = dmin * byte_float(mw, b0);
-                        const float ds_hi = d * byte_float(scw, b0 + 1) * 0.0625f;
-                        const float dm_hi = dmin * byte_float(mw, b0 + 1);
-                        const float2 sl = make_float2(ds_lo, ds_lo), bl = make_float2(-dm_lo, -dm_lo);
-                        const float2 sh = make_float2(ds_hi, ds_hi), bh = make_float2(-dm_hi, -dm_hi);
-                        const uint4 v0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * cc);
-                        const uint4 v1 = *reinterpret_cast<const uint4 *>(blk + 32 + 32 * cc);
-                        const uint32_t qw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                        const int cc = st * CPS + c;   // 64-K chunk of the raw unit
                         uint32_t out[32];
-                        #pragma unroll
-                        for (int wd = 0; wd < 8; ++wd) {
-                            decode4(qw[wd] & 0x0F0F0F0Fu, sl, bl, out[2 * wd], out[2 * wd + 1]);
-                            decode4(qw[wd] & 0xF0F0F0F0u, sh, bh, out[16 + 2 * wd], out[17 + 2 * wd]);
+                        if constexpr (FMT == KQ_TQ1_G128) {
+                            tq1_decode_chunk(blk, cc, out);
+                        } else {
+                            const uint32_t scw = cc < 2 ? sc_lo : sc_hi, mw = cc < 2 ? m_lo : m_hi;
+                            const int b0 = (2 * cc) & 3;
+                            // exact products: d*sc (17 bits), dmin*m (17 bits); high
+                            // nibbles arrive as 16*q, so their scale is divided by 16
+                            const float ds_lo = d * byte_float(scw, b0), dm_lo = dmin * byte_float(mw, b0);
+                            const float ds_hi = d * byte_float(scw, b0 + 1) * 0.0625f;
+                            const float dm_hi = dmin * byte_float(mw, b0 + 1);
+                            const float2 sl = make_float2(ds_lo, ds_lo), bl = make_float2(-dm_lo, -dm_lo);
+                            const float2 sh = make_float2(ds_hi, ds_hi), bh = make_float2(-dm_hi, -dm_hi);
+                            const uint4 v0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * cc);
+                            const uint4 v1 = *reinterpret_cast<const uint4 *>(blk + 32 + 32 * cc);
+                            const uint32_t qw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                            #pragma unroll
+                            for (int wd = 0; wd < 8; ++wd) {
+                                decode4(qw[wd] & 0x0F0F0F0Fu, sl, bl, out[2 * wd], out[2 * wd + 1]);
+                                decode4(qw[wd] & 0xF0F0F0F0u, sh, bh, out[16 + 2 * wd], out[17 + 2 * wd]);
+                            }
                         }
                         tmem_st32(t_lane + a_slot_col<CPS>(slot, p.a_col0) + 32 * c, out);
                       }
@@ -477,6 +576,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, 512);
     }
+}
+
+template <typename YT, bool ID, int CPS>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_q4k_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                    const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+    gemm_body<YT, ID, CPS, KQ_Q4_K>(tmap_x, tmap_w, tmap_y, p);
+}
+
+template <typename YT, bool ID, int CPS>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tq1_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                    const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+    gemm_body<YT, ID, CPS, KQ_TQ1_G128>(tmap_x, tmap_w, tmap_y, p);
 }
 
 // ---------------------------------------------------------------- host side
@@ -527,12 +640,12 @@ constexpr int SMEM_RINGS = SMEM_BUDGET - 1024 - 2560 - EPI_STAGE_BYTES;  // less
 #ifndef KQ_GEMM_MIN_RAW
 #define KQ_GEMM_MIN_RAW 2
 #endif
-int b_stages_for(int b_stage_bytes) {
-    const int st = (SMEM_RINGS - KQ_GEMM_MIN_RAW * RAW_STAGE_BYTES) / b_stage_bytes;
+int b_stages_for(int b_stage_bytes, int raw_bytes) {
+    const int st = (SMEM_RINGS - KQ_GEMM_MIN_RAW * raw_bytes) / b_stage_bytes;
     return st < MAX_B_STAGES ? st : MAX_B_STAGES;
 }
-int raw_stages_for(int b_stage_bytes, int b_stages) {
-    const int st = (SMEM_RINGS - b_stages * b_stage_bytes) / RAW_STAGE_BYTES;
+int raw_stages_for(int b_stage_bytes, int b_stages, int raw_bytes) {
+    const int st = (SMEM_RINGS - b_stages * b_stage_bytes) / raw_bytes;
     return st < MAX_RAW_STAGES ? st : MAX_RAW_STAGES;
 }
 
@@ -562,24 +675,34 @@ bool encode_x_map(CUtensorMap *m, const void *x, int64_t rows, int64_t k, int bo
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Raw Q4_K rows of one or more experts: (row bytes, rows, experts), one
-// super-block column of BM rows per box.
+// Raw rows of one or more experts: (row bytes, rows, experts), one raw unit
+// column (a Q4_K super-block, or four TQ1_G128 blocks) of BM rows per box.
 bool encode_w_map(CUtensorMap *m, const void *w, int64_t n, int64_t k, int64_t n_experts,
-                  int64_t expert_stride) {
-    const int64_t rb = (k / 256) * SB_BYTES;
+                  int64_t expert_stride, int type) {
+    const int ub = type == KQ_TQ1_G128 ? RawUnit<KQ_TQ1_G128>::BYTES : RawUnit<KQ_Q4_K>::BYTES;
+    const int uk = type == KQ_TQ1_G128 ? RawUnit<KQ_TQ1_G128>::K : RawUnit<KQ_Q4_K>::K;
+    if (k % uk) return false;
+    const int64_t rb = (k / uk) * ub;
     cuuint64_t dims[3] = {(cuuint64_t)rb, (cuuint64_t)n, (cuuint64_t)n_experts};
     cuuint64_t strides[2] = {(cuuint64_t)rb, (cuuint64_t)expert_stride};
-    cuuint32_t box[3] = {SB_BYTES, BM, 1};
+    cuuint32_t box[3] = {(cuuint32_t)ub, BM, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(w), dims, strides, box, es,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool gemm_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype) {
-    if (type != KQ_Q4_K || x_dtype != KQ_BF16) return false;
+bool gemm_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype, bool expert_indexed) {
+    if (x_dtype != KQ_BF16) return false;
     if (y_dtype != KQ_F32 && y_dtype != KQ_BF16) return false;
-    if (k % 256 || k > (1 << 24) || n < 1 || n > (1 << 30)) return false;
+    if (k > (1 << 24) || n < 1 || n > (1 << 30)) return false;
+    if (type == KQ_Q4_K) {
+        if (k % 256) return false;
+    } else if (type == KQ_TQ1_G128 && !expert_indexed) {
+        if (k % 512) return false;   // the row pitch and box rows must be multiples of 16 bytes
+    } else {
+        return false;
+    }
     return encode_fn() != nullptr;
 }
 
@@ -604,23 +727,26 @@ bool encode_y_map(CUtensorMap *mp, void *y, int64_t m, int64_t n, int ydt) {
 // the single MMA thread's per-stage waits and commits dominate), else one.
 int cps_for(int bn) { return bn <= 64 ? 2 : 1; }
 
-bool fill_ring(GemmParams *p, int cps) {
+bool fill_ring(GemmParams *p, int cps, int type) {
+    const int rbytes = raw_stage_bytes(type);
     p->b_stage_bytes = p->bn * 128 * cps;
     p->a_stages = a_stages_for(p->bn, cps);
-    p->b_stages = b_stages_for(p->b_stage_bytes);
-    p->raw_stages = raw_stages_for(p->b_stage_bytes, p->b_stages);
+    p->b_stages = b_stages_for(p->b_stage_bytes, rbytes);
+    p->raw_stages = raw_stages_for(p->b_stage_bytes, p->b_stages, rbytes);
     p->a_col0 = a_col0_for(p->bn);
     return p->bn <= MAX_BN && p->bn % 16 == 0 && p->a_stages >= 2 && p->b_stages >= 2 && p->raw_stages >= 2;
 }
 
-template <typename YT, bool ID, int CPS>
+template <typename YT, bool ID, int CPS, int FMT = KQ_Q4_K>
 cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CUtensorMap &ty,
                           const GemmParams &p, int grid, cudaStream_t s) {
     // alignment slack, activation ring, raw ring, epilogue staging, barriers
     // (384 B) and the expert-indexed row list (768 B)
-    const size_t smem = 1024 + (size_t)p.b_stages * p.b_stage_bytes + (size_t)p.raw_stages * RAW_STAGE_BYTES +
-                        EPI_STAGE_BYTES + 2560;
-    auto kern = gemm_q4k_kernel<YT, ID, CPS>;
+    const size_t smem = 1024 + (size_t)p.b_stages * p.b_stage_bytes +
+                        (size_t)p.raw_stages * raw_stage_bytes(FMT) + EPI_STAGE_BYTES + 2560;
+    void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
+    if constexpr (FMT == KQ_TQ1_G128) kern = gemm_tq1_kernel<YT, ID, CPS>;
+    else kern = gemm_q4k_kernel<YT, ID, CPS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -640,8 +766,8 @@ cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CU
 
 cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const void *x, int64_t m,
                         void *y, int ydt, cudaStream_t s) {
-    (void)type;
     if (!encode_fn() || m < 1 || m > (1 << 30)) return cudaErrorNotSupported;
+    if (type != KQ_Q4_K && type != KQ_TQ1_G128) return cudaErrorNotSupported;
     const int sms = sm_count();
     GemmParams p = {};
     p.n = (int)n; p.k = (int)k; p.m = (int)m;
@@ -650,15 +776,23 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
     p.m_tiles = (int)((m + p.bn - 1) / p.bn);
     p.tiles = p.n_tiles * p.m_tiles;
     const int cps = cps_for(p.bn);
-    if (!fill_ring(&p, cps)) return cudaErrorNotSupported;
+    if (!fill_ring(&p, cps, type)) return cudaErrorNotSupported;
     p.y = y;
     p.err = error_word();
     CUtensorMap tx, tw, ty;
-    if (!encode_x_map(&tx, x, m, k, p.bn) || !encode_w_map(&tw, w, n, k, 1, n * ((k / 256) * SB_BYTES)))
+    const int64_t row_bytes = type == KQ_TQ1_G128 ? (k / 128) * 28 : (k / 256) * 144;
+    if (!encode_x_map(&tx, x, m, k, p.bn) || !encode_w_map(&tw, w, n, k, 1, n * row_bytes, type))
         return cudaErrorInvalidValue;
     p.y_tma = encode_y_map(&ty, y, m, n, ydt) ? 1 : 0;
     if (!p.y_tma) ty = tx;   // unused
     const int grid = p.tiles < sms ? p.tiles : sms;
+    if (type == KQ_TQ1_G128) {
+        if (cps == 2)
+            return ydt == KQ_F32 ? launch_kernel<float, false, 2, KQ_TQ1_G128>(tx, tw, ty, p, grid, s)
+                                 : launch_kernel<__nv_bfloat16, false, 2, KQ_TQ1_G128>(tx, tw, ty, p, grid, s);
+        return ydt == KQ_F32 ? launch_kernel<float, false, 1, KQ_TQ1_G128>(tx, tw, ty, p, grid, s)
+                             : launch_kernel<__nv_bfloat16, false, 1, KQ_TQ1_G128>(tx, tw, ty, p, grid, s);
+    }
     if (cps == 2)
         return ydt == KQ_F32 ? launch_kernel<float, false, 2>(tx, tw, ty, p, grid, s)
                              : launch_kernel<__nv_bfloat16, false, 2>(tx, tw, ty, p, grid, s);
@@ -682,8 +816,9 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     p.n = (int)a.n; p.k = (int)a.k; p.m = (int)a.n_tokens;
     p.n_tiles = (int)((a.n + BM - 1) / BM);
     p.bn = bn;
+    if (a.type != KQ_Q4_K) return cudaErrorNotSupported;
     const int cps = cps_for(bn);
-    if (!fill_ring(&p, cps)) return cudaErrorNotSupported;
+    if (!fill_ring(&p, cps, KQ_Q4_K)) return cudaErrorNotSupported;
     p.y = a.y;
     p.err = error_word();
     p.perm = a.perm;
@@ -695,7 +830,7 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     p.n_experts = (int)a.n_experts;
     CUtensorMap tx, tw;
     if (!encode_x_map(&tx, a.x, a.x_rows(), a.k, 1) ||
-        !encode_w_map(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride))
+        !encode_w_map(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride, KQ_Q4_K))
         return cudaErrorInvalidValue;
     // persistent grid: the number of token tiles is only known on the device
     const int64_t max_units = (a.n_tokens * a.top_k / bn + a.n_experts) * p.n_tiles;

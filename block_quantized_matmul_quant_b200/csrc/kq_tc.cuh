@@ -164,9 +164,10 @@ __device__ __forceinline__ void tmem_ld4x8(uint32_t base, uint32_t r[32]) {
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
 // Activations [rows, k] bf16: 64-column boxes of box_rows rows, 128-byte swizzle.
 bool encode_x_map(CUtensorMap *m, const void *x, int64_t rows, int64_t k, int box_rows);
-// Raw Q4_K rows of one or more experts: (row bytes, rows, experts), one
-// super-block column of 128 rows per box.
+// Raw rows of one or more experts: (row bytes, rows, experts), one raw unit
+// column of 128 rows per box: a Q4_K super-block (type KQ_Q4_K) or four
+// TQ1_G128 blocks (KQ_TQ1_G128, K % 512 == 0).
 bool encode_w_map(CUtensorMap *m, const void *w, int64_t n, int64_t k, int64_t n_experts,
-                  int64_t expert_stride);
+                  int64_t expert_stride, int type);
 
 }  // namespace kq

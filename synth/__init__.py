@@ -204,6 +204,7 @@ WORKLOADS = {
         Workload("moe_q4_k_e64_1408x2048_t32_top6", "moe", Q4_K, 1408, 2048, 32, "bf16", "f32",
                  n_experts=64, top_k=6),
         Workload("tq1_g128_gemv_5120x17408", "gemv", TQ1_G128, 5120, 17408, 1, "bf16", "f32"),
+        Workload("tq1_g128_gemm_512x5120x17408", "gemm", TQ1_G128, 5120, 17408, 512, "bf16", "bf16"),
     )
 }
 

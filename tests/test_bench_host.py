@@ -127,7 +127,7 @@ def test_secondary_metrics_call_site(monkeypatch):
     fake_torch = types.SimpleNamespace(cuda=types.SimpleNamespace(empty_cache=lambda: None))
     out = bench.secondary_metrics(fake_torch, None, 0, PEAKS)
     assert set(out) == {"q4_k_gemm_512x11008x4096", "moe_q4_k_e64_1408x2048_t32_top6",
-                        "tq1_g128_gemv_5120x17408", "q8_0_gemv_256x1024",
+                        "tq1_g128_gemv_5120x17408", "tq1_g128_gemm_512x5120x17408", "q8_0_gemv_256x1024",
                         "moe_q4_k_e64_1408x2048_t32_top6_glu"}
     glu = out["moe_q4_k_e64_1408x2048_t32_top6_glu"]
     assert glu["vs_gate_up_pair_us"] == out["moe_q4_k_e64_1408x2048_t32_top6"]["gate_up_pair_us"]

@@ -321,12 +321,12 @@ GEMM_CASES = [
 ]
 
 
-def _bf16_weight_reference(w, k, x):
+def _bf16_weight_reference(w, k, x, codec=synth.Q4_K):
     """x @ bf16(decode_f32(w))^T in fp64: what the tensor-core path computes up
     to fp32 accumulation (weights rounded to nearest-even bf16)."""
     import torch
 
-    dec = oracle.decode_f32(synth.Q4_K, w, k)
+    dec = oracle.decode_f32(codec, w, k)
     wb = torch.from_numpy(dec).to(torch.bfloat16).to(torch.float64).numpy()
     return x.astype(np.float64) @ wb.T
 
@@ -346,6 +346,87 @@ def test_matmul_gemm_q4_k(kq, n, k, m):
     assert row_rel_err(y, _bf16_weight_reference(w, k, x)) <= FP32_PATH_TOL
     yb = kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMM, out_dtype=torch.bfloat16).float().cpu().numpy()
     assert row_rel_err(yb, ref) <= TOL["bf16"] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+TQ1_GEMM_CASES = [
+    # one tile and one raw unit; ragged weight rows and tokens with narrow
+    # token tiles (two 64-K atoms a stage); tokens past one tile; wide tiles
+    # (one atom a stage) over several tiles each way; the long rows of the
+    # measured TQ1 shape (34 raw units a tile, the raw ring lapped)
+    (128, 512, 5), (300, 1024, 37), (129, 2048, 64), (1000, 4096, 300), (640, 17408, 24),
+]
+
+
+@pytest.mark.parametrize("n,k,m", TQ1_GEMM_CASES)
+def test_matmul_gemm_tq1(kq, n, k, m):
+    """TQ1_G128 on the tensor cores: the weights enter the MMA as
+    bf16(scale) * (t - 1), the round-to-nearest-even bf16 of the decoded
+    weight, so the product equals the bf16-weight product up to fp32
+    accumulation; illegal code bytes (a full byte above 242, a tail byte
+    above 26) decode to zeros as everywhere else."""
+    import torch
+
+    r = rng(2000 + n + k + m)
+    w = synth.gen_weights(synth.TQ1_G128, n, k, r)
+    w[0, 5] = 243
+    w[n - 1, (k // 128 - 1) * 28 + 25] = 27
+    w[n // 2, 28 + 12] = 255    # the byte shared by both 64-weight halves of a block
+    x = synth.gen_x(m, k, "bf16", r)
+    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    y = kq.matmul(wd, synth.TQ1_G128, xd, path=kq.PATH_GEMM).cpu().numpy()
+    ref = oracle.matmul(synth.TQ1_G128, w, k, x, threads=8)
+    assert row_rel_err(y, ref) <= TOL["bf16"]
+    assert row_rel_err(y, _bf16_weight_reference(w, k, x, synth.TQ1_G128)) <= FP32_PATH_TOL
+    yb = kq.matmul(wd, synth.TQ1_G128, xd, path=kq.PATH_GEMM,
+                   out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert row_rel_err(yb, ref) <= TOL["bf16"] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+def test_matmul_gemm_tq1_decodes_every_byte_exactly(kq):
+    """Every byte value at every code position (full bytes 0..24 and the tail
+    byte 25 of each block, legal or not) under scales of both signs: with the
+    identity as activations each output is one decoded weight, which must be
+    the round-to-nearest-even bf16 of the oracle's decode."""
+    import torch
+
+    n, k = 128, 512
+    r = rng(43)
+    w = np.zeros((n, k // 128 * 28), dtype=np.uint8)
+    for row in range(n):
+        for b in range(k // 128):
+            pos = np.arange(26)
+            w[row, 28 * b + pos] = (pos * 37 + row * 2 + b * 128 + row // 64) % 256
+            sc = np.float16(r.uniform(0.01, 2.0) * (-1.0 if (row + b) % 3 == 0 else 1.0))
+            w[row, 28 * b + 26: 28 * b + 28] = np.frombuffer(sc.tobytes(), dtype=np.uint8)
+    # every (value, position) pair occurs: 256 values, 26 positions, 512 blocks
+    seen = {(int(w[i, 28 * b + j]), j) for i in range(n) for b in range(k // 128) for j in range(26)}
+    assert len(seen) == 256 * 26
+    x = np.eye(k, dtype=np.float32)
+    y = kq.matmul(to_device_w(w), synth.TQ1_G128, to_device_x(x, "bf16"), path=kq.PATH_GEMM).cpu().numpy()
+    dec = torch.from_numpy(oracle.decode_f32(synth.TQ1_G128, w, k)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(y, dec.T)   # -0 and +0 compare equal
+    assert kq.device_status() == 0
+
+
+def test_matmul_tq1_auto_prefill_uses_the_tensor_cores(kq):
+    r = rng(41)
+    n, k, m = 384, 2048, 40
+    w = synth.gen_weights(synth.TQ1_G128, n, k, r)
+    x = synth.gen_x(m, k, "bf16", r)
+    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    a = kq.matmul(wd, synth.TQ1_G128, xd).cpu().numpy()
+    g = kq.matmul(wd, synth.TQ1_G128, xd, path=kq.PATH_GEMM).cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), g.view(np.uint32))
+    assert row_rel_err(a, oracle.matmul(synth.TQ1_G128, w, k, x, threads=8)) <= TOL["bf16"]
+    # K not a multiple of 512: the plain kernel
+    w2 = synth.gen_weights(synth.TQ1_G128, n, 1280, r)
+    x2 = synth.gen_x(m, 1280, "bf16", r)
+    with pytest.raises(kq.KQError):
+        kq.matmul(to_device_w(w2), synth.TQ1_G128, to_device_x(x2, "bf16"), path=kq.PATH_GEMM)
+    y2 = kq.matmul(to_device_w(w2), synth.TQ1_G128, to_device_x(x2, "bf16")).cpu().numpy()
+    assert row_rel_err(y2, oracle.matmul(synth.TQ1_G128, w2, 1280, x2, threads=8)) <= TOL["bf16"]
     assert kq.device_status() == 0
 
 
@@ -391,10 +472,11 @@ def test_workload_full_size(kq, name):
     assert err <= TOL[wl.x_dtype], err
 
 
-def test_workload_prefill_gemm_sampled_rows(kq):
-    wl = synth.WORKLOADS["q4_k_gemm_512x11008x4096"]
+@pytest.mark.parametrize("name", ["q4_k_gemm_512x11008x4096", "tq1_g128_gemm_512x5120x17408"])
+def test_workload_prefill_gemm_sampled_rows(kq, name):
+    wl = synth.WORKLOADS[name]
     # rows at tile boundaries plus a random sample
-    rows = np.concatenate([np.arange(0, wl.n, 997), [127, 128, 255, 256, 11007 - 128],
+    rows = np.concatenate([np.arange(0, wl.n, 997), [127, 128, 255, 256, wl.n - 1 - 128],
                            rng(3).integers(0, wl.n, 40)])
     err = _workload_check(kq, wl.name, sample_rows=rows)
     assert err <= TOL[wl.x_dtype], err
