@@ -253,7 +253,7 @@ int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, i
                                            : const_w ? GemvOrder::kConstWeights : GemvOrder::kStream,
                                      s));
     default:
-        return to_status(launch_simple_matmul(type, w, n, k, x, x_dtype, m, y, y_dtype, s));
+        return to_status(launch_simple_matmul(type, w, n, k, x, x_dtype, m, y, y_dtype, s, indep));
     }
 }
 

@@ -29,8 +29,10 @@ struct IdArgs {
 
 cudaError_t launch_dequant(int type, const void *w, int64_t rows, int64_t k, void *out, int dt,
                            cudaStream_t s);
+// The plain product; `independent`: the call may overlap the preceding
+// kernel (KQ_FLAG_INDEPENDENT), else it runs after it.
 cudaError_t launch_simple_matmul(int type, const void *w, int64_t n, int64_t k, const void *x,
-                                 int xdt, int64_t m, void *y, int ydt, cudaStream_t s);
+                                 int xdt, int64_t m, void *y, int ydt, cudaStream_t s, bool independent = false);
 cudaError_t launch_tq1_scan(const void *w, int64_t blocks, unsigned long long *first_bad,
                             cudaStream_t s);
 cudaError_t launch_get_rows(int type, const void *w, int64_t rows, int64_t k, const int32_t *ids,

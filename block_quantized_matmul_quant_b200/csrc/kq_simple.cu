@@ -6,6 +6,7 @@
 // fp32.  The plain product is the general-purpose path; the shape-specialised
 // kernels (kq_gemv.cu, kq_gemm_sm100.cu) serve the measured workloads.
 #include "kq_decode.cuh"
+#include "kq_ptx.cuh"
 #include "kq_launch.h"
 
 namespace kq {
@@ -44,9 +45,8 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict_
 // One warp per (weight row, group of up to 4 activation rows).  Lanes stride
 // over the row's 8-weight units; a warp shuffle reduces the partial sums.
 template <int TYPE, typename XT, typename YT>
-__global__ void __launch_bounds__(256) simple_matmul_kernel(
-    const uint8_t *__restrict__ w, int64_t n, int64_t k, const XT *__restrict__ x, int64_t m,
-    YT *__restrict__ y) {
+__device__ __forceinline__ void simple_matmul_rows(const uint8_t *__restrict__ w, int64_t n, int64_t k,
+                                                   const XT *__restrict__ x, int64_t m, YT *__restrict__ y) {
     using G = Geom<TYPE>;
     using U = Unit<TYPE>;
     constexpr int TB = 4;
@@ -84,6 +84,20 @@ __global__ void __launch_bounds__(256) simple_matmul_kernel(
         const int64_t xm = mg * TB + t;
         if (lane == 0 && xm < m) store_out(y + xm * n + row, v);
     }
+}
+
+// Launched as a programmatic dependent: it lets the next kernel launch at
+// once and waits for the preceding one before touching memory, or, for an
+// independent call (`indep`), only before it completes (stream order of
+// completion), so that consecutive independent calls overlap.
+template <int TYPE, typename XT, typename YT>
+__global__ void __launch_bounds__(256) simple_matmul_kernel(
+    const uint8_t *__restrict__ w, int64_t n, int64_t k, const XT *__restrict__ x, int64_t m,
+    YT *__restrict__ y, int indep) {
+    griddep_launch_dependents();
+    if (!indep) griddep_wait();
+    simple_matmul_rows<TYPE>(w, n, k, x, m, y);
+    if (indep) griddep_wait();
 }
 
 // ---------------------------------------------------------------- row gather
@@ -178,34 +192,43 @@ cudaError_t launch_dequant(int type, const void *w, int64_t rows, int64_t k, voi
 
 template <int TYPE, typename XT, typename YT>
 static cudaError_t simple_t(const void *w, int64_t n, int64_t k, const void *x, int64_t m, void *y,
-                            cudaStream_t s) {
+                            bool indep, cudaStream_t s) {
     const int64_t warps = n * ((m + 3) / 4);
     const int64_t blocks = (warps + 7) / 8;
-    simple_matmul_kernel<TYPE, XT, YT><<<(unsigned)blocks, 256, 0, s>>>(
-        static_cast<const uint8_t *>(w), n, k, static_cast<const XT *>(x), m, static_cast<YT *>(y));
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, simple_matmul_kernel<TYPE, XT, YT>, static_cast<const uint8_t *>(w), n, k,
+                              static_cast<const XT *>(x), m, static_cast<YT *>(y), indep ? 1 : 0);
 }
 
 template <int TYPE>
 static cudaError_t simple_xy(const void *w, int64_t n, int64_t k, const void *x, int xdt, int64_t m,
-                             void *y, int ydt, cudaStream_t s) {
+                             void *y, int ydt, bool indep, cudaStream_t s) {
     if (xdt == KQ_F32) {
-        if (ydt == KQ_F32) return simple_t<TYPE, float, float>(w, n, k, x, m, y, s);
-        return simple_t<TYPE, float, __nv_bfloat16>(w, n, k, x, m, y, s);
+        if (ydt == KQ_F32) return simple_t<TYPE, float, float>(w, n, k, x, m, y, indep, s);
+        return simple_t<TYPE, float, __nv_bfloat16>(w, n, k, x, m, y, indep, s);
     }
-    if (ydt == KQ_F32) return simple_t<TYPE, __nv_bfloat16, float>(w, n, k, x, m, y, s);
-    return simple_t<TYPE, __nv_bfloat16, __nv_bfloat16>(w, n, k, x, m, y, s);
+    if (ydt == KQ_F32) return simple_t<TYPE, __nv_bfloat16, float>(w, n, k, x, m, y, indep, s);
+    return simple_t<TYPE, __nv_bfloat16, __nv_bfloat16>(w, n, k, x, m, y, indep, s);
 }
 
 cudaError_t launch_simple_matmul(int type, const void *w, int64_t n, int64_t k, const void *x,
-                                 int xdt, int64_t m, void *y, int ydt, cudaStream_t s) {
+                                 int xdt, int64_t m, void *y, int ydt, cudaStream_t s, bool independent) {
+    const bool ind = independent;
     switch (type) {
-    case KQ_Q8_0: return simple_xy<KQ_Q8_0>(w, n, k, x, xdt, m, y, ydt, s);
-    case KQ_Q4_K: return simple_xy<KQ_Q4_K>(w, n, k, x, xdt, m, y, ydt, s);
-    case KQ_Q2_K: return simple_xy<KQ_Q2_K>(w, n, k, x, xdt, m, y, ydt, s);
-    case KQ_Q5_K: return simple_xy<KQ_Q5_K>(w, n, k, x, xdt, m, y, ydt, s);
-    case KQ_Q6_K: return simple_xy<KQ_Q6_K>(w, n, k, x, xdt, m, y, ydt, s);
-    case KQ_TQ1_G128: return simple_xy<KQ_TQ1_G128>(w, n, k, x, xdt, m, y, ydt, s);
+    case KQ_Q8_0: return simple_xy<KQ_Q8_0>(w, n, k, x, xdt, m, y, ydt, ind, s);
+    case KQ_Q4_K: return simple_xy<KQ_Q4_K>(w, n, k, x, xdt, m, y, ydt, ind, s);
+    case KQ_Q2_K: return simple_xy<KQ_Q2_K>(w, n, k, x, xdt, m, y, ydt, ind, s);
+    case KQ_Q5_K: return simple_xy<KQ_Q5_K>(w, n, k, x, xdt, m, y, ydt, ind, s);
+    case KQ_Q6_K: return simple_xy<KQ_Q6_K>(w, n, k, x, xdt, m, y, ydt, ind, s);
+    case KQ_TQ1_G128: return simple_xy<KQ_TQ1_G128>(w, n, k, x, xdt, m, y, ydt, ind, s);
     default: return cudaErrorInvalidValue;
     }
 }

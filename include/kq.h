@@ -98,8 +98,8 @@ extern "C" {
  * writes y (e.g. separate projections of one activation, or a batch of
  * weight matrices).  The kernel then never waits for the preceding kernel:
  * consecutive independent calls stream their weights concurrently.  Implies
- * KQ_FLAG_CONST_WEIGHTS.  Honoured by the bandwidth kernel; other paths
- * keep stream order. */
+ * KQ_FLAG_CONST_WEIGHTS.  Honoured by the bandwidth kernels and the plain
+ * kernel (KQ_PATH_SIMPLE); the tensor-core paths keep stream order. */
 #define KQ_FLAG_INDEPENDENT 0x200
 
 /* Weights per block and bytes per block of a codec; 0 for an unknown codec. */

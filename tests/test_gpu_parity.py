@@ -227,36 +227,40 @@ def test_matmul_gemv_nonfinite_activations(kq, codec, n, k):
     assert kq.device_status() == 0
 
 
-def test_matmul_gemv_independent_calls_back_to_back(kq):
+@pytest.mark.parametrize("codec,n,path_name,tol", [(synth.Q4_K, 4096, "PATH_GEMV", GEMV_TOL),
+                                                   (synth.Q8_0, 1024, "PATH_SIMPLE", FP32_PATH_TOL)])
+def test_matmul_independent_calls_back_to_back(kq, codec, n, path_name, tol):
     """Many independent calls queued on one stream (they run side by side),
     then an ordinary call, queued right behind them, that reads the first
     call's output as its activations: every result must be the one computed
-    alone, and the ordinary call must see the finished output."""
+    alone, and the ordinary call must see the finished output (the bandwidth
+    kernel, and the plain kernel that serves Q8_0)."""
     import torch
 
+    path = getattr(kq, path_name)
     r = rng(23)
-    n = k = 4096
-    ws = [synth.gen_weights(synth.Q4_K, n, k, r) for _ in range(3)]
+    k = n
+    ws = [synth.gen_weights(codec, n, k, r) for _ in range(3)]
     x = synth.gen_x(1, k, "bf16", r)
     wds = [to_device_w(w) for w in ws]
     xd = to_device_x(x, "bf16")
-    alone = [kq.matmul(wd, synth.Q4_K, xd, path=kq.PATH_GEMV).cpu().numpy() for wd in wds]
+    alone = [kq.matmul(wd, codec, xd, path=path).cpu().numpy() for wd in wds]
     outs = [torch.full((1, n), float("nan"), device="cuda") for _ in range(24)]
     y2 = torch.empty((1, n), device="cuda")
     torch.cuda.synchronize()
     for i, o in enumerate(outs):
-        kq.matmul(wds[i % 3], synth.Q4_K, xd, out=o, path=kq.PATH_GEMV, independent=True)
-    kq.matmul(wds[1], synth.Q4_K, outs[0], out=y2, path=kq.PATH_GEMV)   # fp32 x = outs[0]
+        kq.matmul(wds[i % 3], codec, xd, out=o, path=path, independent=True)
+    kq.matmul(wds[1], codec, outs[0], out=y2, path=path)   # fp32 x = outs[0]
     for i, o in enumerate(outs):
         assert np.array_equal(o.cpu().numpy().view(np.uint32), alone[i % 3].view(np.uint32))
-    ref2 = oracle.matmul(synth.Q4_K, ws[1], k, alone[0].astype(np.float64), threads=8)
-    assert row_rel_err(y2.cpu().numpy(), ref2) <= GEMV_TOL
+    ref2 = oracle.matmul(codec, ws[1], k, alone[0].astype(np.float64), threads=8)
+    assert row_rel_err(y2.cpu().numpy(), ref2) <= tol
     assert kq.device_status() == 0
 
 
 def test_independent_flag_on_other_paths_keeps_stream_order(kq):
-    """The flag is honoured by the bandwidth kernels only; the plain and the
-    tensor-core kernels keep stream order and give their usual result."""
+    """The flag lets the plain kernel overlap the preceding kernel and leaves
+    the tensor-core kernels in stream order; both give their usual result."""
     import torch
 
     r = rng(31)
