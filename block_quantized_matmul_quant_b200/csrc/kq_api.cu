@@ -184,10 +184,10 @@ constexpr int64_t ID_TC_I8_MAX_PAIRS_PER_EXPERT = 1;
 constexpr int64_t TQ1_GEMV_MAX_M = 8;
 // Activation rows from which the tensor-core kernel serves TQ1 products.
 // Measured on B200 (TQ1_G128 5120 x 17408, bf16, us per call, bandwidth vs
-// tensor-core kernel): 4 rows 56.4 vs 116.2, 8 rows 111.9 vs 116.2, 12 rows
-// 167.5 vs 116.3 (the tensor-core kernel has only 40 weight-row tiles here,
-// so its time stays flat up to 16 rows; 512 rows 167.9).
-constexpr int64_t TQ1_GEMM_MIN_M = TQ1_GEMV_MAX_M + 1;
+// tensor-core kernel): 6 rows 84.5 vs 101.1, 8 rows 112.4 vs 101.2, 12 rows
+// 168.3 vs 101.2 (the tensor-core kernel has only 40 weight-row tiles here,
+// so its time stays flat up to 128 rows; 512 rows 136.3).
+constexpr int64_t TQ1_GEMM_MIN_M = 8;
 
 }  // namespace kq
 

@@ -202,24 +202,24 @@ __device__ __forceinline__ uint32_t tq1_word(uint32_t dd, __nv_bfloat162 s2) {
     return *reinterpret_cast<const uint32_t *>(&t);
 }
 
-// Weights 64 H .. 64 H + 63 of block B of a row's raw TQ1 unit (four
-// 28-byte blocks, 112 bytes from `row`, 16-byte aligned) as 32 bf16x2 words
-// of bf16(scale) * (t - 1), word j holding weights 64 H + 2 j and + 1.
-// Weight i of a block is digit i % 5 of byte i / 5 (the tail byte 25 holds
-// weights 125..127); a full byte above 242 or a tail byte above 26 is not a
-// code and decodes to zeros (as byte 121, all digits 1).
-template <int B, int H>
-__device__ __forceinline__ void tq1_decode64(const uint8_t *row, uint32_t out[32]) {
-    constexpr int LO = 28 * B + 12 * H;         // first byte needed (byte 12 of a block is in both halves)
-    constexpr int C0 = LO / 16, C1 = (28 * B + 27) / 16;   // 16-byte chunks through the scale
-    uint32_t wv[4 * (C1 - C0 + 1)];
+// Weights 64 H .. 64 H + 63 of the TQ1_G128 block at `blk` (4-byte aligned)
+// as 32 bf16x2 words of bf16(scale) * (t - 1), word j holding weights
+// 64 H + 2 j and + 1.  Weight i of a block is digit i % 5 of byte i / 5 (the
+// tail byte 25 holds weights 125..127); a full byte above 242 or a tail
+// byte above 26 is not a code and decodes to zeros (as byte 121, all digits
+// 1).  The block's position in the raw unit is a runtime offset, so the
+// decoders hold two copies of this code (one per half), not one per chunk
+// position: fewer instructions to fetch.
+template <int H>
+__device__ __forceinline__ void tq1_decode64(const uint8_t *blk, uint32_t out[32]) {
+    // block words: half 0 needs bytes 0..12 (words 0..3) and the scale (word
+    // 6), half 1 bytes 12..27 (words 3..6)
+    const uint32_t *bw = reinterpret_cast<const uint32_t *>(blk);
+    uint32_t wv[7];
     #pragma unroll
-    for (int c = C0; c <= C1; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(row + 16 * c);
-        wv[4 * (c - C0)] = v.x; wv[4 * (c - C0) + 1] = v.y; wv[4 * (c - C0) + 2] = v.z; wv[4 * (c - C0) + 3] = v.w;
-    }
-    const uint32_t sbits = wv[(28 * B + 26) / 4 - 4 * C0] >> 16;   // bytes 26..27: fp16 scale
-    const __nv_bfloat16 sb = __float2bfloat16_rn(half_bits_to_float(sbits));
+    for (int q = 0; q < 7; ++q)
+        if ((H == 0 && (q <= 3 || q == 6)) || (H == 1 && q >= 3)) wv[q] = bw[q];
+    const __nv_bfloat16 sb = __float2bfloat16_rn(half_bits_to_float(wv[6] >> 16));   // bytes 26..27
     const __nv_bfloat162 s2 = __halves2bfloat162(sb, sb);
     // digit words of block bytes J0 .. J0 + 13 (13 used by half 0)
     constexpr int J0 = H == 0 ? 0 : 12;
@@ -228,8 +228,7 @@ __device__ __forceinline__ void tq1_decode64(const uint8_t *row, uint32_t out[32
     for (int jj = 0; jj < 14; ++jj) {
         const int j = J0 + jj;
         if (j > 25 || (H == 0 && j > 12)) continue;
-        const int i = 28 * B + j;
-        uint32_t b = (wv[i / 4 - 4 * C0] >> (8 * (i % 4))) & 0xFFu;
+        uint32_t b = (wv[j / 4] >> (8 * (j % 4))) & 0xFFu;
         b = b > (j == 25 ? 26u : 242u) ? 121u : b;
         tq1_digits(b, dg[jj][0], dg[jj][1], dg[jj][2]);
     }
@@ -248,16 +247,9 @@ __device__ __forceinline__ void tq1_decode64(const uint8_t *row, uint32_t out[32
 
 // 64-K chunk cc (0..7) of a row's raw TQ1 unit: half cc % 2 of block cc / 2.
 __device__ __forceinline__ void tq1_decode_chunk(const uint8_t *row, int cc, uint32_t out[32]) {
-    switch (cc) {
-    case 0: tq1_decode64<0, 0>(row, out); break;
-    case 1: tq1_decode64<0, 1>(row, out); break;
-    case 2: tq1_decode64<1, 0>(row, out); break;
-    case 3: tq1_decode64<1, 1>(row, out); break;
-    case 4: tq1_decode64<2, 0>(row, out); break;
-    case 5: tq1_decode64<2, 1>(row, out); break;
-    case 6: tq1_decode64<3, 0>(row, out); break;
-    default: tq1_decode64<3, 1>(row, out); break;
-    }
+    const uint8_t *blk = row + 28 * (cc >> 1);
+    if (cc & 1) tq1_decode64<1>(blk, out);
+    else tq1_decode64<0>(blk, out);
 }
 
 // CPS: 64-K swizzle atoms per pipeline stage (1, or 2 for narrow token tiles,
@@ -520,7 +512,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
                 const uint32_t sc_lo = hd.y & 0x3F3F3F3Fu, m_lo = hd.z & 0x3F3F3F3Fu;
                 const uint32_t sc_hi = (hd.w & 0x0F0F0F0Fu) | ((hd.y >> 2) & 0x30303030u);
                 const uint32_t m_hi = ((hd.w >> 4) & 0x0F0F0F0Fu) | ((hd.z >> 2) & 0x30303030u);
-                #pragma unroll
+                // A rolled loop: the chunk position stays a runtime value and
+                // the decode code is not copied per stage.  Instruction fetch
+                // was the top stall of the unrolled TQ1 decoders (eight
+                // chunk-specific copies); rolled, the TQ1 prefill went from
+                // 167.9 to 136.3 us and the Q4_K one from 68.5 to 65.7 us.
+                #pragma unroll 1
                 for (int st = 0; st < SPS; ++st) {
                     if ((int)(g & (DEC_GROUPS - 1)) == grp) {
                         // warp-uniform outcome: the TMEM stores below are .sync.aligned

@@ -133,7 +133,7 @@ KQ_API int kq_dequantize(int type, const void *w, int64_t rows, int64_t k,
  *   y[i][j] = sum_k dequant(w)[j][k] * x[i][k], fp32 accumulation.
  * Small m runs the bandwidth-bound kernel that decodes weights in
  * registers; large m with bf16 x (Q4_K from 5 rows, TQ1_G128 with
- * K % 512 == 0 from 9 rows) runs the tensor-core kernel, which rounds
+ * K % 512 == 0 from 8 rows) runs the tensor-core kernel, which rounds
  * decoded weights to bf16 before the bf16 x bf16 -> fp32 MMA (for TQ1:
  * (t - 1) times the bf16 rounding of the block scale, the same value).
  */
