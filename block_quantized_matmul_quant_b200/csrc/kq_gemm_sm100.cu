@@ -25,7 +25,8 @@
 //                         tcgen05.commit's to the stage / accumulator barriers;
 //                 warps 2-5  epilogue -- tcgen05.ld from TMEM, convert, store;
 //                 warps 7..  decoders, in groups of four warps (one per TMEM
-//                         lane quadrant, so lane = weight row): group j
+//                         lane quadrant, so lane = weight row; two groups
+//                         for Q4_K, four for TQ1_G128): group j
 //                         decodes the stages s with s % groups == j, 64 K
 //                         positions of its 32 rows per warp.  Q4_K: exact
 //                         fp32 (d*sc*q - dmin*m, one rounding) -> bf16 (round
@@ -63,14 +64,15 @@ template <int FMT> struct RawUnit;
 template <> struct RawUnit<KQ_Q4_K> { static constexpr int BYTES = 144, K = 256; };
 template <> struct RawUnit<KQ_TQ1_G128> { static constexpr int BYTES = 112, K = 512; };
 constexpr int raw_stage_bytes(int type) { return BM * (type == KQ_TQ1_G128 ? 112 : 144); }
-#ifndef KQ_GEMM_DEC_WARPS
-#define KQ_GEMM_DEC_WARPS 16
-#endif
 constexpr int RAW_WARP = 6;  // raw weight producer
-constexpr int DEC_WARP0 = 7, DEC_WARPS = KQ_GEMM_DEC_WARPS;  // 8 or 16
-constexpr int DEC_GROUPS = DEC_WARPS / 4;                    // 2 or 4
-static_assert(DEC_GROUPS == 2 || DEC_GROUPS == 4, "decoder warps come in 2 or 4 groups of 4");
-constexpr int NUM_THREADS = (DEC_WARP0 + DEC_WARPS) * 32;
+constexpr int DEC_WARP0 = 7;
+// Decoder warps per format: eight (two groups) for Q4_K; sixteen (four
+// groups) for TQ1_G128, whose integer digit decode bounds the narrow tiles.
+// Measured on B200 (µs): Q4_K 512x11008x4096 65.9 with eight against 67.7
+// with sixteen, 16 rows 25.8 against 26.3; TQ1 512x5120x17408 135.9 against
+// 140.0 but 16 rows 108.0 against 101.0.
+template <int FMT> constexpr int dec_warps() { return FMT == KQ_TQ1_G128 ? 16 : 8; }
+template <int FMT> constexpr int num_threads() { return (DEC_WARP0 + dec_warps<FMT>()) * 32; }
 constexpr int EPI_WARP0 = 2;
 constexpr int MAX_RAW_STAGES = 8;
 constexpr int MAX_A_STAGES = 8;   // TMEM A slots
@@ -285,6 +287,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int SPS = UNIT_K / (BK * CPS);   // stages per raw unit
+    constexpr int DEC_WARPS_T = dec_warps<FMT>(), DEC_GROUPS_T = DEC_WARPS_T / 4;
+    static_assert(DEC_GROUPS_T == 2 || DEC_GROUPS_T == 4, "decoder warps come in 2 or 4 groups of 4");
     const int nk = p.k / (BK * CPS);       // stages per tile
 
     if (threadIdx.x == 0) {
@@ -298,7 +302,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
         }
         for (int r = 0; r < SR; ++r) {
             mbar_init(&raw_full[r], 1);
-            mbar_init(&raw_empty[r], DEC_WARPS);
+            mbar_init(&raw_empty[r], DEC_WARPS_T);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
@@ -487,7 +491,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
     } else {
         // ---------------- decoders ----------------
         // Group grp (four consecutive warps, one per TMEM lane quadrant)
-        // decodes stage g when g % DEC_GROUPS == grp.  Lane l of a warp in
+        // decodes stage g when g % DEC_GROUPS_T == grp.  Lane l of a warp in
         // quadrant q owns weight row r = 32 q + l: per stage it reads the
         // row's 32 quant bytes of chunk cc = g % 4 (low nibbles: K positions
         // 0..31 of the stage = sub-block 2cc, high nibbles: K 32..63 =
@@ -519,7 +523,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
                 // 167.9 to 136.3 us and the Q4_K one from 68.5 to 65.7 us.
                 #pragma unroll 1
                 for (int st = 0; st < SPS; ++st) {
-                    if ((int)(g & (DEC_GROUPS - 1)) == grp) {
+                    if ((int)(g & (DEC_GROUPS_T - 1)) == grp) {
                         // warp-uniform outcome: the TMEM stores below are .sync.aligned
                         ok = warp_wait(&empty_a[slot], phase ^ 1, p.err);
                         if (!ok) break;
@@ -576,14 +580,14 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
 }
 
 template <typename YT, bool ID, int CPS>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(num_threads<KQ_Q4_K>(), 1)
     gemm_q4k_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                     const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
     gemm_body<YT, ID, CPS, KQ_Q4_K>(tmap_x, tmap_w, tmap_y, p);
 }
 
 template <typename YT, bool ID, int CPS>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(num_threads<KQ_TQ1_G128>(), 1)
     gemm_tq1_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                     const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
     gemm_body<YT, ID, CPS, KQ_TQ1_G128>(tmap_x, tmap_w, tmap_y, p);
@@ -748,7 +752,7 @@ cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CU
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.blockDim = dim3(num_threads<FMT>());
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
