@@ -559,15 +559,18 @@ __global__ void __launch_bounds__(MM_THREADS, 1)
                     dm[j] = dmin * mm_byte_f(j < 4 ? m_lo : m_hi, j & 3);    // exact
                     c[j] = fmaf(128.0f, a[j], dm[j]);
                 }
-                const bool gate = p.glu && s < nk;
-                if (nf) {
-                    if (gate) exact(accg, blk, dm, s);
-                    else exact(acc, blk, dm, s);
-                } else if (gate) {
-                    apply(accg, b, s);
-                } else {
-                    apply(acc, b, s);
+                // every stage adds into acc; the GLU form's gate sums move to
+                // accg when its up pass starts (one copy of each accumulate
+                // path in the code, not one per target)
+                if (p.glu && s == nk) {
+                    #pragma unroll
+                    for (int t = 0; t < MM_BN; ++t) {
+                        accg[t] = acc[t];
+                        acc[t] = 0.f;
+                    }
                 }
+                if (nf) exact(acc, blk, dm, s);
+                else apply(acc, b, s);
                 tc_fence_before();
                 fence_proxy_async_smem();   // generic reads of the raw slot before TMA refills it
                 __syncwarp();
