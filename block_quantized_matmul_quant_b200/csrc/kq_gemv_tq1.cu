@@ -111,7 +111,6 @@ struct Tq1SplitParams {
     int slot_bytes;
     int row_bytes;
     int smem_bytes;     // dynamic shared memory of the launch
-    int early;          // weights constant: copies go out before griddepcontrol.wait
     int indep;          // independent call: never wait for the preceding kernel
     unsigned int *err;
 };
@@ -248,14 +247,10 @@ __global__ void __launch_bounds__(T1_THREADS, 1) gemv_tq1_split_kernel(const Tq1
         fence_mbar_init();
         mbar_arrive_expect_tx(tbar, T1_TABLE_BYTES);
         bulk_g2s(sp(lay.tab), &g_prefix_table, T1_TABLE_BYTES, tbar);
-        if (p.early)
-            for (int i = 0; i < min(S, n_batches); ++i) issue(i);
     }
     if (tid < 4) s_flags[tid] = 0;
     for (int i = tid; i < S; i += blockDim.x) s_slot[i] = slot_addr(i);
     if (!p.indep) griddep_wait();
-    if (!p.early && warp == T1_PRODUCER_WARP && lane == 0)
-        for (int i = 0; i < min(S, n_batches); ++i) issue(i);
     __syncthreads();
 
     // ---- activations: thread (b, c) of four per block takes positions
@@ -331,6 +326,13 @@ __global__ void __launch_bounds__(T1_THREADS, 1) gemv_tq1_split_kernel(const Tq1
             for (int i = 0; i < 4; ++i) zb[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
     }
+    // The ring's first copies go out only now, after the activations were
+    // read: issued earlier (before the wait for the preceding kernel, or
+    // before the activation loads), their 15 MB across the CTAs delayed the
+    // activation loads by more than they gained (measured 14.1 -> 13.6 us
+    // for independent calls, 14.8 -> 13.6 for ordered ones).
+    if (warp == T1_PRODUCER_WARP && lane == 0)
+        for (int i = 0; i < min(S, n_batches); ++i) issue(i);
     __syncthreads();
 
     // ---- step 2: item (b, j) turns the five codes of code byte j of block
@@ -850,7 +852,6 @@ cudaError_t launch_gemv_tq1(const void *w, int64_t n, int64_t k, const void *x, 
     Tq1SplitParams sp = {};
     if (plan_tq1_split(n, k, sms, &sp)) {
         sp.w = static_cast<const uint8_t *>(w);
-        sp.early = order != GemvOrder::kStream ? 1 : 0;
         sp.indep = order == GemvOrder::kIndependent ? 1 : 0;
         sp.err = error_word();
         for (int64_t m0 = 0; m0 < m; ++m0) {
