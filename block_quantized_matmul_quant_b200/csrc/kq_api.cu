@@ -188,6 +188,12 @@ constexpr int64_t TQ1_GEMV_MAX_M = 8;
 // 168.3 vs 101.2 (the tensor-core kernel has only 40 weight-row tiles here,
 // so its time stays flat up to 128 rows; 512 rows 136.3).
 constexpr int64_t TQ1_GEMM_MIN_M = 8;
+// Activation rows from which the tensor-core kernel serves Q8_0 products
+// (bf16 activations, K % 256 == 0); below it the plain kernel.  Measured on
+// B200 (Q8_0 4096 x 4096, us per call, plain vs tensor-core kernel): 1 row
+// 18.7 vs 24.6, 4 rows 31.4 vs 24.9, 16 rows 68.2 vs 24.9, 512 rows 1825 vs
+// 34.8.
+constexpr int64_t Q8_0_GEMM_MIN_M = 3;
 
 }  // namespace kq
 
@@ -231,7 +237,8 @@ int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, i
     const bool can_gemm = gemm_supported(type, n, k, x_dtype, y_dtype);
     const bool can_gemv = gemv_supported(type, n, k, x_dtype, m);
     if (path == KQ_PATH_AUTO) {
-        if (can_gemm && m >= (type == KQ_TQ1_G128 ? TQ1_GEMM_MIN_M : GEMM_MIN_M)) path = KQ_PATH_GEMM;
+        if (can_gemm && m >= (type == KQ_TQ1_G128 ? TQ1_GEMM_MIN_M : type == KQ_Q8_0 ? Q8_0_GEMM_MIN_M : GEMM_MIN_M))
+            path = KQ_PATH_GEMM;
         // fp32 activations past one pass of the bandwidth kernel: the
         // few-rows tensor-core kernel reads the weights once per 8 rows of a
         // tile instead of once per 8-row launch

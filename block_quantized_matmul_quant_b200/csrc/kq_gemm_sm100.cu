@@ -18,8 +18,9 @@
 //  * Warp roles:  warp 0  TMA producer of bf16 activation tiles (64 K x BN,
 //                         128-byte swizzle) into a shared-memory ring;
 //                 warp 6  TMA producer of raw weight units (128 rows x one
-//                         Q4_K super-block, 144 bytes, or four TQ1_G128
-//                         blocks, 112 bytes) into their own ring;
+//                         Q4_K super-block, 144 bytes, eight Q8_0 blocks,
+//                         272 bytes, or four TQ1_G128 blocks, 112 bytes)
+//                         into their own ring;
 //                 warp 1  MMA issuer -- one thread issues tcgen05.mma
 //                         (kind::f16, bf16 x bf16 -> fp32 in TMEM) and
 //                         tcgen05.commit's to the stage / accumulator barriers;
@@ -30,7 +31,8 @@
 //                         decodes the stages s with s % groups == j, 64 K
 //                         positions of its 32 rows per warp.  Q4_K: exact
 //                         fp32 (d*sc*q - dmin*m, one rounding) -> bf16 (round
-//                         to nearest even).  TQ1_G128 (Ternary Bonsai
+//                         to nearest even); Q8_0 likewise (d * q).
+//                         TQ1_G128 (Ternary Bonsai
 //                         `tq1_gemm`, the prefill form of the ternary
 //                         product): base-3 digits by integer arithmetic, two
 //                         bytes' digits a 32-bit word, then (t - 1) * bf16(scale)
@@ -60,14 +62,21 @@ constexpr int BK = 64;             // K per swizzle atom (128 bytes of bf16); a 
 // Raw weights move in units of one TMA box row: a Q4_K super-block (144
 // bytes, 256 K) or four TQ1_G128 blocks (112 bytes, 512 K; a box row must be
 // a multiple of 16 bytes, so TQ1 rows need K % 512 == 0).
+// Q8_0: eight 34-byte blocks (272 bytes, 256 K), copied as 16-bit elements
+// (a box row holds at most 256 elements).  ELEM: bytes per tensor-map
+// element.
 template <int FMT> struct RawUnit;
-template <> struct RawUnit<KQ_Q4_K> { static constexpr int BYTES = 144, K = 256; };
-template <> struct RawUnit<KQ_TQ1_G128> { static constexpr int BYTES = 112, K = 512; };
-constexpr int raw_stage_bytes(int type) { return BM * (type == KQ_TQ1_G128 ? 112 : 144); }
+template <> struct RawUnit<KQ_Q4_K> { static constexpr int BYTES = 144, K = 256, ELEM = 1; };
+template <> struct RawUnit<KQ_TQ1_G128> { static constexpr int BYTES = 112, K = 512, ELEM = 1; };
+template <> struct RawUnit<KQ_Q8_0> { static constexpr int BYTES = 272, K = 256, ELEM = 2; };
+constexpr int raw_unit_bytes(int type) { return type == KQ_TQ1_G128 ? 112 : type == KQ_Q8_0 ? 272 : 144; }
+constexpr int raw_unit_k(int type) { return type == KQ_TQ1_G128 ? 512 : 256; }
+constexpr int raw_stage_bytes(int type) { return BM * raw_unit_bytes(type); }
 constexpr int RAW_WARP = 6;  // raw weight producer
 constexpr int DEC_WARP0 = 7;
-// Decoder warps per format: eight (two groups) for Q4_K; sixteen (four
-// groups) for TQ1_G128, whose integer digit decode bounds the narrow tiles.
+// Decoder warps per format: eight (two groups) for Q4_K and Q8_0; sixteen
+// (four groups) for TQ1_G128, whose integer digit decode bounds the narrow
+// tiles.
 // Measured on B200 (µs): Q4_K 512x11008x4096 65.9 with eight against 67.7
 // with sixteen, 16 rows 25.8 against 26.3; TQ1 512x5120x17408 135.9 against
 // 140.0 but 16 rows 108.0 against 101.0.
@@ -248,6 +257,32 @@ __device__ __forceinline__ void tq1_decode64(const uint8_t *blk, uint32_t out[32
 }
 
 // 64-K chunk cc (0..7) of a row's raw TQ1 unit: half cc % 2 of block cc / 2.
+__device__ __forceinline__ void tq1_decode_chunk(const uint8_t *row, int cc, uint32_t out[32]);
+
+// 64-K chunk cc (0..3) of a row's raw Q8_0 unit (eight 34-byte blocks: fp16
+// d, then 32 int8 q; weight d * q): blocks 2 cc and 2 cc + 1, bytes
+// 68 cc .. 68 cc + 67 of the row (4-byte aligned), as 32 bf16x2 words of the
+// round-to-nearest-even bf16 of d * q.  The second block's codes are
+// word-aligned; the first block's sit two bytes in and are realigned with
+// funnel shifts.  Each code goes in as the byte q + 128 (xor 0x80) and
+// comes out as d * (q + 128) - 128 d in one fused rounding (decode4).
+__device__ __forceinline__ void q8_0_decode_chunk(const uint8_t *row, int cc, uint32_t out[32]) {
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(row + 68 * cc);
+    uint32_t v[17];
+    #pragma unroll
+    for (int i = 0; i < 17; ++i) v[i] = w[i];
+    const float d0 = half_f(v[0] & 0xFFFFu), d1 = half_f(v[8] >> 16);
+    const float2 s0 = make_float2(d0, d0), b0 = make_float2(-128.0f * d0, -128.0f * d0);
+    const float2 s1 = make_float2(d1, d1), b1 = make_float2(-128.0f * d1, -128.0f * d1);
+    #pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t qa = __funnelshift_r(v[j], v[j + 1], 16);   // block 2 cc: codes 4 j .. 4 j + 3
+        decode4(qa ^ 0x80808080u, s0, b0, out[2 * j], out[2 * j + 1]);
+        decode4(v[9 + j] ^ 0x80808080u, s1, b1, out[16 + 2 * j], out[17 + 2 * j]);
+    }
+}
+
+// 64-K chunk cc (0..7) of a row's raw TQ1 unit: half cc % 2 of block cc / 2.
 __device__ __forceinline__ void tq1_decode_chunk(const uint8_t *row, int cc, uint32_t out[32]) {
     const uint8_t *blk = row + 28 * (cc >> 1);
     if (cc & 1) tq1_decode64<1>(blk, out);
@@ -339,8 +374,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
                     ok = mbar_wait(&raw_empty[rslot], rphase ^ 1, p.err);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&raw_full[rslot], RAW_STAGE_BYTES);
-                    tma_load_3d(raw_ring + rslot * RAW_STAGE_BYTES, &tmap_w, sb * UNIT_BYTES, t.n0, t.e,
-                                &raw_full[rslot]);
+                    tma_load_3d(raw_ring + rslot * RAW_STAGE_BYTES, &tmap_w, sb * (UNIT_BYTES / RawUnit<FMT>::ELEM),
+                                t.n0, t.e, &raw_full[rslot]);
                     if (++rslot == (uint32_t)SR) { rslot = 0; rphase ^= 1; }
                 }
             }
@@ -534,6 +569,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
                         uint32_t out[32];
                         if constexpr (FMT == KQ_TQ1_G128) {
                             tq1_decode_chunk(blk, cc, out);
+                        } else if constexpr (FMT == KQ_Q8_0) {
+                            q8_0_decode_chunk(blk, cc, out);
                         } else {
                             const uint32_t scw = cc < 2 ? sc_lo : sc_hi, mw = cc < 2 ? m_lo : m_hi;
                             const int b0 = (2 * cc) & 3;
@@ -591,6 +628,13 @@ __global__ void __launch_bounds__(num_threads<KQ_TQ1_G128>(), 1)
     gemm_tq1_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                     const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
     gemm_body<YT, ID, CPS, KQ_TQ1_G128>(tmap_x, tmap_w, tmap_y, p);
+}
+
+template <typename YT, bool ID, int CPS>
+__global__ void __launch_bounds__(num_threads<KQ_Q8_0>(), 1)
+    gemm_q8_0_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                     const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+    gemm_body<YT, ID, CPS, KQ_Q8_0>(tmap_x, tmap_w, tmap_y, p);
 }
 
 // ---------------------------------------------------------------- host side
@@ -680,15 +724,16 @@ bool encode_x_map(CUtensorMap *m, const void *x, int64_t rows, int64_t k, int bo
 // column (a Q4_K super-block, or four TQ1_G128 blocks) of BM rows per box.
 bool encode_w_map(CUtensorMap *m, const void *w, int64_t n, int64_t k, int64_t n_experts,
                   int64_t expert_stride, int type) {
-    const int ub = type == KQ_TQ1_G128 ? RawUnit<KQ_TQ1_G128>::BYTES : RawUnit<KQ_Q4_K>::BYTES;
-    const int uk = type == KQ_TQ1_G128 ? RawUnit<KQ_TQ1_G128>::K : RawUnit<KQ_Q4_K>::K;
+    const int ub = raw_unit_bytes(type), uk = raw_unit_k(type);
+    const int el = type == KQ_Q8_0 ? 2 : 1;   // bytes per element of the map
     if (k % uk) return false;
     const int64_t rb = (k / uk) * ub;
-    cuuint64_t dims[3] = {(cuuint64_t)rb, (cuuint64_t)n, (cuuint64_t)n_experts};
+    cuuint64_t dims[3] = {(cuuint64_t)(rb / el), (cuuint64_t)n, (cuuint64_t)n_experts};
     cuuint64_t strides[2] = {(cuuint64_t)rb, (cuuint64_t)expert_stride};
-    cuuint32_t box[3] = {(cuuint32_t)ub, BM, 1};
+    cuuint32_t box[3] = {(cuuint32_t)(ub / el), BM, 1};
     cuuint32_t es[3] = {1, 1, 1};
-    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(w), dims, strides, box, es,
+    return encode_fn()(m, el == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                       const_cast<void *>(w), dims, strides, box, es,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -701,6 +746,8 @@ bool gemm_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype, bo
         if (k % 256) return false;
     } else if (type == KQ_TQ1_G128 && !expert_indexed) {
         if (k % 512) return false;   // the row pitch and box rows must be multiples of 16 bytes
+    } else if (type == KQ_Q8_0 && !expert_indexed) {
+        if (k % 256) return false;   // likewise: eight 34-byte blocks are 272 bytes
     } else {
         return false;
     }
@@ -747,6 +794,7 @@ cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CU
                         (size_t)p.raw_stages * raw_stage_bytes(FMT) + EPI_STAGE_BYTES + 2560;
     void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
     if constexpr (FMT == KQ_TQ1_G128) kern = gemm_tq1_kernel<YT, ID, CPS>;
+    else if constexpr (FMT == KQ_Q8_0) kern = gemm_q8_0_kernel<YT, ID, CPS>;
     else kern = gemm_q4k_kernel<YT, ID, CPS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -768,7 +816,7 @@ cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CU
 cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const void *x, int64_t m,
                         void *y, int ydt, cudaStream_t s) {
     if (!encode_fn() || m < 1 || m > (1 << 30)) return cudaErrorNotSupported;
-    if (type != KQ_Q4_K && type != KQ_TQ1_G128) return cudaErrorNotSupported;
+    if (type != KQ_Q4_K && type != KQ_TQ1_G128 && type != KQ_Q8_0) return cudaErrorNotSupported;
     const int sms = sm_count();
     GemmParams p = {};
     p.n = (int)n; p.k = (int)k; p.m = (int)m;
@@ -781,7 +829,7 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
     p.y = y;
     p.err = error_word();
     CUtensorMap tx, tw, ty;
-    const int64_t row_bytes = type == KQ_TQ1_G128 ? (k / 128) * 28 : (k / 256) * 144;
+    const int64_t row_bytes = (k / raw_unit_k(type)) * raw_unit_bytes(type);
     if (!encode_x_map(&tx, x, m, k, p.bn) || !encode_w_map(&tw, w, n, k, 1, n * row_bytes, type))
         return cudaErrorInvalidValue;
     p.y_tma = encode_y_map(&ty, y, m, n, ydt) ? 1 : 0;
@@ -793,6 +841,13 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
                                  : launch_kernel<__nv_bfloat16, false, 2, KQ_TQ1_G128>(tx, tw, ty, p, grid, s);
         return ydt == KQ_F32 ? launch_kernel<float, false, 1, KQ_TQ1_G128>(tx, tw, ty, p, grid, s)
                              : launch_kernel<__nv_bfloat16, false, 1, KQ_TQ1_G128>(tx, tw, ty, p, grid, s);
+    }
+    if (type == KQ_Q8_0) {
+        if (cps == 2)
+            return ydt == KQ_F32 ? launch_kernel<float, false, 2, KQ_Q8_0>(tx, tw, ty, p, grid, s)
+                                 : launch_kernel<__nv_bfloat16, false, 2, KQ_Q8_0>(tx, tw, ty, p, grid, s);
+        return ydt == KQ_F32 ? launch_kernel<float, false, 1, KQ_Q8_0>(tx, tw, ty, p, grid, s)
+                             : launch_kernel<__nv_bfloat16, false, 1, KQ_Q8_0>(tx, tw, ty, p, grid, s);
     }
     if (cps == 2)
         return ydt == KQ_F32 ? launch_kernel<float, false, 2>(tx, tw, ty, p, grid, s)

@@ -414,6 +414,58 @@ def test_matmul_gemm_tq1_decodes_every_byte_exactly(kq):
     assert kq.device_status() == 0
 
 
+Q8_0_GEMM_CASES = [
+    # one tile and one raw unit (eight blocks); ragged rows and tokens with
+    # narrow token tiles; wide tiles over several tiles each way; long rows
+    (128, 256, 5), (300, 1024, 37), (1000, 4096, 300), (129, 8192, 64),
+]
+
+
+@pytest.mark.parametrize("n,k,m", Q8_0_GEMM_CASES)
+def test_matmul_gemm_q8_0(kq, n, k, m):
+    """Q8_0 on the tensor cores: each weight enters the MMA as the
+    round-to-nearest-even bf16 of d * q, so the product equals the
+    bf16-weight product up to fp32 accumulation."""
+    import torch
+
+    r = rng(3000 + n + k + m)
+    w = synth.gen_weights(synth.Q8_0, n, k, r)
+    x = synth.gen_x(m, k, "bf16", r)
+    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    y = kq.matmul(wd, synth.Q8_0, xd, path=kq.PATH_GEMM).cpu().numpy()
+    ref = oracle.matmul(synth.Q8_0, w, k, x, threads=8)
+    assert row_rel_err(y, ref) <= TOL["bf16"]
+    assert row_rel_err(y, _bf16_weight_reference(w, k, x, synth.Q8_0)) <= FP32_PATH_TOL
+    yb = kq.matmul(wd, synth.Q8_0, xd, path=kq.PATH_GEMM, out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert row_rel_err(yb, ref) <= TOL["bf16"] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+def test_matmul_gemm_q8_0_decodes_every_code_exactly(kq):
+    """Every int8 code at every position of the eight-block raw unit, under
+    scales of both signs (normal and subnormal fp16): with the identity as
+    activations each output is one decoded weight, which must be the
+    round-to-nearest-even bf16 of the oracle's decode."""
+    import torch
+
+    n, k = 256, 256
+    r = rng(47)
+    w = np.zeros((n, k // 32 * 34), dtype=np.uint8)
+    scales = [0.5, -0.25, 1.0e-3, -3.0e-2, 6.0e-8, -1.5, 7.0, 2.0 ** -14]
+    for row in range(n):
+        for b in range(k // 32):
+            sc = np.float16(scales[(row + b) % len(scales)] * (1.0 + (row % 7) / 16.0))
+            w[row, 34 * b: 34 * b + 2] = np.frombuffer(sc.tobytes(), dtype=np.uint8)
+            w[row, 34 * b + 2: 34 * b + 34] = (np.arange(32) * 8 + row + 3 * b) % 256
+    seen = {(int(w[i, 34 * b + 2 + j]), 32 * b + j) for i in range(n) for b in range(k // 32) for j in range(32)}
+    assert len(seen) == 256 * k
+    x = np.eye(k, dtype=np.float32)
+    y = kq.matmul(to_device_w(w), synth.Q8_0, to_device_x(x, "bf16"), path=kq.PATH_GEMM).cpu().numpy()
+    dec = torch.from_numpy(oracle.decode_f32(synth.Q8_0, w, k)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(y, dec.T)
+    assert kq.device_status() == 0
+
+
 def test_matmul_tq1_auto_prefill_uses_the_tensor_cores(kq):
     r = rng(41)
     n, k, m = 384, 2048, 40
