@@ -669,25 +669,26 @@ def run_tq1_sweep(torch, kq, l2):
 
 
 def run_q8_0_sweep(torch, kq, l2):
-    """Q8_0 4096 x 4096 (bf16 activations): the plain kernel against the
-    tensor-core kernel over the activation-row count."""
-    dense = synth.Workload("sweep_q8_0", "gemm", synth.Q8_0, 4096, 4096, 1, "bf16", "f32")
-    w, _, _ = synth.make_inputs(dense)
-    wd = torch.from_numpy(w).cuda()
-    pool = [wd.clone() for _ in range(pool_size(w.nbytes, l2))]
-    r = np.random.Generator(np.random.PCG64(3))
-    for m in (1, 4, 8, 12, 16, 24, 32, 64, 128, 512):
-        x = torch.from_numpy(synth.gen_x(m, dense.k, "bf16", r)).to(torch.bfloat16).cuda()
-        y = torch.empty((m, dense.n), device="cuda")
-        line = {"sweep": "dense_q8_0_4096x4096", "m": m, "pool": len(pool)}
-        for name, path in (("plain", kq.PATH_SIMPLE), ("gemm", kq.PATH_GEMM)):
-            def fn():
-                for wi in pool:
-                    kq.matmul(wi, synth.Q8_0, x, out=y, path=path, const_weights=True)
-            line[name + "_us"] = round(time_graph(torch, fn, 5, 3, None) * 1e3 / (5 * len(pool)), 2)
-        print(json.dumps(line), flush=True)
-    del pool, wd
-    torch.cuda.empty_cache()
+    """Q8_0 and Q2_K, 4096 x 4096 (bf16 activations): the plain kernel
+    against the tensor-core kernel over the activation-row count."""
+    for codec, cname in ((synth.Q8_0, "q8_0"), (synth.Q2_K, "q2_k")):
+        dense = synth.Workload("sweep_" + cname, "gemm", codec, 4096, 4096, 1, "bf16", "f32")
+        w, _, _ = synth.make_inputs(dense)
+        wd = torch.from_numpy(w).cuda()
+        pool = [wd.clone() for _ in range(pool_size(w.nbytes, l2))]
+        r = np.random.Generator(np.random.PCG64(3))
+        for m in (1, 2, 3, 4, 8, 16, 32, 64, 128, 512):
+            x = torch.from_numpy(synth.gen_x(m, dense.k, "bf16", r)).to(torch.bfloat16).cuda()
+            y = torch.empty((m, dense.n), device="cuda")
+            line = {"sweep": f"dense_{cname}_4096x4096", "m": m, "pool": len(pool)}
+            for name, path in (("plain", kq.PATH_SIMPLE), ("gemm", kq.PATH_GEMM)):
+                def fn():
+                    for wi in pool:
+                        kq.matmul(wi, codec, x, out=y, path=path, const_weights=True)
+                line[name + "_us"] = round(time_graph(torch, fn, 5, 3, None) * 1e3 / (5 * len(pool)), 2)
+            print(json.dumps(line), flush=True)
+        del pool, wd
+        torch.cuda.empty_cache()
 
 
 def run_sweep(args):

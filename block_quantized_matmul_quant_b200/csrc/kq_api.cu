@@ -194,6 +194,9 @@ constexpr int64_t TQ1_GEMM_MIN_M = 8;
 // 18.7 vs 24.6, 4 rows 31.4 vs 24.9, 16 rows 68.2 vs 24.9, 512 rows 1825 vs
 // 34.8.
 constexpr int64_t Q8_0_GEMM_MIN_M = 3;
+// Likewise for Q2_K (K % 1024 == 0): 1 row 22.9 vs 25.2, 2 rows 26.1 vs
+// 25.2, 16 rows 75.4 vs 25.2, 512 rows 2076 vs 35.2.
+constexpr int64_t Q2_K_GEMM_MIN_M = 2;
 
 }  // namespace kq
 
@@ -237,7 +240,10 @@ int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k, const void *x, i
     const bool can_gemm = gemm_supported(type, n, k, x_dtype, y_dtype);
     const bool can_gemv = gemv_supported(type, n, k, x_dtype, m);
     if (path == KQ_PATH_AUTO) {
-        if (can_gemm && m >= (type == KQ_TQ1_G128 ? TQ1_GEMM_MIN_M : type == KQ_Q8_0 ? Q8_0_GEMM_MIN_M : GEMM_MIN_M))
+        if (can_gemm && m >= (type == KQ_TQ1_G128 ? TQ1_GEMM_MIN_M
+                              : type == KQ_Q8_0   ? Q8_0_GEMM_MIN_M
+                              : type == KQ_Q2_K   ? Q2_K_GEMM_MIN_M
+                                                  : GEMM_MIN_M))
             path = KQ_PATH_GEMM;
         // fp32 activations past one pass of the bandwidth kernel: the
         // few-rows tensor-core kernel reads the weights once per 8 rows of a

@@ -19,8 +19,9 @@
 //                         128-byte swizzle) into a shared-memory ring;
 //                 warp 6  TMA producer of raw weight units (128 rows x one
 //                         Q4_K super-block, 144 bytes, eight Q8_0 blocks,
-//                         272 bytes, or four TQ1_G128 blocks, 112 bytes)
-//                         into their own ring;
+//                         272 bytes, four Q2_K super-blocks, 336 bytes, or
+//                         four TQ1_G128 blocks, 112 bytes) into their own
+//                         ring;
 //                 warp 1  MMA issuer -- one thread issues tcgen05.mma
 //                         (kind::f16, bf16 x bf16 -> fp32 in TMEM) and
 //                         tcgen05.commit's to the stage / accumulator barriers;
@@ -31,7 +32,8 @@
 //                         decodes the stages s with s % groups == j, 64 K
 //                         positions of its 32 rows per warp.  Q4_K: exact
 //                         fp32 (d*sc*q - dmin*m, one rounding) -> bf16 (round
-//                         to nearest even); Q8_0 likewise (d * q).
+//                         to nearest even); Q8_0 (d * q) and Q2_K
+//                         (d*sc*q - dmin*m) likewise.
 //                         TQ1_G128 (Ternary Bonsai
 //                         `tq1_gemm`, the prefill form of the ternary
 //                         product): base-3 digits by integer arithmetic, two
@@ -69,12 +71,16 @@ template <int FMT> struct RawUnit;
 template <> struct RawUnit<KQ_Q4_K> { static constexpr int BYTES = 144, K = 256, ELEM = 1; };
 template <> struct RawUnit<KQ_TQ1_G128> { static constexpr int BYTES = 112, K = 512, ELEM = 1; };
 template <> struct RawUnit<KQ_Q8_0> { static constexpr int BYTES = 272, K = 256, ELEM = 2; };
-constexpr int raw_unit_bytes(int type) { return type == KQ_TQ1_G128 ? 112 : type == KQ_Q8_0 ? 272 : 144; }
-constexpr int raw_unit_k(int type) { return type == KQ_TQ1_G128 ? 512 : 256; }
+// Q2_K: four 84-byte super-blocks (336 bytes, 1024 K, 16-bit elements).
+template <> struct RawUnit<KQ_Q2_K> { static constexpr int BYTES = 336, K = 1024, ELEM = 2; };
+constexpr int raw_unit_bytes(int type) {
+    return type == KQ_TQ1_G128 ? 112 : type == KQ_Q8_0 ? 272 : type == KQ_Q2_K ? 336 : 144;
+}
+constexpr int raw_unit_k(int type) { return type == KQ_TQ1_G128 ? 512 : type == KQ_Q2_K ? 1024 : 256; }
 constexpr int raw_stage_bytes(int type) { return BM * raw_unit_bytes(type); }
 constexpr int RAW_WARP = 6;  // raw weight producer
 constexpr int DEC_WARP0 = 7;
-// Decoder warps per format: eight (two groups) for Q4_K and Q8_0; sixteen
+// Decoder warps per format: eight (two groups) for Q4_K, Q8_0 and Q2_K; sixteen
 // (four groups) for TQ1_G128, whose integer digit decode bounds the narrow
 // tiles.
 // Measured on B200 (µs): Q4_K 512x11008x4096 65.9 with eight against 67.7
@@ -279,6 +285,40 @@ __device__ __forceinline__ void q8_0_decode_chunk(const uint8_t *row, int cc, ui
         const uint32_t qa = __funnelshift_r(v[j], v[j + 1], 16);   // block 2 cc: codes 4 j .. 4 j + 3
         decode4(qa ^ 0x80808080u, s0, b0, out[2 * j], out[2 * j + 1]);
         decode4(v[9 + j] ^ 0x80808080u, s1, b1, out[16 + 2 * j], out[17 + 2 * j]);
+    }
+}
+
+// 64-K chunk cc (0..15) of a row's raw Q2_K unit (four 84-byte super-blocks:
+// scale/min bytes at 0 (low nibble scale, high nibble min, one per 16
+// weights), 2-bit codes at 16 (bit pair j of byte 32 h + l is weight
+// 128 h + 32 j + l), fp16 d and dmin at 80; weight d*sc*q - dmin*m): chunk
+// c4 = cc % 4 of super-block cc / 4 is weights 128 h + 32 j + l with
+// h = c4 / 2, j = 2 (c4 % 2) + jj (jj = 0, 1), l = 0..31, as 32 bf16x2 words
+// of the round-to-nearest-even bf16 of the exact weight (decode4: one fused
+// rounding of q * (d*sc) - dmin*m, both products exact).
+__device__ __forceinline__ void q2_k_decode_chunk(const uint8_t *row, int cc, uint32_t out[32]) {
+    const uint32_t *bw = reinterpret_cast<const uint32_t *>(row + 84 * (cc >> 2));   // 4-byte aligned
+    const int c4 = cc & 3, h = c4 >> 1, j0 = 2 * (c4 & 1);
+    const uint32_t dd = bw[20];
+    const float d = half_f(dd & 0xFFFFu), dmin = half_f(dd >> 16);
+    const uint32_t sw = bw[2 * h + (c4 & 1)];   // scale/min bytes of sub-blocks 8 h + 2 j0 .. + 3
+    uint32_t q[8];
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = bw[4 + 8 * h + i];
+    #pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+        const int shift = 2 * (j0 + jj);
+        #pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {   // positions l < 16, l >= 16: one scale each
+            const uint32_t sb = (sw >> (8 * (2 * jj + hf))) & 0xFFu;
+            const float a = d * (float)(sb & 15u), bm = dmin * (float)(sb >> 4);
+            const float2 sc = make_float2(a, a), bi = make_float2(-bm, -bm);
+            #pragma unroll
+            for (int qi = 0; qi < 4; ++qi) {
+                const int i = 4 * hf + qi;   // positions 4 i .. 4 i + 3
+                decode4((q[i] >> shift) & 0x03030303u, sc, bi, out[16 * jj + 2 * i], out[16 * jj + 2 * i + 1]);
+            }
+        }
     }
 }
 
@@ -571,6 +611,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
                             tq1_decode_chunk(blk, cc, out);
                         } else if constexpr (FMT == KQ_Q8_0) {
                             q8_0_decode_chunk(blk, cc, out);
+                        } else if constexpr (FMT == KQ_Q2_K) {
+                            q2_k_decode_chunk(blk, cc, out);
                         } else {
                             const uint32_t scw = cc < 2 ? sc_lo : sc_hi, mw = cc < 2 ? m_lo : m_hi;
                             const int b0 = (2 * cc) & 3;
@@ -635,6 +677,13 @@ __global__ void __launch_bounds__(num_threads<KQ_Q8_0>(), 1)
     gemm_q8_0_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
     gemm_body<YT, ID, CPS, KQ_Q8_0>(tmap_x, tmap_w, tmap_y, p);
+}
+
+template <typename YT, bool ID, int CPS>
+__global__ void __launch_bounds__(num_threads<KQ_Q2_K>(), 1)
+    gemm_q2_k_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                     const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+    gemm_body<YT, ID, CPS, KQ_Q2_K>(tmap_x, tmap_w, tmap_y, p);
 }
 
 // ---------------------------------------------------------------- host side
@@ -725,7 +774,7 @@ bool encode_x_map(CUtensorMap *m, const void *x, int64_t rows, int64_t k, int bo
 bool encode_w_map(CUtensorMap *m, const void *w, int64_t n, int64_t k, int64_t n_experts,
                   int64_t expert_stride, int type) {
     const int ub = raw_unit_bytes(type), uk = raw_unit_k(type);
-    const int el = type == KQ_Q8_0 ? 2 : 1;   // bytes per element of the map
+    const int el = (type == KQ_Q8_0 || type == KQ_Q2_K) ? 2 : 1;   // bytes per element of the map
     if (k % uk) return false;
     const int64_t rb = (k / uk) * ub;
     cuuint64_t dims[3] = {(cuuint64_t)(rb / el), (cuuint64_t)n, (cuuint64_t)n_experts};
@@ -748,6 +797,8 @@ bool gemm_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype, bo
         if (k % 512) return false;   // the row pitch and box rows must be multiples of 16 bytes
     } else if (type == KQ_Q8_0 && !expert_indexed) {
         if (k % 256) return false;   // likewise: eight 34-byte blocks are 272 bytes
+    } else if (type == KQ_Q2_K && !expert_indexed) {
+        if (k % 1024) return false;   // and four 84-byte super-blocks are 336 bytes
     } else {
         return false;
     }
@@ -795,6 +846,7 @@ cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CU
     void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
     if constexpr (FMT == KQ_TQ1_G128) kern = gemm_tq1_kernel<YT, ID, CPS>;
     else if constexpr (FMT == KQ_Q8_0) kern = gemm_q8_0_kernel<YT, ID, CPS>;
+    else if constexpr (FMT == KQ_Q2_K) kern = gemm_q2_k_kernel<YT, ID, CPS>;
     else kern = gemm_q4k_kernel<YT, ID, CPS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -816,7 +868,7 @@ cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CU
 cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const void *x, int64_t m,
                         void *y, int ydt, cudaStream_t s) {
     if (!encode_fn() || m < 1 || m > (1 << 30)) return cudaErrorNotSupported;
-    if (type != KQ_Q4_K && type != KQ_TQ1_G128 && type != KQ_Q8_0) return cudaErrorNotSupported;
+    if (type != KQ_Q4_K && type != KQ_TQ1_G128 && type != KQ_Q8_0 && type != KQ_Q2_K) return cudaErrorNotSupported;
     const int sms = sm_count();
     GemmParams p = {};
     p.n = (int)n; p.k = (int)k; p.m = (int)m;
@@ -848,6 +900,13 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
                                  : launch_kernel<__nv_bfloat16, false, 2, KQ_Q8_0>(tx, tw, ty, p, grid, s);
         return ydt == KQ_F32 ? launch_kernel<float, false, 1, KQ_Q8_0>(tx, tw, ty, p, grid, s)
                              : launch_kernel<__nv_bfloat16, false, 1, KQ_Q8_0>(tx, tw, ty, p, grid, s);
+    }
+    if (type == KQ_Q2_K) {
+        if (cps == 2)
+            return ydt == KQ_F32 ? launch_kernel<float, false, 2, KQ_Q2_K>(tx, tw, ty, p, grid, s)
+                                 : launch_kernel<__nv_bfloat16, false, 2, KQ_Q2_K>(tx, tw, ty, p, grid, s);
+        return ydt == KQ_F32 ? launch_kernel<float, false, 1, KQ_Q2_K>(tx, tw, ty, p, grid, s)
+                             : launch_kernel<__nv_bfloat16, false, 1, KQ_Q2_K>(tx, tw, ty, p, grid, s);
     }
     if (cps == 2)
         return ydt == KQ_F32 ? launch_kernel<float, false, 2>(tx, tw, ty, p, grid, s)

@@ -466,6 +466,60 @@ def test_matmul_gemm_q8_0_decodes_every_code_exactly(kq):
     assert kq.device_status() == 0
 
 
+Q2_K_GEMM_CASES = [
+    # one tile and one raw unit (four super-blocks); ragged rows and tokens;
+    # wide tiles over several tiles each way; long rows
+    (128, 1024, 5), (300, 2048, 37), (1000, 4096, 300), (129, 8192, 64),
+]
+
+
+@pytest.mark.parametrize("n,k,m", Q2_K_GEMM_CASES)
+def test_matmul_gemm_q2_k(kq, n, k, m):
+    """Q2_K on the tensor cores: the bf16 rounding of d*sc*q - dmin*m per
+    weight, so the product equals the bf16-weight product up to fp32
+    accumulation."""
+    import torch
+
+    r = rng(4000 + n + k + m)
+    w = synth.gen_weights(synth.Q2_K, n, k, r)
+    x = synth.gen_x(m, k, "bf16", r)
+    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    y = kq.matmul(wd, synth.Q2_K, xd, path=kq.PATH_GEMM).cpu().numpy()
+    ref = oracle.matmul(synth.Q2_K, w, k, x, threads=8)
+    assert row_rel_err(y, ref) <= TOL["bf16"]
+    assert row_rel_err(y, _bf16_weight_reference(w, k, x, synth.Q2_K)) <= FP32_PATH_TOL
+    yb = kq.matmul(wd, synth.Q2_K, xd, path=kq.PATH_GEMM, out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert row_rel_err(yb, ref) <= TOL["bf16"] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+def test_matmul_gemm_q2_k_decodes_every_weight_exactly(kq):
+    """Every scale/min byte at every sub-block position and every 2-bit code
+    at every position of the four-super-block raw unit, under d and dmin of
+    both signs: with the identity as activations each output is one decoded
+    weight, which must be the round-to-nearest-even bf16 of the oracle's
+    decode."""
+    import torch
+
+    n, k = 256, 1024
+    r = rng(53)
+    w = r.integers(0, 256, size=(n, k // 256 * 84), dtype=np.uint8)
+    ds = [0.25, -0.5, 1.0e-3, -2.0e-2, 6.0e-8, 3.0]
+    for row in range(n):
+        for b in range(k // 256):
+            o = 84 * b
+            w[row, o: o + 16] = (np.arange(16) * 16 + row + 5 * b) % 256   # every scale/min byte per position
+            dd = np.array([ds[(row + b) % len(ds)], -ds[(row + 2 * b + 1) % len(ds)]], dtype=np.float16)
+            w[row, o + 80: o + 84] = np.frombuffer(dd.tobytes(), dtype=np.uint8)
+    seen = {(int(w[i, 84 * b + j]), j) for i in range(n) for b in range(k // 256) for j in range(16)}
+    assert len(seen) == 256 * 16
+    x = np.eye(k, dtype=np.float32)
+    y = kq.matmul(to_device_w(w), synth.Q2_K, to_device_x(x, "bf16"), path=kq.PATH_GEMM).cpu().numpy()
+    dec = torch.from_numpy(oracle.decode_f32(synth.Q2_K, w, k)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(y, dec.T)
+    assert kq.device_status() == 0
+
+
 def test_matmul_tq1_auto_prefill_uses_the_tensor_cores(kq):
     r = rng(41)
     n, k, m = 384, 2048, 40
