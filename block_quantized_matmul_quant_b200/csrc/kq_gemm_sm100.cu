@@ -18,10 +18,10 @@
 //  * Warp roles:  warp 0  TMA producer of bf16 activation tiles (64 K x BN,
 //                         128-byte swizzle) into a shared-memory ring;
 //                 warp 6  TMA producer of raw weight units (128 rows x one
-//                         Q4_K super-block, 144 bytes, eight Q8_0 blocks,
-//                         272 bytes, four Q2_K super-blocks, 336 bytes, or
-//                         four TQ1_G128 blocks, 112 bytes) into their own
-//                         ring;
+//                         Q4_K super-block, 144 bytes, one Q5_K super-block,
+//                         176 bytes, eight Q8_0 blocks, 272 bytes, four Q2_K
+//                         super-blocks, 336 bytes, or four TQ1_G128 blocks,
+//                         112 bytes) into their own ring;
 //                 warp 1  MMA issuer -- one thread issues tcgen05.mma
 //                         (kind::f16, bf16 x bf16 -> fp32 in TMEM) and
 //                         tcgen05.commit's to the stage / accumulator barriers;
@@ -32,8 +32,8 @@
 //                         decodes the stages s with s % groups == j, 64 K
 //                         positions of its 32 rows per warp.  Q4_K: exact
 //                         fp32 (d*sc*q - dmin*m, one rounding) -> bf16 (round
-//                         to nearest even); Q8_0 (d * q) and Q2_K
-//                         (d*sc*q - dmin*m) likewise.
+//                         to nearest even); Q5_K (five-bit q), Q8_0 (d * q)
+//                         and Q2_K (d*sc*q - dmin*m) likewise.
 //                         TQ1_G128 (Ternary Bonsai
 //                         `tq1_gemm`, the prefill form of the ternary
 //                         product): base-3 digits by integer arithmetic, two
@@ -73,14 +73,16 @@ template <> struct RawUnit<KQ_TQ1_G128> { static constexpr int BYTES = 112, K = 
 template <> struct RawUnit<KQ_Q8_0> { static constexpr int BYTES = 272, K = 256, ELEM = 2; };
 // Q2_K: four 84-byte super-blocks (336 bytes, 1024 K, 16-bit elements).
 template <> struct RawUnit<KQ_Q2_K> { static constexpr int BYTES = 336, K = 1024, ELEM = 2; };
+// Q5_K: one 176-byte super-block (256 K).
+template <> struct RawUnit<KQ_Q5_K> { static constexpr int BYTES = 176, K = 256, ELEM = 1; };
 constexpr int raw_unit_bytes(int type) {
-    return type == KQ_TQ1_G128 ? 112 : type == KQ_Q8_0 ? 272 : type == KQ_Q2_K ? 336 : 144;
+    return type == KQ_TQ1_G128 ? 112 : type == KQ_Q8_0 ? 272 : type == KQ_Q2_K ? 336 : type == KQ_Q5_K ? 176 : 144;
 }
 constexpr int raw_unit_k(int type) { return type == KQ_TQ1_G128 ? 512 : type == KQ_Q2_K ? 1024 : 256; }
 constexpr int raw_stage_bytes(int type) { return BM * raw_unit_bytes(type); }
 constexpr int RAW_WARP = 6;  // raw weight producer
 constexpr int DEC_WARP0 = 7;
-// Decoder warps per format: eight (two groups) for Q4_K, Q8_0 and Q2_K; sixteen
+// Decoder warps per format: eight (two groups) for the K-quants and Q8_0; sixteen
 // (four groups) for TQ1_G128, whose integer digit decode bounds the narrow
 // tiles.
 // Measured on B200 (µs): Q4_K 512x11008x4096 65.9 with eight against 67.7
@@ -584,8 +586,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
                 ok = warp_wait(&raw_full[rs], rph, p.err);
                 if (!ok) break;
                 const uint8_t *blk = raw_ring + rs * RAW_STAGE_BYTES + r * UNIT_BYTES;
-                // Q4_K super-block header (unused for TQ1)
-                const uint4 hd = FMT == KQ_Q4_K ? *reinterpret_cast<const uint4 *>(blk) : make_uint4(0u, 0u, 0u, 0u);
+                // Q4_K / Q5_K super-block header (fp16 d, dmin, packed 6-bit
+                // scales and mins; unused by the other formats)
+                const uint4 hd = (FMT == KQ_Q4_K || FMT == KQ_Q5_K) ? *reinterpret_cast<const uint4 *>(blk)
+                                                                     : make_uint4(0u, 0u, 0u, 0u);
                 const float d = half_f(hd.x), dmin = half_f(hd.x >> 16);
                 // packed 6-bit scales / mins of sub-blocks 0..3 and 4..7
                 const uint32_t sc_lo = hd.y & 0x3F3F3F3Fu, m_lo = hd.z & 0x3F3F3F3Fu;
@@ -613,6 +617,30 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
                             q8_0_decode_chunk(blk, cc, out);
                         } else if constexpr (FMT == KQ_Q2_K) {
                             q2_k_decode_chunk(blk, cc, out);
+                        } else if constexpr (FMT == KQ_Q5_K) {
+                            // chunk cc: low nibbles (sub-block 2cc) and high
+                            // nibbles (2cc+1) of qs bytes 32cc.. at 48, each
+                            // with its fifth bit, bit 2cc (+1) of qh byte l at 16
+                            const uint32_t scw = cc < 2 ? sc_lo : sc_hi, mw = cc < 2 ? m_lo : m_hi;
+                            const int b0 = (2 * cc) & 3;
+                            const float ds_lo = d * byte_float(scw, b0), dm_lo = dmin * byte_float(mw, b0);
+                            const float ds_hi = d * byte_float(scw, b0 + 1), dm_hi = dmin * byte_float(mw, b0 + 1);
+                            const float2 sl = make_float2(ds_lo, ds_lo), bl = make_float2(-dm_lo, -dm_lo);
+                            const float2 sh = make_float2(ds_hi, ds_hi), bh = make_float2(-dm_hi, -dm_hi);
+                            const uint4 v0 = *reinterpret_cast<const uint4 *>(blk + 48 + 32 * cc);
+                            const uint4 v1 = *reinterpret_cast<const uint4 *>(blk + 64 + 32 * cc);
+                            const uint4 h0 = *reinterpret_cast<const uint4 *>(blk + 16);
+                            const uint4 h1 = *reinterpret_cast<const uint4 *>(blk + 32);
+                            const uint32_t qw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                            const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+                            #pragma unroll
+                            for (int wd = 0; wd < 8; ++wd) {
+                                const uint32_t lo = (qw[wd] & 0x0F0F0F0Fu) | (((hw[wd] >> (2 * cc)) & 0x01010101u) << 4);
+                                const uint32_t hi =
+                                    ((qw[wd] >> 4) & 0x0F0F0F0Fu) | (((hw[wd] >> (2 * cc + 1)) & 0x01010101u) << 4);
+                                decode4(lo, sl, bl, out[2 * wd], out[2 * wd + 1]);
+                                decode4(hi, sh, bh, out[16 + 2 * wd], out[17 + 2 * wd]);
+                            }
                         } else {
                             const uint32_t scw = cc < 2 ? sc_lo : sc_hi, mw = cc < 2 ? m_lo : m_hi;
                             const int b0 = (2 * cc) & 3;
@@ -684,6 +712,13 @@ __global__ void __launch_bounds__(num_threads<KQ_Q2_K>(), 1)
     gemm_q2_k_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
     gemm_body<YT, ID, CPS, KQ_Q2_K>(tmap_x, tmap_w, tmap_y, p);
+}
+
+template <typename YT, bool ID, int CPS>
+__global__ void __launch_bounds__(num_threads<KQ_Q5_K>(), 1)
+    gemm_q5_k_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                     const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+    gemm_body<YT, ID, CPS, KQ_Q5_K>(tmap_x, tmap_w, tmap_y, p);
 }
 
 // ---------------------------------------------------------------- host side
@@ -799,6 +834,8 @@ bool gemm_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype, bo
         if (k % 256) return false;   // likewise: eight 34-byte blocks are 272 bytes
     } else if (type == KQ_Q2_K && !expert_indexed) {
         if (k % 1024) return false;   // and four 84-byte super-blocks are 336 bytes
+    } else if (type == KQ_Q5_K && !expert_indexed) {
+        if (k % 256) return false;
     } else {
         return false;
     }
@@ -847,6 +884,7 @@ cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CU
     if constexpr (FMT == KQ_TQ1_G128) kern = gemm_tq1_kernel<YT, ID, CPS>;
     else if constexpr (FMT == KQ_Q8_0) kern = gemm_q8_0_kernel<YT, ID, CPS>;
     else if constexpr (FMT == KQ_Q2_K) kern = gemm_q2_k_kernel<YT, ID, CPS>;
+    else if constexpr (FMT == KQ_Q5_K) kern = gemm_q5_k_kernel<YT, ID, CPS>;
     else kern = gemm_q4k_kernel<YT, ID, CPS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -868,7 +906,8 @@ cudaError_t launch_kernel(const CUtensorMap &tx, const CUtensorMap &tw, const CU
 cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const void *x, int64_t m,
                         void *y, int ydt, cudaStream_t s) {
     if (!encode_fn() || m < 1 || m > (1 << 30)) return cudaErrorNotSupported;
-    if (type != KQ_Q4_K && type != KQ_TQ1_G128 && type != KQ_Q8_0 && type != KQ_Q2_K) return cudaErrorNotSupported;
+    if (type != KQ_Q4_K && type != KQ_TQ1_G128 && type != KQ_Q8_0 && type != KQ_Q2_K && type != KQ_Q5_K)
+        return cudaErrorNotSupported;
     const int sms = sm_count();
     GemmParams p = {};
     p.n = (int)n; p.k = (int)k; p.m = (int)m;
@@ -907,6 +946,13 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
                                  : launch_kernel<__nv_bfloat16, false, 2, KQ_Q2_K>(tx, tw, ty, p, grid, s);
         return ydt == KQ_F32 ? launch_kernel<float, false, 1, KQ_Q2_K>(tx, tw, ty, p, grid, s)
                              : launch_kernel<__nv_bfloat16, false, 1, KQ_Q2_K>(tx, tw, ty, p, grid, s);
+    }
+    if (type == KQ_Q5_K) {
+        if (cps == 2)
+            return ydt == KQ_F32 ? launch_kernel<float, false, 2, KQ_Q5_K>(tx, tw, ty, p, grid, s)
+                                 : launch_kernel<__nv_bfloat16, false, 2, KQ_Q5_K>(tx, tw, ty, p, grid, s);
+        return ydt == KQ_F32 ? launch_kernel<float, false, 1, KQ_Q5_K>(tx, tw, ty, p, grid, s)
+                             : launch_kernel<__nv_bfloat16, false, 1, KQ_Q5_K>(tx, tw, ty, p, grid, s);
     }
     if (cps == 2)
         return ydt == KQ_F32 ? launch_kernel<float, false, 2>(tx, tw, ty, p, grid, s)

@@ -81,8 +81,8 @@ bool moe_gemv_supported(int type, int64_t n, int64_t k, int64_t n_experts);
 cudaError_t launch_moe_gemv(const IdArgs &a, cudaStream_t s);
 
 // Tensor-core kernels (kq_gemm_sm100.cu): Q4_K dense and expert-indexed,
-// Q8_0 dense (K % 256 == 0), Q2_K dense (K % 1024 == 0), TQ1_G128 dense
-// (K % 512 == 0).
+// Q8_0 and Q5_K dense (K % 256 == 0), Q2_K dense (K % 1024 == 0), TQ1_G128
+// dense (K % 512 == 0).
 bool gemm_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype, bool expert_indexed = false);
 cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const void *x, int64_t m,
                         void *y, int ydt, cudaStream_t s);

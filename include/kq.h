@@ -80,8 +80,8 @@ extern "C" {
 #define KQ_PATH_SIMPLE   1  /* plain CUDA-core kernel, any codec/shape               */
 #define KQ_PATH_GEMV     2  /* bandwidth kernel: weights decoded in registers         */
 /* TMA + tcgen05 tensor-core kernel: bf16 x only; Q4_K (K % 256 == 0), or,
- * dense only, Q8_0 with K % 256 == 0, Q2_K with K % 1024 == 0 and TQ1_G128
- * with K % 512 == 0 (Ternary Bonsai `tq1_gemm`). */
+ * dense only, Q8_0 and Q5_K with K % 256 == 0, Q2_K with K % 1024 == 0 and
+ * TQ1_G128 with K % 512 == 0 (Ternary Bonsai `tq1_gemm`). */
 #define KQ_PATH_GEMM     3
 /* Tensor-core kernel for few activation rows / pairs per expert: 4-bit codes
  * through the MMA, one accumulator per 32-weight sub-block, the scales
@@ -133,9 +133,9 @@ KQ_API int kq_dequantize(int type, const void *w, int64_t rows, int64_t k,
  *   y  [m, n] of y_dtype (KQ_F32 or KQ_BF16) (device), fully overwritten
  *   y[i][j] = sum_k dequant(w)[j][k] * x[i][k], fp32 accumulation.
  * Small m runs the bandwidth-bound kernel that decodes weights in
- * registers; large m with bf16 x (Q4_K from 5 rows, Q8_0 with K % 256 == 0
- * from 3 rows, Q2_K with K % 1024 == 0 from 2 rows, TQ1_G128 with
- * K % 512 == 0 from 8 rows) runs the tensor-core kernel, which rounds
+ * registers; large m with bf16 x (Q4_K and Q5_K from 5 rows, Q8_0 with
+ * K % 256 == 0 from 3 rows, Q2_K with K % 1024 == 0 from 2 rows, TQ1_G128
+ * with K % 512 == 0 from 8 rows) runs the tensor-core kernel, which rounds
  * decoded weights to bf16 before the bf16 x bf16 -> fp32 MMA (for TQ1:
  * (t - 1) times the bf16 rounding of the block scale, the same value).
  */

@@ -520,6 +520,63 @@ def test_matmul_gemm_q2_k_decodes_every_weight_exactly(kq):
     assert kq.device_status() == 0
 
 
+@pytest.mark.parametrize("n,k,m", [(128, 256, 5), (300, 1024, 37), (1000, 4096, 300), (129, 8192, 64)])
+def test_matmul_gemm_q5_k(kq, n, k, m):
+    """Q5_K on the tensor cores: the bf16 rounding of d*sc*q - dmin*m per
+    weight (q the five-bit code), so the product equals the bf16-weight
+    product up to fp32 accumulation."""
+    import torch
+
+    r = rng(5000 + n + k + m)
+    w = synth.gen_weights(synth.Q5_K, n, k, r)
+    x = synth.gen_x(m, k, "bf16", r)
+    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    y = kq.matmul(wd, synth.Q5_K, xd, path=kq.PATH_GEMM).cpu().numpy()
+    ref = oracle.matmul(synth.Q5_K, w, k, x, threads=8)
+    assert row_rel_err(y, ref) <= TOL["bf16"]
+    assert row_rel_err(y, _bf16_weight_reference(w, k, x, synth.Q5_K)) <= FP32_PATH_TOL
+    yb = kq.matmul(wd, synth.Q5_K, xd, path=kq.PATH_GEMM, out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert row_rel_err(yb, ref) <= TOL["bf16"] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+def test_matmul_gemm_q5_k_decodes_every_code_exactly(kq):
+    """Every five-bit code (four low bits from qs, the fifth from qh) at every
+    position of a super-block, random packed scales and mins, d and dmin of
+    both signs: with the identity as activations each output is one decoded
+    weight, which must be the round-to-nearest-even bf16 of the oracle's
+    decode."""
+    import torch
+
+    n, k = 256, 256
+    r = rng(59)
+    w = r.integers(0, 256, size=(n, 176), dtype=np.uint8)
+    ds = [0.25, -0.5, 1.0e-3, -2.0e-2, 6.0e-8, 3.0]
+    codes = np.zeros((n, 256), dtype=np.int64)
+    for row in range(n):
+        dd = np.array([ds[row % len(ds)], -ds[(row // 3) % len(ds)]], dtype=np.float16)
+        w[row, 0:4] = np.frombuffer(dd.tobytes(), dtype=np.uint8)
+        for c in range(4):
+            for l in range(32):
+                w[row, 48 + 32 * c + l] = (row + 7 * l + 3 * c) % 256
+        # fifth bits: low-nibble codes (even bits) follow row // 16, the
+        # high-nibble ones (odd bits) row % 2, so every (q4, bit) pair occurs
+        w[row, 16:48] = ((row >> 4) & 1) * 0x55 | (row & 1) * 0xAA
+        for c in range(4):
+            for h in range(2):
+                for l in range(32):
+                    q4 = (int(w[row, 48 + 32 * c + l]) >> (4 * h)) & 15
+                    hb = (int(w[row, 16 + l]) >> (2 * c + h)) & 1
+                    codes[row, 64 * c + 32 * h + l] = q4 + 16 * hb
+    seen = {(int(codes[i, j]), j) for i in range(n) for j in range(256)}
+    assert len(seen) == 32 * 256
+    x = np.eye(k, dtype=np.float32)
+    y = kq.matmul(to_device_w(w), synth.Q5_K, to_device_x(x, "bf16"), path=kq.PATH_GEMM).cpu().numpy()
+    dec = torch.from_numpy(oracle.decode_f32(synth.Q5_K, w, k)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(y, dec.T)
+    assert kq.device_status() == 0
+
+
 def test_matmul_tq1_auto_prefill_uses_the_tensor_cores(kq):
     r = rng(41)
     n, k, m = 384, 2048, 40
