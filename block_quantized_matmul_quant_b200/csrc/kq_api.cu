@@ -348,7 +348,8 @@ static int id_setup(int type, const void *w, int64_t n_experts, int64_t n, int64
 // none).
 static int id_path(IdArgs &a, int path, int64_t pairs, int *bn) {
     const bool can_gemv = moe_gemv_supported(a.type, a.n, a.k, a.n_experts);
-    const bool can_gemm = gemm_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype, true);
+    // (the weights' tensor map needs an expert stride of whole 16-byte units)
+    const bool can_gemm = gemm_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype, true) && a.expert_stride % 16 == 0;
     const bool can_tc = moe_mma_supported(a.type, a.n, a.k, a.x_dtype, a.y_dtype);
     if (path == KQ_PATH_AUTO) {
         const bool f32x = a.x_dtype == KQ_F32;

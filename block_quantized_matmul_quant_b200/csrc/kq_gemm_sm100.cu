@@ -830,11 +830,11 @@ bool gemm_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype, bo
         if (k % 256) return false;
     } else if (type == KQ_TQ1_G128 && !expert_indexed) {
         if (k % 512) return false;   // the row pitch and box rows must be multiples of 16 bytes
-    } else if (type == KQ_Q8_0 && !expert_indexed) {
+    } else if (type == KQ_Q8_0) {
         if (k % 256) return false;   // likewise: eight 34-byte blocks are 272 bytes
-    } else if (type == KQ_Q2_K && !expert_indexed) {
+    } else if (type == KQ_Q2_K) {
         if (k % 1024) return false;   // and four 84-byte super-blocks are 336 bytes
-    } else if (type == KQ_Q5_K && !expert_indexed) {
+    } else if (type == KQ_Q5_K) {
         if (k % 256) return false;
     } else {
         return false;
@@ -970,6 +970,20 @@ int gemm_id_bn(int64_t n_tokens, int64_t top_k, int64_t n_experts) {
     return (int)bn;
 }
 
+namespace {
+
+template <int FMT>
+cudaError_t launch_id_fmt(const CUtensorMap &tx, const CUtensorMap &tw, const GemmParams &p, int grid, int cps,
+                          int ydt, cudaStream_t s) {
+    if (cps == 2)
+        return ydt == KQ_F32 ? launch_kernel<float, true, 2, FMT>(tx, tw, tx, p, grid, s)
+                             : launch_kernel<__nv_bfloat16, true, 2, FMT>(tx, tw, tx, p, grid, s);
+    return ydt == KQ_F32 ? launch_kernel<float, true, 1, FMT>(tx, tw, tx, p, grid, s)
+                         : launch_kernel<__nv_bfloat16, true, 1, FMT>(tx, tw, tx, p, grid, s);
+}
+
+}  // namespace
+
 cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     if (!encode_fn()) return cudaErrorNotSupported;
     const int sms = sm_count();
@@ -977,9 +991,10 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     p.n = (int)a.n; p.k = (int)a.k; p.m = (int)a.n_tokens;
     p.n_tiles = (int)((a.n + BM - 1) / BM);
     p.bn = bn;
-    if (a.type != KQ_Q4_K) return cudaErrorNotSupported;
+    if (a.type != KQ_Q4_K && a.type != KQ_Q8_0 && a.type != KQ_Q2_K && a.type != KQ_Q5_K)
+        return cudaErrorNotSupported;
     const int cps = cps_for(bn);
-    if (!fill_ring(&p, cps, KQ_Q4_K)) return cudaErrorNotSupported;
+    if (!fill_ring(&p, cps, a.type)) return cudaErrorNotSupported;
     p.y = a.y;
     p.err = error_word();
     p.perm = a.perm;
@@ -991,16 +1006,17 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     p.n_experts = (int)a.n_experts;
     CUtensorMap tx, tw;
     if (!encode_x_map(&tx, a.x, a.x_rows(), a.k, 1) ||
-        !encode_w_map(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride, KQ_Q4_K))
+        !encode_w_map(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride, (int)a.type))
         return cudaErrorInvalidValue;
     // persistent grid: the number of token tiles is only known on the device
     const int64_t max_units = (a.n_tokens * a.top_k / bn + a.n_experts) * p.n_tiles;
     const int grid = (int)(max_units < sms ? max_units : sms);
-    if (cps == 2)
-        return a.y_dtype == KQ_F32 ? launch_kernel<float, true, 2>(tx, tw, tx, p, grid, s)
-                                   : launch_kernel<__nv_bfloat16, true, 2>(tx, tw, tx, p, grid, s);
-    return a.y_dtype == KQ_F32 ? launch_kernel<float, true, 1>(tx, tw, tx, p, grid, s)
-                               : launch_kernel<__nv_bfloat16, true, 1>(tx, tw, tx, p, grid, s);
+    switch (a.type) {
+    case KQ_Q8_0: return launch_id_fmt<KQ_Q8_0>(tx, tw, p, grid, cps, a.y_dtype, s);
+    case KQ_Q2_K: return launch_id_fmt<KQ_Q2_K>(tx, tw, p, grid, cps, a.y_dtype, s);
+    case KQ_Q5_K: return launch_id_fmt<KQ_Q5_K>(tx, tw, p, grid, cps, a.y_dtype, s);
+    default: return launch_id_fmt<KQ_Q4_K>(tx, tw, p, grid, cps, a.y_dtype, s);
+    }
 }
 
 }  // namespace kq

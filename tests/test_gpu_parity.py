@@ -698,9 +698,22 @@ def test_matmul_id_small(kq, codec, path):
         outs = [kq.matmul_id(to_device_w(w), codec, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
                              path=pp).cpu().numpy() for pp in (kq.PATH_GEMV, kq.PATH_GEMM, kq.PATH_GEMV_TC)]
         assert any(np.array_equal(y.view(np.uint32), o.view(np.uint32)) for o in outs)
+    elif path == "auto" and _grouped_gemm_takes(codec, k):
+        # bf16 activations: the grouped tensor-core GEMM, bit for bit
+        assert row_rel_err(y, ref) <= TOL["bf16"]
+        g = kq.matmul_id(to_device_w(w), codec, to_device_x(x, "bf16"), torch.from_numpy(ids).cuda(),
+                         path=kq.PATH_GEMM).cpu().numpy()
+        assert np.array_equal(y.view(np.uint32), g.view(np.uint32))
     else:
         assert row_rel_err(y, ref) <= FP32_PATH_TOL
     assert kq.device_status() == 0
+
+
+def _grouped_gemm_takes(codec, k):
+    """Whether the grouped tensor-core GEMM serves bf16 activations of this
+    codec and K (the automatic path's choice for the codecs without a
+    grouped bandwidth kernel)."""
+    return (codec in (synth.Q8_0, synth.Q5_K) and k % 256 == 0) or (codec == synth.Q2_K and k % 1024 == 0)
 
 
 @pytest.mark.parametrize("t,top_k,e,n,k", [
@@ -838,7 +851,8 @@ def test_matmul_id_mix(kq, codec, path, xdt, t, top_k, e, n, k):
     wd, xd = to_device_w(w), to_device_x(xs, xdt)
     idd, sd = torch.from_numpy(ids).cuda(), torch.from_numpy(scores).cuda()
     y = kq.matmul_id_mix(wd, codec, xd, idd, sd, path=path).cpu().numpy()
-    if path == 3 or (path == 0 and codec == synth.Q4_K and xdt == "bf16" and t * top_k > e):
+    if path == 3 or (path == 0 and codec == synth.Q4_K and xdt == "bf16" and t * top_k > e) or \
+            (path == 0 and xdt == "bf16" and _grouped_gemm_takes(codec, k)):
         tol = TOL["bf16"]
     elif codec == synth.Q4_K and path in (0, 2):
         tol = GEMV_TOL
@@ -1018,7 +1032,7 @@ def test_matmul_dense_tensor_core_few_rows(kq, n, k, m, xdt):
     assert kq.device_status() == 0
 
 
-def _bf16_weight_reference_id(w, k, x, ids):
+def _bf16_weight_reference_id(w, k, x, ids, codec=synth.Q4_K):
     """y[t, s] = x[t] @ bf16(decode_f32(w[ids[t, s]]))^T in fp64 (NaN rows for
     ids outside [0, E)): the tensor-core expert product up to fp32 accumulation."""
     e_n = w.shape[0]
@@ -1026,7 +1040,7 @@ def _bf16_weight_reference_id(w, k, x, ids):
     for e in range(e_n):
         hit = ids == e
         if hit.any():
-            ye = _bf16_weight_reference(w[e], k, x)   # [T, n]
+            ye = _bf16_weight_reference(w[e], k, x, codec)   # [T, n]
             ref[hit] = ye[np.nonzero(hit)[0]]
     return ref
 
@@ -1057,6 +1071,31 @@ def test_matmul_id_grouped_gemm(kq, t, top_k, e, n, k, skew):
     yb = kq.matmul_id(wd, synth.Q4_K, xd, idd, path=kq.PATH_GEMM,
                       out_dtype=torch.bfloat16).float().cpu().numpy()
     assert row_rel_err(yb, ref) <= TOL["bf16"] + BF16_OUT
+    assert kq.device_status() == 0
+
+
+@pytest.mark.parametrize("codec,t,top_k,e,n,k", [
+    (synth.Q8_0, 64, 4, 8, 300, 1024), (synth.Q8_0, 7, 3, 4, 129, 256),
+    (synth.Q2_K, 64, 4, 8, 300, 2048), (synth.Q2_K, 200, 2, 5, 128, 1024),
+    (synth.Q5_K, 64, 4, 8, 300, 1024), (synth.Q5_K, 9, 2, 3, 70, 512),
+])
+def test_matmul_id_grouped_gemm_other_codecs(kq, codec, t, top_k, e, n, k):
+    """The grouped tensor-core GEMM for Q8_0, Q2_K and Q5_K experts (the
+    automatic path for bf16 activations): the bf16-weight product per pair,
+    deterministic, in stream order with the grouping."""
+    import torch
+
+    r = rng(11 * t + e + n + codec)
+    w = synth.gen_weights(codec, e * n, k, r).reshape(e, n, -1)
+    x = synth.gen_x(t, k, "bf16", r)
+    ids = synth.gen_ids(t, top_k, e, r)
+    ref = oracle.matmul_id(codec, w, k, x, ids)
+    wd, xd, idd = to_device_w(w), to_device_x(x, "bf16"), torch.from_numpy(ids).cuda()
+    y = kq.matmul_id(wd, codec, xd, idd, path=kq.PATH_GEMM).cpu().numpy()
+    assert row_rel_err(y, ref) <= TOL["bf16"]
+    assert row_rel_err(y, _bf16_weight_reference_id(w, k, x, ids, codec)) <= FP32_PATH_TOL
+    ya = kq.matmul_id(wd, codec, xd, idd).cpu().numpy()   # automatic: the same kernel
+    assert np.array_equal(y.view(np.uint32), ya.view(np.uint32))
     assert kq.device_status() == 0
 
 
