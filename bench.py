@@ -691,6 +691,31 @@ def run_q8_0_sweep(torch, kq, l2):
         torch.cuda.empty_cache()
 
 
+def run_id_codecs_sweep(torch, kq, l2):
+    """Expert-indexed Q2_K, Q8_0 and Q5_K (64 experts of 1408 x 2048, top-6,
+    bf16 activations): the plain grouped kernel against the grouped
+    tensor-core GEMM over the token count."""
+    for codec, cname in ((synth.Q2_K, "q2_k"), (synth.Q8_0, "q8_0"), (synth.Q5_K, "q5_k")):
+        for t in (1, 4, 8, 32, 128):
+            wl = synth.Workload("sweep_id", "moe", codec, 1408, 2048, t, "bf16", "f32", n_experts=64, top_k=6)
+            w, x, ids = synth.make_inputs(wl)
+            wd = torch.from_numpy(w).cuda()
+            pool = [wd.clone() for _ in range(max(4, -(-4 * l2 // w.nbytes)))]
+            xd = torch.from_numpy(x).to(torch.bfloat16).cuda()
+            idd = torch.from_numpy(ids).cuda()
+            y = torch.empty((t, 6, 1408), device="cuda")
+            ws = torch.empty(kq.matmul_id_workspace_bytes(t, 6, 64), dtype=torch.uint8, device="cuda")
+            line = {"sweep": f"moe_{cname}_e64_1408x2048_top6", "tokens": t, "pool": len(pool)}
+            for name, path in (("plain", kq.PATH_SIMPLE), ("gemm", kq.PATH_GEMM)):
+                def fn():
+                    for wi in pool:
+                        kq.matmul_id(wi, codec, xd, idd, out=y, workspace=ws, path=path)
+                line[name + "_us"] = round(time_graph(torch, fn, 5, 3, None) * 1e3 / (5 * len(pool)), 2)
+            print(json.dumps(line), flush=True)
+            del pool, wd
+            torch.cuda.empty_cache()
+
+
 def run_sweep(args):
     """Dispatch evidence: per-call time of the bandwidth kernel against the
     tensor-core kernel over the activation-row count (dense Q4_K product,
@@ -704,8 +729,8 @@ def run_sweep(args):
 
     kq.lib()
     l2 = l2_bytes(0)
-    if args.sweep == "q8_0":
-        run_q8_0_sweep(torch, kq, l2)
+    if args.sweep in ("q8_0", "id_codecs"):
+        (run_q8_0_sweep if args.sweep == "q8_0" else run_id_codecs_sweep)(torch, kq, l2)
         status = kq.device_status()
         if status != 0:
             raise SystemExit(f"device status {status} after the sweep")
@@ -772,7 +797,7 @@ def main():
                     help="GEMV call ordering in --profile (the headline step uses independent calls)")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the other workloads' numbers (prefill GEMM, MoE, TQ1, Q8_0)")
-    ap.add_argument("--sweep", default=None, choices=["dispatch", "tq1", "q8_0"],
+    ap.add_argument("--sweep", default=None, choices=["dispatch", "tq1", "q8_0", "id_codecs"],
                     help="print the dispatch sweep (bandwidth vs tensor-core kernel) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
