@@ -173,9 +173,13 @@ KQ_API int kq_matmul_ex(int type, const void *w, int64_t n, int64_t k,
  * Tokens routed to one expert are grouped before the decode, so each hit
  * expert's weights are streamed once per group of tokens; the result of a
  * (t, s) row does not depend on the other tokens' ids.
- * Paths: Q4_K with bf16 x runs the grouped tensor-core GEMM (weights
- * rounded to bf16, like kq_matmul's GEMM); Q4_K with fp32 x the grouped
- * mat-vec (exact fp32 weights); other codecs the plain grouped kernel.
+ * Paths: Q4_K with bf16 x runs the few-pairs tensor-core kernel or, past
+ * 32 routed pairs per expert, the grouped tensor-core GEMM (weights rounded
+ * to bf16, like kq_matmul's GEMM); Q4_K with fp32 x the grouped mat-vec up
+ * to one pair per expert (exact fp32 weights), else the few-pairs kernel;
+ * Q8_0 and Q5_K (K % 256 == 0) and Q2_K (K % 1024 == 0) with bf16 x the
+ * grouped tensor-core GEMM (expert_stride a multiple of 16 bytes); other
+ * codecs and shapes the plain grouped kernel.
  */
 KQ_API size_t kq_matmul_id_workspace_bytes(int64_t n_tokens, int64_t top_k, int64_t n_experts);
 KQ_API int kq_matmul_id(int type, const void *w, int64_t n_experts, int64_t n, int64_t k,
