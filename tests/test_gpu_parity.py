@@ -577,6 +577,34 @@ def test_matmul_gemm_q5_k_decodes_every_code_exactly(kq):
     assert kq.device_status() == 0
 
 
+@pytest.mark.parametrize("codec,k", [(synth.Q8_0, 1408), (synth.Q2_K, 512), (synth.Q5_K, 256 * 3)])
+def test_matmul_gemm_shapes_it_cannot_take(kq, codec, k):
+    """K that the tensor-core kernel's raw units do not tile (Q8_0: 44
+    blocks, Q2_K: two super-blocks) is refused on the explicit path and
+    served by the plain kernel on the automatic one; Q5_K at K = 768 is
+    taken (one super-block a unit)."""
+    import torch
+
+    r = rng(61 + k + codec)
+    n, m = 200, 24
+    w = synth.gen_weights(codec, n, k, r)
+    x = synth.gen_x(m, k, "bf16", r)
+    wd, xd = to_device_w(w), to_device_x(x, "bf16")
+    ref = oracle.matmul(codec, w, k, x, threads=8)
+    y = kq.matmul(wd, codec, xd).cpu().numpy()
+    if codec == synth.Q5_K:
+        g = kq.matmul(wd, codec, xd, path=kq.PATH_GEMM).cpu().numpy()
+        assert np.array_equal(y.view(np.uint32), g.view(np.uint32))
+        assert row_rel_err(y, ref) <= TOL["bf16"]
+    else:
+        with pytest.raises(kq.KQError):
+            kq.matmul(wd, codec, xd, path=kq.PATH_GEMM)
+        ys = kq.matmul(wd, codec, xd, path=kq.PATH_SIMPLE).cpu().numpy()
+        assert np.array_equal(y.view(np.uint32), ys.view(np.uint32))
+        assert row_rel_err(y, ref) <= FP32_PATH_TOL
+    assert kq.device_status() == 0
+
+
 def test_matmul_tq1_auto_prefill_uses_the_tensor_cores(kq):
     r = rng(41)
     n, k, m = 384, 2048, 40
