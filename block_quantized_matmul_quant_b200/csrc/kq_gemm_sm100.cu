@@ -61,20 +61,18 @@ namespace {
 
 constexpr int BM = 128;            // weight rows per tile (MMA M)
 constexpr int BK = 64;             // K per swizzle atom (128 bytes of bf16); a stage holds CPS atoms
-// Raw weights move in units of one TMA box row: a Q4_K super-block (144
-// bytes, 256 K) or four TQ1_G128 blocks (112 bytes, 512 K; a box row must be
-// a multiple of 16 bytes, so TQ1 rows need K % 512 == 0).
-// Q8_0: eight 34-byte blocks (272 bytes, 256 K), copied as 16-bit elements
-// (a box row holds at most 256 elements).  ELEM: bytes per tensor-map
-// element.
+// Raw weights move in units of one TMA box row, the fewest whole blocks
+// whose bytes are a multiple of 16 (so K must be a multiple of the unit's
+// K): a Q4_K super-block (144 bytes, 256 K), a Q5_K super-block (176, 256),
+// eight Q8_0 blocks (272, 256), four Q2_K super-blocks (336, 1024) or four
+// TQ1_G128 blocks (112, 512).  ELEM: bytes per tensor-map element -- 2 for
+// the units above 256 bytes, since a box row holds at most 256 elements.
 template <int FMT> struct RawUnit;
 template <> struct RawUnit<KQ_Q4_K> { static constexpr int BYTES = 144, K = 256, ELEM = 1; };
-template <> struct RawUnit<KQ_TQ1_G128> { static constexpr int BYTES = 112, K = 512, ELEM = 1; };
-template <> struct RawUnit<KQ_Q8_0> { static constexpr int BYTES = 272, K = 256, ELEM = 2; };
-// Q2_K: four 84-byte super-blocks (336 bytes, 1024 K, 16-bit elements).
-template <> struct RawUnit<KQ_Q2_K> { static constexpr int BYTES = 336, K = 1024, ELEM = 2; };
-// Q5_K: one 176-byte super-block (256 K).
 template <> struct RawUnit<KQ_Q5_K> { static constexpr int BYTES = 176, K = 256, ELEM = 1; };
+template <> struct RawUnit<KQ_Q8_0> { static constexpr int BYTES = 272, K = 256, ELEM = 2; };
+template <> struct RawUnit<KQ_Q2_K> { static constexpr int BYTES = 336, K = 1024, ELEM = 2; };
+template <> struct RawUnit<KQ_TQ1_G128> { static constexpr int BYTES = 112, K = 512, ELEM = 1; };
 constexpr int raw_unit_bytes(int type) {
     return type == KQ_TQ1_G128 ? 112 : type == KQ_Q8_0 ? 272 : type == KQ_Q2_K ? 336 : type == KQ_Q5_K ? 176 : 144;
 }
@@ -82,12 +80,11 @@ constexpr int raw_unit_k(int type) { return type == KQ_TQ1_G128 ? 512 : type == 
 constexpr int raw_stage_bytes(int type) { return BM * raw_unit_bytes(type); }
 constexpr int RAW_WARP = 6;  // raw weight producer
 constexpr int DEC_WARP0 = 7;
-// Decoder warps per format: eight (two groups) for the K-quants and Q8_0; sixteen
-// (four groups) for TQ1_G128, whose integer digit decode bounds the narrow
-// tiles.
-// Measured on B200 (µs): Q4_K 512x11008x4096 65.9 with eight against 67.7
-// with sixteen, 16 rows 25.8 against 26.3; TQ1 512x5120x17408 135.9 against
-// 140.0 but 16 rows 108.0 against 101.0.
+// Decoder warps per format: eight (two groups) for the K-quants and Q8_0,
+// sixteen (four groups) for TQ1_G128, whose integer digit decode bounds the
+// narrow tiles.  Measured on B200 (µs): Q4_K 512x11008x4096 65.9 with eight
+// against 67.7 with sixteen, 16 rows 25.8 against 26.3; TQ1 512x5120x17408
+// 135.9 against 140.0 but 16 rows 108.0 against 101.0.
 template <int FMT> constexpr int dec_warps() { return FMT == KQ_TQ1_G128 ? 16 : 8; }
 template <int FMT> constexpr int num_threads() { return (DEC_WARP0 + dec_warps<FMT>()) * 32; }
 constexpr int EPI_WARP0 = 2;
