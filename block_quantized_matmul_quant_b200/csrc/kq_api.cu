@@ -427,13 +427,25 @@ int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_e
     cudaStream_t s = (cudaStream_t)stream;
     // Q4_K: the few-pairs tensor-core kernel (a gate pass and an up pass per
     // unit), except fp32 activations up to one pair per expert (the
-    // bandwidth kernel); other codecs the plain kernel
+    // bandwidth kernel).  Q8_0, Q2_K and Q5_K with bf16 activations: the
+    // grouped tensor-core GEMM twice over one grouping -- the up projection
+    // into y, then the gate projection, whose epilogue writes
+    // act(gate) * y.  Other codecs and shapes: the plain kernel.
     const bool few = x_dtype == KQ_F32 && pairs <= ID_GEMV_MAX_PAIRS_PER_EXPERT * n_experts;
     const bool tc = moe_mma_supported(type, n, k, x_dtype, y_dtype) && !(few && moe_gemv_supported(type, n, k, n_experts));
+    const bool gemm = !tc && type != KQ_Q4_K && gemm_supported(type, n, k, x_dtype, y_dtype, true) &&
+                      expert_stride % 16 == 0;
     a.tc_i8 = tc && pairs <= ID_TC_I8_MAX_PAIRS_PER_EXPERT * n_experts;
-    if (id_group(a, ids, pairs, y, y_dtype, tc ? moe_mma_bn(x_dtype, a.tc_i8) : 0, s) != cudaSuccess)
-        return KQ_ERR_CUDA;
+    const int bn = tc ? moe_mma_bn(x_dtype, a.tc_i8) : gemm ? gemm_id_bn(n_tokens, top_k, n_experts) : 0;
+    if (id_group(a, ids, pairs, y, y_dtype, bn, s) != cudaSuccess) return KQ_ERR_CUDA;
     if (tc) return to_status(launch_moe_mma(a, s));
+    if (gemm) {
+        IdArgs up = a;
+        up.w = w_up;
+        const cudaError_t e = launch_gemm_id(up, bn, s, false);
+        if (e != cudaSuccess) return to_status(e);
+        return to_status(launch_gemm_id(a, bn, s, true));
+    }
     if (moe_gemv_supported(type, n, k, n_experts)) return to_status(launch_moe_gemv(a, s));
     return to_status(launch_simple_glu(a, s));
 }

@@ -116,7 +116,14 @@ struct GemmParams {
     const int32_t *id_n_tiles;
     int top_k;
     int n_pairs, n_experts;   // entries of perm; experts of the stack
+    // expert-indexed GLU, second pass: y = act(this product) * y, y holding
+    // the up projection written by the first pass (glu: 0 plain store, 1
+    // combine; act: KQ_ACT_*)
+    int glu, act;
 };
+
+__device__ __forceinline__ float load_out(const float *p) { return *p; }
+__device__ __forceinline__ float load_out(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
 
 // One output tile: weight rows n0.. of expert e times BN activation rows.
 // Dense: activation rows m0..m0+rows-1.  Expert-indexed: the activation rows
@@ -551,8 +558,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmap_x, const CUten
                         if (c0 + j < t.rows) {
                             // output row: the activation row, or the (token, slot) pair
                             const int64_t m = ID ? (int64_t)__ldg(p.perm + t.m0 + c0 + j) : (int64_t)(t.m0 + c0 + j);
-                            if (!ID || KQ_DCHECK(m >= 0 && m < p.n_pairs, p.err))
-                                store_out(y + m * p.n + n, __uint_as_float(r[j]));
+                            if (!ID || KQ_DCHECK(m >= 0 && m < p.n_pairs, p.err)) {
+                                YT *dst = y + m * p.n + n;
+                                const float v = __uint_as_float(r[j]);
+                                if (ID && p.glu) store_out(dst, glu_activation(v, p.act) * load_out(dst));
+                                else store_out(dst, v);
+                            }
                         }
                     }
                 }
@@ -981,7 +992,7 @@ cudaError_t launch_id_fmt(const CUtensorMap &tx, const CUtensorMap &tw, const Ge
 
 }  // namespace
 
-cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
+cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s, bool glu_combine) {
     if (!encode_fn()) return cudaErrorNotSupported;
     const int sms = sm_count();
     GemmParams p = {};
@@ -1001,6 +1012,8 @@ cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s) {
     p.top_k = a.x_div();
     p.n_pairs = (int)(a.n_tokens * a.top_k);
     p.n_experts = (int)a.n_experts;
+    p.glu = glu_combine ? 1 : 0;
+    p.act = a.act;
     CUtensorMap tx, tw;
     if (!encode_x_map(&tx, a.x, a.x_rows(), a.k, 1) ||
         !encode_w_map(&tw, a.w, a.n, a.k, a.n_experts, a.expert_stride, (int)a.type))

@@ -89,7 +89,8 @@ cudaError_t launch_gemm(int type, const void *w, int64_t n, int64_t k, const voi
 // Expert-indexed form over the grouping's token tiles (a.tiles / a.n_tiles,
 // written by launch_moe_tiles with the same bn).
 int gemm_id_bn(int64_t n_tokens, int64_t top_k, int64_t n_experts);
-cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s);
+// glu_combine: the GLU's second pass, y = act(this product) * y (a.act).
+cudaError_t launch_gemm_id(const IdArgs &a, int bn, cudaStream_t s, bool glu_combine = false);
 // Expert-indexed tensor-core kernel for few pairs per expert
 // (kq_moe_mma.cu), over token tiles of moe_mma_bn(x_dtype) pairs.
 bool moe_mma_supported(int type, int64_t n, int64_t k, int x_dtype, int y_dtype);

@@ -239,11 +239,15 @@ KQ_API int kq_matmul_id_noalloc(int type, const void *w, int64_t n_experts, int6
  *                 out as kq_matmul_id's w (device)
  *   act           KQ_ACT_SILU or KQ_ACT_GELU_TANH
  * Other arguments, the workspace (kq_matmul_id_workspace_bytes), invalid
- * ids (NaN rows, device error word) and errors as kq_matmul_id.  Q4_K up to
- * one routed pair per expert runs the grouped bandwidth kernel (a tile
- * holding each output row's gate and up weights), beyond it the few-pairs
- * tensor-core kernel (a gate pass and an up pass per unit over the same
- * activation tile); other codecs the plain grouped kernel.
+ * ids (NaN rows, device error word) and errors as kq_matmul_id.  Q4_K with
+ * fp32 x up to one routed pair per expert runs the grouped bandwidth kernel
+ * (a tile holding each output row's gate and up weights), otherwise the
+ * few-pairs tensor-core kernel (a gate pass and an up pass per unit over
+ * the same activation tile).  Q8_0 and Q5_K (K % 256 == 0) and Q2_K
+ * (K % 1024 == 0) with bf16 x run the grouped tensor-core GEMM twice over
+ * one grouping: the up projection into y, then the gate projection, whose
+ * epilogue writes act(gate) * y (a bf16 y holds the up projection rounded
+ * to bf16 in between).  Other codecs and shapes: the plain grouped kernel.
  */
 KQ_API int kq_matmul_id_glu(int type, const void *w_gate, const void *w_up, int64_t n_experts,
                             int64_t n, int64_t k, int64_t expert_stride, const void *x, int x_dtype,

@@ -807,7 +807,10 @@ def test_matmul_id_grouped_gemv_skewed_and_nonfinite(kq):
     (synth.Q4_K, 32, 6, 64, 1408, 2048),   # the MoE workload's shape, gate and up stacks
     (synth.Q4_K, 20, 4, 5, 300, 1024),     # several rounds per expert
     (synth.Q4_K, 7, 3, 4, 129, 1280),      # ragged tiles, a group with idle lanes
-    (synth.Q8_0, 9, 2, 3, 70, 256),        # other codecs: the plain fused kernel
+    (synth.Q8_0, 9, 2, 3, 70, 256),        # Q8_0, Q2_K, Q5_K: two grouped GEMMs with bf16
+    (synth.Q2_K, 40, 4, 6, 300, 2048),     # activations (up, then gate combined in the
+    (synth.Q5_K, 9, 2, 3, 130, 512),       # epilogue), the plain fused kernel with fp32
+    (synth.Q8_0, 9, 2, 3, 70, 1408),       # K the GEMM does not tile: the plain kernel
     (synth.Q6_K, 9, 2, 3, 70, 512),
     (synth.TQ1_G128, 9, 2, 3, 70, 384),
 ])
@@ -830,10 +833,26 @@ def test_matmul_id_glu(kq, codec, t, top_k, e, n, k, act, xdt):
     assert np.all(np.isnan(y[t // 2, 0]))
     good = ~np.isnan(ref[..., 0])
     # the product of two results each within its path's bound
-    tol = 2 * (GEMV_TOL if codec == synth.Q4_K else FP32_PATH_TOL)
+    if xdt == "bf16" and _grouped_gemm_takes(codec, k):
+        tol = 2 * TOL["bf16"]   # bf16 weights on the tensor cores
+    else:
+        tol = 2 * (GEMV_TOL if codec == synth.Q4_K else FP32_PATH_TOL)
     assert row_rel_err(y[good], ref[good]) <= tol
     assert kq.device_status() == -9
     assert kq.device_status() == 0
+    if xdt == "bf16" and _grouped_gemm_takes(codec, k):
+        # tight: act(gate) * up from the two grouped GEMM products themselves
+        # (each checked against the oracle elsewhere), so a swapped or
+        # misplaced operand of the combine cannot hide in the bf16 bound
+        xd, idd = to_device_x(x, xdt), torch.from_numpy(ids).cuda()
+        g = kq.matmul_id(to_device_w(wg), codec, xd, idd, path=kq.PATH_GEMM).cpu().numpy().astype(np.float64)
+        u = kq.matmul_id(to_device_w(wu), codec, xd, idd, path=kq.PATH_GEMM).cpu().numpy().astype(np.float64)
+        kq.device_status()   # the invalid id flagged again
+        if act == "silu":
+            a = g / (1.0 + np.exp(-g))
+        else:
+            a = 0.5 * g * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (g + 0.044715 * g ** 3)))
+        assert row_rel_err(y[good], (a * u)[good]) <= 1e-5
 
 
 def _pair_refs(codec, w, k, xs, ids):
