@@ -714,6 +714,16 @@ def run_id_codecs_sweep(torch, kq, l2):
             print(json.dumps(line), flush=True)
             del pool, wd
             torch.cuda.empty_cache()
+        # the fused GLU at 32 tokens (two grouped GEMMs over one grouping)
+        # beside one expert product on the same routing
+        wl = synth.Workload("sweep_id", "moe", codec, 1408, 2048, 32, "bf16", "f32", n_experts=64, top_k=6)
+        line = {"sweep": f"moe_{cname}_e64_1408x2048_top6_glu", "tokens": 32}
+        for glu in (False, True):
+            st = PoolStep(torch, kq, wl, l2, glu=glu)
+            line["glu_us" if glu else "product_us"] = round(time_graph(torch, st.run, 5, 3, None) * 1e3 / (5 * st.pool), 2)
+            del st
+            torch.cuda.empty_cache()
+        print(json.dumps(line), flush=True)
 
 
 def run_sweep(args):
